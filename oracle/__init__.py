@@ -1,0 +1,10 @@
+"""fp64 CPU oracle for Heavily Compressed Attention (HCA).
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package.  It shares no code with
+the CUDA library in ``compressed_long_context_b200``.
+"""
+from .oracle import (  # noqa: F401
+    compress, round_bf16, visible_entries, prefill_rows, decode, num_threads,
+    bf16_bits, bits_to_f64,
+)
