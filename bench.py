@@ -1,0 +1,451 @@
+"""Benchmark of the HCA hot path on B200 (one JSON line on stdout).
+
+Workload (the decode configuration the headline metric is quoted on): 64 sequences of
+131072 tokens, Hq=64 query heads sharing one 512-dim KV head, blocks of 128, a raw
+window of 128 tokens; pooling weights ~N(0, 0.5); bf16 inputs ~N(0, 1); seed 1.
+
+One step = the whole path for one batch:
+    hca_compress  (raw K/V [64, 131072, 1, 512] -> 1024 cached entries per sequence)
+    hca_decode    (one query per sequence over 1023 entries + 128 raw tokens;
+                   split kernel + combine kernel)
+value = queries of all ranks / device time of the step (max over ranks).
+
+Also reported, measured in the same run: the decode kernels alone (cache resident,
+L2 flushed before each call) and the 128K prefill (T=131072, Hq=64, d=512, W=128,
+1% of raw keys x8; seed 2) in TFLOP/s.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU: torchrun, one rank per GPU, each rank a full batch (weak scaling).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "HCA decode queries/s, prefill TFLOP/s, % of HBM/TC roofline (1 B200)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def compress_bytes(B, T, Hkv, d, dv, blk):
+    Nc = T // blk
+    return B * Nc * Hkv * (blk * (d + dv) * 2 + 2 * (d + dv)) + B * Nc * blk * 4
+
+
+def decode_bytes(B, L, Hq, Hkv, d, dv, blk, W):
+    nc = max(0, (L - W) // blk)
+    nw = min(W, L)
+    per = Hq * d * 2 + (nc + nw) * Hkv * (d + dv) * 2 + Hq * dv * 4 + 4
+    return B * per
+
+
+def prefill_flops(B, T, Hq, d, dv, blk, W):
+    t = np.arange(T, dtype=np.int64)
+    a = t - W + 1
+    nc = np.where(a > 0, a // blk, 0)
+    keys = int((nc + np.minimum(W, t + 1)).sum())
+    return 2.0 * B * Hq * keys * (d + dv), keys
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if len(s) > 2 + i and s[2 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def l2_flush_buffer():
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    return torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+
+
+def traffic_for(kernel_key, source_files):
+    """Per-launch DRAM bytes from the committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent:
+        return None
+    h = hashlib.sha256()
+    for rel in source_files:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if ent.get("source_sha256") != h.hexdigest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- reference arm (the CPU oracle)
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    sys.path.insert(0, ROOT)
+    import oracle
+    from compressed_long_context_b200 import workloads as wl
+    cfg = wl.DECODE_128K
+    one = cfg.scaled(B=1)
+    inp = wl.decode_inputs(one, "cpu")
+    kb, vb = oracle.bf16_bits(inp["k"]), oracle.bf16_bits(inp["v"])
+    wn, qb = inp["w"].numpy(), oracle.bf16_bits(inp["q"])
+    kwb, vwb = oracle.bf16_bits(inp["kw"]), oracle.bf16_bits(inp["vw"])
+    seq = inp["seqlens"].numpy()
+    scale = 1.0 / np.sqrt(cfg.d)
+
+    def step():
+        kc, vc = oracle.compress(kb, vb, wn, cfg.blk)
+        out = oracle.decode(qb, oracle.round_bf16(kc), oracle.round_bf16(vc), kwb, vwb, seq, cfg.blk, cfg.W,
+                            scale)
+        return out
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    qps = 1.0 / dt
+    cores = oracle.num_threads()
+    sample = ("oracle fp64 compress of one 131072-token sequence (K and V, d=512) + decode of its query "
+              "(64 heads, 1023 entries + 128 window), per step")
+    line = {"metric": METRIC, "value": qps, "unit": "queries/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "L": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
+                       "blk": cfg.blk, "W": cfg.W, "sample_sequences_per_step": 1},
+            "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_sample():
+    """The oracle as it stands, on this host, for a bounded sample: 2 sequences of the workload."""
+    import oracle
+    from compressed_long_context_b200 import workloads as wl
+    cfg = wl.DECODE_128K
+    n = 2
+    inp = wl.decode_inputs(cfg.scaled(B=n), "cpu")
+    kb, vb = oracle.bf16_bits(inp["k"]), oracle.bf16_bits(inp["v"])
+    scale = 1.0 / np.sqrt(cfg.d)
+    t0 = time.perf_counter()
+    kc, vc = oracle.compress(kb, vb, inp["w"].numpy(), cfg.blk)
+    oracle.decode(oracle.bf16_bits(inp["q"]), oracle.round_bf16(kc), oracle.round_bf16(vc),
+                  oracle.bf16_bits(inp["kw"]), oracle.bf16_bits(inp["vw"]), inp["seqlens"].numpy(), cfg.blk,
+                  cfg.W, scale)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "queries/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d sequences of the workload: oracle fp64 compress (131072 raw tokens, K and V) + decode "
+                      "(64 heads, 1023 entries + 128 window), %.1f s" % (n, dt)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    world, rank, local = dist_setup(args)
+    sys.path.insert(0, ROOT)
+    import compressed_long_context_b200 as hca
+    from compressed_long_context_b200 import _lib, workloads as wl
+
+    pk, pk_kind = peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = wl.DECODE_128K
+    scale = 1.0 / np.sqrt(cfg.d)
+    inp = wl.decode_inputs(cfg, dev)
+    k, v, w, q, kw, vw, seq = (inp[x] for x in ("k", "v", "w", "q", "kw", "vw", "seqlens"))
+    B, L = cfg.B, cfg.T
+    Nc = L // cfg.blk
+    kc = torch.empty((B, Nc, 1, cfg.d), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty((B, Nc, 1, cfg.dv), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((B, cfg.Hq, cfg.dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(hca.decode_workspace_size(B, cfg.Hq, cfg.Hkv, cfg.dv), dtype=torch.uint8, device=dev)
+    flush = l2_flush_buffer()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hca.compress(k, v, w, cfg.blk, kc=kc, vc=vc)
+        hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+
+    # ---- timed region: K steps, each bracketed by events; L2 flushed between steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(args.steps):
+            flush.zero_()
+            a, m, b = ev[i]
+            a.record(stream)
+            hca.compress(k, v, w, cfg.blk, kc=kc, vc=vc)
+            m.record(stream)
+            hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
+            b.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, _, b in ev]
+    comp_ms = [a.elapsed_time(m) for a, m, _ in ev]
+    dec_in_step_ms = [m.elapsed_time(b) for _, m, b in ev]
+    hca.get_device_error()
+    t_step = max_over_ranks(sum(step_ms) / 1e3, world)
+    ms_per_step = t_step * 1e3 / args.steps
+    value = world * B * args.steps / t_step
+
+    # compress roofline (dominant kernel of the step)
+    cbytes = compress_bytes(B, L, 1, cfg.d, cfg.dv, cfg.blk)
+    c_avg = sum(comp_ms) / len(comp_ms) / 1e3
+    c_gbs = cbytes / c_avg / 1e9
+    roof = {"bound": "hbm", "kernel": "compress_kernel<512,512>", "achieved": c_gbs, "peak": pk["hbm_gbs"],
+            "unit": "GB/s", "frac": c_gbs / pk["hbm_gbs"],
+            "traffic": traffic_for("compress_decode_B64_L131072",
+                                   ["compressed_long_context_b200/csrc/compress.cuh"]),
+            "algorithmic_bytes_per_launch": cbytes, "peak_kind": pk_kind + " (hbm_gbs)"}
+
+    # ---- decode alone: cache resident, L2 flushed before each call
+    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        a, b = dev_ev[i]
+        a.record(stream)
+        hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    d_ms = [a.elapsed_time(b) for a, b in dev_ev]
+    d_avg = max_over_ranks(sum(d_ms) / len(d_ms) / 1e3, world)
+    dbytes = decode_bytes(B, L, cfg.Hq, 1, cfg.d, cfg.dv, cfg.blk, cfg.W)
+    d_gbs = dbytes / d_avg / 1e9
+    decode_part = {"queries_per_s": world * B / d_avg, "us_per_call": d_avg * 1e6,
+                   "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + decode_combine_kernel",
+                                "achieved": d_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                "frac": d_gbs / pk["hbm_gbs"], "algorithmic_bytes_per_call": dbytes,
+                                "traffic": traffic_for("decode_B64_L131072",
+                                                       ["compressed_long_context_b200/csrc/decode.cuh"])},
+                   "median_us_per_call": statistics.median(d_ms) * 1e3,
+                   "decode_in_step_us": statistics.median(dec_in_step_ms) * 1e3}
+
+    # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+        hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+        hk.copy_(k)
+        hv.copy_(v)
+        hw, hq, hkw, hvw, hs = (x.cpu().pin_memory() for x in (w, q, kw, vw, seq))
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dk, dvv = torch.empty_like(k), torch.empty_like(v)
+        dw, dq, dkw, dvw, ds = (torch.empty_like(x) for x in (w, q, kw, vw, seq))
+        h2d = sum(x.numel() * x.element_size() for x in (hk, hv, hw, hq, hkw, hvw, hs))
+        d2h = hout.numel() * hout.element_size()
+        del k, v
+        torch.cuda.empty_cache()
+
+        def e2e_step():
+            for hsrc, ddst in ((hk, dk), (hv, dvv), (hw, dw), (hq, dq), (hkw, dkw), (hvw, dvw), (hs, ds)):
+                ddst.copy_(hsrc, non_blocking=True)
+            hca.compress(dk, dvv, dw, cfg.blk, kc=kc, vc=vc)
+            hca.decode(dq, kc, vc, dkw, dvw, ds, cfg.blk, cfg.W, scale, out=out, workspace=ws)
+            hout.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ne = max(2, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        te = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+        e2e = {"value": world * B * ne / te, "unit": "queries/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": ne}
+        del hk, hv, dk, dvv
+        torch.cuda.empty_cache()
+    else:
+        del k, v
+        torch.cuda.empty_cache()
+
+    # ---- prefill 128K (TFLOP/s)
+    prefill_part = None
+    if not args.no_prefill:
+        pc = wl.PREFILL_128K
+        pin = wl.prefill_inputs(pc, dev)
+        pkc, pvc = hca.compress(pin["k"], pin["v"], pin["w"], pc.blk)
+        pout = torch.empty((1, pc.T, pc.Hq, pc.dv), dtype=torch.bfloat16, device=dev)
+        for _ in range(2):
+            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
+        torch.cuda.synchronize()
+        hca.get_device_error()
+        np_steps = max(2, min(args.steps, 5))
+        pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True)) for _ in range(np_steps)]
+        for i in range(np_steps):
+            flush.zero_()
+            a, m, b = pev[i]
+            a.record(stream)
+            hca.compress(pin["k"], pin["v"], pin["w"], pc.blk, kc=pkc, vc=pvc)
+            m.record(stream)
+            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
+            b.record(stream)
+        torch.cuda.synchronize()
+        hca.get_device_error()
+        p_ms = max_over_ranks(statistics.median([m.elapsed_time(b) for _, m, b in pev]), world)
+        c3_ms = statistics.median([a.elapsed_time(m) for a, m, _ in pev])
+        flops, keys = prefill_flops(1, pc.T, pc.Hq, pc.d, pc.dv, pc.blk, pc.W)
+        tf = flops / (p_ms / 1e3) / 1e12
+        peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        prefill_part = {"workload": pc.name, "tflops": tf, "ms": p_ms, "compress_ms": c3_ms,
+                        "algorithmic_flops": flops, "keys_per_head": keys,
+                        "roofline": {"bound": "tensor", "kernel": "prefill_kernel<512>", "achieved": tf,
+                                     "peak": peak_tf, "unit": "TFLOP/s", "frac": tf / peak_tf,
+                                     "peak_kind": pk_kind + " (bf16_tflops_sustained)",
+                                     "frac_of_burst": tf / pk["bf16_tflops"],
+                                     "traffic": traffic_for("prefill_T131072",
+                                                            ["compressed_long_context_b200/csrc/prefill.cuh"])}}
+        del pin, pkc, pvc, pout
+        torch.cuda.empty_cache()
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = cpu_baseline_sample()
+
+    clocks = sampler.summary()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded; no dataset)",
+                "config": {"workload": cfg.name, "B": B, "L": L, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
+                           "blk": cfg.blk, "W": cfg.W, "step": "hca_compress(raw K/V) + hca_decode",
+                           "l2": "flushed (2x L2 memset) before every timed step; raw K/V 17.2 GB > L2",
+                           "parallelism": "dp%d (independent batches, no collective)" % world},
+                "roofline": roof, "decode": decode_part, "prefill": prefill_part,
+                "cpu_baseline": cpu_base, "e2e": e2e,
+                "gpu_launches": 3 * args.steps, "clocks": clocks,
+                "libhca": os.path.relpath(_lib.LIB_PATH, ROOT)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+"""compressed_long_context_b200 -- Heavily Compressed Attention (HCA) on B200.
+
+A thin PyTorch-facing binding over the C ABI of ``libhca.so`` (include/hca.h).
+Every step of the computation runs in the library's CUDA kernels; this module only
+checks dtypes/devices, allocates outputs with PyTorch and passes raw device pointers
+and the current CUDA stream.  If the library is missing, calls fail loudly.
+
+The layer (web pages on ERNIE 5.5 Flash Base: official blog, section 2.1; Zhidx
+article, section "1. Latent-Gated Sparse Attention"): every 128 tokens of K/V are
+pooled into one cached entry, and each query attends, in one causal softmax, to all
+completed entries plus a window of the W most recent raw tokens.
+"""
+import torch
+
+from . import _lib
+from ._lib import (HCA_OUT_F32, HCA_OUT_GATE, HCA_PAGED, HCA_QK_NORM,  # noqa: F401
+                   HCA_WRITE_LSE)
+
+__all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "get_device_error",
+           "status_string"]
+
+
+class HCAError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__("%s: %s" % (where, status_string(code)))
+
+
+def status_string(code: int) -> str:
+    return _lib.load().hca_status_string(int(code)).decode()
+
+
+def _check(code, where):
+    if code != _lib.HCA_OK:
+        raise HCAError(code, where)
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t, dtype, name, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def get_device_error(device=None) -> None:
+    """Synchronise the current stream and raise if a kernel recorded a device-side error."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    _check(_lib.load().hca_get_device_error(_stream(device)), "device")
+
+
+def compress(k, v, w=None, blk=128, kc=None, vc=None):
+    """Pool every complete block of ``blk`` raw rows into one cache entry.
+
+    k [B,T,Hkv,d], v [B,T,Hkv,dv] bf16; w [B,T] fp32 or None (mean pooling).
+    Returns (kc, vc) of shape [B, T // blk, Hkv, d|dv] bf16.
+    """
+    _need(k, torch.bfloat16, "k")
+    _need(v, torch.bfloat16, "v", k.device)
+    B, T, Hkv, d = k.shape
+    dv = v.shape[3]
+    if w is not None:
+        _need(w, torch.float32, "w", k.device)
+    Nc = T // blk
+    if kc is None:
+        kc = torch.empty((B, Nc, Hkv, d), dtype=torch.bfloat16, device=k.device)
+    if vc is None:
+        vc = torch.empty((B, Nc, Hkv, dv), dtype=torch.bfloat16, device=k.device)
+    _need(kc, torch.bfloat16, "kc", k.device)
+    _need(vc, torch.bfloat16, "vc", k.device)
+    rc = _lib.load().hca_compress(_p(k), _p(v), _p(w), _p(kc), _p(vc), B, T, Hkv, d, dv, blk, _stream(k.device))
+    _check(rc, "hca_compress")
+    return kc, vc
+
+
+def prefill(q, k, v, kc, vc, blk, W, scale, out=None, want_lse=False, out_f32=False):
+    """Causal HCA attention for every position.  Returns out [B,T,Hq,dv] (and lse [B,Hq,T])."""
+    _need(q, torch.bfloat16, "q")
+    for name, t in (("k", k), ("v", v), ("kc", kc), ("vc", vc)):
+        _need(t, torch.bfloat16, name, q.device)
+    B, T, Hq, d = q.shape
+    Hkv, dv = k.shape[2], v.shape[3]
+    if out is None:
+        out = torch.empty((B, T, Hq, dv), dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
+    _need(out, torch.float32 if out_f32 else torch.bfloat16, "out", q.device)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device) if want_lse else None
+    flags = (HCA_WRITE_LSE if want_lse else 0) | (HCA_OUT_F32 if out_f32 else 0)
+    rc = _lib.load().hca_prefill(_p(q), _p(k), _p(v), _p(kc), _p(vc), _p(out), _p(lse), B, T, Hq, Hkv, d, dv,
+                                 blk, W, float(scale), flags, _stream(q.device))
+    _check(rc, "hca_prefill")
+    return (out, lse) if want_lse else out
+
+
+def decode_workspace_size(B, Hq, Hkv, dv) -> int:
+    """Bytes of scratch ``decode`` needs on the current device."""
+    return int(_lib.load().hca_decode_workspace_size(B, Hq, Hkv, dv))
+
+
+def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size=0,
+           gq=None, gk=None, eps=1e-6, gate=None, out=None, workspace=None):
+    """One query per sequence at position seqlens[b]-1 over its compressed cache + raw window.
+
+    q [B,Hq,d] bf16; kc/vc contiguous [B,Nmax,Hkv,d|dv] or page pools [P,page_size,Hkv,d|dv]
+    with page_table [B,max_pages] int32; kw/vw [B,W,Hkv,d|dv] bf16; seqlens [B] int32;
+    gq/gk [d] fp32 for QK RMSNorm; gate [B,Hq,dv] bf16 logits.  Returns out [B,Hq,dv] fp32.
+    """
+    _need(q, torch.bfloat16, "q")
+    dev = q.device
+    for name, t in (("kc", kc), ("vc", vc), ("kw", kw), ("vw", vw)):
+        _need(t, torch.bfloat16, name, dev)
+    _need(seqlens, torch.int32, "seqlens", dev)
+    B, Hq, d = q.shape
+    Hkv, dv = kc.shape[2], vc.shape[3]
+    flags = 0
+    max_pages = num_pages = 0
+    Nmax = kc.shape[1]
+    if page_table is not None:
+        _need(page_table, torch.int32, "page_table", dev)
+        flags |= HCA_PAGED
+        max_pages = page_table.shape[1]
+        num_pages = kc.shape[0]
+        page_size = kc.shape[1]
+        Nmax = 0
+    if gq is not None or gk is not None:
+        _need(gq, torch.float32, "gq", dev)
+        _need(gk, torch.float32, "gk", dev)
+        flags |= HCA_QK_NORM
+    if gate is not None:
+        _need(gate, torch.bfloat16, "gate", dev)
+        flags |= HCA_OUT_GATE
+    if out is None:
+        out = torch.empty((B, Hq, dv), dtype=torch.float32, device=dev)
+    _need(out, torch.float32, "out", dev)
+    ws_bytes = decode_workspace_size(B, Hq, Hkv, dv)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
+    _need(workspace, torch.uint8, "workspace", dev)
+    rc = _lib.load().hca_decode(_p(q), _p(kc), _p(vc), _p(page_table), int(page_size), int(max_pages),
+                                int(num_pages), _p(kw), _p(vw), _p(seqlens), _p(gq), _p(gk), float(eps), _p(gate), _p(out),
+                                _p(workspace), workspace.numel(), B, Hq, Hkv, d, dv, blk, W, Nmax,
+                                float(scale), flags, _stream(dev))
+    _check(rc, "hca_decode")
+    return out

@@ -1,0 +1,728 @@
+// decode.cuh -- split-KV HCA decode on tcgen05 tensor cores (sm_100a).
+//
+// One new query per sequence attends, in one softmax, to its n_c visible compressed
+// entries and to its raw window of the last W tokens (official blog "ERNIE 5.5 Flash
+// Base . ERNIE", section 2.1; Zhidx article, section "1. Latent-Gated Sparse
+// Attention").  With 64 query heads sharing one KV head, every cached byte feeds 64
+// heads, so the dot products run on the tensor cores and the kernel is bound by HBM.
+//
+// Work decomposition.  A unit is one (sequence, KV head) pair; its keys are cut into
+// tiles of 128 (compressed tiles first, then window tiles).  All tiles of the batch are
+// laid end to end and cut into one contiguous range per CTA (one CTA per SM), so ragged
+// batches balance to within one tile.  A CTA may cover the tail of one unit and the
+// head of the next; for each (CTA, unit) piece it writes a partial record (running max
+// m, sum l, unnormalised O) into the workspace, and the combine kernel merges the
+// records of each unit with a log-sum-exp and applies the optional output gate.
+//
+// Per tile, inside a CTA (warp-specialised):
+//   warp 0 (1 thread)  TMA: K tile then V tile as eight 16 KB slabs of 128 keys x 64
+//                      channels (128-byte swizzle) into a ring of shared-memory slots;
+//   warp 1 (1 thread)  tcgen05.mma:  S^T[128 keys x 64 heads] = K . Q^T   (TMEM)
+//                                    O^T[512 ch x 64 heads] += V^T . P^T (TMEM, 4 x 128)
+//                      and, with QK normalisation, diag(K K^T) for the key norms;
+//   warps 2-5          softmax: thread = key row; per-head running max with lazy
+//                      rescaling (only when a logit exceeds the max by 2^8), P^T in bf16
+//                      to shared memory; the end-of-piece epilogue writes the record.
+// Every mbarrier wait is bounded (see common.cuh).
+#pragma once
+
+#include "common.cuh"
+
+namespace hca {
+
+constexpr int kDecD = 512;                 // head dim (d == dv)
+constexpr int kDecSlabs = kDecD / 64;      // 64-channel slabs per key row
+constexpr int kDecTile = 128;              // keys per tile (MMA M of S^T)
+constexpr int kDecHeads = 64;              // MMA N: query heads of one KV group (padded)
+constexpr int kDecRing = 8;                // ring slots (even, see the V^T descriptor)
+constexpr int kDecThreads = 192;
+constexpr uint32_t kSlabBytes = 128 * 128;                 // 128 rows x 128 B
+constexpr uint32_t kDecQBytes = kDecHeads * kDecD * 2;     // 64 KB
+constexpr uint32_t kDecPBytes = kDecTile * kDecHeads * 2;  // 16 KB
+constexpr float kRescaleThreshold = 8.0f;                  // log2 units
+
+// TMEM columns
+constexpr uint32_t kTmS = 0;      // 2 x 64  S^T buffers
+constexpr uint32_t kTmO = 128;    // 4 x 64  O^T chunks (128 channels each)
+constexpr uint32_t kTmKK = 384;   // 128     K K^T (QK normalisation only)
+
+// shared-memory layout (offsets from a 1024-aligned base)
+constexpr uint32_t kSmQ = 0;
+constexpr uint32_t kSmP = kSmQ + kDecQBytes;
+constexpr uint32_t kSmRing = kSmP + 2 * kDecPBytes;
+constexpr uint32_t kSmBar = kSmRing + kDecRing * kSlabBytes;
+constexpr int kNumBars = 2 * kDecRing + 12;
+constexpr uint32_t kSmRed = kSmBar + kNumBars * 8;          // float[4][64]
+constexpr uint32_t kSmFin = kSmRed + 4 * 64 * 4;            // float[64] reduction result
+constexpr uint32_t kSmMax = kSmFin + 64 * 4;                // float[64] running max per head
+constexpr uint32_t kSmAlpha = kSmMax + 64 * 4;              // float[64] rescale factors
+constexpr uint32_t kSmSum = kSmAlpha + 64 * 4;              // float[64] running sum per head
+constexpr uint32_t kSmMisc = kSmSum + 64 * 4;               // ints
+constexpr uint32_t kDecSmemBytes = kSmMisc + 64 + 1024;     // + alignment slack
+
+struct DecodeParams {
+    const __nv_bfloat16* q;      // [B, Hq, 512]
+    const int* seqlens;          // [B]
+    const int* page_table;       // [B, max_pages] or null
+    const float* gq;             // [512] or null
+    const float* gk;
+    const __nv_bfloat16* gate;   // [B, Hq, 512] or null
+    float* out;                  // [B, Hq, 512]
+    long long* total;            // workspace header: total tiles of the batch
+    int* meta;                   // [U][2]: first and last CTA holding a piece of unit u
+    float* rec_m;                // [R][64]  running max (log2 units)
+    float* rec_l;                // [R][64]
+    float* rec_o;                // [R][64][512]
+    int B, Hq, Hkv, G, blk, W, Nmax, page_size, max_pages, num_pages, flags, nsplit;
+    float scale_log2, eps;
+};
+
+struct UnitTiles {
+    int b, g, nc, nw, nct, nwt, s0;
+};
+
+// Visible entries and tiles of unit u.  Out-of-range lengths are clamped and reported.
+__device__ __forceinline__ UnitTiles unit_tiles(const DecodeParams& p, int u, bool report) {
+    UnitTiles t;
+    t.b = u / p.Hkv;
+    t.g = u - t.b * p.Hkv;
+    int L = __ldg(p.seqlens + t.b);
+    if (L < 1) {
+        if (report) record_error(HCA_ERR_DEVICE_INPUT);
+        L = 1;
+    }
+    const long long a = (long long)L - p.W;          // (t - W + 1) with t = L - 1
+    long long nc = a > 0 ? a / p.blk : 0;
+    const long long cap = (p.flags & HCA_PAGED) ? (long long)p.max_pages * p.page_size : (long long)p.Nmax;
+    if (nc > cap) {
+        if (report) record_error(HCA_ERR_DEVICE_INPUT);
+        nc = cap;
+    }
+    t.nc = (int)nc;
+    t.nw = L < p.W ? L : p.W;
+    t.nct = (t.nc + kDecTile - 1) / kDecTile;
+    t.nwt = (t.nw + kDecTile - 1) / kDecTile;
+    t.s0 = p.W - t.nw;
+    return t;
+}
+
+// Block-wide (all 192 threads) inclusive scan of one int per thread.
+__device__ __forceinline__ int block_scan_incl(int v, int* warp_tot, int* total_out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    int pre = 0, tot = 0;
+    for (int w = 0; w < kDecThreads / 32; ++w) {
+        if (w < warp) pre += warp_tot[w];
+        tot += warp_tot[w];
+    }
+    __syncthreads();
+    *total_out = tot;
+    return v + pre;
+}
+
+// Named barrier among the 128 softmax threads (warps 2-5).
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ bool softmax_any(bool pred) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "barrier.red.or.pred q, 2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)pred) : "memory");
+    return r != 0;
+}
+
+// Column reduction over the 128 softmax threads of a 64-vector held by every thread:
+// warp reduce-scatter with shuffles (lane l ends with heads 2l, 2l+1), then the four
+// warps meet in shared memory.  Result (all 64 heads) left in fin[] for every thread.
+template <bool kMax>
+__device__ __forceinline__ void colreduce64(const float (&v)[64], float* red, float* fin, int q, int lane) {
+    float t[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const bool hi = lane & 16;
+        const float send = hi ? v[i] : v[i + 32];
+        const float keep = hi ? v[i + 32] : v[i];
+        const float o = __shfl_xor_sync(0xffffffffu, send, 16);
+        t[i] = kMax ? fmaxf(keep, o) : keep + o;
+    }
+    // 32 -> 16 -> 8 -> 4 -> 2 values per lane, exchanging with lane ^ 8, ^4, ^2, ^1
+#pragma unroll
+    for (int w = 32; w >= 4; w >>= 1) {
+        const int hf = w / 2, x = w / 4;
+        const bool hi = lane & x;
+#pragma unroll
+        for (int i = 0; i < hf; ++i) {
+            const float send = hi ? t[i] : t[i + hf];
+            const float keep = hi ? t[i + hf] : t[i];
+            const float o = __shfl_xor_sync(0xffffffffu, send, x);
+            t[i] = kMax ? fmaxf(keep, o) : keep + o;
+        }
+    }
+    red[q * 64 + 2 * lane] = t[0];
+    red[q * 64 + 2 * lane + 1] = t[1];
+    softmax_bar();
+    const int idx = q * 32 + lane;
+    if (idx < 64) {
+        float a = red[idx], b = red[64 + idx], c = red[128 + idx], d = red[192 + idx];
+        fin[idx] = kMax ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
+    }
+    softmax_bar();
+}
+
+// Byte offset of 16-byte chunk `c` of row `r` in a 128-byte-swizzled slab.
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) {
+    return r * 128u + (((c ^ r) & 7u) << 4);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kw,
+                    const __grid_constant__ CUtensorMap tm_vw) {
+    extern __shared__ uint8_t dsmem[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSmBar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kDecRing;
+    uint64_t* q_full = bars + 2 * kDecRing;
+    uint64_t* q_empty = q_full + 1;
+    uint64_t* s_full = q_full + 2;    // [2]
+    uint64_t* s_empty = q_full + 4;   // [2]
+    uint64_t* p_full = q_full + 6;    // [2]
+    uint64_t* p_empty = q_full + 8;   // [2]
+    uint64_t* o_full = q_full + 10;
+    uint64_t* o_empty = q_full + 11;
+    float* red = reinterpret_cast<float*>(sm + kSmRed);
+    float* fin = reinterpret_cast<float*>(sm + kSmFin);
+    float* m_s = reinterpret_cast<float*>(sm + kSmMax);
+    float* al_s = reinterpret_cast<float*>(sm + kSmAlpha);
+    float* l_s = reinterpret_cast<float*>(sm + kSmSum);
+    int* misc = reinterpret_cast<int*>(sm + kSmMisc);
+    volatile int* abort_flag = misc + 0;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
+    int* sched = misc + 2;          // [0] = first unit, [1] = its first tile index (global), [2..7] scan scratch
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool norm = (p.flags & HCA_QK_NORM) != 0;
+    const bool paged = (p.flags & HCA_PAGED) != 0;
+    const int U = p.B * p.Hkv;
+    const int cta = blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int i = 0; i < kDecRing; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(q_full, 4);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_empty[i], 4);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&p_empty[i], 1);
+        }
+        mbar_init(o_full, 1);
+        mbar_init(o_empty, 4);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_kw);
+        prefetch_tmap(&tm_vw);
+    }
+
+    // ---- this CTA's tile range [ts, te) of the batch, and the unit holding tile ts
+    long long total = 0;
+    for (int u = threadIdx.x; u < U; u += kDecThreads) {
+        UnitTiles t = unit_tiles(p, u, true);
+        total += t.nct + t.nwt;
+    }
+    {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+        long long* wt = reinterpret_cast<long long*>(red);
+        if (lane == 0) wt[warp] = total;
+        __syncthreads();
+        total = 0;
+        for (int w = 0; w < kDecThreads / 32; ++w) total += wt[w];
+        __syncthreads();
+    }
+    const long long ts = total * cta / p.nsplit;
+    const long long te = total * (cta + 1) / p.nsplit;
+    if (cta == 0 && threadIdx.x == 0) *p.total = total;
+    if (threadIdx.x == 0) { sched[0] = -1; sched[1] = 0; }
+    __syncthreads();
+    {
+        long long base = 0;
+        for (int c0 = 0; c0 < U; c0 += kDecThreads) {
+            const int u = c0 + threadIdx.x;
+            int n = 0;
+            if (u < U) {
+                UnitTiles t = unit_tiles(p, u, false);
+                n = t.nct + t.nwt;
+            }
+            int tot;
+            const int incl = block_scan_incl(n, sched + 2, &tot);
+            const long long pu = base + incl - n;
+            if (u < U && pu <= ts && ts < pu + n) {
+                sched[0] = u;
+                reinterpret_cast<long long*>(red + 64)[0] = pu;
+            }
+            base += tot;
+        }
+        __syncthreads();
+    }
+    const int u_first = sched[0];
+    const long long p_first = reinterpret_cast<long long*>(red + 64)[0];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool have_work = (ts < te) && u_first >= 0;
+
+    if (have_work && warp == 0) {
+        // ===================================================== TMA producer
+        if (lane == 0) {
+            uint32_t ring = 0;
+            // Slab order: K(n0) ; K(n1) V(n0) ; K(n2) V(n1) ; ... ; V(last) -- the MMA
+            // issuer consumes in the same order.
+            struct Pend { int u, tile; };
+            Pend prev = {-1, 0};
+            int u = u_first;
+            long long pu = p_first;
+            bool ok = true;
+            auto load_tile = [&](int uu, int tile, bool is_v) -> bool {
+                UnitTiles t = unit_tiles(p, uu, false);
+                const CUtensorMap* m;
+                const bool comp = tile < t.nct;
+                if (comp) m = is_v ? &tm_v : &tm_k;
+                else m = is_v ? &tm_vw : &tm_kw;
+                for (int s = 0; s < kDecSlabs; ++s) {
+                    const uint32_t st = ring % kDecRing;
+                    if (!mbar_wait(&empty[st], ((ring / kDecRing) & 1) ^ 1, abort_flag)) return false;
+                    uint8_t* dst = sm + kSmRing + st * kSlabBytes;
+                    if (comp && paged) {
+                        uint32_t bytes = 0;
+                        const int j0 = tile * kDecTile;
+                        const bool h1 = j0 + 64 < t.nc;
+                        bytes = h1 ? 2 * 8192 : 8192;
+                        mbar_arrive_expect_tx(&full[st], bytes);
+                        for (int h = 0; h < (h1 ? 2 : 1); ++h) {
+                            const int j = j0 + 64 * h;
+                            const int pg = __ldg(p.page_table + (size_t)t.b * p.max_pages + j / p.page_size);
+                            if (pg < 0 || pg >= p.num_pages) record_error(HCA_ERR_DEVICE_INPUT);
+                            tma_load_4d(dst + h * 8192, m, &full[st], 64 * s, t.g, j % p.page_size, pg);
+                        }
+                    } else {
+                        mbar_arrive_expect_tx(&full[st], kSlabBytes);
+                        const int row = comp ? tile * kDecTile : t.s0 + (tile - t.nct) * kDecTile;
+                        tma_load_4d(dst, m, &full[st], 64 * s, t.g, row, t.b);
+                    }
+                    ++ring;
+                }
+                return true;
+            };
+            while (ok && pu < te) {
+                UnitTiles t = unit_tiles(p, u, false);
+                const int ntiles = t.nct + t.nwt;
+                const int tb = (int)((ts > pu ? ts : pu) - pu);
+                const int tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
+                for (int tile = tb; ok && tile < tend; ++tile) {
+                    if (tile == tb && prev.u >= 0) {
+                        ok = load_tile(prev.u, prev.tile, true);
+                        prev.u = -1;
+                    }
+                    if (ok) ok = load_tile(u, tile, false);
+                    if (ok && prev.u >= 0) ok = load_tile(prev.u, prev.tile, true);
+                    prev = {u, tile};
+                }
+                pu += ntiles;
+                ++u;
+            }
+            if (ok && prev.u >= 0) load_tile(prev.u, prev.tile, true);
+        }
+    } else if (have_work && warp == 1) {
+        // ===================================================== MMA issuer (whole warp waits, lane 0 issues)
+        const uint32_t id_s = idesc_bf16(128, kDecHeads, 0, 0);
+        const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+        const uint32_t id_o = idesc_bf16(128, kDecHeads, 1, 1);
+        const uint32_t q_base = smem_u32(sm + kSmQ);
+        uint32_t ring = 0;
+        int n = 0;          // tiles issued (S side)
+        int item = 0;
+        bool ok = true;
+        // pending PV tile
+        int pv_n = -1, pv_item = 0, pv_nvalid = 128;
+        bool pv_first = false, pv_last = false, pv_partial = false;
+
+        auto issue_pv = [&]() -> bool {
+            const int b = pv_n & 1;
+            if (!mbar_wait(&p_full[b], (pv_n >> 1) & 1, abort_flag)) return false;
+            if (pv_first && !mbar_wait(o_empty, (pv_item & 1) ^ 1, abort_flag)) return false;
+            tc_fence_after();
+            const uint32_t p_base = smem_u32(sm + kSmP + b * kDecPBytes);
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t st0 = ring % kDecRing, st1 = (ring + 1) % kDecRing;
+                if (!mbar_wait(&full[st0], (ring / kDecRing) & 1, abort_flag)) return false;
+                if (!mbar_wait(&full[st1], ((ring + 1) / kDecRing) & 1, abort_flag)) return false;
+                if (pv_partial) {
+                    // rows >= nvalid may hold anything (caller memory past the visible
+                    // entries): zero them so 0-probability keys contribute exactly 0
+                    const int nz = (kDecTile - pv_nvalid) * 8;
+                    for (int i = lane; i < 2 * nz; i += 32) {
+                        const int sl = i / nz, k = i - sl * nz;
+                        const int r = pv_nvalid + (k >> 3);
+                        uint8_t* slab = sm + kSmRing + (sl ? st1 : st0) * kSlabBytes;
+                        *reinterpret_cast<uint4*>(slab + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    const uint32_t v_base = smem_u32(sm + kSmRing + st0 * kSlabBytes);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(v_base + kk * 2048, kSlabBytes, 1024);
+                        const uint64_t bd = smem_desc_sw128(p_base + kk * 2048, 8192, 1024);
+                        mma_ss(tmem + kTmO + 64 * c, ad, bd, id_o, (pv_first && kk == 0) ? 0u : 1u);
+                    }
+                    mma_commit(&empty[st0]);
+                    mma_commit(&empty[st1]);
+                }
+                __syncwarp();
+                ring += 2;
+            }
+            if (lane == 0) {
+                mma_commit(&p_empty[b]);
+                if (pv_last) mma_commit(o_full);
+            }
+            __syncwarp();
+            return true;
+        };
+
+        int u = u_first;
+        long long pu = p_first;
+        while (ok && pu < te) {
+            UnitTiles t = unit_tiles(p, u, false);
+            const int ntiles = t.nct + t.nwt;
+            const int tb = (int)((ts > pu ? ts : pu) - pu);
+            const int tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
+            for (int tile = tb; ok && tile < tend; ++tile, ++n) {
+                const bool first = tile == tb, last = tile == tend - 1;
+                const int sb = n & 1;
+                if (first && pv_n >= 0) {
+                    // close the previous piece first: its epilogue waits for this PV
+                    if (!issue_pv()) { ok = false; break; }
+                    pv_n = -1;
+                }
+                if (first && !mbar_wait(q_full, item & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                // the K K^T accumulator has one buffer: wait until tile n-1's softmax has read it
+                if (norm && n > 0 && !mbar_wait(&s_empty[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int s = 0; s < kDecSlabs; ++s) {
+                    const uint32_t st = ring % kDecRing;
+                    if (!mbar_wait(&full[st], (ring / kDecRing) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t k_base = smem_u32(sm + kSmRing + st * kSlabBytes);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t ad = smem_desc_sw128(k_base + kk * 32, 16, 1024);
+                            const uint64_t bd = smem_desc_sw128(q_base + s * 8192 + kk * 32, 16, 1024);
+                            mma_ss(tmem + kTmS + 64 * sb, ad, bd, id_s, (s | kk) ? 1u : 0u);
+                            if (norm) mma_ss(tmem + kTmKK, ad, ad, id_kk, (s | kk) ? 1u : 0u);
+                        }
+                        mma_commit(&empty[st]);
+                    }
+                    __syncwarp();
+                    ++ring;
+                }
+                if (!ok) break;
+                if (lane == 0) {
+                    mma_commit(&s_full[sb]);
+                    if (last) mma_commit(q_empty);
+                }
+                __syncwarp();
+                // PV of the previous tile (its V slabs follow this tile's K slabs in the ring)
+                if (pv_n >= 0 && !issue_pv()) { ok = false; break; }
+                pv_n = n;
+                pv_item = item;
+                pv_first = first;
+                pv_last = last;
+                pv_partial = tile < t.nct && (t.nc - tile * kDecTile) < kDecTile;
+                pv_nvalid = tile < t.nct ? min(kDecTile, t.nc - tile * kDecTile) : kDecTile;
+                if (last) ++item;
+            }
+            pu += ntiles;
+            ++u;
+        }
+        if (ok && pv_n >= 0) issue_pv();
+    } else if (have_work) {
+        // ===================================================== softmax / epilogue (warps 2-5)
+        const int q4 = warp & 3;                 // TMEM lane quarter
+        const int r = q4 * 32 + lane;            // key row within the tile / channel within a chunk
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int sidx = threadIdx.x - 64;       // 0..127
+        int n = 0, item = 0;
+        bool ok = true;
+        int u = u_first;
+        long long pu = p_first;
+        while (ok && pu < te) {
+            UnitTiles t = unit_tiles(p, u, false);
+            const int ntiles = t.nct + t.nwt;
+            const int tb = (int)((ts > pu ? ts : pu) - pu);
+            const int tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
+
+            // ---- stage this unit's queries (64 rows, zero past G) into Q smem
+            if (!mbar_wait(q_empty, (item & 1) ^ 1, abort_flag)) { ok = false; break; }
+            {
+                const int h = sidx >> 1, half = sidx & 1;
+                const bool live = h < p.G;
+                const __nv_bfloat16* qrow = p.q + ((size_t)t.b * p.Hq + (size_t)t.g * p.G + h) * kDecD + 256 * half;
+                float inv = 1.f;
+                if (norm && live) {
+                    float ss = 0.f;
+                    for (int c = 0; c < 256; c += 8) {
+                        const uint4 x = __ldg(reinterpret_cast<const uint4*>(qrow + c));
+                        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float a = bf16lo(w4[i]), b2 = bf16hi(w4[i]);
+                            ss = fmaf(a, a, fmaf(b2, b2, ss));
+                        }
+                    }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    inv = rsqrtf(ss * (1.f / kDecD) + p.eps);
+                }
+                for (int c = 0; c < 256; c += 8) {
+                    uint4 x = make_uint4(0, 0, 0, 0);
+                    if (live) {
+                        x = __ldg(reinterpret_cast<const uint4*>(qrow + c));
+                        if (norm) {
+                            const int cc = 256 * half + c;
+                            uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int ch = cc + 2 * i;
+                                const float a = bf16lo(w4[i]) * inv * __ldg(p.gq + ch) * __ldg(p.gk + ch);
+                                const float b2 = bf16hi(w4[i]) * inv * __ldg(p.gq + ch + 1) * __ldg(p.gk + ch + 1);
+                                w4[i] = pack_bf16x2(a, b2);
+                            }
+                            x = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    }
+                    const int cc = 256 * half + c;
+                    uint8_t* slab = sm + kSmQ + (cc >> 6) * 8192;
+                    *reinterpret_cast<uint4*>(slab + sw128(h, (cc & 63) >> 3)) = x;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_full);
+            }
+
+            for (int tile = tb; ok && tile < tend; ++tile, ++n) {
+                const bool first = tile == tb, last = tile == tend - 1;
+                const int sb = n & 1;
+                const bool comp = tile < t.nct;
+                const int nvalid = comp ? min(kDecTile, t.nc - tile * kDecTile)
+                                        : min(kDecTile, p.W - (t.s0 + (tile - t.nct) * kDecTile));
+                const bool valid = r < nvalid;
+
+                if (!mbar_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                float z[64];
+#pragma unroll
+                for (int c = 0; c < 64; c += 16) tmem_ld16(tmem + lane_off + kTmS + 64 * sb + c, z + c);
+                float kscale = p.scale_log2;
+                if (norm) {
+                    float d[32];
+                    tmem_ld16(tmem + lane_off + kTmKK + q4 * 32, d);
+                    tmem_ld16(tmem + lane_off + kTmKK + q4 * 32 + 16, d + 16);
+                    tmem_wait_ld();
+                    float diag = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) diag = (j == lane) ? d[j] : diag;
+                    kscale *= rsqrtf(diag * (1.f / kDecD) + p.eps);
+                } else {
+                    tmem_wait_ld();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[sb]);
+#pragma unroll
+                for (int h = 0; h < 64; ++h) z[h] = valid ? z[h] * kscale : -INFINITY;
+
+                // ---- running max (shared m_s[64]): full reduction on the first tile of a
+                // piece; afterwards only when some logit exceeds the max by 2^threshold
+                bool need;
+                if (first) {
+                    need = true;
+                } else {
+                    bool mine = false;
+#pragma unroll
+                    for (int h = 0; h < 64; h += 4) {
+                        const float4 mm = *reinterpret_cast<const float4*>(m_s + h);
+                        mine |= (z[h] > mm.x + kRescaleThreshold) | (z[h + 1] > mm.y + kRescaleThreshold) |
+                                (z[h + 2] > mm.z + kRescaleThreshold) | (z[h + 3] > mm.w + kRescaleThreshold);
+                    }
+                    need = softmax_any(mine);
+                }
+                if (need) {
+                    colreduce64<true>(z, red, fin, q4, lane);
+                    if (sidx < 64) {
+                        const float mo = first ? -INFINITY : m_s[sidx];
+                        const float mn = fmaxf(mo, fin[sidx]);
+                        const float al = first ? 0.f : ex2(mo - mn);
+                        al_s[sidx] = al;
+                        m_s[sidx] = mn;
+                        l_s[sidx] = first ? 0.f : l_s[sidx] * al;
+                    }
+                    softmax_bar();
+                    if (!first) {
+                        // rescale O^T once the previous PV has landed
+                        const int pb = (n - 1) & 1;
+                        if (!mbar_wait(&p_empty[pb], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                            for (int c16 = 0; c16 < 64; c16 += 16) {
+                                float o[16];
+                                const uint32_t ta = tmem + lane_off + kTmO + 64 * c + c16;
+                                tmem_ld16(ta, o);
+                                tmem_wait_ld();
+                                uint32_t w[16];
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) w[j] = __float_as_uint(o[j] * al_s[c16 + j]);
+                                tmem_st16(ta, w);
+                            }
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                    }
+                }
+                // ---- probabilities
+                uint32_t pk[32];
+#pragma unroll
+                for (int h = 0; h < 64; h += 4) {
+                    const float4 mm = *reinterpret_cast<const float4*>(m_s + h);
+                    z[h] = ex2(z[h] - mm.x);
+                    z[h + 1] = ex2(z[h + 1] - mm.y);
+                    z[h + 2] = ex2(z[h + 2] - mm.z);
+                    z[h + 3] = ex2(z[h + 3] - mm.w);
+                    pk[h >> 1] = pack_bf16x2(z[h], z[h + 1]);
+                    pk[(h >> 1) + 1] = pack_bf16x2(z[h + 2], z[h + 3]);
+                }
+                const int pbuf = n & 1;
+                if (!mbar_wait(&p_empty[pbuf], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                uint8_t* pt = sm + kSmP + pbuf * kDecPBytes;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(pt + sw128(r, c)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[pbuf]);
+                // row sums of this tile (off the MMA's critical path)
+                colreduce64<false>(z, red, fin, q4, lane);
+                if (sidx < 64) l_s[sidx] += fin[sidx];
+
+                if (last) {
+                    // ---- end of this CTA's piece of unit u: write the partial record
+                    const int rec = cta + u;
+                    if (sidx < 64) {
+                        p.rec_m[(size_t)rec * 64 + sidx] = m_s[sidx];
+                        p.rec_l[(size_t)rec * 64 + sidx] = l_s[sidx];
+                    }
+                    if (sidx == 0) {
+                        if (tb == 0) p.meta[2 * u] = cta;
+                        if (tend == ntiles) p.meta[2 * u + 1] = cta;
+                    }
+                    if (!mbar_wait(o_full, item & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    float* orec = p.rec_o + (size_t)rec * 64 * kDecD;
+                    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                        for (int c16 = 0; c16 < 64; c16 += 16) {
+                            float o[16];
+                            tmem_ld16(tmem + lane_off + kTmO + 64 * c + c16, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int h = c16 + j;
+                                if (h < p.G) orec[(size_t)h * kDecD + 128 * c + r] = o[j];
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(o_empty);
+                    ++item;
+                }
+            }
+            pu += ntiles;
+            ++u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// Merge the partial records of each unit (log-sum-exp), normalise, apply the gate.
+// Grid: (units, heads / 8); 256 threads, two channels each.
+__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeParams p) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int u = blockIdx.x;
+    const int b = u / p.Hkv, g = u - (u / p.Hkv) * p.Hkv;
+    const int first = p.meta[2 * u], last = p.meta[2 * u + 1];
+    const long long total = *p.total;
+    const int c = 2 * threadIdx.x;
+    if (first < 0 || last < first || last >= p.nsplit) {
+        record_error(HCA_ERR_DEVICE_INPUT);
+        return;
+    }
+    for (int h = blockIdx.y * 8; h < min(p.G, blockIdx.y * 8 + 8); ++h) {
+        float M = -INFINITY;
+        for (int i = first; i <= last; ++i) {
+            if (total * i / p.nsplit == total * (i + 1) / p.nsplit) continue;   // empty range
+            M = fmaxf(M, p.rec_m[(size_t)(i + u) * 64 + h]);
+        }
+        float L = 0.f, a0 = 0.f, a1 = 0.f;
+        for (int i = first; i <= last; ++i) {
+            if (total * i / p.nsplit == total * (i + 1) / p.nsplit) continue;
+            const size_t rec = (size_t)(i + u);
+            const float w = exp2f(p.rec_m[rec * 64 + h] - M);
+            L = fmaf(w, p.rec_l[rec * 64 + h], L);
+            const float2 o = *reinterpret_cast<const float2*>(p.rec_o + (rec * 64 + h) * kDecD + c);
+            a0 = fmaf(w, o.x, a0);
+            a1 = fmaf(w, o.y, a1);
+        }
+        const float inv = 1.f / L;
+        float o0 = a0 * inv, o1 = a1 * inv;
+        const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h) * kDecD + c;
+        if (p.flags & HCA_OUT_GATE) {
+            const uint32_t gv = *reinterpret_cast<const uint32_t*>(p.gate + orow);
+            o0 *= 1.f / (1.f + __expf(-bf16lo(gv)));
+            o1 *= 1.f / (1.f + __expf(-bf16hi(gv)));
+        }
+        *reinterpret_cast<float2*>(p.out + orow) = make_float2(o0, o1);
+    }
+}
+
+}  // namespace hca

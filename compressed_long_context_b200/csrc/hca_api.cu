@@ -1,0 +1,332 @@
+// hca_api.cu -- the C ABI of libhca (declared in include/hca.h): argument checks,
+// TMA tensor maps and kernel launches.  Everything here is host code except the
+// kernels pulled in from the .cuh files of this directory.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "compress.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+using hca::g_error;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hca_status_t launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? HCA_OK : HCA_ERR_CUDA;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+namespace hca {
+
+// 4-D bf16 tensor map over a [d3][d2][d1][d0] array (d0 innermost, contiguous), box
+// {b0, b1, b2, b3}, 128-byte swizzle (b0 * 2 bytes must be 128).  Strides are in
+// elements for dims 1..3.  Returns false if the driver rejects the map.
+bool make_tmap_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                  uint64_t s1, uint64_t s2, uint64_t s3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {d0, d1, d2, d3};
+    cuuint64_t strides[3] = {s1 * 2, s2 * 2, s3 * 2};
+    cuuint32_t box[4] = {b0, b1, b2, b3};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel slot, device).
+bool set_smem_attr_once(const void* fn, int bytes, int slot) {
+    static std::mutex mu;
+    static bool done[8][64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 8) return false;
+    std::lock_guard<std::mutex> g(mu);
+    if (done[slot][dev]) return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done[slot][dev] = true;
+    return true;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+}  // namespace hca
+
+extern "C" {
+
+const char* hca_status_string(hca_status_t s) {
+    switch (s) {
+        case HCA_OK: return "HCA_OK";
+        case HCA_ERR_INVALID_ARG: return "HCA_ERR_INVALID_ARG: null/misaligned pointer or size out of range";
+        case HCA_ERR_UNSUPPORTED: return "HCA_ERR_UNSUPPORTED: shape or flag combination not supported";
+        case HCA_ERR_CUDA: return "HCA_ERR_CUDA: a CUDA launch or query failed";
+        case HCA_ERR_TIMEOUT: return "HCA_ERR_TIMEOUT: a bounded device wait ran out";
+        case HCA_ERR_DEVICE_INPUT: return "HCA_ERR_DEVICE_INPUT: a device-resident input was out of range";
+    }
+    return "unknown hca_status_t";
+}
+
+hca_status_t hca_get_device_error(hca_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&word, g_error, sizeof word, 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return HCA_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(g_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return HCA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HCA_ERR_CUDA;
+    if (word == HCA_ERR_TIMEOUT || word == HCA_ERR_DEVICE_INPUT) return static_cast<hca_status_t>(word);
+    return word == 0 ? HCA_OK : HCA_ERR_CUDA;
+}
+
+hca_status_t hca_compress(const void* k, const void* v, const float* w, void* kc, void* vc,
+                          int B, int T, int Hkv, int d, int dv, int blk, hca_stream_t stream) {
+    if (B < 0 || T < 0 || Hkv < 1 || blk < 1) return HCA_ERR_INVALID_ARG;
+    auto ok_dim = [](int x) { return x == 64 || x == 128 || x == 256 || x == 512; };
+    if (!ok_dim(d) || !ok_dim(dv) || blk > 128) return HCA_ERR_UNSUPPORTED;
+    const int64_t Nc = T / blk;
+    const int64_t entries = (int64_t)B * Nc * Hkv;
+    if (entries == 0) return HCA_OK;
+    if (entries > 0x7fffffffLL) return HCA_ERR_INVALID_ARG;
+    if (!k || !v || !kc || !vc) return HCA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc) || (w && !aligned16(w)))
+        return HCA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)entries);
+    const auto* K = static_cast<const __nv_bfloat16*>(k);
+    const auto* V = static_cast<const __nv_bfloat16*>(v);
+    auto* KC = static_cast<__nv_bfloat16*>(kc);
+    auto* VC = static_cast<__nv_bfloat16*>(vc);
+#define HCA_COMPRESS_CASE(DK, DV)                                                                       \
+    if (d == DK && dv == DV) {                                                                          \
+        hca::compress_kernel<DK, DV><<<grid, hca::kCompressThreads, 0, s>>>(K, V, w, KC, VC, T, Hkv, blk, \
+                                                                            (int)Nc);                   \
+        return launch_status();                                                                         \
+    }
+#define HCA_COMPRESS_ROW(DK) \
+    HCA_COMPRESS_CASE(DK, 64) HCA_COMPRESS_CASE(DK, 128) HCA_COMPRESS_CASE(DK, 256) HCA_COMPRESS_CASE(DK, 512)
+    HCA_COMPRESS_ROW(64) HCA_COMPRESS_ROW(128) HCA_COMPRESS_ROW(256) HCA_COMPRESS_ROW(512)
+#undef HCA_COMPRESS_ROW
+#undef HCA_COMPRESS_CASE
+    return HCA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace layout of hca_decode: [header 256 B: total tiles][meta: U x 2 int][records]
+struct DecodeWs {
+    size_t meta_off, m_off, l_off, o_off, bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+DecodeWs decode_ws_layout(long long U, long long nsplit) {
+    DecodeWs w;
+    const long long R = nsplit + U;
+    w.meta_off = 256;
+    w.m_off = align256(w.meta_off + (size_t)U * 2 * sizeof(int));
+    w.l_off = align256(w.m_off + (size_t)R * 64 * sizeof(float));
+    w.o_off = align256(w.l_off + (size_t)R * 64 * sizeof(float));
+    w.bytes = align256(w.o_off + (size_t)R * 64 * hca::kDecD * sizeof(float));
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hca_decode_workspace_size(int B, int Hq, int Hkv, int dv) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || dv < 1) return 0;
+    const int ns = hca::num_sms();
+    if (ns <= 0) return 0;
+    return decode_ws_layout((long long)B * Hkv, ns).bytes;
+}
+
+hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int* page_table, int page_size,
+                        int max_pages, int num_pages, const void* kw, const void* vw, const int* seqlens,
+                        const float* gq, const float* gk, float eps, const void* gate, float* out,
+                        void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int d, int dv, int blk, int W,
+                        int Nmax, float scale, unsigned flags, hca_stream_t stream) {
+    using namespace hca;
+    if (B < 0 || Hq < 1 || Hkv < 1 || blk < 1 || W < 1) return HCA_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(HCA_QK_NORM | HCA_OUT_GATE | HCA_PAGED)) return HCA_ERR_UNSUPPORTED;
+    if (d != kDecD || dv != kDecD || Hq % Hkv != 0 || Hq / Hkv > kDecHeads || blk > 128)
+        return HCA_ERR_UNSUPPORTED;
+    if (!(scale == scale) || !(eps >= 0.f)) return HCA_ERR_INVALID_ARG;
+    if (B == 0) return HCA_OK;
+    const bool paged = flags & HCA_PAGED;
+    const bool norm = flags & HCA_QK_NORM;
+    const bool gated = flags & HCA_OUT_GATE;
+    if (!q || !kc || !vc || !kw || !vw || !seqlens || !out || !workspace) return HCA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(kw) || !aligned16(vw) ||
+        !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(seqlens) & 3))
+        return HCA_ERR_INVALID_ARG;
+    if (paged) {
+        if (!page_table || page_size < 64 || page_size % 64 || max_pages < 1 || num_pages < 1)
+            return HCA_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(page_table) & 3) return HCA_ERR_INVALID_ARG;
+    } else if (Nmax < 1) {
+        return HCA_ERR_INVALID_ARG;
+    }
+    if (norm && (!gq || !gk || (reinterpret_cast<uintptr_t>(gq) & 3) || (reinterpret_cast<uintptr_t>(gk) & 3)))
+        return HCA_ERR_INVALID_ARG;
+    if (gated && (!gate || (reinterpret_cast<uintptr_t>(gate) & 3))) return HCA_ERR_INVALID_ARG;
+    const int nsplit = num_sms();
+    if (nsplit <= 0) return HCA_ERR_CUDA;
+    const long long U = (long long)B * Hkv;
+    if (U > (1 << 24)) return HCA_ERR_INVALID_ARG;
+    const DecodeWs lay = decode_ws_layout(U, nsplit);
+    if (ws_bytes < lay.bytes) return HCA_ERR_INVALID_ARG;
+
+    const uint64_t hd = (uint64_t)Hkv * kDecD;
+    CUtensorMap tk, tv, tkw, tvw;
+    bool ok = true;
+    if (paged) {
+        ok &= make_tmap_4d(&tk, kc, kDecD, Hkv, page_size, num_pages, kDecD, hd, hd * page_size, 64, 1, 64, 1);
+        ok &= make_tmap_4d(&tv, vc, kDecD, Hkv, page_size, num_pages, kDecD, hd, hd * page_size, 64, 1, 64, 1);
+    } else {
+        ok &= make_tmap_4d(&tk, kc, kDecD, Hkv, Nmax, B, kDecD, hd, hd * Nmax, 64, 1, 128, 1);
+        ok &= make_tmap_4d(&tv, vc, kDecD, Hkv, Nmax, B, kDecD, hd, hd * Nmax, 64, 1, 128, 1);
+    }
+    ok &= make_tmap_4d(&tkw, kw, kDecD, Hkv, W, B, kDecD, hd, hd * W, 64, 1, 128, 1);
+    ok &= make_tmap_4d(&tvw, vw, kDecD, Hkv, W, B, kDecD, hd, hd * W, 64, 1, 128, 1);
+    if (!ok) return HCA_ERR_CUDA;
+
+    DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.seqlens = seqlens;
+    p.page_table = paged ? page_table : nullptr;
+    p.gq = norm ? gq : nullptr;
+    p.gk = norm ? gk : nullptr;
+    p.gate = gated ? static_cast<const __nv_bfloat16*>(gate) : nullptr;
+    p.out = out;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.total = reinterpret_cast<long long*>(ws);
+    p.meta = reinterpret_cast<int*>(ws + lay.meta_off);
+    p.rec_m = reinterpret_cast<float*>(ws + lay.m_off);
+    p.rec_l = reinterpret_cast<float*>(ws + lay.l_off);
+    p.rec_o = reinterpret_cast<float*>(ws + lay.o_off);
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.blk = blk; p.W = W; p.Nmax = paged ? 0 : Nmax;
+    p.page_size = paged ? page_size : 0; p.max_pages = paged ? max_pages : 0; p.num_pages = paged ? num_pages : 0;
+    p.flags = (int)flags; p.nsplit = nsplit;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.eps = eps;
+
+    if (!set_smem_attr_once(reinterpret_cast<const void*>(&decode_split_kernel), (int)kDecSmemBytes, 0))
+        return HCA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    decode_split_kernel<<<nsplit, kDecThreads, kDecSmemBytes, s>>>(p, tk, tv, tkw, tvw);
+    if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)U, (unsigned)((p.G + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel, p) != cudaSuccess) {
+        cudaGetLastError();
+        return HCA_ERR_CUDA;
+    }
+    return HCA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int D>
+hca_status_t launch_prefill(const hca::PrefillParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const CUtensorMap& tkc, const CUtensorMap& tvc,
+                            cudaStream_t s) {
+    using C = hca::PfCfg<D>;
+    if (!hca::set_smem_attr_once(reinterpret_cast<const void*>(&hca::prefill_kernel<D>), (int)C::kSmem,
+                                 D == 512 ? 1 : 2))
+        return HCA_ERR_CUDA;
+    const int ns = hca::num_sms();
+    if (ns <= 0) return HCA_ERR_CUDA;
+    const long long grid = p.items < ns ? p.items : ns;
+    hca::prefill_kernel<D><<<(unsigned)grid, hca::kPfThreads, C::kSmem, s>>>(p, tq, tk, tv, tkc, tvc);
+    return cudaGetLastError() == cudaSuccess ? HCA_OK : HCA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v, const void* kc, const void* vc,
+                                    void* out, float* lse, int B, int T, int Hq, int Hkv, int d, int dv, int blk,
+                                    int W, float scale, unsigned flags, hca_stream_t stream) {
+    using namespace hca;
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || blk < 1 || W < 1) return HCA_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(HCA_WRITE_LSE | HCA_OUT_F32)) return HCA_ERR_UNSUPPORTED;
+    if (d != dv || (d != 64 && d != 512) || blk > 128 || Hq % Hkv) return HCA_ERR_UNSUPPORTED;
+    const int G = Hq / Hkv;
+    if (G > 128 || (G & (G - 1))) return HCA_ERR_UNSUPPORTED;
+    if (!(scale == scale)) return HCA_ERR_INVALID_ARG;
+    if ((long long)B * T == 0) return HCA_OK;
+    const int Nc = T / blk;
+    const bool want_lse = flags & HCA_WRITE_LSE;
+    if (!q || !k || !v || !out || (Nc > 0 && (!kc || !vc)) || (want_lse && !lse)) return HCA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (Nc > 0 && (!aligned16(kc) ||
+        !aligned16(vc))) || (want_lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+        return HCA_ERR_INVALID_ARG;
+
+    PrefillParams p;
+    p.out = out;
+    p.lse = want_lse ? lse : nullptr;
+    p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.tpt = 128 / G; p.blk = blk; p.W = W; p.Nc = Nc;
+    p.ntile_t = (T + p.tpt - 1) / p.tpt;
+    p.flags = (int)flags;
+    const int NS = d == 512 ? 2 : 1;
+    p.items = (long long)p.ntile_t * B * Hkv * NS;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    const uint64_t D = (uint64_t)d;
+    CUtensorMap tq, tk, tv, tkc, tvc;
+    bool ok = true;
+    ok &= make_tmap_4d(&tq, q, D, Hq, T, B, D, D * Hq, D * Hq * T, 64, G, p.tpt, 1);
+    ok &= make_tmap_4d(&tk, k, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, 128, 1);
+    ok &= make_tmap_4d(&tv, v, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, 128, 1);
+    if (Nc > 0) {
+        ok &= make_tmap_4d(&tkc, kc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, 128, 1);
+        ok &= make_tmap_4d(&tvc, vc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, 128, 1);
+    } else {   // never read: no entry is visible when T < blk
+        tkc = tk;
+        tvc = tv;
+    }
+    if (!ok) return HCA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return d == 512 ? launch_prefill<512>(p, tq, tk, tv, tkc, tvc, s) : launch_prefill<64>(p, tq, tk, tv, tkc, tvc, s);
+}
+

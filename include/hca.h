@@ -1,0 +1,164 @@
+/*
+ * hca.h -- C ABI of libhca, a B200 (sm_100a) implementation of Heavily Compressed
+ * Attention (HCA).
+ *
+ * The operation (web pages describing ERNIE 5.5 Flash Base):
+ *  - "ERNIE 5.5 Flash Base . ERNIE" (official blog), section 2.1: an HCA layer
+ *    compresses every 128 tokens into a single cached entry, then attends to all of
+ *    these entries plus a short window of recent, uncompressed tokens; it still sees
+ *    the whole sequence while caching only a small fraction of it.
+ *  - Zhidx article "280B Total Parameters, 14B Activated ...", section
+ *    "1. Latent-Gated Sparse Attention": 37 of 43 layers are HCA; attention is
+ *    computed only over the compressed entries and a window of recent raw tokens.
+ *  - Model-card page "ERNIE 5.5 Flash Base", architecture paragraph: HCA layers use
+ *    512-dim heads, 64 attention heads; every attention layer uses QK normalization
+ *    and a gated output (Low-Rank Gated Attention).
+ *
+ * Readings where the pages are silent (the same in the kernels and in the tests):
+ *  - compression of block j (raw positions blk*j .. blk*j+blk-1) is a softmax-weighted
+ *    pooling: alpha = softmax(w over the block), Kc[j] = sum alpha_i K[i], Vc[j] likewise;
+ *    w == NULL means all-zero weights, i.e. the mean.  Only complete blocks are written.
+ *  - a query at position t attends, in one softmax, to compressed entries
+ *    j < n_c(t) = max(0, floor((t - W + 1) / blk)) and to raw tokens t-W+1 .. t.
+ *  - logits are scale * q.k; query head h reads KV head h / (Hq / Hkv).
+ *  - QK normalization (decode): per-head RMSNorm x / sqrt(mean(x^2) + eps) * g with gains
+ *    g_q, g_k of length d shared by all heads, applied to q and to every key used.
+ *  - output gate (decode): out *= sigmoid(gate), element-wise, gate logits [B,Hq,dv].
+ *
+ * Conventions for every entry point:
+ *  - all tensor pointers are DEVICE pointers owned by the caller, dense row-major in the
+ *    stated layout, 16-byte aligned; bf16 means IEEE bfloat16 bit patterns;
+ *  - the library allocates no device memory and copies nothing between host and device
+ *    (hca_get_device_error excepted); work is queued on `stream` and the call returns
+ *    without waiting for it;
+ *  - a call returns HCA_OK once the work is queued; HCA_ERR_INVALID_ARG for a NULL
+ *    pointer, a misaligned pointer or a size out of range; HCA_ERR_UNSUPPORTED for a
+ *    shape outside the supported set (nothing is launched in either case);
+ *    HCA_ERR_CUDA if a launch failed (the CUDA error is consumed);
+ *  - errors found on the device (a bounded wait that ran out, a sequence length or page
+ *    index out of range) are recorded in a per-device error word read by
+ *    hca_get_device_error; the affected outputs are then unspecified.
+ *  - nothing is printed, nothing aborts, no C++ exception crosses the boundary.
+ */
+#ifndef HCA_H_
+#define HCA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st* hca_stream_t;
+
+typedef enum {
+    HCA_OK = 0,
+    HCA_ERR_INVALID_ARG = 1,
+    HCA_ERR_UNSUPPORTED = 2,
+    HCA_ERR_CUDA = 3,
+    HCA_ERR_TIMEOUT = 4,       /* a bounded device wait ran out (reported by hca_get_device_error) */
+    HCA_ERR_DEVICE_INPUT = 5   /* a device-resident input was out of range (seqlens, page table) */
+} hca_status_t;
+
+enum {
+    HCA_QK_NORM = 1,    /* decode: RMSNorm q and k with gains gq, gk */
+    HCA_OUT_GATE = 2,   /* decode: multiply the output by sigmoid(gate) */
+    HCA_PAGED = 4,      /* decode: compressed cache is a page pool addressed by page_table */
+    HCA_WRITE_LSE = 8,  /* prefill: also write the natural-log sum-exp of the logits */
+    HCA_OUT_F32 = 16    /* prefill: output in fp32 instead of bf16 */
+};
+
+/*
+ * hca_compress -- build the compressed cache (official blog, section 2.1: every 128
+ * tokens become one cached entry).
+ *   k  [B,T,Hkv,d]  bf16     raw keys
+ *   v  [B,T,Hkv,dv] bf16     raw values
+ *   w  [B,T]        fp32     pooling weights, one per position, shared by K, V and all
+ *                            KV heads; NULL = all zero (mean pooling)
+ *   kc [B,Nc,Hkv,d]  bf16    output, Nc = floor(T / blk); a trailing partial block is
+ *   vc [B,Nc,Hkv,dv] bf16    not written
+ * Supported: d, dv in {64, 128, 256, 512}; 1 <= blk <= 128; B, T >= 0, Hkv >= 1.
+ * Arithmetic: fp32 accumulation, one rounding to bf16 (nearest even) per output.
+ */
+hca_status_t hca_compress(const void* k, const void* v, const float* w,
+                          void* kc, void* vc,
+                          int B, int T, int Hkv, int d, int dv, int blk,
+                          hca_stream_t stream);
+
+/*
+ * hca_prefill -- causal HCA attention for every position of B sequences of T tokens
+ * (official blog, section 2.1; Zhidx article, section 1).
+ *   q  [B,T,Hq,d]    bf16
+ *   k  [B,T,Hkv,d]   bf16    raw keys (the window segment)
+ *   v  [B,T,Hkv,dv]  bf16
+ *   kc [B,Nc,Hkv,d]  bf16    compressed cache from hca_compress, Nc = floor(T / blk)
+ *   vc [B,Nc,Hkv,dv] bf16
+ *   out [B,T,Hq,dv]  bf16, or fp32 with HCA_OUT_F32
+ *   lse [B,Hq,T]     fp32 natural-log sum-exp of the logits, written iff HCA_WRITE_LSE
+ *                    (may be NULL otherwise)
+ *   scale            logit scale (typically 1/sqrt(d))
+ * Supported: d == dv in {64, 512}; Hq % Hkv == 0 with Hq / Hkv a power of two <= 128;
+ * 1 <= blk <= 128; W >= 1; flags among HCA_WRITE_LSE | HCA_OUT_F32.
+ */
+hca_status_t hca_prefill(const void* q, const void* k, const void* v,
+                         const void* kc, const void* vc,
+                         void* out, float* lse,
+                         int B, int T, int Hq, int Hkv, int d, int dv, int blk, int W,
+                         float scale, unsigned flags, hca_stream_t stream);
+
+/*
+ * hca_decode_workspace_size -- bytes of device workspace hca_decode needs for a batch
+ * of B sequences on the CURRENT device (split-KV partial results).  Returns 0 for
+ * invalid sizes.
+ */
+size_t hca_decode_workspace_size(int B, int Hq, int Hkv, int dv);
+
+/*
+ * hca_decode -- one new query per sequence over its compressed cache and raw window
+ * (official blog, section 2.1), split over keys across the whole GPU and merged in a
+ * second pass.
+ *   q        [B,Hq,d] bf16        the query at position t = seqlens[b] - 1
+ *   kc, vc   contiguous: [B,Nmax,Hkv,d|dv] bf16, entry j of sequence b at row (b, j);
+ *            with HCA_PAGED: page pools [P,page_size,Hkv,d|dv], entry j of sequence b at
+ *            pool[page_table[b*max_pages + j/page_size], j % page_size]
+ *   page_table [B,max_pages] int32 (HCA_PAGED only, else NULL); num_pages = P, the
+ *            number of pages in the pools (entries outside [0, P) are reported as
+ *            HCA_ERR_DEVICE_INPUT and read as zeros)
+ *   kw, vw   [B,W,Hkv,d|dv] bf16  raw window: slot i holds position seqlens[b] - W + i;
+ *            slots with a negative position are ignored
+ *   seqlens  [B] int32            context length L_b >= 1 including the new token; the
+ *            visible entry count n_c(L_b - 1) must not exceed Nmax (or the pages)
+ *   gq, gk   [d] fp32 gains, eps  (HCA_QK_NORM only, else NULL)
+ *   gate     [B,Hq,dv] bf16 logits (HCA_OUT_GATE only, else NULL)
+ *   out      [B,Hq,dv] fp32
+ *   workspace, ws_bytes           device scratch of at least
+ *            hca_decode_workspace_size(B, Hq, Hkv, dv) bytes, owned by the caller; its
+ *            contents need no initialisation and are overwritten
+ * Supported: d == dv == 512; Hq % Hkv == 0 with Hq / Hkv <= 64; 1 <= blk <= 128; W >= 1;
+ * page_size a multiple of 64 with HCA_PAGED.
+ */
+hca_status_t hca_decode(const void* q, const void* kc, const void* vc,
+                        const int* page_table, int page_size, int max_pages, int num_pages,
+                        const void* kw, const void* vw, const int* seqlens,
+                        const float* gq, const float* gk, float eps,
+                        const void* gate, float* out,
+                        void* workspace, size_t ws_bytes,
+                        int B, int Hq, int Hkv, int d, int dv, int blk, int W, int Nmax,
+                        float scale, unsigned flags, hca_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* hca_status_string(hca_status_t status);
+
+/*
+ * hca_get_device_error -- wait for `stream`, then read and clear the current device's
+ * error word: HCA_OK if no kernel recorded an error since the last call,
+ * HCA_ERR_TIMEOUT or HCA_ERR_DEVICE_INPUT otherwise, HCA_ERR_CUDA if the read failed.
+ */
+hca_status_t hca_get_device_error(hca_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HCA_H_ */

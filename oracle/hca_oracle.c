@@ -162,7 +162,8 @@ static void attend(const double* qv, const double* keys, const double* vals, int
 }
 
 /*
- * Prefill rows.  q [B,T,Hq,d], k [B,T,Hkv,d], v [B,T,Hkv,dv] bf16;
+ * Prefill rows.  q [B,T,Hq,d] (or, with q_rows != 0, [n_rows,Hq,d]: one query row per
+ * requested (b, t)), k [B,T,Hkv,d], v [B,T,Hkv,dv] bf16;
  * kc [B,Nc,Hkv,d], vc [B,Nc,Hkv,dv] bf16 (the stored cache), Nc = T / blk.
  * rows: n_rows pairs (b, t).  out: [n_rows, Hq, dv] fp64; lse: [n_rows, Hq] or NULL.
  * Query head h reads KV head h / (Hq / Hkv).
@@ -171,7 +172,7 @@ int oracle_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         const uint16_t* kc, const uint16_t* vc,
                         int64_t B, int64_t T, int64_t Hq, int64_t Hkv, int64_t d, int64_t dv,
                         int64_t blk, int64_t W, double scale,
-                        const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+                        const int64_t* rows, int64_t n_rows, int q_rows, double* out, double* lse) {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv || blk <= 0 || W <= 0) return 1;
     int64_t Nc = T / blk, grp = Hq / Hkv;
     #pragma omp parallel
@@ -196,7 +197,8 @@ int oracle_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     for (int64_t c = 0; c < dv; ++c) vals[n * dv + c] = bf(v[((b * T + u) * Hkv + g) * dv + c]);
                 }
                 for (int64_t h = g * grp; h < (g + 1) * grp; ++h) {
-                    for (int64_t c = 0; c < d; ++c) qv[c] = bf(q[((b * T + t) * Hq + h) * d + c]);
+                    const uint16_t* qr = q_rows ? q + (r * Hq + h) * d : q + ((b * T + t) * Hq + h) * d;
+                    for (int64_t c = 0; c < d; ++c) qv[c] = bf(qr[c]);
                     attend(qv, keys, vals, n, d, dv, scale, out + (r * Hq + h) * dv,
                            lse ? lse + r * Hq + h : NULL, z);
                 }

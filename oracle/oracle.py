@@ -32,7 +32,7 @@ def _load():
         lib.oracle_compress.argtypes = [_u16p, _u16p, _vp] + [_i64] * 6 + [_f64p, _f64p]
         lib.oracle_prefill_rows.restype = ctypes.c_int
         lib.oracle_prefill_rows.argtypes = ([_u16p] * 5 + [_i64] * 8 + [ctypes.c_double, _i64p, _i64,
-                                            _f64p, _vp])
+                                            ctypes.c_int, _f64p, _vp])
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode.argtypes = ([_u16p, _u16p, _u16p, _vp, _i64, _i64, _u16p, _u16p, _i32p,
                                        _vp, _vp, ctypes.c_double, _vp] + [_i64] * 8
@@ -99,14 +99,15 @@ def compress(k, v, w, blk):
     return kc, vc
 
 
-def prefill_rows(q, k, v, kc, vc, blk, W, scale, rows, want_lse=False):
+def prefill_rows(q, k, v, kc, vc, blk, W, scale, rows, want_lse=False, q_rows=False):
     """Attention output of prefill rows.
 
-    q [B,T,Hq,d], k [B,T,Hkv,d], v [B,T,Hkv,dv], kc [B,Nc,Hkv,d], vc [B,Nc,Hkv,dv]: uint16 bf16 bits.
+    q [B,T,Hq,d] (or [n_rows,Hq,d] with q_rows=True), k [B,T,Hkv,d], v [B,T,Hkv,dv],
+    kc [B,Nc,Hkv,d], vc [B,Nc,Hkv,dv]: uint16 bf16 bits.
     rows: iterable of (b, t).  Returns out [n_rows, Hq, dv] fp64 (and lse [n_rows, Hq]).
     """
-    B, T, Hq, d = q.shape
-    Hkv = k.shape[2]
+    B, T, Hkv, _ = k.shape
+    Hq, d = q.shape[-2], q.shape[-1]
     dv = v.shape[3]
     Nc = T // blk
     assert kc.shape == (B, Nc, Hkv, d) and vc.shape == (B, Nc, Hkv, dv)
@@ -115,8 +116,12 @@ def prefill_rows(q, k, v, kc, vc, blk, W, scale, rows, want_lse=False):
     out = np.zeros((n, Hq, dv), dtype=np.float64)
     lse = np.zeros((n, Hq), dtype=np.float64) if want_lse else None
     args = [np.ascontiguousarray(a, dtype=np.uint16) for a in (q, k, v, kc, vc)]
+    if q_rows:
+        assert q.shape[0] == n
+    else:
+        assert q.shape[:2] == (B, T)
     rc = _load().oracle_prefill_rows(*args, B, T, Hq, Hkv, d, dv, blk, W, float(scale), rows, n,
-                                     out, _ptr(lse))
+                                     1 if q_rows else 0, out, _ptr(lse))
     if rc:
         raise ValueError("oracle_prefill_rows rejected its arguments (%d)" % rc)
     return (out, lse) if want_lse else out

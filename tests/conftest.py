@@ -18,3 +18,11 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def libhca():
+    """Build (if stale) and load the in-tree libhca.so."""
+    from compressed_long_context_b200 import _lib, build
+    build.build()
+    return _lib.load()

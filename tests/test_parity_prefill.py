@@ -1,0 +1,156 @@
+"""GPU parity of hca_compress + hca_prefill (through the C ABI) against the fp64 oracle.
+
+Bar: max abs error <= 1e-2 and mean abs error <= 1e-3 (output), same for the LSE.
+The oracle builds its own compressed cache from the raw K/V (rounded to bf16 as the
+stored cache is); nothing it reads comes from the CUDA path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import compressed_long_context_b200 as hca
+import oracle
+from compressed_long_context_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+MAX_TOL, MEAN_TOL = 1e-2, 1e-3
+
+
+def check(got, ref, what="out"):
+    g = got.detach().float().cpu().numpy().astype(np.float64)
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    assert np.isfinite(g).all(), what
+    err = np.abs(g - ref)
+    assert err.max() <= MAX_TOL, (what, "max", err.max())
+    assert err.mean() <= MEAN_TOL, (what, "mean", err.mean())
+
+
+def bits(t):
+    return oracle.bf16_bits(t)
+
+
+def oracle_cache(k, v, w, blk):
+    kc, vc = oracle.compress(bits(k), bits(v), None if w is None else w.cpu().numpy(), blk)
+    return oracle.round_bf16(kc), oracle.round_bf16(vc)
+
+
+def run_case(dev, B, T, Hq, Hkv, d, blk, W, seed, out_f32=False, lse=True, wstd=0.5, rows=None):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    q = torch.randn((B, T, Hq, d), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((B, T, Hkv, d), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((B, T, Hkv, d), generator=g, device=dev).to(torch.bfloat16)
+    w = torch.randn((B, T), generator=g, device=dev) * wstd
+    scale = 1.0 / np.sqrt(d)
+    kc, vc = hca.compress(k, v, w, blk)
+    res = hca.prefill(q, k, v, kc, vc, blk, W, scale, want_lse=lse, out_f32=out_f32)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    out, l = res if lse else (res, None)
+    kcb, vcb = oracle_cache(k, v, w, blk)
+    if rows is None:
+        rows = [(b, t) for b in range(B) for t in range(T)]
+    qb = bits(q)
+    ro, rl = oracle.prefill_rows(qb, bits(k), bits(v), kcb, vcb, blk, W, scale, rows, want_lse=True)
+    idx_b = torch.tensor([r[0] for r in rows])
+    idx_t = torch.tensor([r[1] for r in rows])
+    check(out.cpu()[idx_b, idx_t], ro)
+    if lse:
+        check(l.cpu()[idx_b, :, idx_t], rl, "lse")
+
+
+def test_tiny_prefill_workload(cuda_device, libhca):
+    """B=1, T=1024, Hq=4, Hkv=1, d=64, W=128, mean pooling, fp32 output: every row."""
+    cfg = wl.TINY_PREFILL
+    inp = wl.prefill_inputs(cfg, cuda_device)
+    scale = 1.0 / np.sqrt(cfg.d)
+    kc, vc = hca.compress(inp["k"], inp["v"], inp["w"], cfg.blk)
+    out, lse = hca.prefill(inp["q"], inp["k"], inp["v"], kc, vc, cfg.blk, cfg.W, scale, want_lse=True,
+                           out_f32=True)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    assert kc.shape == (1, 8, 1, 64) and out.dtype == torch.float32
+    kcb, vcb = oracle_cache(inp["k"], inp["v"], inp["w"], cfg.blk)
+    rows = [(0, t) for t in range(cfg.T)]
+    ro, rl = oracle.prefill_rows(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]), kcb, vcb, cfg.blk, cfg.W,
+                                 scale, rows, want_lse=True)
+    check(out[0], ro)
+    check(lse[0].transpose(0, 1), rl, "lse")
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,blk,W", [
+    (2, 1000, 8, 2, 128, 128),
+    (1, 777, 4, 1, 1, 5),
+    (1, 500, 16, 1, 2, 300),
+    (2, 300, 2, 2, 128, 1),
+    (1, 200, 4, 4, 16, 1000),     # window covers everything
+    (1, 1300, 128, 1, 64, 100),   # 128 heads per group: one token per tile
+    (1, 129, 1, 1, 128, 128),     # one head per group: 128 tokens per tile
+])
+def test_prefill_d64(cuda_device, libhca, B, T, Hq, Hkv, blk, W):
+    run_case(cuda_device, B, T, Hq, Hkv, 64, blk, W, seed=T + Hq, out_f32=(T % 2 == 0))
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,blk,W", [
+    (1, 600, 64, 1, 128, 128),
+    (1, 450, 64, 1, 128, 256),
+    (2, 333, 16, 2, 32, 40),
+    (1, 260, 32, 1, 1, 3),
+])
+def test_prefill_d512(cuda_device, libhca, B, T, Hq, Hkv, blk, W):
+    run_case(cuda_device, B, T, Hq, Hkv, 512, blk, W, seed=T + 7 * Hq, out_f32=(Hq == 16))
+
+
+def test_prefill_d512_long_sampled(cuda_device, libhca):
+    T = 6000
+    rs = np.random.RandomState(1)
+    rows = [(0, t) for t in sorted(set([0, 1, 127, 128, 254, 255, 256, 383, 384, 5999, 5998]
+                                        + list(rs.randint(0, T, 20))))]
+    run_case(cuda_device, 1, T, 64, 1, 512, 128, 128, seed=3, rows=rows)
+
+
+def test_prefill_large_logits(cuda_device, libhca):
+    """Raw keys boosted x8 on a few rows: the running max jumps mid-sequence."""
+    dev = cuda_device
+    B, T, Hq, d = 1, 900, 64, 512
+    g = torch.Generator(device=dev).manual_seed(99)
+    q = torch.randn((B, T, Hq, d), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((B, T, 1, d), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((B, T, 1, d), generator=g, device=dev).to(torch.bfloat16)
+    k[0, ::37] = (k[0, ::37].float() * 8).to(torch.bfloat16)
+    w = torch.randn((B, T), generator=g, device=dev) * 0.5
+    kc, vc = hca.compress(k, v, w, 128)
+    out = hca.prefill(q, k, v, kc, vc, 128, 128, 1.0 / np.sqrt(d))
+    torch.cuda.synchronize()
+    kcb, vcb = oracle_cache(k, v, w, 128)
+    rows = [(0, t) for t in range(T)]
+    ro = oracle.prefill_rows(bits(q), bits(k), bits(v), kcb, vcb, 128, 128, 1.0 / np.sqrt(d), rows)
+    check(out[0], ro)
+
+
+def test_prefill_128k_workload_sampled(cuda_device, libhca):
+    """Full-size 128K prefill (T=131072, Hq=64, d=512, 1% boosted keys) in the benchmark's
+    launch configuration; sampled rows checked against oracle compress + oracle prefill."""
+    cfg = wl.PREFILL_128K
+    inp = wl.prefill_inputs(cfg, cuda_device)
+    scale = 1.0 / np.sqrt(cfg.d)
+    kc, vc = hca.compress(inp["k"], inp["v"], inp["w"], cfg.blk)
+    out, lse = hca.prefill(inp["q"], inp["k"], inp["v"], kc, vc, cfg.blk, cfg.W, scale, want_lse=True)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    T = cfg.T
+    kb = inp["k"][0, :, 0].float().abs().amax(dim=1)
+    boosted = torch.nonzero(kb > 6.0).flatten().tolist()[:40]
+    rs = np.random.RandomState(2)
+    ts = set([0, 1, 2, 126, 127, 128, 129, 254, 255, 256, 257, 1000, T - 3, T - 2, T - 1])
+    ts |= set(int(x) for x in rs.randint(0, T, 60))
+    ts |= set(min(T - 1, b + o) for b in boosted for o in (0, 1, 100, 127))
+    rows = [(0, t) for t in sorted(ts)]
+    kcb, vcb = oracle_cache(inp["k"], inp["v"], inp["w"], cfg.blk)
+    qsel = bits(inp["q"][0, [t for _, t in rows]])
+    ro, rl = oracle.prefill_rows(qsel, bits(inp["k"]), bits(inp["v"]), kcb, vcb, cfg.blk, cfg.W, scale, rows,
+                                 want_lse=True, q_rows=True)
+    idx = torch.tensor([t for _, t in rows], device=cuda_device)
+    check(out[0, idx], ro)
+    check(lse[0][:, idx].transpose(0, 1), rl, "lse")
+    del inp, kc, vc, out, lse
+    torch.cuda.empty_cache()
