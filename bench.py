@@ -146,13 +146,19 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Max of a host scalar over all ranks (timing only; not on the data path)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(per_rank_units, world, seconds):
+    """Whole-job throughput: units processed by all ranks / max-over-ranks device time."""
+    return per_rank_units * world / seconds
 
 
 def l2_flush_buffer():
@@ -304,7 +310,7 @@ def main():
     hca.get_device_error()
     t_step = max_over_ranks(sum(step_ms) / 1e3, world)
     ms_per_step = t_step * 1e3 / args.steps
-    value = world * B * args.steps / t_step
+    value = weak_scaling_value(B * args.steps, world, t_step)
 
     # compress roofline (dominant kernel of the step)
     cbytes = compress_bytes(B, L, 1, cfg.d, cfg.dv, cfg.blk)

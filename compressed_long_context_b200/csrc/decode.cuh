@@ -34,7 +34,7 @@ constexpr int kDecD = 512;                 // head dim (d == dv)
 constexpr int kDecSlabs = kDecD / 64;      // 64-channel slabs per key row
 constexpr int kDecTile = 128;              // keys per tile (MMA M of S^T)
 constexpr int kDecHeads = 64;              // MMA N: query heads of one KV group (padded)
-constexpr int kDecRing = 8;                // ring slots (even, see the V^T descriptor)
+constexpr int kDecRing = 6;                // ring slots (even, see the V^T descriptor)
 constexpr int kDecThreads = 192;
 constexpr uint32_t kSlabBytes = 128 * 128;                 // 128 rows x 128 B
 constexpr uint32_t kDecQBytes = kDecHeads * kDecD * 2;     // 64 KB
@@ -59,6 +59,8 @@ constexpr uint32_t kSmAlpha = kSmMax + 64 * 4;              // float[64] rescale
 constexpr uint32_t kSmSum = kSmAlpha + 64 * 4;              // float[64] running sum per head
 constexpr uint32_t kSmMisc = kSmSum + 64 * 4;               // ints
 constexpr uint32_t kDecSmemBytes = kSmMisc + 64 + 1024;     // + alignment slack
+static_assert(kDecSmemBytes <= 232448, "decode shared memory exceeds the 227 KB per-block limit");
+static_assert(kDecRing % 2 == 0, "V^T operand pairs need an even ring");
 
 struct DecodeParams {
     const __nv_bfloat16* q;      // [B, Hq, 512]

@@ -47,6 +47,7 @@ struct PfCfg {
     static constexpr int kNumBars = 2 * kRing + 10;
     static constexpr uint32_t kSmMisc = kSmBar + kNumBars * 8;
     static constexpr uint32_t kSmem = kSmMisc + 64 + 1024;
+    static_assert(kSmem <= 232448, "prefill shared memory exceeds the 227 KB per-block limit");
     static constexpr uint32_t kTmS = 0;       // 2 x 128 columns
     static constexpr uint32_t kTmO = 256;     // kDVC columns
 };

@@ -35,6 +35,9 @@ def oracle_cache(k, v, w, blk):
 
 
 def run_case(dev, B, T, Hq, Hkv, d, blk, W, seed, out_f32=False, lse=True, wstd=0.5, rows=None):
+    # With only a handful of keys per row (tiny W and blk) outputs reach |o| ~ 3, where a bf16
+    # output alone is off by up to 2^-8 |o| > 1e-2: such stress cases return fp32.
+    out_f32 = out_f32 or W <= 8
     g = torch.Generator(device=dev).manual_seed(seed)
     q = torch.randn((B, T, Hq, d), generator=g, device=dev).to(torch.bfloat16)
     k = torch.randn((B, T, Hkv, d), generator=g, device=dev).to(torch.bfloat16)
