@@ -51,7 +51,7 @@ constexpr uint32_t kSmQ = 0;
 constexpr uint32_t kSmP = kSmQ + kDecQBytes;
 constexpr uint32_t kSmRing = kSmP + 2 * kDecPBytes;
 constexpr uint32_t kSmBar = kSmRing + kDecRing * kSlabBytes;
-constexpr int kNumBars = 2 * kDecRing + 12;
+constexpr int kNumBars = 2 * kDecRing + 13;
 constexpr uint32_t kSmRed = kSmBar + kNumBars * 8;          // float[4][64]
 constexpr uint32_t kSmFin = kSmRed + 4 * 64 * 4;            // float[64] reduction result
 constexpr uint32_t kSmMax = kSmFin + 64 * 4;                // float[64] running max per head
@@ -139,6 +139,18 @@ __device__ __forceinline__ bool softmax_any(bool pred) {
     return r != 0;
 }
 
+// Wait by all 128 softmax threads with one verdict for the group (barrier.red.and), so
+// the four warps either all go on or all unwind -- their named barriers never strand a
+// warp.
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    const bool ok = mbar_wait(bar, parity, abort);
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "barrier.red.and.pred q, 3, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)ok) : "memory");
+    return r != 0;
+}
+
 // Column reduction over the 128 softmax threads of a 64-vector held by every thread:
 // warp reduce-scatter with shuffles (lane l ends with heads 2l, 2l+1), then the four
 // warps meet in shared memory.  Result (all 64 heads) left in fin[] for every thread.
@@ -183,7 +195,8 @@ __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) {
 }
 
 __global__ void __launch_bounds__(kDecThreads, 1)
-decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
+decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kw,
                     const __grid_constant__ CUtensorMap tm_vw) {
     extern __shared__ uint8_t dsmem[];
@@ -199,6 +212,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     uint64_t* p_empty = q_full + 8;   // [2]
     uint64_t* o_full = q_full + 10;
     uint64_t* o_empty = q_full + 11;
+    uint64_t* q_tma = q_full + 12;    // Q slabs landed (TMA)
     float* red = reinterpret_cast<float*>(sm + kSmRed);
     float* fin = reinterpret_cast<float*>(sm + kSmFin);
     float* m_s = reinterpret_cast<float*>(sm + kSmMax);
@@ -231,10 +245,12 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         }
         mbar_init(o_full, 1);
         mbar_init(o_empty, 4);
+        mbar_init(q_tma, 1);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, 512);
     if (threadIdx.x == 0) {
+        prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_kw);
@@ -332,6 +348,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 }
                 return true;
             };
+            int item = 0;
             while (ok && pu < te) {
                 UnitTiles t = unit_tiles(p, u, false);
                 const int ntiles = t.nct + t.nwt;
@@ -341,6 +358,16 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     if (tile == tb && prev.u >= 0) {
                         ok = load_tile(prev.u, prev.tile, true);
                         prev.u = -1;
+                    }
+                    if (ok && tile == tb) {
+                        // this piece's 64 query rows (heads g*G ..), eight 8 KB slabs
+                        ok = mbar_wait(q_empty, (item & 1) ^ 1, abort_flag);
+                        if (ok) {
+                            mbar_arrive_expect_tx(q_tma, kDecQBytes);
+                            for (int s = 0; s < kDecSlabs; ++s)
+                                tma_load_4d(sm + kSmQ + s * 8192, &tm_q, q_tma, 64 * s, t.g * p.G, t.b, 0);
+                        }
+                        ++item;
                     }
                     if (ok) ok = load_tile(u, tile, false);
                     if (ok && prev.u >= 0) ok = load_tile(prev.u, prev.tile, true);
@@ -367,14 +394,14 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 
         auto issue_pv = [&]() -> bool {
             const int b = pv_n & 1;
-            if (!mbar_wait(&p_full[b], (pv_n >> 1) & 1, abort_flag)) return false;
-            if (pv_first && !mbar_wait(o_empty, (pv_item & 1) ^ 1, abort_flag)) return false;
+            if (!warp_wait(&p_full[b], (pv_n >> 1) & 1, abort_flag)) return false;
+            if (pv_first && !warp_wait(o_empty, (pv_item & 1) ^ 1, abort_flag)) return false;
             tc_fence_after();
             const uint32_t p_base = smem_u32(sm + kSmP + b * kDecPBytes);
             for (int c = 0; c < 4; ++c) {
                 const uint32_t st0 = ring % kDecRing, st1 = (ring + 1) % kDecRing;
-                if (!mbar_wait(&full[st0], (ring / kDecRing) & 1, abort_flag)) return false;
-                if (!mbar_wait(&full[st1], ((ring + 1) / kDecRing) & 1, abort_flag)) return false;
+                if (!warp_wait(&full[st0], (ring / kDecRing) & 1, abort_flag)) return false;
+                if (!warp_wait(&full[st1], ((ring + 1) / kDecRing) & 1, abort_flag)) return false;
                 if (pv_partial) {
                     // rows >= nvalid may hold anything (caller memory past the visible
                     // entries): zero them so 0-probability keys contribute exactly 0
@@ -425,17 +452,17 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     if (!issue_pv()) { ok = false; break; }
                     pv_n = -1;
                 }
-                if (first && !mbar_wait(q_full, item & 1, abort_flag)) { ok = false; break; }
-                if (!mbar_wait(&s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                if (first && !warp_wait(q_full, item & 1, abort_flag)) { ok = false; break; }
+                if (!warp_wait(&s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 // the K K^T accumulator has one buffer: wait until tile n-1's softmax has read it
-                if (norm && n > 0 && !mbar_wait(&s_empty[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) {
+                if (norm && n > 0 && !warp_wait(&s_empty[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int s = 0; s < kDecSlabs; ++s) {
                     const uint32_t st = ring % kDecRing;
-                    if (!mbar_wait(&full[st], (ring / kDecRing) & 1, abort_flag)) { ok = false; break; }
+                    if (!warp_wait(&full[st], (ring / kDecRing) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     if (lane == 0) {
                         const uint32_t k_base = smem_u32(sm + kSmRing + st * kSlabBytes);
@@ -487,52 +514,44 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             const int tb = (int)((ts > pu ? ts : pu) - pu);
             const int tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
 
-            // ---- stage this unit's queries (64 rows, zero past G) into Q smem
-            if (!mbar_wait(q_empty, (item & 1) ^ 1, abort_flag)) { ok = false; break; }
-            {
+            // ---- this piece's queries arrive by TMA; with QK normalisation they are
+            // rewritten in place as q' = q / rms(q) * g_q * g_k (bf16), since
+            // q_hat . k_hat = (q' . k) / rms(k)
+            if (!group_wait(q_tma, item & 1, abort_flag)) { ok = false; break; }
+            if (norm) {
                 const int h = sidx >> 1, half = sidx & 1;
-                const bool live = h < p.G;
-                const __nv_bfloat16* qrow = p.q + ((size_t)t.b * p.Hq + (size_t)t.g * p.G + h) * kDecD + 256 * half;
-                float inv = 1.f;
-                if (norm && live) {
-                    float ss = 0.f;
-                    for (int c = 0; c < 256; c += 8) {
-                        const uint4 x = __ldg(reinterpret_cast<const uint4*>(qrow + c));
-                        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float a = bf16lo(w4[i]), b2 = bf16hi(w4[i]);
-                            ss = fmaf(a, a, fmaf(b2, b2, ss));
-                        }
-                    }
-                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                    inv = rsqrtf(ss * (1.f / kDecD) + p.eps);
-                }
+                float ss = 0.f;
                 for (int c = 0; c < 256; c += 8) {
-                    uint4 x = make_uint4(0, 0, 0, 0);
-                    if (live) {
-                        x = __ldg(reinterpret_cast<const uint4*>(qrow + c));
-                        if (norm) {
-                            const int cc = 256 * half + c;
-                            uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int ch = cc + 2 * i;
-                                const float a = bf16lo(w4[i]) * inv * __ldg(p.gq + ch) * __ldg(p.gk + ch);
-                                const float b2 = bf16hi(w4[i]) * inv * __ldg(p.gq + ch + 1) * __ldg(p.gk + ch + 1);
-                                w4[i] = pack_bf16x2(a, b2);
-                            }
-                            x = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                        }
-                    }
                     const int cc = 256 * half + c;
-                    uint8_t* slab = sm + kSmQ + (cc >> 6) * 8192;
-                    *reinterpret_cast<uint4*>(slab + sw128(h, (cc & 63) >> 3)) = x;
+                    const uint4 x = *reinterpret_cast<const uint4*>(sm + kSmQ + (cc >> 6) * 8192 +
+                                                                  sw128(h, (cc & 63) >> 3));
+                    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float a = bf16lo(w4[i]), b2 = bf16hi(w4[i]);
+                        ss = fmaf(a, a, fmaf(b2, b2, ss));
+                    }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                const float inv = rsqrtf(ss * (1.f / kDecD) + p.eps);
+                for (int c = 0; c < 256; c += 8) {
+                    const int cc = 256 * half + c;
+                    uint4* ptr = reinterpret_cast<uint4*>(sm + kSmQ + (cc >> 6) * 8192 + sw128(h, (cc & 63) >> 3));
+                    const uint4 x = *ptr;
+                    uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int ch = cc + 2 * i;
+                        const float a = bf16lo(w4[i]) * inv * __ldg(p.gq + ch) * __ldg(p.gk + ch);
+                        const float b2 = bf16hi(w4[i]) * inv * __ldg(p.gq + ch + 1) * __ldg(p.gk + ch + 1);
+                        w4[i] = pack_bf16x2(a, b2);
+                    }
+                    *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
                 fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(q_full);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_full);
 
             for (int tile = tb; ok && tile < tend; ++tile, ++n) {
                 const bool first = tile == tb, last = tile == tend - 1;
@@ -542,7 +561,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                                         : min(kDecTile, p.W - (t.s0 + (tile - t.nct) * kDecTile));
                 const bool valid = r < nvalid;
 
-                if (!mbar_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (!group_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 float z[64];
 #pragma unroll
@@ -595,7 +614,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     if (!first) {
                         // rescale O^T once the previous PV has landed
                         const int pb = (n - 1) & 1;
-                        if (!mbar_wait(&p_empty[pb], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                        if (!group_wait(&p_empty[pb], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -627,7 +646,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     pk[(h >> 1) + 1] = pack_bf16x2(z[h + 2], z[h + 3]);
                 }
                 const int pbuf = n & 1;
-                if (!mbar_wait(&p_empty[pbuf], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                if (!group_wait(&p_empty[pbuf], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 uint8_t* pt = sm + kSmP + pbuf * kDecPBytes;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
@@ -651,7 +670,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                         if (tb == 0) p.meta[2 * u] = cta;
                         if (tend == ntiles) p.meta[2 * u + 1] = cta;
                     }
-                    if (!mbar_wait(o_full, item & 1, abort_flag)) { ok = false; break; }
+                    if (!group_wait(o_full, item & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     float* orec = p.rec_o + (size_t)rec * 64 * kDecD;
                     for (int c = 0; c < 4; ++c) {

@@ -207,8 +207,10 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     if (ws_bytes < lay.bytes) return HCA_ERR_INVALID_ARG;
 
     const uint64_t hd = (uint64_t)Hkv * kDecD;
-    CUtensorMap tk, tv, tkw, tvw;
+    CUtensorMap tq, tk, tv, tkw, tvw;
     bool ok = true;
+    // queries [B, Hq, 512]: a box of 64 heads starting at the group's first head
+    ok &= make_tmap_4d(&tq, q, kDecD, Hq, B, 1, kDecD, (uint64_t)Hq * kDecD, (uint64_t)B * Hq * kDecD, 64, 64, 1, 1);
     if (paged) {
         ok &= make_tmap_4d(&tk, kc, kDecD, Hkv, page_size, num_pages, kDecD, hd, hd * page_size, 64, 1, 64, 1);
         ok &= make_tmap_4d(&tv, vc, kDecD, Hkv, page_size, num_pages, kDecD, hd, hd * page_size, 64, 1, 64, 1);
@@ -243,7 +245,7 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     if (!set_smem_attr_once(reinterpret_cast<const void*>(&decode_split_kernel), (int)kDecSmemBytes, 0))
         return HCA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    decode_split_kernel<<<nsplit, kDecThreads, kDecSmemBytes, s>>>(p, tk, tv, tkw, tvw);
+    decode_split_kernel<<<nsplit, kDecThreads, kDecSmemBytes, s>>>(p, tq, tk, tv, tkw, tvw);
     if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};

@@ -97,8 +97,6 @@ __device__ __forceinline__ int pf_tile_keys(const PfItem& it, int j) {
     return j < it.nct ? min(128, it.ncomp - 128 * j) : min(128, it.nwin - 128 * (j - it.nct));
 }
 
-__device__ __forceinline__ void tmem_st16_u(uint32_t taddr, const uint32_t* r) { tmem_st16(taddr, r); }
-
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
@@ -204,7 +202,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
         for (long long i = blockIdx.x; ok && i < p.items; i += stride, ++item_n) {
             const PfItem it = pf_item<D>(p, i);
             const int nt = it.nct + it.nwt;
-            if (!mbar_wait(q_full, item_n & 1, abort_flag)) { ok = false; break; }
+            if (!warp_wait(q_full, item_n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             auto issue_qk = [&](int j, int nn) -> bool {
                 const int N = (pf_tile_keys(it, j) + 15) & ~15;
@@ -212,7 +210,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                 const uint32_t dst = tmem + C::kTmS + 128 * (nn & 1);
                 for (int s = 0; s < C::kSlabs; ++s) {
                     const uint32_t st = ring % C::kRing;
-                    if (!mbar_wait(&full[st], (ring / C::kRing) & 1, abort_flag)) return false;
+                    if (!warp_wait(&full[st], (ring / C::kRing) & 1, abort_flag)) return false;
                     tc_fence_after();
                     if (lane == 0) {
                         const uint32_t kb = smem_u32(sm + C::kSmRing + st * kPfSlab);
@@ -238,12 +236,12 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                 const int ksteps = (pf_tile_keys(it, j) + 15) >> 4;
                 const uint32_t id = idesc_bf16(128, 64, 0, 1);
                 const uint32_t pa = tmem + C::kTmS + 128 * (nn & 1);
-                if (!mbar_wait(&p_full[nn & 1], (nn >> 1) & 1, abort_flag)) return false;
-                if (j == 0 && !mbar_wait(o_empty, (item_n & 1) ^ 1, abort_flag)) return false;
+                if (!warp_wait(&p_full[nn & 1], (nn >> 1) & 1, abort_flag)) return false;
+                if (j == 0 && !warp_wait(o_empty, (item_n & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
                 for (int v = 0; v < C::kVSlabs; ++v) {
                     const uint32_t st = ring % C::kRing;
-                    if (!mbar_wait(&full[st], (ring / C::kRing) & 1, abort_flag)) return false;
+                    if (!warp_wait(&full[st], (ring / C::kRing) & 1, abort_flag)) return false;
                     tc_fence_after();
                     if (lane == 0) {
                         const uint32_t vb = smem_u32(sm + C::kSmRing + st * kPfSlab);
@@ -300,7 +298,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                     lo = max(0, t - p.W + 1 - u0);
                     hi = min(nk, t - u0 + 1);
                 }
-                if (!mbar_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (!warp_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 float s[128];
                 const uint32_t sa = tmem + lane_off + C::kTmS + 128 * sb;
@@ -315,27 +313,32 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                     s[c] = v ? s[c] * p.scale_log2 : -INFINITY;
                     tmax = fmaxf(tmax, s[c]);
                 }
-                // lazy max: move the reference only when the new max exceeds it by 2^8
-                if (tmax > m + kPfRescale || (m == -INFINITY && tmax > -INFINITY)) {
-                    if (m != -INFINITY) {
-                        const float al = ex2(m - tmax);
-                        l *= al;
-                        // this row's O, once the previous PV has landed
-                        if (!mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
+                // lazy max: a row moves its reference only when the new max exceeds it by
+                // 2^8 (or on its first visible key).  tcgen05.ld/st are warp-collective, so the
+                // O rescale runs for the whole warp whenever any of its rows needs it, with
+                // factor 1 for the others.
+                const bool rescale = m != -INFINITY && tmax > m + kPfRescale;
+                float al = 1.f;
+                if (rescale) {
+                    al = ex2(m - tmax);
+                    l *= al;
+                }
+                if (rescale || (m == -INFINITY && tmax > -INFINITY)) m = tmax;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O, once the previous PV has landed
+                    if (!warp_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
-                        for (int c = 0; c < C::kDVC; c += 16) {
-                            float o[16];
-                            uint32_t w[16];
-                            tmem_ld16(tmem + lane_off + C::kTmO + c, o);
-                            tmem_wait_ld();
+                    for (int c = 0; c < C::kDVC; c += 16) {
+                        float o[16];
+                        uint32_t w[16];
+                        tmem_ld16(tmem + lane_off + C::kTmO + c, o);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int k = 0; k < 16; ++k) w[k] = __float_as_uint(o[k] * al);
-                            tmem_st16(tmem + lane_off + C::kTmO + c, w);
-                        }
-                        tmem_wait_st();
+                        for (int k = 0; k < 16; ++k) w[k] = __float_as_uint(o[k] * al);
+                        tmem_st16(tmem + lane_off + C::kTmO + c, w);
                     }
-                    m = tmax;
+                    tmem_wait_st();
                 }
                 const float mref = m == -INFINITY ? 0.f : m;
                 float rs = 0.f;
@@ -361,7 +364,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
             }
             if (!ok) break;
             // ---- epilogue: out = O / l, lse = ln(sum exp(logits))
-            if (!mbar_wait(o_full, item_n & 1, abort_flag)) { ok = false; break; }
+            if (!warp_wait(o_full, item_n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const float inv = 1.f / l;
             const size_t orow = (((size_t)it.b * p.T + tok) * p.Hq + head) * (size_t)(C::kDVC * C::kNS) +

@@ -1,0 +1,109 @@
+"""Small, self-contained launches of one HCA kernel for profiling (ncu) and quick timing.
+
+    python -m compressed_long_context_b200.profile_cases compress [--reps N]
+    python -m compressed_long_context_b200.profile_cases decode   [--reps N]
+    python -m compressed_long_context_b200.profile_cases prefill  [--reps N]
+    python -m compressed_long_context_b200.profile_cases paged    [--reps N]
+
+Each case keeps its working set larger than the 126 MB L2 (so DRAM counters mean
+something) but a few GB at most, and launches the kernel `--reps` times after one
+warm-up launch.  Prints the per-launch time from CUDA events (not meaningful under a
+profiler).
+"""
+import argparse
+import json
+import math
+
+import torch
+
+from . import compress, decode, decode_workspace_size, get_device_error, prefill
+from . import workloads as wl
+
+
+def _events():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def run(case: str, reps: int) -> dict:
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g = torch.Generator(device=dev).manual_seed(123)
+    if case == "compress":
+        # 8 sequences x 131072 tokens x 512: 2.1 GB of raw K/V
+        B, T, d = 8, 131072, 512
+        k = torch.randn((B, T, 1, d), generator=g, device=dev).to(torch.bfloat16)
+        v = torch.randn((B, T, 1, d), generator=g, device=dev).to(torch.bfloat16)
+        w = torch.randn((B, T), generator=g, device=dev) * 0.5
+        kc = torch.empty((B, T // 128, 1, d), dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        fn = lambda: compress(k, v, w, 128, kc=kc, vc=vc)  # noqa: E731
+        nbytes = B * (T // 128) * (128 * 2 * d * 2 + 2 * d * 2) + B * T * 4
+    elif case in ("decode", "paged"):
+        # the 128K decode batch with its cache drawn directly (134 MB of entries)
+        B, L, Hq, d, W = 64, 131072, 64, 512, 128
+        nc = (L - W) // 128
+        q = torch.randn((B, Hq, d), generator=g, device=dev).to(torch.bfloat16)
+        kw = torch.randn((B, W, 1, d), generator=g, device=dev).to(torch.bfloat16)
+        vw = torch.randn((B, W, 1, d), generator=g, device=dev).to(torch.bfloat16)
+        seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+        ws = torch.empty(decode_workspace_size(B, Hq, 1, d), dtype=torch.uint8, device=dev)
+        if case == "decode":
+            kc = torch.randn((B, L // 128, 1, d), generator=g, device=dev).to(torch.bfloat16)
+            vc = torch.randn((B, L // 128, 1, d), generator=g, device=dev).to(torch.bfloat16)
+            fn = lambda: decode(q, kc, vc, kw, vw, seq, 128, W, 1 / math.sqrt(d), out=out,  # noqa: E731
+                                workspace=ws)
+        else:
+            ps = 64
+            npg = (L // 128 + ps - 1) // ps
+            kc = torch.randn((B * npg, ps, 1, d), generator=g, device=dev).to(torch.bfloat16)
+            vc = torch.randn((B * npg, ps, 1, d), generator=g, device=dev).to(torch.bfloat16)
+            perm = torch.randperm(B * npg, generator=torch.Generator().manual_seed(5)).to(torch.int32)
+            table = perm.view(B, npg).to(dev)
+            gq = torch.rand((d,), generator=g, device=dev) + 0.5
+            gk = torch.rand((d,), generator=g, device=dev) + 0.5
+            gate = torch.randn((B, Hq, d), generator=g, device=dev).to(torch.bfloat16)
+            fn = lambda: decode(q, kc, vc, kw, vw, seq, 128, W, 1 / math.sqrt(d), page_table=table,  # noqa: E731
+                                page_size=ps, gq=gq, gk=gk, gate=gate, out=out, workspace=ws)
+        nbytes = B * (Hq * d * 2 + (nc + W) * 2 * d * 2 + Hq * d * 4)
+    elif case == "prefill":
+        # T = 16384 tokens, 64 heads of 512: 1 GB of Q, 1 GB of output
+        cfg = wl.PREFILL_128K.scaled(T=16384)
+        inp = wl.prefill_inputs(cfg, dev)
+        kc, vc = compress(inp["k"], inp["v"], inp["w"], 128)
+        out = torch.empty((1, cfg.T, cfg.Hq, cfg.dv), dtype=torch.bfloat16, device=dev)
+        fn = lambda: prefill(inp["q"], inp["k"], inp["v"], kc, vc, 128, cfg.W, 1 / math.sqrt(cfg.d),  # noqa: E731
+                             out=out)
+        keys = sum(max(0, (t - cfg.W + 1) // 128) + min(cfg.W, t + 1) for t in range(cfg.T))
+        nbytes = None
+        flops = 2.0 * cfg.Hq * keys * (cfg.d + cfg.dv)
+    else:
+        raise ValueError(case)
+    fn()
+    torch.cuda.synchronize()
+    get_device_error()
+    a, b = _events()
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    get_device_error()
+    ms = a.elapsed_time(b) / reps
+    res = {"case": case, "reps": reps, "ms_per_launch": ms}
+    if nbytes:
+        res["GB_per_s"] = nbytes / (ms / 1e3) / 1e9
+    if case == "prefill":
+        res["TFLOP_per_s"] = flops / (ms / 1e3) / 1e12
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["compress", "decode", "paged", "prefill"])
+    ap.add_argument("--reps", type=int, default=3)
+    args = ap.parse_args()
+    print(json.dumps(run(args.case, args.reps)))
+
+
+if __name__ == "__main__":
+    main()
