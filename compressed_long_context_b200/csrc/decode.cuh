@@ -52,7 +52,7 @@ constexpr uint32_t kSmP = kSmQ + kDecQBytes;
 constexpr uint32_t kSmRing = kSmP + 2 * kDecPBytes;
 constexpr uint32_t kSmBar = kSmRing + kDecRing * kSlabBytes;
 constexpr int kNumBars = 2 * kDecRing + 13;
-constexpr uint32_t kSmRed = kSmBar + kNumBars * 8;          // float[4][64]
+constexpr uint32_t kSmRed = (kSmBar + kNumBars * 8 + 127) & ~127u;   // float[4][64] (read as float4)
 constexpr uint32_t kSmFin = kSmRed + 4 * 64 * 4;            // float[64] reduction result
 constexpr uint32_t kSmMax = kSmFin + 64 * 4;                // float[64] running max per head
 constexpr uint32_t kSmAlpha = kSmMax + 64 * 4;              // float[64] rescale factors
@@ -60,6 +60,9 @@ constexpr uint32_t kSmSum = kSmAlpha + 64 * 4;              // float[64] running
 constexpr uint32_t kSmMisc = kSmSum + 64 * 4;               // ints
 constexpr uint32_t kDecSmemBytes = kSmMisc + 64 + 1024;     // + alignment slack
 static_assert(kDecSmemBytes <= 232448, "decode shared memory exceeds the 227 KB per-block limit");
+static_assert(kSmRed % 16 == 0 && kSmFin % 16 == 0 && kSmMax % 16 == 0 && kSmAlpha % 16 == 0 &&
+              kSmSum % 16 == 0 && kSmMisc % 16 == 0, "vector-accessed shared arrays must be 16-byte aligned");
+static_assert(kSmP % 1024 == 0 && kSmRing % 1024 == 0, "swizzled operand tiles must be 1024-byte aligned");
 static_assert(kDecRing % 2 == 0, "V^T operand pairs need an even ring");
 
 struct DecodeParams {

@@ -48,6 +48,7 @@ struct PfCfg {
     static constexpr uint32_t kSmMisc = kSmBar + kNumBars * 8;
     static constexpr uint32_t kSmem = kSmMisc + 64 + 1024;
     static_assert(kSmem <= 232448, "prefill shared memory exceeds the 227 KB per-block limit");
+    static_assert(kSmRing % 1024 == 0 && kSmBar % 8 == 0, "operand tiles 1024-aligned, barriers 8-aligned");
     static constexpr uint32_t kTmS = 0;       // 2 x 128 columns
     static constexpr uint32_t kTmO = 256;     // kDVC columns
 };

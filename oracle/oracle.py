@@ -20,25 +20,34 @@ _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
 
 
+def _bind(path):
+    """Load an oracle shared object and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    _declare(lib)
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(_build.build())
-        lib.oracle_num_threads.restype = ctypes.c_int
-        lib.oracle_visible_entries.restype = _i64
-        lib.oracle_visible_entries.argtypes = [_i64, _i64, _i64]
-        lib.oracle_round_bf16.argtypes = [_f64p, _u16p, _i64]
-        lib.oracle_compress.restype = ctypes.c_int
-        lib.oracle_compress.argtypes = [_u16p, _u16p, _vp] + [_i64] * 6 + [_f64p, _f64p]
-        lib.oracle_prefill_rows.restype = ctypes.c_int
-        lib.oracle_prefill_rows.argtypes = ([_u16p] * 5 + [_i64] * 8 + [ctypes.c_double, _i64p, _i64,
-                                            ctypes.c_int, _f64p, _vp])
-        lib.oracle_decode.restype = ctypes.c_int
-        lib.oracle_decode.argtypes = ([_u16p, _u16p, _u16p, _vp, _i64, _i64, _u16p, _u16p, _i32p,
-                                       _vp, _vp, ctypes.c_double, _vp] + [_i64] * 8
-                                      + [ctypes.c_double, _f64p, _vp])
-        _lib = lib
+        _lib = _bind(_build.build())
     return _lib
+
+
+def _declare(lib):
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_visible_entries.restype = _i64
+    lib.oracle_visible_entries.argtypes = [_i64, _i64, _i64]
+    lib.oracle_round_bf16.argtypes = [_f64p, _u16p, _i64]
+    lib.oracle_compress.restype = ctypes.c_int
+    lib.oracle_compress.argtypes = [_u16p, _u16p, _vp] + [_i64] * 6 + [_f64p, _f64p]
+    lib.oracle_prefill_rows.restype = ctypes.c_int
+    lib.oracle_prefill_rows.argtypes = ([_u16p] * 5 + [_i64] * 8 + [ctypes.c_double, _i64p, _i64,
+                                        ctypes.c_int, _f64p, _vp])
+    lib.oracle_decode.restype = ctypes.c_int
+    lib.oracle_decode.argtypes = ([_u16p, _u16p, _u16p, _vp, _i64, _i64, _u16p, _u16p, _i32p,
+                                   _vp, _vp, ctypes.c_double, _vp] + [_i64] * 8
+                                  + [ctypes.c_double, _f64p, _vp])
 
 
 def _ptr(a):
