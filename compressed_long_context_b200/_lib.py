@@ -19,7 +19,7 @@ HCA_WRITE_LSE = 8
 HCA_OUT_F32 = 16
 
 # Names of every entry point declared in include/hca.h.
-EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_decode",
+EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_decode", "hca_decode_noalloc",
            "hca_status_string", "hca_get_device_error")
 
 _lib = None
@@ -53,5 +53,8 @@ def load():
     lib.hca_decode.restype = _i
     lib.hca_decode.argtypes = ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _sz]
                                + [_i] * 8 + [_f, _u, _vp])
+    lib.hca_decode_noalloc.restype = _i
+    lib.hca_decode_noalloc.argtypes = ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp]
+                                       + [_i] * 8 + [_f, _u, _vp])
     _lib = lib
     return lib

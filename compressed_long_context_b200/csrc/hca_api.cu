@@ -332,3 +332,53 @@ extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v,
     return d == 512 ? launch_prefill<512>(p, tq, tk, tv, tkc, tvc, s) : launch_prefill<64>(p, tq, tk, tv, tkc, tvc, s);
 }
 
+
+// ---------------------------------------------------------------------------------------
+// hca_decode_noalloc: hca_decode with library-owned scratch.
+//
+// The split records live in a fixed array in the library's device image instead of a
+// caller-provided workspace, for callers that cannot allocate device memory when they
+// decode.  Host code must not pass the array's name to a kernel (on the host it is only
+// a stand-in for the symbol); its device address is looked up once per device.
+static __device__ __align__(256) unsigned char hca_decode_scratch[HCA_DECODE_NOALLOC_MAX_BYTES];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+
+// Device address of hca_decode_scratch on the current device; nullptr on failure.
+void* decode_scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> g(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, hca_decode_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_scratch_addr[dev] = ptr;
+    }
+    return g_scratch_addr[dev];
+}
+
+}  // namespace
+
+extern "C" hca_status_t hca_decode_noalloc(const void* q, const void* kc, const void* vc, const int* page_table,
+                                           int page_size, int max_pages, int num_pages, const void* kw,
+                                           const void* vw, const int* seqlens, const float* gq, const float* gk,
+                                           float eps, const void* gate, float* out, int B, int Hq, int Hkv, int d,
+                                           int dv, int blk, int W, int Nmax, float scale, unsigned flags,
+                                           hca_stream_t stream) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || dv < 1) return HCA_ERR_INVALID_ARG;
+    if (B == 0) return HCA_OK;
+    const size_t need = hca_decode_workspace_size(B, Hq, Hkv, dv);
+    if (need == 0) return HCA_ERR_CUDA;
+    if (need > (size_t)HCA_DECODE_NOALLOC_MAX_BYTES) return HCA_ERR_INVALID_ARG;
+    void* ws = decode_scratch_address();
+    if (!ws) return HCA_ERR_CUDA;
+    return hca_decode(q, kc, vc, page_table, page_size, max_pages, num_pages, kw, vw, seqlens, gq, gk, eps, gate,
+                      out, ws, (size_t)HCA_DECODE_NOALLOC_MAX_BYTES, B, Hq, Hkv, d, dv, blk, W, Nmax, scale, flags,
+                      stream);
+}

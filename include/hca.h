@@ -147,6 +147,39 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc,
                         int B, int Hq, int Hkv, int d, int dv, int blk, int W, int Nmax,
                         float scale, unsigned flags, hca_stream_t stream);
 
+/*
+ * hca_decode_noalloc -- hca_decode without a workspace argument.  There is no counterpart
+ * in the paper: this entry point exists for callers that cannot allocate device memory
+ * when they decode -- an inference-engine plugin that must not allocate inside its
+ * enqueue call, a latency-critical server that forbids allocation after warm-up, or host
+ * code that only ever receives pre-allocated buffers -- and so cannot provide the
+ * workspace hca_decode needs.
+ *
+ * Arguments, layouts, supported shapes and results are those of hca_decode.  The split
+ * records live in a fixed array of HCA_DECODE_NOALLOC_MAX_BYTES inside the library's
+ * device image, which every GPU that loads the library holds until the process exits.
+ * The call allocates nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+ *  - Returns HCA_ERR_INVALID_ARG, before any launch, when the batch needs more scratch
+ *    than the array holds, i.e. when hca_decode_workspace_size(B, Hq, Hkv, dv) exceeds
+ *    HCA_DECODE_NOALLOC_MAX_BYTES (on a 148-SM B200 this allows up to about 200
+ *    (sequence, KV head) units).
+ *  - The first call on a device looks up the array's device address on that device
+ *    (once per device, with that device current); make that first call before any stream
+ *    capture.
+ *  - Every call on a device shares the same array, and the array keeps the previous
+ *    call's contents; nothing in it needs to start at zero.  Calls whose work overlaps
+ *    on the GPU (for example on two streams at once) race on it: serialise them.
+ */
+#define HCA_DECODE_NOALLOC_MAX_BYTES (48u << 20)
+
+hca_status_t hca_decode_noalloc(const void* q, const void* kc, const void* vc,
+                                const int* page_table, int page_size, int max_pages, int num_pages,
+                                const void* kw, const void* vw, const int* seqlens,
+                                const float* gq, const float* gk, float eps,
+                                const void* gate, float* out,
+                                int B, int Hq, int Hkv, int d, int dv, int blk, int W, int Nmax,
+                                float scale, unsigned flags, hca_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* hca_status_string(hca_status_t status);
 
