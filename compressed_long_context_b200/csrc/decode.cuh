@@ -15,14 +15,17 @@
 // records of each unit with a log-sum-exp and applies the optional output gate.
 //
 // Per tile, inside a CTA (warp-specialised):
-//   warp 0 (1 thread)  TMA: K tile then V tile as eight 16 KB slabs of 128 keys x 64
-//                      channels (128-byte swizzle) into a ring of shared-memory slots;
-//   warp 1 (1 thread)  tcgen05.mma:  S^T[128 keys x 64 heads] = K . Q^T   (TMEM)
-//                                    O^T[512 ch x 64 heads] += V^T . P^T (TMEM, 4 x 128)
-//                      and, with QK normalisation, diag(K K^T) for the key norms;
+//   warp 0 (1 thread)  TMA: K and V tiles as 16 KB slabs (128 keys x 64 channels,
+//                      128-byte swizzle) into two separate rings, polled without blocking
+//                      so the K stream never waits behind V slabs that are still waiting
+//                      for their probabilities; the query rows of each piece;
+//   warp 1 (1 thread)  tcgen05.mma  S^T[128 keys x 64 heads] = K . Q^T into TMEM (and, with
+//                      QK normalisation, diag(K K^T) for the key norms);
+//   warp 6 (1 thread)  tcgen05.mma  O^T[512 ch x 64 heads] += V^T . P^T (TMEM, 4 x 128);
 //   warps 2-5          softmax: thread = key row; per-head running max with lazy
 //                      rescaling (only when a logit exceeds the max by 2^8), P^T in bf16
 //                      to shared memory; the end-of-piece epilogue writes the record.
+// Two MMA issuers keep QK^T of the next tile from queueing behind PV of this one.
 // Every mbarrier wait is bounded (see common.cuh).
 #pragma once
 
@@ -34,8 +37,9 @@ constexpr int kDecD = 512;                 // head dim (d == dv)
 constexpr int kDecSlabs = kDecD / 64;      // 64-channel slabs per key row
 constexpr int kDecTile = 128;              // keys per tile (MMA M of S^T)
 constexpr int kDecHeads = 64;              // MMA N: query heads of one KV group (padded)
-constexpr int kDecRing = 6;                // ring slots (even, see the V^T descriptor)
-constexpr int kDecThreads = 192;
+constexpr int kDecRingK = 3;               // K slab slots
+constexpr int kDecRingV = 4;               // V slab slots (even: V^T operands are slab pairs)
+constexpr int kDecThreads = 224;           // 7 warps
 constexpr uint32_t kSlabBytes = 128 * 128;                 // 128 rows x 128 B
 constexpr uint32_t kDecQBytes = kDecHeads * kDecD * 2;     // 64 KB
 constexpr uint32_t kDecPBytes = kDecTile * kDecHeads * 2;  // 16 KB
@@ -49,9 +53,10 @@ constexpr uint32_t kTmKK = 384;   // 128     K K^T (QK normalisation only)
 // shared-memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t kSmQ = 0;
 constexpr uint32_t kSmP = kSmQ + kDecQBytes;
-constexpr uint32_t kSmRing = kSmP + 2 * kDecPBytes;
-constexpr uint32_t kSmBar = kSmRing + kDecRing * kSlabBytes;
-constexpr int kNumBars = 2 * kDecRing + 13;
+constexpr uint32_t kSmRingK = kSmP + 2 * kDecPBytes;
+constexpr uint32_t kSmRingV = kSmRingK + kDecRingK * kSlabBytes;
+constexpr uint32_t kSmBar = kSmRingV + kDecRingV * kSlabBytes;
+constexpr int kNumBars = 2 * kDecRingK + 2 * kDecRingV + 13;
 constexpr uint32_t kSmRed = (kSmBar + kNumBars * 8 + 127) & ~127u;   // float[4][64] (read as float4)
 constexpr uint32_t kSmFin = kSmRed + 4 * 64 * 4;            // float[64] reduction result
 constexpr uint32_t kSmMax = kSmFin + 64 * 4;                // float[64] running max per head
@@ -62,8 +67,10 @@ constexpr uint32_t kDecSmemBytes = kSmMisc + 64 + 1024;     // + alignment slack
 static_assert(kDecSmemBytes <= 232448, "decode shared memory exceeds the 227 KB per-block limit");
 static_assert(kSmRed % 16 == 0 && kSmFin % 16 == 0 && kSmMax % 16 == 0 && kSmAlpha % 16 == 0 &&
               kSmSum % 16 == 0 && kSmMisc % 16 == 0, "vector-accessed shared arrays must be 16-byte aligned");
-static_assert(kSmP % 1024 == 0 && kSmRing % 1024 == 0, "swizzled operand tiles must be 1024-byte aligned");
-static_assert(kDecRing % 2 == 0, "V^T operand pairs need an even ring");
+static_assert(kSmP % 1024 == 0 && kSmRingK % 1024 == 0 && kSmRingV % 1024 == 0,
+              "swizzled operand tiles must be 1024-byte aligned");
+static_assert(kDecRingV % 2 == 0, "V^T operand pairs need an even V ring");
+constexpr int kMaxRecords = 512;           // records one unit may have (<= SMs)
 
 struct DecodeParams {
     const __nv_bfloat16* q;      // [B, Hq, 512]
@@ -111,7 +118,7 @@ __device__ __forceinline__ UnitTiles unit_tiles(const DecodeParams& p, int u, bo
     return t;
 }
 
-// Block-wide (all 192 threads) inclusive scan of one int per thread.
+// Block-wide (all threads) inclusive scan of one int per thread.
 __device__ __forceinline__ int block_scan_incl(int v, int* warp_tot, int* total_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -197,17 +204,72 @@ __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) {
     return r * 128u + (((c ^ r) & 7u) << 4);
 }
 
+// This CTA's tiles, in order: (unit u, tile index) pairs of the range [ts, te).
+struct TileIter {
+    const DecodeParams* p;
+    long long te, pu;
+    UnitTiles t;
+    int u, ntiles, tb, tend, tile, item;
+    bool done;
+
+    __device__ void load_unit(long long from) {
+        t = unit_tiles(*p, u, false);
+        ntiles = t.nct + t.nwt;
+        tb = (int)((from > pu ? from : pu) - pu);
+        tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
+        tile = tb;
+    }
+    __device__ void init(const DecodeParams* pp, int u0, long long p0, long long ts, long long te_) {
+        p = pp;
+        te = te_;
+        u = u0;
+        pu = p0;
+        item = 0;
+        done = u0 < 0 || ts >= te_;
+        if (!done) load_unit(ts);
+    }
+    __device__ bool first() const { return tile == tb; }
+    __device__ bool last() const { return tile == tend - 1; }
+    __device__ bool comp() const { return tile < t.nct; }
+    // keys of the current tile that belong to the sequence
+    __device__ int nvalid() const {
+        return comp() ? min(kDecTile, t.nc - tile * kDecTile)
+                      : min(kDecTile, p->W - (t.s0 + (tile - t.nct) * kDecTile));
+    }
+    __device__ void next() {
+        if (++tile < tend) return;
+        ++item;
+        pu += ntiles;
+        ++u;
+        if (pu >= te) {
+            done = true;
+            return;
+        }
+        load_unit(pu);
+    }
+};
+
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_q,
-                    const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kw,
-                    const __grid_constant__ CUtensorMap tm_vw) {
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw) {
     extern __shared__ uint8_t dsmem[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSmBar);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + kDecRing;
-    uint64_t* q_full = bars + 2 * kDecRing;
+    uint64_t* kfull = bars;
+    uint64_t* kempty = kfull + kDecRingK;
+    uint64_t* vfull = kempty + kDecRingK;
+    uint64_t* vempty = vfull + kDecRingV;
+    uint64_t* q_full = vempty + kDecRingV;
     uint64_t* q_empty = q_full + 1;
     uint64_t* s_full = q_full + 2;    // [2]
     uint64_t* s_empty = q_full + 4;   // [2]
@@ -215,7 +277,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     uint64_t* p_empty = q_full + 8;   // [2]
     uint64_t* o_full = q_full + 10;
     uint64_t* o_empty = q_full + 11;
-    uint64_t* q_tma = q_full + 12;    // Q slabs landed (TMA)
+    uint64_t* q_tma = q_full + 12;    // query slabs landed (TMA)
     float* red = reinterpret_cast<float*>(sm + kSmRed);
     float* fin = reinterpret_cast<float*>(sm + kSmFin);
     float* m_s = reinterpret_cast<float*>(sm + kSmMax);
@@ -224,7 +286,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     int* misc = reinterpret_cast<int*>(sm + kSmMisc);
     volatile int* abort_flag = misc + 0;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
-    int* sched = misc + 2;          // [0] = first unit, [1] = its first tile index (global), [2..7] scan scratch
+    int* sched = misc + 2;          // [0] = first unit, [2..8] scan scratch
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool norm = (p.flags & HCA_QK_NORM) != 0;
@@ -234,9 +296,13 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < kDecRing; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
+        for (int i = 0; i < kDecRingK; ++i) {
+            mbar_init(&kfull[i], 1);
+            mbar_init(&kempty[i], 1);
+        }
+        for (int i = 0; i < kDecRingV; ++i) {
+            mbar_init(&vfull[i], 1);
+            mbar_init(&vempty[i], 1);
         }
         mbar_init(q_full, 4);
         mbar_init(q_empty, 1);
@@ -252,7 +318,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, 512);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 32) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -279,7 +345,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const long long ts = total * cta / p.nsplit;
     const long long te = total * (cta + 1) / p.nsplit;
     if (cta == 0 && threadIdx.x == 0) *p.total = total;
-    if (threadIdx.x == 0) { sched[0] = -1; sched[1] = 0; }
+    if (threadIdx.x == 0) sched[0] = -1;
     __syncthreads();
     {
         long long base = 0;
@@ -310,393 +376,385 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const bool have_work = (ts < te) && u_first >= 0;
 
     if (have_work && warp == 0) {
-        // ===================================================== TMA producer
+        // ===================================================== TMA producer (one thread)
         if (lane == 0) {
-            uint32_t ring = 0;
-            // Slab order: K(n0) ; K(n1) V(n0) ; K(n2) V(n1) ; ... ; V(last) -- the MMA
-            // issuer consumes in the same order.
-            struct Pend { int u, tile; };
-            Pend prev = {-1, 0};
-            int u = u_first;
-            long long pu = p_first;
-            bool ok = true;
-            auto load_tile = [&](int uu, int tile, bool is_v) -> bool {
-                UnitTiles t = unit_tiles(p, uu, false);
-                const CUtensorMap* m;
-                const bool comp = tile < t.nct;
-                if (comp) m = is_v ? &tm_v : &tm_k;
-                else m = is_v ? &tm_vw : &tm_kw;
-                for (int s = 0; s < kDecSlabs; ++s) {
-                    const uint32_t st = ring % kDecRing;
-                    if (!mbar_wait(&empty[st], ((ring / kDecRing) & 1) ^ 1, abort_flag)) return false;
-                    uint8_t* dst = sm + kSmRing + st * kSlabBytes;
-                    if (comp && paged) {
-                        uint32_t bytes = 0;
-                        const int j0 = tile * kDecTile;
-                        const bool h1 = j0 + 64 < t.nc;
-                        bytes = h1 ? 2 * 8192 : 8192;
-                        mbar_arrive_expect_tx(&full[st], bytes);
-                        for (int h = 0; h < (h1 ? 2 : 1); ++h) {
-                            const int j = j0 + 64 * h;
-                            const int pg = __ldg(p.page_table + (size_t)t.b * p.max_pages + j / p.page_size);
-                            if (pg < 0 || pg >= p.num_pages) record_error(HCA_ERR_DEVICE_INPUT);
-                            tma_load_4d(dst + h * 8192, m, &full[st], 64 * s, t.g, j % p.page_size, pg);
-                        }
-                    } else {
-                        mbar_arrive_expect_tx(&full[st], kSlabBytes);
-                        const int row = comp ? tile * kDecTile : t.s0 + (tile - t.nct) * kDecTile;
-                        tma_load_4d(dst, m, &full[st], 64 * s, t.g, row, t.b);
+            TileIter ki, vi;
+            ki.init(&p, u_first, p_first, ts, te);
+            vi.init(&p, u_first, p_first, ts, te);
+            int ks = 0, vs = 0, kdone = 0, vdone = 0, qitem = 0;
+            uint32_t kring = 0, vring = 0;
+            bool q_issued = false;
+            uint64_t t_prog = globaltimer_ns();
+            uint32_t idle = 0;
+            // One slab of the current tile of iterator `it` (K or V) into slot `dst`.
+            auto issue = [&](const TileIter& it, int s, bool is_v, uint8_t* dst, uint64_t* bar) {
+                const CUtensorMap* m = it.comp() ? (is_v ? &tm_v : &tm_k) : (is_v ? &tm_vw : &tm_kw);
+                if (it.comp() && paged) {
+                    const int j0 = it.tile * kDecTile;
+                    const bool h1 = j0 + 64 < it.t.nc;
+                    mbar_arrive_expect_tx(bar, h1 ? 2 * 8192 : 8192);
+                    for (int h = 0; h < (h1 ? 2 : 1); ++h) {
+                        const int j = j0 + 64 * h;
+                        const int pg = __ldg(p.page_table + (size_t)it.t.b * p.max_pages + j / p.page_size);
+                        if (pg < 0 || pg >= p.num_pages) record_error(HCA_ERR_DEVICE_INPUT);
+                        tma_load_4d(dst + h * 8192, m, bar, 64 * s, it.t.g, j % p.page_size, pg);
                     }
-                    ++ring;
+                } else {
+                    mbar_arrive_expect_tx(bar, kSlabBytes);
+                    const int row = it.comp() ? it.tile * kDecTile : it.t.s0 + (it.tile - it.t.nct) * kDecTile;
+                    tma_load_4d(dst, m, bar, 64 * s, it.t.g, row, it.t.b);
                 }
-                return true;
             };
-            int item = 0;
-            while (ok && pu < te) {
-                UnitTiles t = unit_tiles(p, u, false);
-                const int ntiles = t.nct + t.nwt;
-                const int tb = (int)((ts > pu ? ts : pu) - pu);
-                const int tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
-                for (int tile = tb; ok && tile < tend; ++tile) {
-                    if (tile == tb && prev.u >= 0) {
-                        ok = load_tile(prev.u, prev.tile, true);
-                        prev.u = -1;
-                    }
-                    if (ok && tile == tb) {
-                        // this piece's 64 query rows (heads g*G ..), eight 8 KB slabs
-                        ok = mbar_wait(q_empty, (item & 1) ^ 1, abort_flag);
-                        if (ok) {
+            while (!ki.done || !vi.done) {
+                bool prog = false;
+                if (!ki.done) {
+                    if (ks == 0 && ki.first() && !q_issued) {
+                        // the piece's 64 query rows (heads g*G ..), eight 8 KB slabs
+                        if (mbar_test(q_empty, (qitem & 1) ^ 1)) {
                             mbar_arrive_expect_tx(q_tma, kDecQBytes);
                             for (int s = 0; s < kDecSlabs; ++s)
-                                tma_load_4d(sm + kSmQ + s * 8192, &tm_q, q_tma, 64 * s, t.g * p.G, t.b, 0);
+                                tma_load_4d(sm + kSmQ + s * 8192, &tm_q, q_tma, 64 * s, ki.t.g * p.G, ki.t.b, 0);
+                            q_issued = true;
+                            ++qitem;
+                            prog = true;
                         }
-                        ++item;
+                    } else {
+                        const uint32_t st = kring % kDecRingK;
+                        if (mbar_test(&kempty[st], ((kring / kDecRingK) & 1) ^ 1)) {
+                            issue(ki, ks, false, sm + kSmRingK + st * kSlabBytes, &kfull[st]);
+                            ++kring;
+                            prog = true;
+                            if (++ks == kDecSlabs) {
+                                ks = 0;
+                                ki.next();
+                                ++kdone;
+                                q_issued = false;
+                            }
+                        }
                     }
-                    if (ok) ok = load_tile(u, tile, false);
-                    if (ok && prev.u >= 0) ok = load_tile(prev.u, prev.tile, true);
-                    prev = {u, tile};
                 }
-                pu += ntiles;
-                ++u;
+                // V of a tile only once its K has started
+                if (!vi.done && (vdone < kdone || ks > 0)) {
+                    const uint32_t st = vring % kDecRingV;
+                    if (mbar_test(&vempty[st], ((vring / kDecRingV) & 1) ^ 1)) {
+                        issue(vi, vs, true, sm + kSmRingV + st * kSlabBytes, &vfull[st]);
+                        ++vring;
+                        prog = true;
+                        if (++vs == kDecSlabs) {
+                            vs = 0;
+                            vi.next();
+                            ++vdone;
+                        }
+                    }
+                }
+                if (prog) {
+                    idle = 0;
+                } else if ((++idle & 255u) != 0) {
+                    __nanosleep(32);
+                } else {
+                    if (*abort_flag) break;
+                    const uint64_t now = globaltimer_ns();
+                    if (idle == 256) t_prog = now;
+                    else if (now - t_prog > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        record_error(HCA_ERR_TIMEOUT);
+                        break;
+                    }
+                }
             }
-            if (ok && prev.u >= 0) load_tile(prev.u, prev.tile, true);
         }
     } else if (have_work && warp == 1) {
-        // ===================================================== MMA issuer (whole warp waits, lane 0 issues)
+        // ===================================================== QK^T issuer (warp waits, lane 0 issues)
         const uint32_t id_s = idesc_bf16(128, kDecHeads, 0, 0);
         const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_o = idesc_bf16(128, kDecHeads, 1, 1);
         const uint32_t q_base = smem_u32(sm + kSmQ);
-        uint32_t ring = 0;
-        int n = 0;          // tiles issued (S side)
-        int item = 0;
-        bool ok = true;
-        // pending PV tile
-        int pv_n = -1, pv_item = 0, pv_nvalid = 128;
-        bool pv_first = false, pv_last = false, pv_partial = false;
-
-        auto issue_pv = [&]() -> bool {
-            const int b = pv_n & 1;
-            if (!warp_wait(&p_full[b], (pv_n >> 1) & 1, abort_flag)) return false;
-            if (pv_first && !warp_wait(o_empty, (pv_item & 1) ^ 1, abort_flag)) return false;
+        TileIter it;
+        it.init(&p, u_first, p_first, ts, te);
+        uint32_t kring = 0;
+        int n = 0;
+        while (!it.done) {
+            const int sb = n & 1;
+            if (it.first() && !warp_wait(q_full, it.item & 1, abort_flag)) break;
+            if (!warp_wait(&s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) break;
+            // the K K^T accumulator has one buffer: wait until tile n-1's softmax has read it
+            if (norm && n > 0 && !warp_wait(&s_empty[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) break;
             tc_fence_after();
+            bool ok = true;
+            for (int s = 0; s < kDecSlabs; ++s) {
+                const uint32_t st = kring % kDecRingK;
+                if (!warp_wait(&kfull[st], (kring / kDecRingK) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t k_base = smem_u32(sm + kSmRingK + st * kSlabBytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(k_base + kk * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(q_base + s * 8192 + kk * 32, 16, 1024);
+                        mma_ss(tmem + kTmS + 64 * sb, ad, bd, id_s, (s | kk) ? 1u : 0u);
+                        if (norm) mma_ss(tmem + kTmKK, ad, ad, id_kk, (s | kk) ? 1u : 0u);
+                    }
+                    mma_commit(&kempty[st]);
+                }
+                __syncwarp();
+                ++kring;
+            }
+            if (!ok) break;
+            if (lane == 0) {
+                mma_commit(&s_full[sb]);
+                if (it.last()) mma_commit(q_empty);
+            }
+            __syncwarp();
+            ++n;
+            it.next();
+        }
+    } else if (have_work && warp == 6) {
+        // ===================================================== PV issuer (warp waits, lane 0 issues)
+        const uint32_t id_o = idesc_bf16(128, kDecHeads, 1, 1);
+        TileIter it;
+        it.init(&p, u_first, p_first, ts, te);
+        uint32_t vring = 0;
+        int n = 0;
+        while (!it.done) {
+            const int b = n & 1;
+            if (!warp_wait(&p_full[b], (n >> 1) & 1, abort_flag)) break;
+            if (it.first() && !warp_wait(o_empty, (it.item & 1) ^ 1, abort_flag)) break;
+            tc_fence_after();
+            const int nvalid = it.nvalid();
+            const bool partial = it.comp() && nvalid < kDecTile;
             const uint32_t p_base = smem_u32(sm + kSmP + b * kDecPBytes);
+            bool ok = true;
             for (int c = 0; c < 4; ++c) {
-                const uint32_t st0 = ring % kDecRing, st1 = (ring + 1) % kDecRing;
-                if (!warp_wait(&full[st0], (ring / kDecRing) & 1, abort_flag)) return false;
-                if (!warp_wait(&full[st1], ((ring + 1) / kDecRing) & 1, abort_flag)) return false;
-                if (pv_partial) {
+                const uint32_t st0 = vring % kDecRingV, st1 = (vring + 1) % kDecRingV;
+                if (!warp_wait(&vfull[st0], (vring / kDecRingV) & 1, abort_flag) ||
+                    !warp_wait(&vfull[st1], ((vring + 1) / kDecRingV) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (partial) {
                     // rows >= nvalid may hold anything (caller memory past the visible
                     // entries): zero them so 0-probability keys contribute exactly 0
-                    const int nz = (kDecTile - pv_nvalid) * 8;
+                    const int nz = (kDecTile - nvalid) * 8;
                     for (int i = lane; i < 2 * nz; i += 32) {
                         const int sl = i / nz, k = i - sl * nz;
-                        const int r = pv_nvalid + (k >> 3);
-                        uint8_t* slab = sm + kSmRing + (sl ? st1 : st0) * kSlabBytes;
+                        const int r = nvalid + (k >> 3);
+                        uint8_t* slab = sm + kSmRingV + (sl ? st1 : st0) * kSlabBytes;
                         *reinterpret_cast<uint4*>(slab + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
+                tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t v_base = smem_u32(sm + kSmRing + st0 * kSlabBytes);
+                    const uint32_t v_base = smem_u32(sm + kSmRingV + st0 * kSlabBytes);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint64_t ad = smem_desc_sw128(v_base + kk * 2048, kSlabBytes, 1024);
                         const uint64_t bd = smem_desc_sw128(p_base + kk * 2048, 8192, 1024);
-                        mma_ss(tmem + kTmO + 64 * c, ad, bd, id_o, (pv_first && kk == 0) ? 0u : 1u);
+                        mma_ss(tmem + kTmO + 64 * c, ad, bd, id_o, (it.first() && kk == 0) ? 0u : 1u);
                     }
-                    mma_commit(&empty[st0]);
-                    mma_commit(&empty[st1]);
+                    mma_commit(&vempty[st0]);
+                    mma_commit(&vempty[st1]);
                 }
                 __syncwarp();
-                ring += 2;
+                vring += 2;
             }
+            if (!ok) break;
             if (lane == 0) {
                 mma_commit(&p_empty[b]);
-                if (pv_last) mma_commit(o_full);
+                if (it.last()) mma_commit(o_full);
             }
             __syncwarp();
-            return true;
-        };
-
-        int u = u_first;
-        long long pu = p_first;
-        while (ok && pu < te) {
-            UnitTiles t = unit_tiles(p, u, false);
-            const int ntiles = t.nct + t.nwt;
-            const int tb = (int)((ts > pu ? ts : pu) - pu);
-            const int tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
-            for (int tile = tb; ok && tile < tend; ++tile, ++n) {
-                const bool first = tile == tb, last = tile == tend - 1;
-                const int sb = n & 1;
-                if (first && pv_n >= 0) {
-                    // close the previous piece first: its epilogue waits for this PV
-                    if (!issue_pv()) { ok = false; break; }
-                    pv_n = -1;
-                }
-                if (first && !warp_wait(q_full, item & 1, abort_flag)) { ok = false; break; }
-                if (!warp_wait(&s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                // the K K^T accumulator has one buffer: wait until tile n-1's softmax has read it
-                if (norm && n > 0 && !warp_wait(&s_empty[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                for (int s = 0; s < kDecSlabs; ++s) {
-                    const uint32_t st = ring % kDecRing;
-                    if (!warp_wait(&full[st], (ring / kDecRing) & 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t k_base = smem_u32(sm + kSmRing + st * kSlabBytes);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t ad = smem_desc_sw128(k_base + kk * 32, 16, 1024);
-                            const uint64_t bd = smem_desc_sw128(q_base + s * 8192 + kk * 32, 16, 1024);
-                            mma_ss(tmem + kTmS + 64 * sb, ad, bd, id_s, (s | kk) ? 1u : 0u);
-                            if (norm) mma_ss(tmem + kTmKK, ad, ad, id_kk, (s | kk) ? 1u : 0u);
-                        }
-                        mma_commit(&empty[st]);
-                    }
-                    __syncwarp();
-                    ++ring;
-                }
-                if (!ok) break;
-                if (lane == 0) {
-                    mma_commit(&s_full[sb]);
-                    if (last) mma_commit(q_empty);
-                }
-                __syncwarp();
-                // PV of the previous tile (its V slabs follow this tile's K slabs in the ring)
-                if (pv_n >= 0 && !issue_pv()) { ok = false; break; }
-                pv_n = n;
-                pv_item = item;
-                pv_first = first;
-                pv_last = last;
-                pv_partial = tile < t.nct && (t.nc - tile * kDecTile) < kDecTile;
-                pv_nvalid = tile < t.nct ? min(kDecTile, t.nc - tile * kDecTile) : kDecTile;
-                if (last) ++item;
-            }
-            pu += ntiles;
-            ++u;
+            ++n;
+            it.next();
         }
-        if (ok && pv_n >= 0) issue_pv();
-    } else if (have_work) {
+    } else if (have_work && warp >= 2 && warp <= 5) {
         // ===================================================== softmax / epilogue (warps 2-5)
         const int q4 = warp & 3;                 // TMEM lane quarter
         const int r = q4 * 32 + lane;            // key row within the tile / channel within a chunk
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const int sidx = threadIdx.x - 64;       // 0..127
-        int n = 0, item = 0;
+        TileIter it;
+        it.init(&p, u_first, p_first, ts, te);
+        int n = 0;
         bool ok = true;
-        int u = u_first;
-        long long pu = p_first;
-        while (ok && pu < te) {
-            UnitTiles t = unit_tiles(p, u, false);
-            const int ntiles = t.nct + t.nwt;
-            const int tb = (int)((ts > pu ? ts : pu) - pu);
-            const int tend = (int)((te < pu + ntiles ? te : pu + ntiles) - pu);
-
-            // ---- this piece's queries arrive by TMA; with QK normalisation they are
-            // rewritten in place as q' = q / rms(q) * g_q * g_k (bf16), since
-            // q_hat . k_hat = (q' . k) / rms(k)
-            if (!group_wait(q_tma, item & 1, abort_flag)) { ok = false; break; }
-            if (norm) {
-                const int h = sidx >> 1, half = sidx & 1;
-                float ss = 0.f;
-                for (int c = 0; c < 256; c += 8) {
-                    const int cc = 256 * half + c;
-                    const uint4 x = *reinterpret_cast<const uint4*>(sm + kSmQ + (cc >> 6) * 8192 +
-                                                                  sw128(h, (cc & 63) >> 3));
-                    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float a = bf16lo(w4[i]), b2 = bf16hi(w4[i]);
-                        ss = fmaf(a, a, fmaf(b2, b2, ss));
-                    }
-                }
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                const float inv = rsqrtf(ss * (1.f / kDecD) + p.eps);
-                for (int c = 0; c < 256; c += 8) {
-                    const int cc = 256 * half + c;
-                    uint4* ptr = reinterpret_cast<uint4*>(sm + kSmQ + (cc >> 6) * 8192 + sw128(h, (cc & 63) >> 3));
-                    const uint4 x = *ptr;
-                    uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int ch = cc + 2 * i;
-                        const float a = bf16lo(w4[i]) * inv * __ldg(p.gq + ch) * __ldg(p.gk + ch);
-                        const float b2 = bf16hi(w4[i]) * inv * __ldg(p.gq + ch + 1) * __ldg(p.gk + ch + 1);
-                        w4[i] = pack_bf16x2(a, b2);
-                    }
-                    *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                }
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(q_full);
-
-            for (int tile = tb; ok && tile < tend; ++tile, ++n) {
-                const bool first = tile == tb, last = tile == tend - 1;
-                const int sb = n & 1;
-                const bool comp = tile < t.nct;
-                const int nvalid = comp ? min(kDecTile, t.nc - tile * kDecTile)
-                                        : min(kDecTile, p.W - (t.s0 + (tile - t.nct) * kDecTile));
-                const bool valid = r < nvalid;
-
-                if (!group_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                float z[64];
-#pragma unroll
-                for (int c = 0; c < 64; c += 16) tmem_ld16(tmem + lane_off + kTmS + 64 * sb + c, z + c);
-                float kscale = p.scale_log2;
+        while (ok && !it.done) {
+            const bool first = it.first(), last = it.last();
+            if (first) {
+                // ---- the piece's queries arrive by TMA; with QK normalisation they are
+                // rewritten in place as q' = q / rms(q) * g_q * g_k (bf16), since
+                // q_hat . k_hat = (q' . k) / rms(k)
+                if (!group_wait(q_tma, it.item & 1, abort_flag)) { ok = false; break; }
                 if (norm) {
-                    float d[32];
-                    tmem_ld16(tmem + lane_off + kTmKK + q4 * 32, d);
-                    tmem_ld16(tmem + lane_off + kTmKK + q4 * 32 + 16, d + 16);
-                    tmem_wait_ld();
-                    float diag = 0.f;
+                    const int h = sidx >> 1, half = sidx & 1;
+                    float ss = 0.f;
+                    for (int c = 0; c < 256; c += 8) {
+                        const int cc = 256 * half + c;
+                        const uint4 x = *reinterpret_cast<const uint4*>(sm + kSmQ + (cc >> 6) * 8192 +
+                                                                      sw128(h, (cc & 63) >> 3));
+                        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) diag = (j == lane) ? d[j] : diag;
-                    kscale *= rsqrtf(diag * (1.f / kDecD) + p.eps);
-                } else {
-                    tmem_wait_ld();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[sb]);
-#pragma unroll
-                for (int h = 0; h < 64; ++h) z[h] = valid ? z[h] * kscale : -INFINITY;
-
-                // ---- running max (shared m_s[64]): full reduction on the first tile of a
-                // piece; afterwards only when some logit exceeds the max by 2^threshold
-                bool need;
-                if (first) {
-                    need = true;
-                } else {
-                    bool mine = false;
-#pragma unroll
-                    for (int h = 0; h < 64; h += 4) {
-                        const float4 mm = *reinterpret_cast<const float4*>(m_s + h);
-                        mine |= (z[h] > mm.x + kRescaleThreshold) | (z[h + 1] > mm.y + kRescaleThreshold) |
-                                (z[h + 2] > mm.z + kRescaleThreshold) | (z[h + 3] > mm.w + kRescaleThreshold);
-                    }
-                    need = softmax_any(mine);
-                }
-                if (need) {
-                    colreduce64<true>(z, red, fin, q4, lane);
-                    if (sidx < 64) {
-                        const float mo = first ? -INFINITY : m_s[sidx];
-                        const float mn = fmaxf(mo, fin[sidx]);
-                        const float al = first ? 0.f : ex2(mo - mn);
-                        al_s[sidx] = al;
-                        m_s[sidx] = mn;
-                        l_s[sidx] = first ? 0.f : l_s[sidx] * al;
-                    }
-                    softmax_bar();
-                    if (!first) {
-                        // rescale O^T once the previous PV has landed
-                        const int pb = (n - 1) & 1;
-                        if (!group_wait(&p_empty[pb], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                            for (int c16 = 0; c16 < 64; c16 += 16) {
-                                float o[16];
-                                const uint32_t ta = tmem + lane_off + kTmO + 64 * c + c16;
-                                tmem_ld16(ta, o);
-                                tmem_wait_ld();
-                                uint32_t w[16];
-#pragma unroll
-                                for (int j = 0; j < 16; ++j) w[j] = __float_as_uint(o[j] * al_s[c16 + j]);
-                                tmem_st16(ta, w);
-                            }
+                        for (int i = 0; i < 4; ++i) {
+                            const float a = bf16lo(w4[i]), b2 = bf16hi(w4[i]);
+                            ss = fmaf(a, a, fmaf(b2, b2, ss));
                         }
-                        tmem_wait_st();
-                        tc_fence_before();
                     }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    const float inv = rsqrtf(ss * (1.f / kDecD) + p.eps);
+                    for (int c = 0; c < 256; c += 8) {
+                        const int cc = 256 * half + c;
+                        uint4* ptr =
+                            reinterpret_cast<uint4*>(sm + kSmQ + (cc >> 6) * 8192 + sw128(h, (cc & 63) >> 3));
+                        const uint4 x = *ptr;
+                        uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int ch = cc + 2 * i;
+                            const float a = bf16lo(w4[i]) * inv * __ldg(p.gq + ch) * __ldg(p.gk + ch);
+                            const float b2 = bf16hi(w4[i]) * inv * __ldg(p.gq + ch + 1) * __ldg(p.gk + ch + 1);
+                            w4[i] = pack_bf16x2(a, b2);
+                        }
+                        *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                    fence_proxy_async_smem();
                 }
-                // ---- probabilities
-                uint32_t pk[32];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_full);
+            }
+
+            const int sb = n & 1;
+            const bool valid = r < it.nvalid();
+            if (!group_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            float z[64];
+#pragma unroll
+            for (int c = 0; c < 64; c += 16) tmem_ld16(tmem + lane_off + kTmS + 64 * sb + c, z + c);
+            float kscale = p.scale_log2;
+            if (norm) {
+                float d[32];
+                tmem_ld16(tmem + lane_off + kTmKK + q4 * 32, d);
+                tmem_ld16(tmem + lane_off + kTmKK + q4 * 32 + 16, d + 16);
+                tmem_wait_ld();
+                float diag = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) diag = (j == lane) ? d[j] : diag;
+                kscale *= rsqrtf(diag * (1.f / kDecD) + p.eps);
+            } else {
+                tmem_wait_ld();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+#pragma unroll
+            for (int h = 0; h < 64; ++h) z[h] = valid ? z[h] * kscale : -INFINITY;
+
+            // ---- running max (shared m_s[64]): full reduction on the first tile of a
+            // piece; afterwards only when some logit exceeds the max by 2^threshold
+            bool need;
+            if (first) {
+                need = true;
+            } else {
+                bool mine = false;
 #pragma unroll
                 for (int h = 0; h < 64; h += 4) {
                     const float4 mm = *reinterpret_cast<const float4*>(m_s + h);
-                    z[h] = ex2(z[h] - mm.x);
-                    z[h + 1] = ex2(z[h + 1] - mm.y);
-                    z[h + 2] = ex2(z[h + 2] - mm.z);
-                    z[h + 3] = ex2(z[h + 3] - mm.w);
-                    pk[h >> 1] = pack_bf16x2(z[h], z[h + 1]);
-                    pk[(h >> 1) + 1] = pack_bf16x2(z[h + 2], z[h + 3]);
+                    mine |= (z[h] > mm.x + kRescaleThreshold) | (z[h + 1] > mm.y + kRescaleThreshold) |
+                            (z[h + 2] > mm.z + kRescaleThreshold) | (z[h + 3] > mm.w + kRescaleThreshold);
                 }
-                const int pbuf = n & 1;
-                if (!group_wait(&p_empty[pbuf], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                uint8_t* pt = sm + kSmP + pbuf * kDecPBytes;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(pt + sw128(r, c)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[pbuf]);
-                // row sums of this tile (off the MMA's critical path)
-                colreduce64<false>(z, red, fin, q4, lane);
-                if (sidx < 64) l_s[sidx] += fin[sidx];
-
-                if (last) {
-                    // ---- end of this CTA's piece of unit u: write the partial record
-                    const int rec = cta + u;
-                    if (sidx < 64) {
-                        p.rec_m[(size_t)rec * 64 + sidx] = m_s[sidx];
-                        p.rec_l[(size_t)rec * 64 + sidx] = l_s[sidx];
-                    }
-                    if (sidx == 0) {
-                        if (tb == 0) p.meta[2 * u] = cta;
-                        if (tend == ntiles) p.meta[2 * u + 1] = cta;
-                    }
-                    if (!group_wait(o_full, item & 1, abort_flag)) { ok = false; break; }
+                need = softmax_any(mine);
+            }
+            if (need) {
+                colreduce64<true>(z, red, fin, q4, lane);
+                if (sidx < 64) {
+                    const float mo = first ? -INFINITY : m_s[sidx];
+                    const float mn = fmaxf(mo, fin[sidx]);
+                    const float al = first ? 0.f : ex2(mo - mn);
+                    al_s[sidx] = al;
+                    m_s[sidx] = mn;
+                    l_s[sidx] = first ? 0.f : l_s[sidx] * al;
+                }
+                softmax_bar();
+                if (!first) {
+                    // rescale O^T once the previous PV has landed
+                    const int pb = (n - 1) & 1;
+                    if (!group_wait(&p_empty[pb], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    float* orec = p.rec_o + (size_t)rec * 64 * kDecD;
                     for (int c = 0; c < 4; ++c) {
 #pragma unroll
                         for (int c16 = 0; c16 < 64; c16 += 16) {
                             float o[16];
-                            tmem_ld16(tmem + lane_off + kTmO + 64 * c + c16, o);
+                            const uint32_t ta = tmem + lane_off + kTmO + 64 * c + c16;
+                            tmem_ld16(ta, o);
                             tmem_wait_ld();
+                            uint32_t w[16];
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int h = c16 + j;
-                                if (h < p.G) orec[(size_t)h * kDecD + 128 * c + r] = o[j];
-                            }
+                            for (int j = 0; j < 16; ++j) w[j] = __float_as_uint(o[j] * al_s[c16 + j]);
+                            tmem_st16(ta, w);
                         }
                     }
+                    tmem_wait_st();
                     tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(o_empty);
-                    ++item;
                 }
             }
-            pu += ntiles;
-            ++u;
+            // ---- probabilities
+            uint32_t pk[32];
+#pragma unroll
+            for (int h = 0; h < 64; h += 4) {
+                const float4 mm = *reinterpret_cast<const float4*>(m_s + h);
+                z[h] = ex2(z[h] - mm.x);
+                z[h + 1] = ex2(z[h + 1] - mm.y);
+                z[h + 2] = ex2(z[h + 2] - mm.z);
+                z[h + 3] = ex2(z[h + 3] - mm.w);
+                pk[h >> 1] = pack_bf16x2(z[h], z[h + 1]);
+                pk[(h >> 1) + 1] = pack_bf16x2(z[h + 2], z[h + 3]);
+            }
+            const int pbuf = n & 1;
+            if (!group_wait(&p_empty[pbuf], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            uint8_t* pt = sm + kSmP + pbuf * kDecPBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(pt + sw128(r, c)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[pbuf]);
+            // row sums of this tile (off the MMA's critical path)
+            colreduce64<false>(z, red, fin, q4, lane);
+            if (sidx < 64) l_s[sidx] += fin[sidx];
+
+            if (last) {
+                // ---- end of this CTA's piece of unit u: write the partial record
+                const int u = it.u;
+                const int rec = cta + u;
+                if (sidx < 64) {
+                    p.rec_m[(size_t)rec * 64 + sidx] = m_s[sidx];
+                    p.rec_l[(size_t)rec * 64 + sidx] = l_s[sidx];
+                }
+                if (sidx == 0) {
+                    if (it.tb == 0) p.meta[2 * u] = cta;
+                    if (it.tend == it.ntiles) p.meta[2 * u + 1] = cta;
+                }
+                if (!group_wait(o_full, it.item & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                float* orec = p.rec_o + (size_t)rec * 64 * kDecD;
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int c16 = 0; c16 < 64; c16 += 16) {
+                        float o[16];
+                        tmem_ld16(tmem + lane_off + kTmO + 64 * c + c16, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int h = c16 + j;
+                            if (h < p.G) orec[(size_t)h * kDecD + 128 * c + r] = o[j];
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(o_empty);
+            }
+            ++n;
+            it.next();
         }
     }
 
@@ -709,36 +767,71 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 }
 
 // Merge the partial records of each unit (log-sum-exp), normalise, apply the gate.
-// Grid: (units, heads / 8); 256 threads, two channels each.
+// Grid: (units, heads / 8); 256 threads, two channels each.  The merge weights of all
+// (record, head) pairs are computed once into shared memory, so the accumulation loop
+// issues independent loads.
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float wgt[kMaxRecords][8];
+    __shared__ int recs[kMaxRecords];
+    __shared__ float inv_l[8];
+    __shared__ int nrec_s;
     const int u = blockIdx.x;
     const int b = u / p.Hkv, g = u - (u / p.Hkv) * p.Hkv;
+    const int h0 = blockIdx.y * 8;
+    const int tid = threadIdx.x;
     const int first = p.meta[2 * u], last = p.meta[2 * u + 1];
     const long long total = *p.total;
-    const int c = 2 * threadIdx.x;
-    if (first < 0 || last < first || last >= p.nsplit) {
-        record_error(HCA_ERR_DEVICE_INPUT);
+    if (first < 0 || last < first || last >= p.nsplit || last - first >= kMaxRecords) {
+        if (tid == 0) record_error(HCA_ERR_DEVICE_INPUT);
         return;
     }
-    for (int h = blockIdx.y * 8; h < min(p.G, blockIdx.y * 8 + 8); ++h) {
+    if (tid == 0) {
+        int n = 0;
+        for (int i = first; i <= last; ++i)
+            if (total * i / p.nsplit != total * (i + 1) / p.nsplit) recs[n++] = i + u;   // CTA had work
+        nrec_s = n;
+    }
+    __syncthreads();
+    const int nrec = nrec_s;
+    for (int idx = tid; idx < nrec * 8; idx += 256) {
+        const int rr = idx >> 3, h = h0 + (idx & 7);
+        wgt[rr][idx & 7] = h < p.G ? p.rec_m[(size_t)recs[rr] * 64 + h] : 0.f;
+    }
+    __syncthreads();
+    if (tid < 8) {
+        const int h = h0 + tid;
         float M = -INFINITY;
-        for (int i = first; i <= last; ++i) {
-            if (total * i / p.nsplit == total * (i + 1) / p.nsplit) continue;   // empty range
-            M = fmaxf(M, p.rec_m[(size_t)(i + u) * 64 + h]);
+        for (int rr = 0; rr < nrec; ++rr) M = fmaxf(M, wgt[rr][tid]);
+        float L = 0.f;
+        for (int rr = 0; rr < nrec; ++rr) {
+            const float w = exp2f(wgt[rr][tid] - M);
+            wgt[rr][tid] = w;
+            L = fmaf(w, h < p.G ? p.rec_l[(size_t)recs[rr] * 64 + h] : 0.f, L);
         }
-        float L = 0.f, a0 = 0.f, a1 = 0.f;
-        for (int i = first; i <= last; ++i) {
-            if (total * i / p.nsplit == total * (i + 1) / p.nsplit) continue;
-            const size_t rec = (size_t)(i + u);
-            const float w = exp2f(p.rec_m[rec * 64 + h] - M);
-            L = fmaf(w, p.rec_l[rec * 64 + h], L);
-            const float2 o = *reinterpret_cast<const float2*>(p.rec_o + (rec * 64 + h) * kDecD + c);
-            a0 = fmaf(w, o.x, a0);
-            a1 = fmaf(w, o.y, a1);
+        inv_l[tid] = 1.f / L;
+    }
+    __syncthreads();
+    const int c = 2 * tid;
+    float a0[8], a1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a0[j] = a1[j] = 0.f;
+    for (int rr = 0; rr < nrec; ++rr) {
+        const float* base = p.rec_o + ((size_t)recs[rr] * 64 + h0) * kDecD + c;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (h0 + j < p.G) {
+                const float2 o = *reinterpret_cast<const float2*>(base + (size_t)j * kDecD);
+                a0[j] = fmaf(wgt[rr][j], o.x, a0[j]);
+                a1[j] = fmaf(wgt[rr][j], o.y, a1[j]);
+            }
         }
-        const float inv = 1.f / L;
-        float o0 = a0 * inv, o1 = a1 * inv;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int h = h0 + j;
+        if (h >= p.G) continue;
+        float o0 = a0[j] * inv_l[j], o1 = a1[j] * inv_l[j];
         const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h) * kDecD + c;
         if (p.flags & HCA_OUT_GATE) {
             const uint32_t gv = *reinterpret_cast<const uint32_t*>(p.gate + orow);
