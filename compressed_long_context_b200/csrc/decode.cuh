@@ -70,7 +70,6 @@ static_assert(kSmRed % 16 == 0 && kSmFin % 16 == 0 && kSmMax % 16 == 0 && kSmAlp
 static_assert(kSmP % 1024 == 0 && kSmRingK % 1024 == 0 && kSmRingV % 1024 == 0,
               "swizzled operand tiles must be 1024-byte aligned");
 static_assert(kDecRingV % 2 == 0, "V^T operand pairs need an even V ring");
-constexpr int kMaxRecords = 512;           // records one unit may have (<= SMs)
 
 struct DecodeParams {
     const __nv_bfloat16* q;      // [B, Hq, 512]
@@ -342,12 +341,19 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         for (int w = 0; w < kDecThreads / 32; ++w) total += wt[w];
         __syncthreads();
     }
-    const long long ts = total * cta / p.nsplit;
-    const long long te = total * (cta + 1) / p.nsplit;
-    if (cta == 0 && threadIdx.x == 0) *p.total = total;
-    if (threadIdx.x == 0) sched[0] = -1;
+    // equal ranges of ceil(total / nsplit) tiles (the last CTAs may get fewer or none); a
+    // range may hold the tail of one unit and the head of the next
+    const long long tpc = (total + p.nsplit - 1) / p.nsplit;
+    long long* sched64 = reinterpret_cast<long long*>(red + 64);   // [0] ts, [1] te, [2] p_first
+    if (threadIdx.x == 0) {
+        sched[0] = -1;
+        sched64[0] = min(total, tpc * cta);
+        sched64[1] = min(total, tpc * (cta + 1));
+    }
     __syncthreads();
     {
+        // the unit holding tile ts (block-wide scan over units)
+        const long long ts0 = sched64[0];
         long long base = 0;
         for (int c0 = 0; c0 < U; c0 += kDecThreads) {
             const int u = c0 + threadIdx.x;
@@ -359,16 +365,19 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             int tot;
             const int incl = block_scan_incl(n, sched + 2, &tot);
             const long long pu = base + incl - n;
-            if (u < U && pu <= ts && ts < pu + n) {
+            if (u < U && pu <= ts0 && ts0 < pu + n) {
                 sched[0] = u;
-                reinterpret_cast<long long*>(red + 64)[0] = pu;
+                sched64[2] = pu;
             }
             base += tot;
         }
         __syncthreads();
     }
+    const long long ts = sched64[0];
+    const long long te = sched64[1];
+    if (cta == 0 && threadIdx.x == 0) *p.total = total;
     const int u_first = sched[0];
-    const long long p_first = reinterpret_cast<long long*>(red + 64)[0];
+    const long long p_first = sched64[2];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -722,16 +731,16 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             if (sidx < 64) l_s[sidx] += fin[sidx];
 
             if (last) {
-                // ---- end of this CTA's piece of unit u: write the partial record
+                // ---- end of this CTA's piece of unit u
                 const int u = it.u;
                 const int rec = cta + u;
-                if (sidx < 64) {
-                    p.rec_m[(size_t)rec * 64 + sidx] = m_s[sidx];
-                    p.rec_l[(size_t)rec * 64 + sidx] = l_s[sidx];
-                }
                 if (sidx == 0) {
                     if (it.tb == 0) p.meta[2 * u] = cta;
                     if (it.tend == it.ntiles) p.meta[2 * u + 1] = cta;
+                }
+                if (sidx < 64) {
+                    p.rec_m[(size_t)rec * 64 + sidx] = m_s[sidx];
+                    p.rec_l[(size_t)rec * 64 + sidx] = l_s[sidx];
                 }
                 if (!group_wait(o_full, it.item & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -767,78 +776,84 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 }
 
 // Merge the partial records of each unit (log-sum-exp), normalise, apply the gate.
-// Grid: (units, heads / 8); 256 threads, two channels each.  The merge weights of all
-// (record, head) pairs are computed once into shared memory, so the accumulation loop
-// issues independent loads.
-__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeParams p) {
+// Grid (units, heads / 4), 128 threads; a thread owns 4 heads x 4 channels.  All the
+// (m, l, O) values of a chunk of records are loaded before any is used, so a merge costs
+// about two memory round trips, and the grid fits in one wave.
+constexpr int kMergeChunk = 4;
+constexpr int kMergeHeads = 4;
+
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    __shared__ float wgt[kMaxRecords][8];
-    __shared__ int recs[kMaxRecords];
-    __shared__ float inv_l[8];
-    __shared__ int nrec_s;
     const int u = blockIdx.x;
+    const int h0 = blockIdx.y * kMergeHeads;
+    const int c = 4 * threadIdx.x;                // channels c .. c+3
     const int b = u / p.Hkv, g = u - (u / p.Hkv) * p.Hkv;
-    const int h0 = blockIdx.y * 8;
-    const int tid = threadIdx.x;
-    const int first = p.meta[2 * u], last = p.meta[2 * u + 1];
-    const long long total = *p.total;
-    if (first < 0 || last < first || last >= p.nsplit || last - first >= kMaxRecords) {
-        if (tid == 0) record_error(HCA_ERR_DEVICE_INPUT);
+    const int first = __ldg(p.meta + 2 * u), last = __ldg(p.meta + 2 * u + 1);
+    if (first < 0 || last < first || last >= p.nsplit) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) record_error(HCA_ERR_DEVICE_INPUT);
         return;
     }
-    if (tid == 0) {
-        int n = 0;
-        for (int i = first; i <= last; ++i)
-            if (total * i / p.nsplit != total * (i + 1) / p.nsplit) recs[n++] = i + u;   // CTA had work
-        nrec_s = n;
-    }
-    __syncthreads();
-    const int nrec = nrec_s;
-    for (int idx = tid; idx < nrec * 8; idx += 256) {
-        const int rr = idx >> 3, h = h0 + (idx & 7);
-        wgt[rr][idx & 7] = h < p.G ? p.rec_m[(size_t)recs[rr] * 64 + h] : 0.f;
-    }
-    __syncthreads();
-    if (tid < 8) {
-        const int h = h0 + tid;
-        float M = -INFINITY;
-        for (int rr = 0; rr < nrec; ++rr) M = fmaxf(M, wgt[rr][tid]);
-        float L = 0.f;
-        for (int rr = 0; rr < nrec; ++rr) {
-            const float w = exp2f(wgt[rr][tid] - M);
-            wgt[rr][tid] = w;
-            L = fmaf(w, h < p.G ? p.rec_l[(size_t)recs[rr] * 64 + h] : 0.f, L);
-        }
-        inv_l[tid] = 1.f / L;
-    }
-    __syncthreads();
-    const int c = 2 * tid;
-    float a0[8], a1[8];
+    float M[kMergeHeads], L[kMergeHeads];
+    float4 acc[kMergeHeads];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a0[j] = a1[j] = 0.f;
-    for (int rr = 0; rr < nrec; ++rr) {
-        const float* base = p.rec_o + ((size_t)recs[rr] * 64 + h0) * kDecD + c;
+    for (int j = 0; j < kMergeHeads; ++j) {
+        M[j] = -INFINITY;
+        L[j] = 0.f;
+        acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int i0 = first; i0 <= last; i0 += kMergeChunk) {
+        float m[kMergeChunk][kMergeHeads], l[kMergeChunk][kMergeHeads];
+        float4 o[kMergeChunk][kMergeHeads];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (h0 + j < p.G) {
-                const float2 o = *reinterpret_cast<const float2*>(base + (size_t)j * kDecD);
-                a0[j] = fmaf(wgt[rr][j], o.x, a0[j]);
-                a1[j] = fmaf(wgt[rr][j], o.y, a1[j]);
+        for (int k = 0; k < kMergeChunk; ++k) {
+            const bool live = i0 + k <= last;     // ranges are contiguous: every CTA in between has a piece
+            const size_t rec = (size_t)(i0 + k + u);
+#pragma unroll
+            for (int j = 0; j < kMergeHeads; ++j) {
+                const int h = h0 + j;
+                const bool ok = live && h < p.G;
+                m[k][j] = ok ? __ldcg(p.rec_m + rec * 64 + h) : -INFINITY;
+                l[k][j] = ok ? __ldcg(p.rec_l + rec * 64 + h) : 0.f;
+                o[k][j] = ok ? __ldcg(reinterpret_cast<const float4*>(p.rec_o + (rec * 64 + h) * kDecD + c))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
+#pragma unroll
+        for (int j = 0; j < kMergeHeads; ++j) {
+            float Mn = M[j];
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) Mn = fmaxf(Mn, m[k][j]);
+            if (Mn == -INFINITY) continue;
+            const float sc = M[j] == -INFINITY ? 0.f : exp2f(M[j] - Mn);
+            L[j] *= sc;
+            acc[j].x *= sc; acc[j].y *= sc; acc[j].z *= sc; acc[j].w *= sc;
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) {
+                const float w = m[k][j] == -INFINITY ? 0.f : exp2f(m[k][j] - Mn);
+                L[j] = fmaf(w, l[k][j], L[j]);
+                acc[j].x = fmaf(w, o[k][j].x, acc[j].x);
+                acc[j].y = fmaf(w, o[k][j].y, acc[j].y);
+                acc[j].z = fmaf(w, o[k][j].z, acc[j].z);
+                acc[j].w = fmaf(w, o[k][j].w, acc[j].w);
+            }
+            M[j] = Mn;
+        }
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kMergeHeads; ++j) {
         const int h = h0 + j;
         if (h >= p.G) continue;
-        float o0 = a0[j] * inv_l[j], o1 = a1[j] * inv_l[j];
+        const float inv = 1.f / L[j];
+        float4 r = make_float4(acc[j].x * inv, acc[j].y * inv, acc[j].z * inv, acc[j].w * inv);
         const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h) * kDecD + c;
         if (p.flags & HCA_OUT_GATE) {
-            const uint32_t gv = *reinterpret_cast<const uint32_t*>(p.gate + orow);
-            o0 *= 1.f / (1.f + __expf(-bf16lo(gv)));
-            o1 *= 1.f / (1.f + __expf(-bf16hi(gv)));
+            const uint2 gv = __ldg(reinterpret_cast<const uint2*>(p.gate + orow));
+            r.x *= 1.f / (1.f + __expf(-bf16lo(gv.x)));
+            r.y *= 1.f / (1.f + __expf(-bf16hi(gv.x)));
+            r.z *= 1.f / (1.f + __expf(-bf16lo(gv.y)));
+            r.w *= 1.f / (1.f + __expf(-bf16hi(gv.y)));
         }
-        *reinterpret_cast<float2*>(p.out + orow) = make_float2(o0, o1);
+        *reinterpret_cast<float4*>(p.out + orow) = r;
     }
 }
 

@@ -249,8 +249,8 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)U, (unsigned)((p.G + 7) / 8));
-    cfg.blockDim = dim3(256);
+    cfg.gridDim = dim3((unsigned)U, (unsigned)((p.G + kMergeHeads - 1) / kMergeHeads));
+    cfg.blockDim = dim3(kDecD / 4);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

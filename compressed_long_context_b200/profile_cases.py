@@ -20,11 +20,14 @@ from . import compress, decode, decode_workspace_size, get_device_error, prefill
 from . import workloads as wl
 
 
+_last_fn = [None]
+
+
 def _events():
     return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
 
-def run(case: str, reps: int) -> dict:
+def run(case: str, reps: int, B_override: int = 0, L_override: int = 0) -> dict:
     dev = torch.device("cuda", torch.cuda.current_device())
     g = torch.Generator(device=dev).manual_seed(123)
     if case == "compress":
@@ -40,6 +43,8 @@ def run(case: str, reps: int) -> dict:
     elif case in ("decode", "paged"):
         # the 128K decode batch with its cache drawn directly (134 MB of entries)
         B, L, Hq, d, W = 64, 131072, 64, 512, 128
+        B = B_override or B
+        L = L_override or L
         nc = (L - W) // 128
         q = torch.randn((B, Hq, d), generator=g, device=dev).to(torch.bfloat16)
         kw = torch.randn((B, W, 1, d), generator=g, device=dev).to(torch.bfloat16)
@@ -78,6 +83,7 @@ def run(case: str, reps: int) -> dict:
         flops = 2.0 * cfg.Hq * keys * (cfg.d + cfg.dv)
     else:
         raise ValueError(case)
+    _last_fn[0] = fn
     fn()
     torch.cuda.synchronize()
     get_device_error()
@@ -90,10 +96,37 @@ def run(case: str, reps: int) -> dict:
     get_device_error()
     ms = a.elapsed_time(b) / reps
     res = {"case": case, "reps": reps, "ms_per_launch": ms}
+    if case in ("decode", "paged"):
+        res["B"], res["L"] = B, L
     if nbytes:
+        res["bytes"] = nbytes
         res["GB_per_s"] = nbytes / (ms / 1e3) / 1e9
     if case == "prefill":
         res["TFLOP_per_s"] = flops / (ms / 1e3) / 1e12
+    return res
+
+
+def run_flushed(args) -> dict:
+    """Per-launch device time with L2 flushed before every launch (a GPU spin is queued first
+    so that launches are enqueued ahead of the GPU)."""
+    import statistics
+    res = run(args.case, 1, args.B, args.L)
+    fn = _last_fn[0]
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    buf = torch.empty(2 * l2, dtype=torch.uint8, device="cuda")
+    evs = [_events() for _ in range(args.reps)]
+    torch.cuda._sleep(int(2e8))
+    for a, b in evs:
+        buf.zero_()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    res["ms_per_launch"] = statistics.median(ms)
+    res["flushed"] = True
+    if "bytes" in res:
+        res["GB_per_s"] = res["bytes"] / (res["ms_per_launch"] / 1e3) / 1e9
     return res
 
 
@@ -101,8 +134,11 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["compress", "decode", "paged", "prefill"])
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--B", type=int, default=0, help="decode batch (default 64)")
+    ap.add_argument("--L", type=int, default=0, help="decode context length (default 131072)")
+    ap.add_argument("--flush", action="store_true", help="flush L2 before every launch (events per launch)")
     args = ap.parse_args()
-    print(json.dumps(run(args.case, args.reps)))
+    print(json.dumps(run(args.case, args.reps, args.B, args.L) if not args.flush else run_flushed(args)))
 
 
 if __name__ == "__main__":
