@@ -11,6 +11,7 @@ HCA_ERR_UNSUPPORTED = 2
 HCA_ERR_CUDA = 3
 HCA_ERR_TIMEOUT = 4
 HCA_ERR_DEVICE_INPUT = 5
+HCA_ERR_INTERNAL = 6
 
 HCA_QK_NORM = 1
 HCA_OUT_GATE = 2

@@ -38,7 +38,8 @@ constexpr int kDecSlabs = kDecD / 64;      // 64-channel slabs per key row
 constexpr int kDecTile = 128;              // keys per tile (MMA M of S^T)
 constexpr int kDecHeads = 64;              // MMA N: query heads of one KV group (padded)
 constexpr int kDecRingK = 3;               // K slab slots
-constexpr int kDecRingV = 4;               // V slab slots (even: V^T operands are slab pairs)
+constexpr int kDecRingV = 6;               // V slab slots (even: V^T operands are slab pairs)
+constexpr int kDecPBufs = 1;               // P^T buffers
 constexpr int kDecThreads = 224;           // 7 warps
 constexpr uint32_t kSlabBytes = 128 * 128;                 // 128 rows x 128 B
 constexpr uint32_t kDecQBytes = kDecHeads * kDecD * 2;     // 64 KB
@@ -53,7 +54,7 @@ constexpr uint32_t kTmKK = 384;   // 128     K K^T (QK normalisation only)
 // shared-memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t kSmQ = 0;
 constexpr uint32_t kSmP = kSmQ + kDecQBytes;
-constexpr uint32_t kSmRingK = kSmP + 2 * kDecPBytes;
+constexpr uint32_t kSmRingK = kSmP + kDecPBufs * kDecPBytes;
 constexpr uint32_t kSmRingV = kSmRingK + kDecRingK * kSlabBytes;
 constexpr uint32_t kSmBar = kSmRingV + kDecRingV * kSlabBytes;
 constexpr int kNumBars = 2 * kDecRingK + 2 * kDecRingV + 13;
@@ -63,7 +64,7 @@ constexpr uint32_t kSmMax = kSmFin + 64 * 4;                // float[64] running
 constexpr uint32_t kSmAlpha = kSmMax + 64 * 4;              // float[64] rescale factors
 constexpr uint32_t kSmSum = kSmAlpha + 64 * 4;              // float[64] running sum per head
 constexpr uint32_t kSmMisc = kSmSum + 64 * 4;               // ints
-constexpr uint32_t kDecSmemBytes = kSmMisc + 64 + 1024;     // + alignment slack
+constexpr uint32_t kDecSmemBytes = kSmMisc + 64;            // the dynamic base is checked to be 1024-aligned
 static_assert(kDecSmemBytes <= 232448, "decode shared memory exceeds the 227 KB per-block limit");
 static_assert(kSmRed % 16 == 0 && kSmFin % 16 == 0 && kSmMax % 16 == 0 && kSmAlpha % 16 == 0 &&
               kSmSum % 16 == 0 && kSmMisc % 16 == 0, "vector-accessed shared arrays must be 16-byte aligned");
@@ -261,8 +262,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_kw, const __grid_constant__ CUtensorMap tm_vw) {
-    extern __shared__ uint8_t dsmem[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t dsmem[];
+    // the swizzled operand tiles need a 1024-byte aligned base; there is no room for slack
+    if (smem_u32(dsmem) & 1023u) {
+        if (threadIdx.x == 0) record_error(HCA_ERR_INTERNAL);
+        return;
+    }
+    uint8_t* sm = dsmem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSmBar);
     uint64_t* kfull = bars;
     uint64_t* kempty = kfull + kDecRingK;
@@ -308,6 +314,8 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&s_empty[i], 4);
+        }
+        for (int i = 0; i < kDecPBufs; ++i) {
             mbar_init(&p_full[i], 4);
             mbar_init(&p_empty[i], 1);
         }
@@ -524,8 +532,8 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         uint32_t vring = 0;
         int n = 0;
         while (!it.done) {
-            const int b = n & 1;
-            if (!warp_wait(&p_full[b], (n >> 1) & 1, abort_flag)) break;
+            const int b = n % kDecPBufs;
+            if (!warp_wait(&p_full[b], (n / kDecPBufs) & 1, abort_flag)) break;
             if (it.first() && !warp_wait(o_empty, (it.item & 1) ^ 1, abort_flag)) break;
             tc_fence_after();
             const int nvalid = it.nvalid();
@@ -684,8 +692,8 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 softmax_bar();
                 if (!first) {
                     // rescale O^T once the previous PV has landed
-                    const int pb = (n - 1) & 1;
-                    if (!group_wait(&p_empty[pb], ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                    const int pb = (n - 1) % kDecPBufs;
+                    if (!group_wait(&p_empty[pb], ((n - 1) / kDecPBufs) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -716,8 +724,8 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 pk[h >> 1] = pack_bf16x2(z[h], z[h + 1]);
                 pk[(h >> 1) + 1] = pack_bf16x2(z[h + 2], z[h + 3]);
             }
-            const int pbuf = n & 1;
-            if (!group_wait(&p_empty[pbuf], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            const int pbuf = n % kDecPBufs;
+            if (!group_wait(&p_empty[pbuf], ((n / kDecPBufs) & 1) ^ 1, abort_flag)) { ok = false; break; }
             uint8_t* pt = sm + kSmP + pbuf * kDecPBytes;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -767,6 +775,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         }
     }
 
+    __syncwarp();      // every role reconverges its warp before the CTA-wide barrier
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -89,6 +89,7 @@ const char* hca_status_string(hca_status_t s) {
         case HCA_ERR_CUDA: return "HCA_ERR_CUDA: a CUDA launch or query failed";
         case HCA_ERR_TIMEOUT: return "HCA_ERR_TIMEOUT: a bounded device wait ran out";
         case HCA_ERR_DEVICE_INPUT: return "HCA_ERR_DEVICE_INPUT: a device-resident input was out of range";
+        case HCA_ERR_INTERNAL: return "HCA_ERR_INTERNAL: a kernel found its launch environment unusable";
     }
     return "unknown hca_status_t";
 }
@@ -101,7 +102,8 @@ hca_status_t hca_get_device_error(hca_stream_t stream) {
     if (cudaMemcpyToSymbolAsync(g_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return HCA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return HCA_ERR_CUDA;
-    if (word == HCA_ERR_TIMEOUT || word == HCA_ERR_DEVICE_INPUT) return static_cast<hca_status_t>(word);
+    if (word == HCA_ERR_TIMEOUT || word == HCA_ERR_DEVICE_INPUT || word == HCA_ERR_INTERNAL)
+        return static_cast<hca_status_t>(word);
     return word == 0 ? HCA_OK : HCA_ERR_CUDA;
 }
 

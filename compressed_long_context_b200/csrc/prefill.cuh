@@ -401,6 +401,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
         }
     }
 
+    __syncwarp();      // every role reconverges its warp before the CTA-wide barrier
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

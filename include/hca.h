@@ -58,7 +58,8 @@ typedef enum {
     HCA_ERR_UNSUPPORTED = 2,
     HCA_ERR_CUDA = 3,
     HCA_ERR_TIMEOUT = 4,       /* a bounded device wait ran out (reported by hca_get_device_error) */
-    HCA_ERR_DEVICE_INPUT = 5   /* a device-resident input was out of range (seqlens, page table) */
+    HCA_ERR_DEVICE_INPUT = 5,  /* a device-resident input was out of range (seqlens, page table) */
+    HCA_ERR_INTERNAL = 6       /* a kernel found its launch environment unusable (e.g. shared-memory alignment) */
 } hca_status_t;
 
 enum {

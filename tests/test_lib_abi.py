@@ -50,7 +50,7 @@ def test_library_exports_every_declared_symbol(libhca):
 
 
 def test_status_strings(libhca):
-    for code in range(6):
+    for code in range(7):
         s = libhca.hca_status_string(code).decode()
         assert s.startswith("HCA_")
     assert b"unknown" in libhca.hca_status_string(99)
