@@ -10,6 +10,7 @@
 #include "compress.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill_pair.cuh"
 
 namespace {
 
@@ -286,6 +287,61 @@ hca_status_t launch_prefill(const hca::PrefillParams& p, const CUtensorMap& tq, 
     return cudaGetLastError() == cudaSuccess ? HCA_OK : HCA_ERR_CUDA;
 }
 
+// Clusters of two CTAs (one per SM) that can be resident at once on the current device.
+int pair_clusters_resident(cudaStream_t s) {
+    static std::mutex mu;
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> g(mu);
+    if (cached[dev] > 0) return cached[dev];
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(hca::kPpThreads, 1, 1);
+    cfg.dynamicSmemBytes = hca::kPpSmem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(&hca::prefill_pair_kernel), &cfg) !=
+        cudaSuccess)
+        return 0;
+    cached[dev] = n;
+    return n;
+}
+
+hca_status_t launch_prefill_pair(const hca::PrefillParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const CUtensorMap& tkc, const CUtensorMap& tvc,
+                                 cudaStream_t s) {
+    if (!hca::set_smem_attr_once(reinterpret_cast<const void*>(&hca::prefill_pair_kernel), (int)hca::kPpSmem, 3))
+        return HCA_ERR_CUDA;
+    const int nc = pair_clusters_resident(s);
+    if (nc <= 0) return HCA_ERR_CUDA;
+    const long long npairs = p.items < nc ? p.items : nc;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * npairs), 1, 1);
+    cfg.blockDim = dim3(hca::kPpThreads, 1, 1);
+    cfg.dynamicSmemBytes = hca::kPpSmem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, hca::prefill_pair_kernel, p, tq, tk, tv, tkc, tvc) != cudaSuccess) {
+        cudaGetLastError();
+        return HCA_ERR_CUDA;
+    }
+    return HCA_OK;
+}
+
 }  // namespace
 
 extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v, const void* kc, const void* vc,
@@ -312,26 +368,28 @@ extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v,
     p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.tpt = 128 / G; p.blk = blk; p.W = W; p.Nc = Nc;
     p.ntile_t = (T + p.tpt - 1) / p.tpt;
     p.flags = (int)flags;
-    const int NS = d == 512 ? 2 : 1;
-    p.items = (long long)p.ntile_t * B * Hkv * NS;
+    // d = 512: one item per row tile, processed by a CTA pair; d = 64: one CTA per row tile
+    p.items = (long long)p.ntile_t * B * Hkv;
     p.scale_log2 = scale * 1.4426950408889634f;
 
     const uint64_t D = (uint64_t)d;
     CUtensorMap tq, tk, tv, tkc, tvc;
     bool ok = true;
     ok &= make_tmap_4d(&tq, q, D, Hq, T, B, D, D * Hq, D * Hq * T, 64, G, p.tpt, 1);
-    ok &= make_tmap_4d(&tk, k, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, 128, 1);
-    ok &= make_tmap_4d(&tv, v, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, 128, 1);
+    // key rows per TMA box: 256 for K (and 64 for V) on the pair kernel, 128 otherwise
+    const uint32_t kbox = d == 512 ? 256 : 128, vbox = d == 512 ? 64 : 128;
+    ok &= make_tmap_4d(&tk, k, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, kbox, 1);
+    ok &= make_tmap_4d(&tv, v, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, vbox, 1);
     if (Nc > 0) {
-        ok &= make_tmap_4d(&tkc, kc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, 128, 1);
-        ok &= make_tmap_4d(&tvc, vc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, 128, 1);
+        ok &= make_tmap_4d(&tkc, kc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, kbox, 1);
+        ok &= make_tmap_4d(&tvc, vc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, vbox, 1);
     } else {   // never read: no entry is visible when T < blk
         tkc = tk;
         tvc = tv;
     }
     if (!ok) return HCA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return d == 512 ? launch_prefill<512>(p, tq, tk, tv, tkc, tvc, s) : launch_prefill<64>(p, tq, tk, tv, tkc, tvc, s);
+    return d == 512 ? launch_prefill_pair(p, tq, tk, tv, tkc, tvc, s) : launch_prefill<64>(p, tq, tk, tv, tkc, tvc, s);
 }
 
 

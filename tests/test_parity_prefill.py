@@ -107,6 +107,9 @@ def test_prefill_d64(cuda_device, libhca, B, T, Hq, Hkv, blk, W):
     (1, 450, 64, 1, 128, 256),
     (2, 333, 16, 2, 32, 40),
     (1, 260, 32, 1, 1, 3),
+    (1, 300, 2, 2, 16, 200),      # one head per KV group: 128 tokens per row tile, two window tiles
+    (1, 131, 128, 1, 8, 17),      # 128 heads per KV group: one token per row tile
+    (1, 700, 64, 1, 1, 64),       # one entry per token: three 256-entry tiles of compressed keys
 ])
 def test_prefill_d512(cuda_device, libhca, B, T, Hq, Hkv, blk, W):
     run_case(cuda_device, B, T, Hq, Hkv, 512, blk, W, seed=T + 7 * Hq, out_f32=(Hq == 16))   # bf16 path too
