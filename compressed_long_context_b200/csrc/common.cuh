@@ -223,8 +223,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
+// 2^x with the hardware approximation (PTX ex2.approx.ftz.f32: relative error about 2^-22,
+// results below 2^-126 flushed to zero, 2^-inf = 0).  The library exp2f adds range handling
+// that doubles the cost of a softmax; nothing here needs denormal results.
 __device__ __forceinline__ float ex2(float x) {
-    return exp2f(x);
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 }  // namespace hca

@@ -12,7 +12,9 @@
 //   S-CTA (cluster rank 0): Q resident in shared memory, K tiles streamed by TMA,
 //       S = Q K^T with N = 256 keys into a double-buffered S (2 x 256 TMEM columns), softmax
 //       (thread = row), and P (bf16) stored straight into the O-CTA's shared memory in the
-//       128-byte-swizzled K-major layout the tensor core reads, together with the per-row
+//       non-swizzled K-major layout the tensor core reads (8 keys of row r at
+//       (key / 8) * 2048 + r * 16, so the 32 rows of a warp fill 512 contiguous bytes per
+//       store instruction: remote stores need that to stream), together with the per-row
 //       rescale factors (and, after the last tile, the row sums);
 //   O-CTA (cluster rank 1): V tiles streamed by TMA, O += P V with N = 256 value columns
 //       (two MMAs per 16 keys cover the 512 columns), rescale of O rows when the S-CTA moved
@@ -43,7 +45,7 @@ constexpr int kPpRing = 3;                       // K units (S-CTA) / V units (O
 constexpr uint32_t kPpQSlab = 128 * 128;         // Q: 128 rows x 64 channels
 constexpr uint32_t kPpUnit = 32768;              // K: 256 keys x 64 ch; V: 64 keys x 256 ch
 constexpr uint32_t kPpVSub = 8192;               // V unit = 4 channel slabs of 64 keys x 64 ch
-constexpr uint32_t kPpPBuf = 65536;              // P: 128 rows x 256 keys, 4 key slabs of 16 KB
+constexpr uint32_t kPpPBuf = 65536;              // P: 128 rows x 256 keys, 32 key chunks of 2 KB
 constexpr uint32_t kPpHdrBytes = 1040;           // alpha[128], l[128], flag[4]
 // shared-memory layout (offsets from a 1024-aligned base); the two ranks reuse offsets
 constexpr uint32_t kPpSmQ = 0;                   // S-CTA: Q, 8 slabs (128 KB)
@@ -163,9 +165,16 @@ __device__ __forceinline__ void pp_drain_wait(uint64_t* bar, uint32_t parity) {
         }
 }
 
-// byte offset of (row r, 16-byte chunk c) inside a 128-byte-swizzled slab of 128-byte rows
-__device__ __forceinline__ uint32_t pp_sw128(int r, int c) {
-    return (uint32_t)(r * 128 + (((c ^ r) & 7) << 4));
+// Shared-memory matrix descriptor for the non-swizzled K-major layout: core matrices of
+// 8 rows x 16 bytes (rows 16 bytes apart), `lbo` bytes between core matrices adjacent in K,
+// `sbo` bytes between core matrices adjacent in M/N; swizzle field 0.
+__device__ __forceinline__ uint64_t pp_desc_noswz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
 }
 
 __device__ __forceinline__ uint32_t pp_ld_cluster_u32(uint32_t raddr) {
@@ -332,7 +341,7 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
             const int q4 = warp & 3;
             const int r = q4 * 32 + lane;
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-            const uint32_t rP = peer_base + kPpSmP + (uint32_t)r * 128u;
+            const uint32_t rP = peer_base + kPpSmP + (uint32_t)r * 16u;
             const uint32_t rHdr = peer_base + kPpSmHdr;
             const uint32_t rPFull = peer_base + kPpSmBar + kBarPFull * 8;
             const float sl2 = p.scale_log2;
@@ -366,67 +375,89 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                     }
                     tc_fence_after();
                     const uint32_t sa = tmem + lane_off + sb * kPpKeys;
-                    // pass 1: the tile's maximum logit of this row (log2 units)
+                    // The reference maximum m of a row is lazy: P = 2^(logit - m) is computed
+                    // against the reference of the earlier tiles, and m moves only when a tile
+                    // exceeds it by 2^8 -- the tile is then redone against the new reference.  A
+                    // warp in which some row has no reference yet takes the tile maximum first.
+                    const bool need_max = __any_sync(0xffffffffu, m == -INFINITY);
                     float tmax = -INFINITY;
+                    if (need_max) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < ncol; c0 += 64) {
-                        float v[64];
+                        for (int c0 = 0; c0 < ncol; c0 += 64) {
+                            float v[64];
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            if (c0 + 16 * k < ncol) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
-                        tmem_wait_ld();
+                            for (int k = 0; k < 4; ++k)
+                                if (c0 + 16 * k < ncol) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int k = 0; k < 64; ++k) {
-                            const int c = c0 + k;
-                            if (c >= lo && c < hi) tmax = fmaxf(tmax, v[k] * sl2);
+                            for (int k = 0; k < 64; ++k) {
+                                const int c = c0 + k;
+                                if (c >= lo && c < hi) tmax = fmaxf(tmax, v[k] * sl2);
+                            }
                         }
                     }
-                    // lazy reference maximum: moved only on the first visible key or when the
-                    // tile exceeds it by 2^8
-                    const bool resc = m != -INFINITY && tmax > m + kPfRescale;
+                    bool resc = false;
                     float al = 1.f;
-                    if (resc) {
-                        al = ex2(m - tmax);
-                        l *= al;
+                    if (need_max) {
+                        resc = m != -INFINITY && tmax > m + kPfRescale;
+                        if (resc) {
+                            al = ex2(m - tmax);
+                            l *= al;
+                        }
+                        if (resc || (m == -INFINITY && tmax > -INFINITY)) m = tmax;
                     }
-                    if (resc || (m == -INFINITY && tmax > -INFINITY)) m = tmax;
-                    const float mref = m == -INFINITY ? 0.f : m;
                     // the O-CTA's P slot is free once the PV of tile n-2 has landed
                     if (!pp_warp_wait_cl(&bars[kBarPEmpty + sb], ((n >> 1) & 1) ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    // pass 2: P = 2^(logit - m) in bf16, stored into the peer in the swizzled
-                    // K-major layout (key slab of 64 = 16 KB, row = 128 B)
+                    // P in bf16, stored into the peer: keys 8c..8c+7 of this row at chunk c
+                    // (2 KB per chunk of 8 keys x 128 rows)
                     const uint32_t pbase = rP + sb * kPpPBuf;
-                    float rs = 0.f;
+                    float rs;
+                    for (int attempt = 0;; ++attempt) {
+                        const float mref = m == -INFINITY ? 0.f : m;
+                        float dmax = -INFINITY;
+                        rs = 0.f;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < ncol; c0 += 64) {
-                        float v[64];
+                        for (int c0 = 0; c0 < ncol; c0 += 64) {
+                            float v[64];
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            if (c0 + 16 * k < ncol) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
-                        tmem_wait_ld();
+                            for (int k = 0; k < 4; ++k)
+                                if (c0 + 16 * k < ncol) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int k16 = 0; k16 < 4; ++k16) {
-                            const int cb = c0 + 16 * k16;
-                            if (cb < ncol) {
-                                uint32_t pk[8];
+                            for (int k16 = 0; k16 < 4; ++k16) {
+                                const int cb = c0 + 16 * k16;
+                                if (cb < ncol) {
+                                    uint32_t pk[8];
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    const int c = cb + 2 * e;
-                                    const float a = (c >= lo && c < hi) ? ex2(fmaf(v[16 * k16 + 2 * e], sl2, -mref)) : 0.f;
-                                    const float b2 = (c + 1 >= lo && c + 1 < hi)
-                                                         ? ex2(fmaf(v[16 * k16 + 2 * e + 1], sl2, -mref)) : 0.f;
-                                    rs += a + b2;
-                                    pk[e] = pack_bf16x2(a, b2);
+                                    for (int e = 0; e < 8; ++e) {
+                                        const int c = cb + 2 * e;
+                                        const float d0 = (c >= lo && c < hi) ? fmaf(v[16 * k16 + 2 * e], sl2, -mref)
+                                                                             : -INFINITY;
+                                        const float d1 = (c + 1 >= lo && c + 1 < hi)
+                                                             ? fmaf(v[16 * k16 + 2 * e + 1], sl2, -mref) : -INFINITY;
+                                        dmax = fmaxf(dmax, fmaxf(d0, d1));
+                                        const float a = ex2(d0), b2 = ex2(d1);
+                                        rs += a + b2;
+                                        pk[e] = pack_bf16x2(a, b2);
+                                    }
+                                    const uint32_t ra = pbase + ((uint32_t)cb >> 3) * 2048u;
+                                    pp_st_cluster_v4(ra, pk[0], pk[1], pk[2], pk[3]);
+                                    pp_st_cluster_v4(ra + 2048u, pk[4], pk[5], pk[6], pk[7]);
                                 }
-                                const uint32_t ra = pbase + ((uint32_t)cb >> 6) * 16384u;
-                                const int ch = (cb & 63) >> 3;
-                                pp_st_cluster_v4(ra + ((((uint32_t)ch ^ (uint32_t)r) & 7u) << 4), pk[0], pk[1], pk[2], pk[3]);
-                                pp_st_cluster_v4(ra + ((((uint32_t)ch + 1u ^ (uint32_t)r) & 7u) << 4), pk[4], pk[5], pk[6],
-                                                 pk[7]);
                             }
+                        }
+                        if (need_max || attempt) break;
+                        // every row of this warp has a reference here; redo if one was exceeded
+                        const bool over = dmax > kPfRescale;
+                        if (!__any_sync(0xffffffffu, over)) break;
+                        if (over) {
+                            al = ex2(-dmax);
+                            l *= al;
+                            m += dmax;
+                            resc = true;
                         }
                     }
                     l += rs;
@@ -511,11 +542,11 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                             tc_fence_after();
                             if (lane == 0) {
                                 const uint32_t vb = smem_u32(sm + kPpSmRing + st * kPpUnit);
-                                const uint32_t pa = p_base + sb * kPpPBuf + u * 16384;
+                                const uint32_t pa = p_base + sb * kPpPBuf + u * 16384;   // 16 keys = 4 KB
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
                                     if (64 * u + 16 * kk < nk)
-                                        mma_ss(tmem + 256 * h, smem_desc_sw128(pa + kk * 32, 16, 1024),
+                                        mma_ss(tmem + 256 * h, pp_desc_noswz(pa + kk * 4096, 2048, 128),
                                                smem_desc_sw128(vb + kk * 2048, kPpVSub, 1024), id,
                                                (j == 0 && u == 0 && kk == 0) ? 0u : 1u);
                                 mma_commit(&bars[kBarVEmpty + st]);
