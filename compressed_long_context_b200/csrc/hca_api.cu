@@ -58,6 +58,22 @@ bool make_tmap_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, ui
     return r == CUDA_SUCCESS;
 }
 
+// 4-D tensor map with 128-byte swizzle for TMA stores of 128-byte rows: element type bf16
+// or fp32 (esize 2 or 4); strides in elements for dims 1..3.
+bool make_tmap_4d_plain(CUtensorMap* m, void* base, int esize, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                        uint64_t s1, uint64_t s2, uint64_t s3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {d0, d1, d2, d3};
+    cuuint64_t strides[3] = {s1 * esize, s2 * esize, s3 * esize};
+    cuuint32_t box[4] = {b0, b1, b2, b3};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel slot, device).
 bool set_smem_attr_once(const void* fn, int bytes, int slot) {
     static std::mutex mu;
@@ -295,6 +311,9 @@ int pair_clusters_resident(cudaStream_t s) {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> g(mu);
     if (cached[dev] > 0) return cached[dev];
+    // the occupancy query needs the kernel's shared-memory opt-in in place
+    if (!hca::set_smem_attr_once(reinterpret_cast<const void*>(&hca::prefill_pair_kernel), (int)hca::kPpSmem, 3))
+        return 0;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -317,12 +336,16 @@ int pair_clusters_resident(cudaStream_t s) {
 
 hca_status_t launch_prefill_pair(const hca::PrefillParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& tkc, const CUtensorMap& tvc,
-                                 cudaStream_t s) {
+                                 const CUtensorMap& tout, size_t ws_bytes, cudaStream_t s) {
     if (!hca::set_smem_attr_once(reinterpret_cast<const void*>(&hca::prefill_pair_kernel), (int)hca::kPpSmem, 3))
         return HCA_ERR_CUDA;
     const int nc = pair_clusters_resident(s);
     if (nc <= 0) return HCA_ERR_CUDA;
     const long long npairs = p.items < nc ? p.items : nc;
+    // the P hand-off slots of every pair
+    if (!p.scratch || (reinterpret_cast<uintptr_t>(p.scratch) & 127) ||
+        ws_bytes < (size_t)npairs * hca::kPpSlots * hca::kPpSlotStride)
+        return HCA_ERR_INVALID_ARG;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -335,7 +358,7 @@ hca_status_t launch_prefill_pair(const hca::PrefillParams& p, const CUtensorMap&
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, hca::prefill_pair_kernel, p, tq, tk, tv, tkc, tvc) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, hca::prefill_pair_kernel, p, tq, tk, tv, tkc, tvc, tout) != cudaSuccess) {
         cudaGetLastError();
         return HCA_ERR_CUDA;
     }
@@ -344,8 +367,16 @@ hca_status_t launch_prefill_pair(const hca::PrefillParams& p, const CUtensorMap&
 
 }  // namespace
 
+extern "C" size_t hca_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d, int dv) {
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || d != dv) return 0;
+    if (d != 512) return 0;       // only the 512-dim (CTA pair) kernel uses scratch
+    const int nc = pair_clusters_resident(nullptr);
+    return nc > 0 ? (size_t)nc * hca::kPpSlots * hca::kPpSlotStride : 0;
+}
+
 extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v, const void* kc, const void* vc,
-                                    void* out, float* lse, int B, int T, int Hq, int Hkv, int d, int dv, int blk,
+                                    void* out, float* lse, void* workspace, size_t ws_bytes,
+                                    int B, int T, int Hq, int Hkv, int d, int dv, int blk,
                                     int W, float scale, unsigned flags, hca_stream_t stream) {
     using namespace hca;
     if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || blk < 1 || W < 1) return HCA_ERR_INVALID_ARG;
@@ -365,6 +396,7 @@ extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v,
     PrefillParams p;
     p.out = out;
     p.lse = want_lse ? lse : nullptr;
+    p.scratch = static_cast<uint8_t*>(workspace);
     p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.tpt = 128 / G; p.blk = blk; p.W = W; p.Nc = Nc;
     p.ntile_t = (T + p.tpt - 1) / p.tpt;
     p.flags = (int)flags;
@@ -389,7 +421,14 @@ extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v,
     }
     if (!ok) return HCA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return d == 512 ? launch_prefill_pair(p, tq, tk, tv, tkc, tvc, s) : launch_prefill<64>(p, tq, tk, tv, tkc, tvc, s);
+    if (d != 512) return launch_prefill<64>(p, tq, tk, tv, tkc, tvc, s);
+    // output boxes of 32 rows x 128 bytes: the 32 rows of a warp are (tokens, heads) in order
+    CUtensorMap tout;
+    const uint32_t bh = G < 32 ? (uint32_t)G : 32u, bt = 32u / bh;
+    const int es = (flags & HCA_OUT_F32) ? 4 : 2;
+    if (!make_tmap_4d_plain(&tout, out, es, D, Hq, T, B, D, D * Hq, D * Hq * T, 128 / es, bh, bt, 1))
+        return HCA_ERR_CUDA;
+    return launch_prefill_pair(p, tq, tk, tv, tkc, tvc, tout, ws_bytes, s);
 }
 
 

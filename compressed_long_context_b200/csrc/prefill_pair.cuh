@@ -11,21 +11,25 @@
 // tile need 256 more.  So the work is split by stage, not by value columns:
 //   S-CTA (cluster rank 0): Q resident in shared memory, K tiles streamed by TMA,
 //       S = Q K^T with N = 256 keys into a double-buffered S (2 x 256 TMEM columns), softmax
-//       (thread = row), and P (bf16) stored straight into the O-CTA's shared memory in the
+//       (thread = row), and P (bf16) written to a per-pair slot in global memory (L2) in the
 //       non-swizzled K-major layout the tensor core reads (8 keys of row r at
 //       (key / 8) * 2048 + r * 16, so the 32 rows of a warp fill 512 contiguous bytes per
-//       store instruction: remote stores need that to stream), together with the per-row
-//       rescale factors (and, after the last tile, the row sums);
+//       store); the per-row rescale factors (and, after the last tile, the row sums) go
+//       straight into the O-CTA's shared memory.  P takes the L2 path because the
+//       SM-to-SM network moves only about 30 GB/s per pair, a third of what a 256-key tile
+//       needs; an O-CTA thread pulls each slot into shared memory with a bulk copy.  The
+//       hand-off granule is a P unit of 128 keys (half an S tile), four units in flight;
 //   O-CTA (cluster rank 1): V tiles streamed by TMA, O += P V with N = 256 value columns
 //       (two MMAs per 16 keys cover the 512 columns), rescale of O rows when the S-CTA moved
 //       a row's reference maximum, and the epilogue out = O / l.
 // Every MMA is M = 128, N = 256 (or the 16-rounded key count of a short tile): the tcgen05
 // issue cost of one M = 128 MMA does not shrink with N, so narrow MMAs waste the pipe.
 //
-// Warps (224 threads, same kernel for both ranks):
-//   S-CTA: 0 TMA (Q, K) | 1 MMA + TMEM | 2-5 softmax | 6 idle
-//   O-CTA: 0 TMA (V)    | 1 MMA + TMEM | 2-5 rescale + epilogue | 6 forwards "P slot
-//          consumed" to the S-CTA
+// Warps (320 threads, same kernel for both ranks):
+//   S-CTA: 0 TMA (Q, K) | 1 MMA + TMEM | 2-9 softmax (two warps per TMEM lane quarter)
+//   O-CTA: 0 TMA (V)    | 1 MMA + TMEM | 2-5 rescale + epilogue | 6 P loads | 7 "P slot
+//          consumed" forwarded to the S-CTA (its own warp, so that a slot is returned the
+//          moment its PV lands, whatever the loads are waiting for) | 8, 9 idle
 //
 // Tiles of one row tile (item): the compressed segment in tiles of 256 entries, then the
 // raw window [wlo, tlast] in tiles of 256 tokens; per-row masks [lo, hi) as in prefill.cuh.
@@ -33,39 +37,53 @@
 // by 2^8, so the O-CTA rarely touches O between MMAs.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "prefill.cuh"
 
 namespace hca {
 
-constexpr int kPpThreads = 224;
-constexpr int kPpKeys = 256;                     // keys per tile (MMA N of S)
+constexpr int kPpThreads = 320;
+constexpr int kPpSoftWarps = 8;                 // S-CTA softmax warps (2..9)
+constexpr int kPpKeys = 256;                     // keys per S tile (MMA N of S)
+constexpr int kPpUKeys = 128;                    // keys per P unit (the hand-off granule)
+constexpr int kPpSlots = 3;                      // P units in flight between the two CTAs
 constexpr int kPpD = 512;
 constexpr int kPpRing = 3;                       // K units (S-CTA) / V units (O-CTA)
 constexpr uint32_t kPpQSlab = 128 * 128;         // Q: 128 rows x 64 channels
 constexpr uint32_t kPpUnit = 32768;              // K: 256 keys x 64 ch; V: 64 keys x 256 ch
 constexpr uint32_t kPpVSub = 8192;               // V unit = 4 channel slabs of 64 keys x 64 ch
-constexpr uint32_t kPpPBuf = 65536;              // P: 128 rows x 256 keys, 32 key chunks of 2 KB
-constexpr uint32_t kPpHdrBytes = 1040;           // alpha[128], l[128], flag[4]
+constexpr uint32_t kPpPBuf = 32768;              // P unit: 128 rows x 128 keys, 16 key chunks of 2 KB
+constexpr uint32_t kPpHdrBytes = 528;            // per P unit: alpha[128], flag[4]
+constexpr uint32_t kPpSlotStride = kPpPBuf + 512; // global slot: P unit, then l[128] after an item's last unit
 // shared-memory layout (offsets from a 1024-aligned base); the two ranks reuse offsets
 constexpr uint32_t kPpSmQ = 0;                   // S-CTA: Q, 8 slabs (128 KB)
-constexpr uint32_t kPpSmP = 0;                   // O-CTA: P, 2 buffers (128 KB)
+constexpr uint32_t kPpSmP = 0;                   // O-CTA: P, 3 units (96 KB)
+constexpr uint32_t kPpSmStage = kPpSmP + kPpSlots * kPpPBuf;   // O-CTA: output staging, 4 warps x 8 KB
+constexpr uint32_t kPpStageWarp = 8192;          // 2 pieces of 4 KB: 32 rows x 64 bf16 or 32 fp32 columns
 constexpr uint32_t kPpSmRing = 131072;           // both: ring of 3 units (96 KB)
-constexpr uint32_t kPpSmHdr = kPpSmRing + kPpRing * kPpUnit;     // O-CTA: 2 headers
-constexpr uint32_t kPpSmBar = kPpSmHdr + 2 * kPpHdrBytes;
-constexpr int kPpNumBars = 32;
+constexpr uint32_t kPpSmHdr = kPpSmRing + kPpRing * kPpUnit;     // O-CTA: unit headers
+constexpr uint32_t kPpSmXch = kPpSmHdr;          // S-CTA: softmax exchange, 2 x 2 x 128 floats
+constexpr uint32_t kPpHdrArea = kPpSlots * kPpHdrBytes > 2048 ? kPpSlots * kPpHdrBytes : 2048;
+constexpr uint32_t kPpSmBar = kPpSmHdr + kPpHdrArea;
+constexpr int kPpNumBars = 42;                  // 41 used; even count keeps misc 16-aligned
 constexpr uint32_t kPpSmMisc = kPpSmBar + kPpNumBars * 8;
-constexpr uint32_t kPpSmem = kPpSmMisc + 64;
+constexpr uint32_t kPpSmem = kPpSmMisc + 16;
 static_assert(kPpSmem <= 232448, "pair prefill shared memory exceeds the 227 KB per-block limit");
-static_assert(kPpSmHdr % 16 == 0 && kPpSmBar % 8 == 0, "header 16-aligned, barriers 8-aligned");
+static_assert(kPpSmHdr % 16 == 0 && kPpSmBar % 8 == 0 && kPpSmMisc % 16 == 0,
+              "header 16-aligned, barriers 8-aligned");
+static_assert(kPpSlotStride % 128 == 0, "global slots 128-aligned");
+static_assert(kPpKeys == 2 * kPpUKeys, "an S tile is two P units");
+static_assert(kPpSmStage + 4 * kPpStageWarp <= kPpSmRing, "output staging fits below the ring");
 
 // barrier indices (both ranks initialise all of them; each rank uses its own)
 enum : int {
     kBarKFull = 0, kBarKEmpty = 3, kBarQFull = 6, kBarQEmpty = 7, kBarSFull = 8, kBarSEmpty = 10,
-    kBarPEmpty = 12,                                           // S-CTA
-    kBarVFull = 14, kBarVEmpty = 17, kBarPFull = 20, kBarCorr = 22, kBarPCons = 24, kBarOFull = 26,
-    kBarOEmpty = 27,                                           // O-CTA
-    kBarDrain = 28
+    kBarPEmpty = 12,                                                       // S-CTA (+ [4])
+    kBarVFull = 16, kBarVEmpty = 19, kBarPFull = 22, kBarCorr = 26, kBarPCons = 30, kBarPLoaded = 34,
+    kBarOFull = 38, kBarOEmpty = 39,                                       // O-CTA
+    kBarDrain = 40
 };
 
 struct PpItem {
@@ -96,6 +114,10 @@ __device__ __forceinline__ int pp_tile_keys(const PpItem& it, int j) {
 __device__ __forceinline__ int pp_tile_row(const PpItem& it, int j) {
     return j < it.nct ? kPpKeys * j : it.wlo + kPpKeys * (j - it.nct);
 }
+// P units of a tile with nk keys, and the keys / 16-rounded columns of unit hh
+__device__ __forceinline__ int pp_units(int nk) { return (nk + kPpUKeys - 1) / kPpUKeys; }
+__device__ __forceinline__ int pp_unit_keys(int nk, int hh) { return min(kPpUKeys, nk - hh * kPpUKeys); }
+__device__ __forceinline__ int pp_unit_cols(int nk, int hh) { return min(kPpUKeys, ((nk + 15) & ~15) - hh * kPpUKeys); }
 
 // ------------------------------------------------------------------ cluster helpers
 
@@ -116,15 +138,44 @@ __device__ __forceinline__ void pp_cluster_sync() {
 __device__ __forceinline__ void pp_remote_arrive(uint32_t rbar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(rbar) : "memory");
 }
-__device__ __forceinline__ void pp_st_cluster_v4(uint32_t raddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(raddr), "r"(a), "r"(b), "r"(c), "r"(d)
+// Asynchronous stores into a peer CTA's shared memory; each completes `bytes` of the peer's
+// mbarrier transaction count (release at cluster scope), so the writer never waits.
+__device__ __forceinline__ void pp_st_async_v4(uint32_t raddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                               uint32_t rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+                 :: "r"(raddr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar) : "memory");
+}
+__device__ __forceinline__ void pp_st_async_u32(uint32_t raddr, uint32_t v, uint32_t rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 :: "r"(raddr), "r"(v), "r"(rbar) : "memory");
+}
+// Arrival + expected bytes on a peer's barrier.  Relaxed: the bytes carry their own release
+// (complete_tx of st.async), and a release here would wait for every store still in flight.
+__device__ __forceinline__ void pp_remote_arrive_expect_tx(uint32_t rbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;"
+                 :: "r"(rbar), "r"(bytes) : "memory");
+}
+// TMA tensor store (shared -> global) of one box, tracked by the issuing thread's bulk groups
+__device__ __forceinline__ void pp_tma_store_4d(const CUtensorMap* m, const void* src, int c0, int c1, int c2,
+                                                int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 :: "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                  : "memory");
 }
+__device__ __forceinline__ void pp_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void pp_bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void pp_bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void pp_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void pp_st_cluster_u32(uint32_t raddr, uint32_t v) {
     asm volatile("st.shared::cluster.b32 [%0], %1;" :: "r"(raddr), "r"(v) : "memory");
 }
-__device__ __forceinline__ void pp_fence_proxy_async_cluster() {
-    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+__device__ __forceinline__ void pp_fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// bulk copy global -> this CTA's shared memory, completion counted in bytes on `bar`
+__device__ __forceinline__ void pp_bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 // try_wait with acquire at cluster scope: for barriers the peer CTA arrives on
 __device__ __forceinline__ bool pp_try_wait_cl(uint64_t* bar, uint32_t parity) {
@@ -189,10 +240,11 @@ __device__ __forceinline__ void pp_drain_ring(uint64_t* full, uint32_t issued) {
         if (issued > st) pp_drain_wait(&full[st], ((issued - 1 - st) / kPpRing) & 1);
 }
 
-__global__ void __launch_bounds__(kPpThreads, 1)
+__global__ void __launch_bounds__(kPpThreads, 1)   // 10 warps: at most 168 registers (3 warps per SMSP)
 prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc) {
+                    const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+                    const __grid_constant__ CUtensorMap tm_out) {
     extern __shared__ __align__(1024) uint8_t dsmem[];
     uint8_t* sm = dsmem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kPpSmBar);
@@ -218,11 +270,14 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
         mbar_init(&bars[kBarQEmpty], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars[kBarSFull + i], 1);
-            mbar_init(&bars[kBarSEmpty + i], 4);
+            mbar_init(&bars[kBarSEmpty + i], kPpSoftWarps);
+        }
+        for (int i = 0; i < kPpSlots; ++i) {
             mbar_init(&bars[kBarPEmpty + i], 1);
-            mbar_init(&bars[kBarPFull + i], 4);
+            mbar_init(&bars[kBarPFull + i], 4);        // armed by each TMEM lane quarter
             mbar_init(&bars[kBarCorr + i], 4);
             mbar_init(&bars[kBarPCons + i], 1);
+            mbar_init(&bars[kBarPLoaded + i], 1);
         }
         mbar_init(&bars[kBarOFull], 1);
         mbar_init(&bars[kBarOEmpty], 4);
@@ -235,6 +290,7 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
         } else {
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_vc);
+            prefetch_tmap(&tm_out);
         }
     }
     if (warp == 1) tmem_alloc(tmem_slot, 512);
@@ -335,17 +391,41 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
             }
             __syncwarp();
         }
-    } else if (s_cta && warp >= 2 && warp <= 5) {
+    } else if (s_cta && warp >= 2 && warp < 2 + kPpSoftWarps) {
         // ===================================================== S-CTA: softmax, P to the O-CTA
+        // Eight warps: warp w owns the 32 rows of TMEM lane quarter w % 4 and one half of the
+        // columns of every unit (hw = 0: the first 64, hw = 1: the last 64).  The two warps of
+        // a quarter keep identical per-row references m (they take the same decisions from
+        // the same exchanged maxima) and their own partial row sums.
         if (go) {
             const int q4 = warp & 3;
+            const int hw = (warp - 2) >> 2;
             const int r = q4 * 32 + lane;
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+            float* xch = reinterpret_cast<float*>(sm + kPpSmXch);     // [2 parities][2 halves][128 rows]
+            int xpar = 0;
+            // a value of this row from both warps of the quarter (64-thread named barrier)
+            auto exchange = [&](float mine, float* other) {
+                xch[(xpar * 2 + hw) * 128 + r] = mine;
+                asm volatile("bar.sync %0, 64;" :: "r"(4 + q4) : "memory");
+                *other = xch[(xpar * 2 + (hw ^ 1)) * 128 + r];
+                xpar ^= 1;
+            };
+            // the two warps of a quarter go on or unwind together: a verdict that differed
+            // would leave one of them at a named barrier the other never reaches
+            auto pair_agree = [&](bool ok_mine) -> bool {
+                uint32_t res;
+                asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                             "barrier.red.and.pred q, %2, 64, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                             : "=r"(res) : "r"((uint32_t)ok_mine), "r"(4 + q4) : "memory");
+                return res != 0;
+            };
             const uint32_t rP = peer_base + kPpSmP + (uint32_t)r * 16u;
             const uint32_t rHdr = peer_base + kPpSmHdr;
             const uint32_t rPFull = peer_base + kPpSmBar + kBarPFull * 8;
             const float sl2 = p.scale_log2;
-            int n = 0;
+            int n = 0;            // S tiles
+            uint32_t un = 0;      // P units
             bool ok = true;
             for (long long i = pair; ok && i < p.items; i += npairs) {
                 const PpItem it = pp_item(p, i);
@@ -355,12 +435,11 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                 const int t = row_live ? tok : p.T - 1;
                 const int head = it.g * p.G + (r % p.G);
                 const int nc_t = pf_visible(t, p.W, p.blk);
-                float m = -INFINITY, l = 0.f;
-                for (int j = 0; j < nt; ++j, ++n) {
+                float m = -INFINITY, l = 0.f;     // l: this warp's partial row sum
+                for (int j = 0; ok && j < nt; ++j, ++n) {
                     const int sb = n & 1;
                     const int nk = pp_tile_keys(it, j);
-                    const int ncol = (nk + 15) & ~15;
-                    int lo, hi;               // valid columns of this row: [lo, hi)
+                    int lo, hi;               // valid columns of this row in the tile: [lo, hi)
                     if (j < it.nct) {
                         lo = 0;
                         hi = min(nk, nc_t - kPpKeys * j);
@@ -369,115 +448,156 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                         lo = max(0, t - p.W + 1 - u0);
                         hi = min(nk, t - u0 + 1);
                     }
-                    if (!warp_wait(&bars[kBarSFull + sb], (n >> 1) & 1, abort_flag)) {
+                    if (!pair_agree(warp_wait(&bars[kBarSFull + sb], (n >> 1) & 1, abort_flag))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t sa = tmem + lane_off + sb * kPpKeys;
-                    // The reference maximum m of a row is lazy: P = 2^(logit - m) is computed
-                    // against the reference of the earlier tiles, and m moves only when a tile
-                    // exceeds it by 2^8 -- the tile is then redone against the new reference.  A
-                    // warp in which some row has no reference yet takes the tile maximum first.
-                    const bool need_max = __any_sync(0xffffffffu, m == -INFINITY);
-                    float tmax = -INFINITY;
-                    if (need_max) {
+                    const int nu = pp_units(nk);
+                    for (int hh = 0; hh < nu; ++hh, ++un) {
+                        const int us = (int)(un % kPpSlots);
+                        const int u_end = hh * kPpUKeys + pp_unit_cols(nk, hh);
+                        const int c_beg = hh * kPpUKeys + 64 * hw;            // this warp's columns
+                        const int c_end = min(c_beg + 64, u_end);             // (may be empty)
+                        // The reference maximum m of a row is lazy: P = 2^(logit - m) is computed
+                        // against the reference of the earlier units, and m moves only when a unit
+                        // exceeds it by 2^8 -- the unit is then redone against the new reference.
+                        // A quarter in which some row has no reference yet takes the maximum first.
+                        const bool need_max = __any_sync(0xffffffffu, m == -INFINITY);
+                        bool resc = false;
+                        float al = 1.f;
+                        if (need_max) {
+                            float tmax = -INFINITY;
 #pragma unroll 1
-                        for (int c0 = 0; c0 < ncol; c0 += 64) {
-                            float v[64];
+                            for (int c0 = c_beg; c0 < c_end; c0 += 32) {
+                                float v[32];
 #pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                if (c0 + 16 * k < ncol) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
-                            tmem_wait_ld();
+                                for (int k = 0; k < 2; ++k)
+                                    if (c0 + 16 * k < c_end) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
+                                tmem_wait_ld();
 #pragma unroll
-                            for (int k = 0; k < 64; ++k) {
-                                const int c = c0 + k;
-                                if (c >= lo && c < hi) tmax = fmaxf(tmax, v[k] * sl2);
-                            }
-                        }
-                    }
-                    bool resc = false;
-                    float al = 1.f;
-                    if (need_max) {
-                        resc = m != -INFINITY && tmax > m + kPfRescale;
-                        if (resc) {
-                            al = ex2(m - tmax);
-                            l *= al;
-                        }
-                        if (resc || (m == -INFINITY && tmax > -INFINITY)) m = tmax;
-                    }
-                    // the O-CTA's P slot is free once the PV of tile n-2 has landed
-                    if (!pp_warp_wait_cl(&bars[kBarPEmpty + sb], ((n >> 1) & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    // P in bf16, stored into the peer: keys 8c..8c+7 of this row at chunk c
-                    // (2 KB per chunk of 8 keys x 128 rows)
-                    const uint32_t pbase = rP + sb * kPpPBuf;
-                    float rs;
-                    for (int attempt = 0;; ++attempt) {
-                        const float mref = m == -INFINITY ? 0.f : m;
-                        float dmax = -INFINITY;
-                        rs = 0.f;
-#pragma unroll 1
-                        for (int c0 = 0; c0 < ncol; c0 += 64) {
-                            float v[64];
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                if (c0 + 16 * k < ncol) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int k16 = 0; k16 < 4; ++k16) {
-                                const int cb = c0 + 16 * k16;
-                                if (cb < ncol) {
-                                    uint32_t pk[8];
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) {
-                                        const int c = cb + 2 * e;
-                                        const float d0 = (c >= lo && c < hi) ? fmaf(v[16 * k16 + 2 * e], sl2, -mref)
-                                                                             : -INFINITY;
-                                        const float d1 = (c + 1 >= lo && c + 1 < hi)
-                                                             ? fmaf(v[16 * k16 + 2 * e + 1], sl2, -mref) : -INFINITY;
-                                        dmax = fmaxf(dmax, fmaxf(d0, d1));
-                                        const float a = ex2(d0), b2 = ex2(d1);
-                                        rs += a + b2;
-                                        pk[e] = pack_bf16x2(a, b2);
-                                    }
-                                    const uint32_t ra = pbase + ((uint32_t)cb >> 3) * 2048u;
-                                    pp_st_cluster_v4(ra, pk[0], pk[1], pk[2], pk[3]);
-                                    pp_st_cluster_v4(ra + 2048u, pk[4], pk[5], pk[6], pk[7]);
+                                for (int k = 0; k < 32; ++k) {
+                                    const int c = c0 + k;
+                                    if (c >= lo && c < hi) tmax = fmaxf(tmax, v[k] * sl2);
                                 }
                             }
+                            float tother;
+                            exchange(tmax, &tother);
+                            tmax = fmaxf(tmax, tother);
+                            resc = m != -INFINITY && tmax > m + kPfRescale;
+                            if (resc) {
+                                al = ex2(m - tmax);
+                                l *= al;
+                            }
+                            if (resc || (m == -INFINITY && tmax > -INFINITY)) m = tmax;
                         }
-                        if (need_max || attempt) break;
-                        // every row of this warp has a reference here; redo if one was exceeded
-                        const bool over = dmax > kPfRescale;
-                        if (!__any_sync(0xffffffffu, over)) break;
-                        if (over) {
-                            al = ex2(-dmax);
-                            l *= al;
-                            m += dmax;
-                            resc = true;
+                        // the O-CTA's slot us is free once the PV of unit un - kPpSlots has landed
+                        if (!pair_agree(pp_warp_wait_cl(&bars[kBarPEmpty + us], ((un / kPpSlots) & 1) ^ 1,
+                                                        abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        // P in bf16 straight into the O-CTA's slot us: keys 8c..8c+7 of the unit,
+                        // this row, at chunk c (2 KB per chunk of 8 keys x 128 rows).  Every store
+                        // counts its bytes on the slot's barrier; each lane quarter arms it once
+                        // it knows how many bytes it stored (a redone unit is stored twice).
+                        const uint32_t pbar = rPFull + us * 8;
+                        const uint32_t pbase = rP + us * kPpPBuf;
+                        int attempts = 1;
+                        // columns valid for every row of the warp (most compressed units) skip
+                        // the per-column mask
+                        const bool unmasked = __all_sync(0xffffffffu, lo <= c_beg && hi >= c_end);
+                        float rs, dmax;
+                        auto pass2 = [&](auto masked_tag, float mref) {
+                            constexpr bool kMasked = decltype(masked_tag)::value;
+                            dmax = -INFINITY;
+                            rs = 0.f;
+#pragma unroll 1
+                            for (int c0 = c_beg; c0 < c_end; c0 += 32) {
+                                float v[32];
+#pragma unroll
+                                for (int k = 0; k < 2; ++k)
+                                    if (c0 + 16 * k < c_end) tmem_ld16(sa + c0 + 16 * k, v + 16 * k);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int k16 = 0; k16 < 2; ++k16) {
+                                    const int cb = c0 + 16 * k16;
+                                    if (cb < c_end) {
+                                        uint32_t pk[8];
+#pragma unroll
+                                        for (int e = 0; e < 8; ++e) {
+                                            const int c = cb + 2 * e;
+                                            float d0 = fmaf(v[16 * k16 + 2 * e], sl2, -mref);
+                                            float d1 = fmaf(v[16 * k16 + 2 * e + 1], sl2, -mref);
+                                            if (kMasked) {
+                                                d0 = (c >= lo && c < hi) ? d0 : -INFINITY;
+                                                d1 = (c + 1 >= lo && c + 1 < hi) ? d1 : -INFINITY;
+                                            }
+                                            dmax = fmaxf(dmax, fmaxf(d0, d1));
+                                            const float a = ex2(d0), b2 = ex2(d1);
+                                            rs += a + b2;
+                                            pk[e] = pack_bf16x2(a, b2);
+                                        }
+                                        const uint32_t ra = pbase + ((uint32_t)(cb - hh * kPpUKeys) >> 3) * 2048u;
+                                        pp_st_async_v4(ra, pk[0], pk[1], pk[2], pk[3], pbar);
+                                        pp_st_async_v4(ra + 2048u, pk[4], pk[5], pk[6], pk[7], pbar);
+                                    }
+                                }
+                            }
+                        };
+                        for (int attempt = 0;; ++attempt) {
+                            const float mref = m == -INFINITY ? 0.f : m;
+                            if (unmasked)
+                                pass2(std::false_type{}, mref);
+                            else
+                                pass2(std::true_type{}, mref);
+                            if (need_max || attempt) break;
+                            // every row has a reference here; redo if a unit exceeded it
+                            float dother;
+                            exchange(dmax, &dother);
+                            dmax = fmaxf(dmax, dother);
+                            const bool over = dmax > kPfRescale;
+                            if (!__any_sync(0xffffffffu, over)) break;
+                            if (over) {
+                                al = ex2(-dmax);
+                                l *= al;
+                                m += dmax;
+                                resc = true;
+                            }
+                            attempts = 2;
+                        }
+                        l += rs;
+                        if (hh == nu - 1) {
+                            // every TMEM load of this warp from the tile has completed
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&bars[kBarSEmpty + sb]);
+                        }
+                        const bool last = j == nt - 1 && hh == nu - 1;
+                        float lrow = 0.f;
+                        if (last) {      // whole-row sums for the epilogue and the LSE
+                            float lother;
+                            exchange(l, &lother);
+                            lrow = l + lother;
+                        }
+                        if (hw == 0) {
+                            // unit header: rescale factor per row, per-quarter flag; then the arm:
+                            // this quarter's P bytes (both warps, every attempt) and header bytes
+                            const uint32_t hdr = rHdr + us * kPpHdrBytes;
+                            pp_st_async_u32(hdr + r * 4, __float_as_uint(al), pbar);
+                            const bool any = __any_sync(0xffffffffu, resc);
+                            if (lane == 0) {
+                                pp_st_async_u32(hdr + 512 + q4 * 4, any ? 1u : 0u, pbar);
+                                pp_remote_arrive_expect_tx(
+                                    pbar, (uint32_t)attempts * (uint32_t)(u_end - hh * kPpUKeys) * 64u + 32u * 4u + 4u);
+                            }
+                            if (last && row_live && p.lse)
+                                p.lse[((size_t)it.b * p.Hq + head) * p.T + tok] =
+                                    (m + log2f(lrow)) * 0.6931471805599453f;
                         }
                     }
-                    l += rs;
-                    // every TMEM load of this warp has completed: S may be overwritten
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[kBarSEmpty + sb]);
-                    // header of the slot: rescale factor per row, per-warp flag, row sums
-                    const uint32_t hdr = rHdr + sb * kPpHdrBytes;
-                    pp_st_cluster_u32(hdr + r * 4, __float_as_uint(al));
-                    if (j == nt - 1) pp_st_cluster_u32(hdr + 512 + r * 4, __float_as_uint(l));
-                    const bool any = __any_sync(0xffffffffu, resc);
-                    if (lane == 0) pp_st_cluster_u32(hdr + 1024 + q4 * 4, any ? 1u : 0u);
-                    pp_fence_proxy_async_cluster();
-                    __syncwarp();
-                    if (lane == 0) pp_remote_arrive(rPFull + sb * 8);
                 }
-                if (!ok) break;
-                if (row_live && p.lse)
-                    p.lse[((size_t)it.b * p.Hq + head) * p.T + tok] = (m + log2f(l)) * 0.6931471805599453f;
             }
         }
     }
@@ -492,20 +612,24 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                 for (int j = 0; ok && j < nt; ++j) {
                     const bool comp = j < it.nct;
                     const int row = pp_tile_row(it, j);
-                    const int nu = (pp_tile_keys(it, j) + 63) >> 6;
-                    for (int h = 0; ok && h < 2; ++h)
-                        for (int u = 0; u < nu; ++u) {
-                            const uint32_t st = vr % kPpRing;
-                            if (!mbar_wait(&bars[kBarVEmpty + st], ((vr / kPpRing) & 1) ^ 1, abort_flag)) {
-                                ok = false;
-                                break;
+                    const int nk = pp_tile_keys(it, j);
+                    for (int hh = 0; ok && hh < pp_units(nk); ++hh) {
+                        const int nv = (pp_unit_keys(nk, hh) + 63) >> 6;
+                        for (int h = 0; ok && h < 2; ++h)
+                            for (int u = 0; u < nv; ++u) {
+                                const uint32_t st = vr % kPpRing;
+                                if (!mbar_wait(&bars[kBarVEmpty + st], ((vr / kPpRing) & 1) ^ 1, abort_flag)) {
+                                    ok = false;
+                                    break;
+                                }
+                                mbar_arrive_expect_tx(&bars[kBarVFull + st], kPpUnit);
+                                for (int c = 0; c < 4; ++c)
+                                    tma_load_4d(sm + kPpSmRing + st * kPpUnit + c * kPpVSub, comp ? &tm_vc : &tm_v,
+                                                &bars[kBarVFull + st], 256 * h + 64 * c, it.g,
+                                                row + kPpUKeys * hh + 64 * u, it.b);
+                                ++vr;
                             }
-                            mbar_arrive_expect_tx(&bars[kBarVFull + st], kPpUnit);
-                            for (int c = 0; c < 4; ++c)
-                                tma_load_4d(sm + kPpSmRing + st * kPpUnit + c * kPpVSub, comp ? &tm_vc : &tm_v,
-                                            &bars[kBarVFull + st], 256 * h + 64 * c, it.g, row + 64 * u, it.b);
-                            ++vr;
-                        }
+                    }
                 }
             }
             pp_drain_ring(&bars[kBarVFull], vr);
@@ -513,53 +637,60 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
     } else if (!s_cta && warp == 1) {
         // ===================================================== O-CTA: O += P V
         if (go) {
-            uint32_t vr = 0;
-            int n = 0, item_n = 0;
+            uint32_t vr = 0, un = 0;
+            int item_n = 0;
             bool ok = true;
             const uint32_t p_base = smem_u32(sm + kPpSmP);
             const uint32_t id = idesc_bf16(128, 256, 0, 1);
             for (long long i = pair; ok && i < p.items; i += npairs, ++item_n) {
                 const PpItem it = pp_item(p, i);
                 const int nt = it.nct + it.nwt;
-                for (int j = 0; ok && j < nt; ++j, ++n) {
-                    const int sb = n & 1;
-                    if (!pp_warp_wait_cl(&bars[kBarPFull + sb], (n >> 1) & 1, abort_flag) ||
-                        !warp_wait(&bars[kBarCorr + sb], (n >> 1) & 1, abort_flag) ||
-                        (j == 0 && !warp_wait(&bars[kBarOEmpty], (item_n & 1) ^ 1, abort_flag))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                for (int j = 0; ok && j < nt; ++j) {
                     const int nk = pp_tile_keys(it, j);
-                    const int nu = (nk + 63) >> 6;
-                    for (int h = 0; ok && h < 2; ++h)
-                        for (int u = 0; u < nu; ++u) {
-                            const uint32_t st = vr % kPpRing;
-                            if (!warp_wait(&bars[kBarVFull + st], (vr / kPpRing) & 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            if (lane == 0) {
-                                const uint32_t vb = smem_u32(sm + kPpSmRing + st * kPpUnit);
-                                const uint32_t pa = p_base + sb * kPpPBuf + u * 16384;   // 16 keys = 4 KB
-#pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    if (64 * u + 16 * kk < nk)
-                                        mma_ss(tmem + 256 * h, pp_desc_noswz(pa + kk * 4096, 2048, 128),
-                                               smem_desc_sw128(vb + kk * 2048, kPpVSub, 1024), id,
-                                               (j == 0 && u == 0 && kk == 0) ? 0u : 1u);
-                                mma_commit(&bars[kBarVEmpty + st]);
-                            }
-                            __syncwarp();
-                            ++vr;
+                    const int nu = pp_units(nk);
+                    for (int hh = 0; hh < nu; ++hh, ++un) {
+                        const int us = (int)(un % kPpSlots);
+                        const uint32_t ph = (un / kPpSlots) & 1;
+                        const bool first = j == 0 && hh == 0;
+                        if (!pp_warp_wait_cl(&bars[kBarPFull + us], ph, abort_flag) ||
+                            !warp_wait(&bars[kBarCorr + us], ph, abort_flag) ||
+                            (first && !warp_wait(&bars[kBarOEmpty], (item_n & 1) ^ 1, abort_flag))) {
+                            ok = false;
+                            break;
                         }
-                    if (!ok) break;
-                    if (lane == 0) {
-                        mma_commit(&bars[kBarPCons + sb]);
-                        if (j == nt - 1) mma_commit(&bars[kBarOFull]);
+                        fence_proxy_async_smem();    // P arrived through the generic proxy
+                        tc_fence_after();
+                        const int nku = pp_unit_keys(nk, hh);
+                        const int nv = (nku + 63) >> 6;
+                        for (int h = 0; ok && h < 2; ++h)
+                            for (int u = 0; u < nv; ++u) {
+                                const uint32_t st = vr % kPpRing;
+                                if (!warp_wait(&bars[kBarVFull + st], (vr / kPpRing) & 1, abort_flag)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after();
+                                if (lane == 0) {
+                                    const uint32_t vb = smem_u32(sm + kPpSmRing + st * kPpUnit);
+                                    const uint32_t pa = p_base + us * kPpPBuf + u * 16384;   // 16 keys = 4 KB
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        if (64 * u + 16 * kk < nku)
+                                            mma_ss(tmem + 256 * h, pp_desc_noswz(pa + kk * 4096, 2048, 128),
+                                                   smem_desc_sw128(vb + kk * 2048, kPpVSub, 1024), id,
+                                                   (first && u == 0 && kk == 0) ? 0u : 1u);
+                                    mma_commit(&bars[kBarVEmpty + st]);
+                                }
+                                __syncwarp();
+                                ++vr;
+                            }
+                        if (!ok) break;
+                        if (lane == 0) {
+                            mma_commit(&bars[kBarPCons + us]);
+                            if (j == nt - 1 && hh == nu - 1) mma_commit(&bars[kBarOFull]);
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
             }
             if (lane == 0) {
@@ -574,103 +705,145 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
             const int q4 = warp & 3;
             const int r = q4 * 32 + lane;
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-            int n = 0, item_n = 0;
+            uint32_t un = 0;
+            int item_n = 0;
             bool ok = true;
             for (long long i = pair; ok && i < p.items; i += npairs, ++item_n) {
                 const PpItem it = pp_item(p, i);
                 const int nt = it.nct + it.nwt;
-                const int tok = it.t0 + r / p.G;
-                const bool row_live = tok < p.T;
-                const int head = it.g * p.G + (r % p.G);
-                float lfin = 1.f;
-                for (int j = 0; j < nt; ++j, ++n) {
-                    const int sb = n & 1;
-                    if (!pp_warp_wait_cl(&bars[kBarPFull + sb], (n >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint8_t* hdr = sm + kPpSmHdr + sb * kPpHdrBytes;
-                    const int flag = *reinterpret_cast<const volatile int*>(hdr + 1024 + q4 * 4);
-                    const float al = *reinterpret_cast<const volatile float*>(hdr + r * 4);
-                    if (j == nt - 1) lfin = *reinterpret_cast<const volatile float*>(hdr + 512 + r * 4);
-                    if (flag) {
-                        // a row of this warp moved its reference maximum (never on a first
-                        // tile): scale O once the PV of tile n-1 has landed
-                        if (!warp_wait(&bars[kBarPCons + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_flag)) {
+                float l = 0.f;            // row sum of the bf16 P this CTA multiplies with
+                for (int j = 0; ok && j < nt; ++j) {
+                    const int nk = pp_tile_keys(it, j);
+                    const int nu = pp_units(nk);
+                    for (int hh = 0; hh < nu; ++hh, ++un) {
+                        const int us = (int)(un % kPpSlots);
+                        if (!pp_warp_wait_cl(&bars[kBarPFull + us], (un / kPpSlots) & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
-                        tc_fence_after();
-#pragma unroll 1
-                        for (int c0 = 0; c0 < kPpD; c0 += 64) {
-                            float o[64];
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) tmem_ld16(tmem + lane_off + c0 + 16 * k, o + 16 * k);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                uint32_t w[16];
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(o[16 * k + e] * al);
-                                tmem_st16(tmem + lane_off + c0 + 16 * k, w);
-                            }
+                        const uint8_t* hdr = sm + kPpSmHdr + us * kPpHdrBytes;
+                        const int flag = *reinterpret_cast<const volatile int*>(hdr + 512 + q4 * 4);
+                        const float al = *reinterpret_cast<const volatile float*>(hdr + r * 4);
+                        // l = l * alpha + the unit's P of this row (8 keys per 16-byte chunk)
+                        float us_sum = 0.f;
+                        const uint8_t* prow = sm + kPpSmP + us * kPpPBuf + r * 16;
+                        const int nch = pp_unit_cols(nk, hh) >> 3;
+#pragma unroll 4
+                        for (int c = 0; c < nch; ++c) {
+                            const uint4 w = *reinterpret_cast<const uint4*>(prow + c * 2048);
+                            us_sum += (bf16lo(w.x) + bf16hi(w.x)) + (bf16lo(w.y) + bf16hi(w.y)) +
+                                      (bf16lo(w.z) + bf16hi(w.z)) + (bf16lo(w.w) + bf16hi(w.w));
                         }
-                        tmem_wait_st();
+                        l = l * al + us_sum;
+                        if (flag) {
+                            // a row of this warp moved its reference maximum (never in the first
+                            // unit of an item): scale O once the PV of unit un-1 has landed
+                            const uint32_t pu = un - 1;
+                            if (!warp_wait(&bars[kBarPCons + pu % kPpSlots], (pu / kPpSlots) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int c0 = 0; c0 < kPpD; c0 += 32) {
+                                float o[32];
+#pragma unroll
+                                for (int k = 0; k < 2; ++k) tmem_ld16(tmem + lane_off + c0 + 16 * k, o + 16 * k);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int k = 0; k < 2; ++k) {
+                                    uint32_t w[16];
+#pragma unroll
+                                    for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(o[16 * k + e] * al);
+                                    tmem_st16(tmem + lane_off + c0 + 16 * k, w);
+                                }
+                            }
+                            tmem_wait_st();
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars[kBarCorr + us]);
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[kBarCorr + sb]);
                 }
                 if (!ok) break;
-                // ---- epilogue: out = O / l
+                // ---- epilogue: out = O / l.  Each warp stages 32 rows x 128 bytes at a time in
+                // shared memory and writes them with one TMA tensor store (a coalesced box);
+                // per-lane row stores would touch 32 lines per instruction.
                 if (!warp_wait(&bars[kBarOFull], item_n & 1, abort_flag)) break;
                 tc_fence_after();
-                const float inv = 1.f / lfin;
-                const size_t orow = (((size_t)it.b * p.T + tok) * p.Hq + head) * (size_t)kPpD;
+                const float inv = 1.f / l;
+                const bool f32 = (p.flags & HCA_OUT_F32) != 0;
+                uint8_t* stg = sm + kPpSmStage + q4 * kPpStageWarp;
+                const int r0 = q4 * 32;                       // first row of this warp's box
+                const int tok0 = it.t0 + r0 / p.G, head0 = it.g * p.G + r0 % p.G;
+                const bool live = tok0 < p.T;                 // rows past T are clipped by the store
+                // a piece is 4 KB: 32 rows x 64 columns of bf16, or x 32 columns of fp32
+                const int pw = f32 ? 32 : 64;
 #pragma unroll 1
-                for (int c0 = 0; c0 < kPpD; c0 += 32) {
-                    float o[32];
-                    tmem_ld16(tmem + lane_off + c0, o);
-                    tmem_ld16(tmem + lane_off + c0 + 16, o + 16);
-                    tmem_wait_ld();
-                    if (row_live) {
-                        if (p.flags & HCA_OUT_F32) {
-                            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + c0);
+                for (int c0 = 0, k = 0; c0 < kPpD; c0 += pw, ++k) {
+                    uint8_t* buf = stg + (k & 1) * (kPpStageWarp / 2);
+                    if (k >= 2 && lane == 0) pp_bulk_wait_read1();     // the store of piece k-2 read it
+                    __syncwarp();
+                    if (f32) {
+                        float o[32];
+                        tmem_ld16(tmem + lane_off + c0, o);
+                        tmem_ld16(tmem + lane_off + c0 + 16, o + 16);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                dst[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv,
-                                                     o[4 * k + 3] * inv);
-                        } else {
-                            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow + c0);
+                        for (int e = 0; e < 8; ++e)       // 128-byte swizzle: chunk e of row lane
+                            *reinterpret_cast<float4*>(buf + lane * 128 + (((e ^ lane) & 7) << 4)) =
+                                make_float4(o[4 * e] * inv, o[4 * e + 1] * inv, o[4 * e + 2] * inv,
+                                            o[4 * e + 3] * inv);
+                    } else {
 #pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                dst[k] = make_uint4(pack_bf16x2(o[8 * k] * inv, o[8 * k + 1] * inv),
-                                                    pack_bf16x2(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
-                                                    pack_bf16x2(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
-                                                    pack_bf16x2(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
+                        for (int hv = 0; hv < 2; ++hv) {
+                            float o[32];
+                            tmem_ld16(tmem + lane_off + c0 + 32 * hv, o);
+                            tmem_ld16(tmem + lane_off + c0 + 32 * hv + 16, o + 16);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)   // 128-byte swizzle: chunk 4 hv + e of row lane
+                                *reinterpret_cast<uint4*>(buf + lane * 128 + ((((4 * hv + e) ^ lane) & 7) << 4)) =
+                                    make_uint4(pack_bf16x2(o[8 * e] * inv, o[8 * e + 1] * inv),
+                                               pack_bf16x2(o[8 * e + 2] * inv, o[8 * e + 3] * inv),
+                                               pack_bf16x2(o[8 * e + 4] * inv, o[8 * e + 5] * inv),
+                                               pack_bf16x2(o[8 * e + 6] * inv, o[8 * e + 7] * inv));
                         }
                     }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && live) {
+                        pp_tma_store_4d(&tm_out, buf, c0, head0, tok0, it.b);
+                        pp_bulk_commit();
+                    }
                 }
+                if (lane == 0) pp_bulk_wait_read0();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[kBarOEmpty]);
             }
+            if (lane == 0) pp_bulk_wait_all();     // every output store has completed
+            __syncwarp();
         }
-    } else if (!s_cta && warp == 6) {
+    } else if (!s_cta && warp == 7) {
         // ===================================================== O-CTA: P slot consumed -> S-CTA
         if (lane == 0 && go) {
             const uint32_t rPEmpty = peer_base + kPpSmBar + kBarPEmpty * 8;
-            int n = 0;
+            uint32_t un = 0;
             bool ok = true;
             for (long long i = pair; ok && i < p.items; i += npairs) {
                 const PpItem it = pp_item(p, i);
                 const int nt = it.nct + it.nwt;
-                for (int j = 0; j < nt; ++j, ++n) {
-                    if (!mbar_wait(&bars[kBarPCons + (n & 1)], (n >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
+                for (int j = 0; ok && j < nt; ++j) {
+                    const int nu = pp_units(pp_tile_keys(it, j));
+                    for (int hh = 0; hh < nu; ++hh, ++un) {
+                        const int us = (int)(un % kPpSlots);
+                        if (!mbar_wait(&bars[kBarPCons + us], (un / kPpSlots) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        pp_remote_arrive(rPEmpty + us * 8);
                     }
-                    pp_remote_arrive(rPEmpty + (n & 1) * 8);
                 }
             }
         }
