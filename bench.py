@@ -400,11 +400,8 @@ def main():
         pin = wl.prefill_inputs(pc, dev)
         pkc, pvc = hca.compress(pin["k"], pin["v"], pin["w"], pc.blk)
         pout = torch.empty((1, pc.T, pc.Hq, pc.dv), dtype=torch.bfloat16, device=dev)
-        pws = torch.empty(max(1, hca.prefill_workspace_size(1, pc.T, pc.Hq, pc.Hkv, pc.d, pc.dv)), dtype=torch.uint8,
-                          device=dev)
         for _ in range(2):
-            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout,
-                        workspace=pws)
+            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
         torch.cuda.synchronize()
         hca.get_device_error()
         np_steps = max(2, min(args.steps, 5))
@@ -416,8 +413,7 @@ def main():
             a.record(stream)
             hca.compress(pin["k"], pin["v"], pin["w"], pc.blk, kc=pkc, vc=pvc)
             m.record(stream)
-            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout,
-                        workspace=pws)
+            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
             b.record(stream)
         torch.cuda.synchronize()
         hca.get_device_error()
@@ -434,7 +430,7 @@ def main():
                                      "frac_of_burst": tf / pk["bf16_tflops"],
                                      "traffic": traffic_for("prefill_T131072",
                                                             ["compressed_long_context_b200/csrc/prefill.cuh"])}}
-        del pin, pkc, pvc, pout, pws
+        del pin, pkc, pvc, pout
         torch.cuda.empty_cache()
 
     cpu_base = None

@@ -16,8 +16,8 @@ from . import _lib
 from ._lib import (HCA_OUT_F32, HCA_OUT_GATE, HCA_PAGED, HCA_QK_NORM,  # noqa: F401
                    HCA_WRITE_LSE)
 
-__all__ = ["HCAError", "compress", "prefill", "prefill_workspace_size", "decode", "decode_workspace_size",
-           "get_device_error", "status_string"]
+__all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "get_device_error",
+           "status_string"]
 
 
 class HCAError(RuntimeError):
@@ -86,16 +86,8 @@ def compress(k, v, w=None, blk=128, kc=None, vc=None):
     return kc, vc
 
 
-def prefill_workspace_size(B, T, Hq, Hkv, d, dv) -> int:
-    """Bytes of scratch ``prefill`` needs on the current device (0 when none)."""
-    return int(_lib.load().hca_prefill_workspace_size(B, T, Hq, Hkv, d, dv))
-
-
-def prefill(q, k, v, kc, vc, blk, W, scale, out=None, want_lse=False, out_f32=False, workspace=None):
-    """Causal HCA attention for every position.  Returns out [B,T,Hq,dv] (and lse [B,Hq,T]).
-
-    ``workspace``: a uint8 device tensor of at least ``prefill_workspace_size`` bytes; one is
-    allocated per call when it is not given."""
+def prefill(q, k, v, kc, vc, blk, W, scale, out=None, want_lse=False, out_f32=False):
+    """Causal HCA attention for every position.  Returns out [B,T,Hq,dv] (and lse [B,Hq,T])."""
     _need(q, torch.bfloat16, "q")
     for name, t in (("k", k), ("v", v), ("kc", kc), ("vc", vc)):
         _need(t, torch.bfloat16, name, q.device)
@@ -106,12 +98,8 @@ def prefill(q, k, v, kc, vc, blk, W, scale, out=None, want_lse=False, out_f32=Fa
     _need(out, torch.float32 if out_f32 else torch.bfloat16, "out", q.device)
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device) if want_lse else None
     flags = (HCA_WRITE_LSE if want_lse else 0) | (HCA_OUT_F32 if out_f32 else 0)
-    if workspace is None:
-        n = prefill_workspace_size(B, T, Hq, Hkv, d, dv)
-        workspace = torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
-    ws_bytes = workspace.numel() if workspace is not None else 0
-    rc = _lib.load().hca_prefill(_p(q), _p(k), _p(v), _p(kc), _p(vc), _p(out), _p(lse), _p(workspace), ws_bytes,
-                                 B, T, Hq, Hkv, d, dv, blk, W, float(scale), flags, _stream(q.device))
+    rc = _lib.load().hca_prefill(_p(q), _p(k), _p(v), _p(kc), _p(vc), _p(out), _p(lse), B, T, Hq, Hkv, d, dv,
+                                 blk, W, float(scale), flags, _stream(q.device))
     _check(rc, "hca_prefill")
     return (out, lse) if want_lse else out
 

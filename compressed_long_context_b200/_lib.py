@@ -20,8 +20,8 @@ HCA_WRITE_LSE = 8
 HCA_OUT_F32 = 16
 
 # Names of every entry point declared in include/hca.h.
-EXPORTS = ("hca_compress", "hca_prefill_workspace_size", "hca_prefill", "hca_decode_workspace_size", "hca_decode",
-           "hca_decode_noalloc", "hca_status_string", "hca_get_device_error")
+EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_decode", "hca_decode_noalloc",
+           "hca_status_string", "hca_get_device_error")
 
 _lib = None
 
@@ -47,10 +47,8 @@ def load():
     lib.hca_get_device_error.argtypes = [_vp]
     lib.hca_compress.restype = _i
     lib.hca_compress.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 6 + [_vp]
-    lib.hca_prefill_workspace_size.restype = _sz
-    lib.hca_prefill_workspace_size.argtypes = [_i] * 6
     lib.hca_prefill.restype = _i
-    lib.hca_prefill.argtypes = [_vp] * 7 + [_vp, _sz] + [_i] * 8 + [_f, _u, _vp]
+    lib.hca_prefill.argtypes = [_vp] * 7 + [_i] * 8 + [_f, _u, _vp]
     lib.hca_decode_workspace_size.restype = _sz
     lib.hca_decode_workspace_size.argtypes = [_i] * 4
     lib.hca_decode.restype = _i

@@ -336,16 +336,12 @@ int pair_clusters_resident(cudaStream_t s) {
 
 hca_status_t launch_prefill_pair(const hca::PrefillParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& tkc, const CUtensorMap& tvc,
-                                 const CUtensorMap& tout, size_t ws_bytes, cudaStream_t s) {
+                                 const CUtensorMap& tout, cudaStream_t s) {
     if (!hca::set_smem_attr_once(reinterpret_cast<const void*>(&hca::prefill_pair_kernel), (int)hca::kPpSmem, 3))
         return HCA_ERR_CUDA;
     const int nc = pair_clusters_resident(s);
     if (nc <= 0) return HCA_ERR_CUDA;
     const long long npairs = p.items < nc ? p.items : nc;
-    // the P hand-off slots of every pair
-    if (!p.scratch || (reinterpret_cast<uintptr_t>(p.scratch) & 127) ||
-        ws_bytes < (size_t)npairs * hca::kPpSlots * hca::kPpSlotStride)
-        return HCA_ERR_INVALID_ARG;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -367,15 +363,8 @@ hca_status_t launch_prefill_pair(const hca::PrefillParams& p, const CUtensorMap&
 
 }  // namespace
 
-extern "C" size_t hca_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d, int dv) {
-    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || d != dv) return 0;
-    if (d != 512) return 0;       // only the 512-dim (CTA pair) kernel uses scratch
-    const int nc = pair_clusters_resident(nullptr);
-    return nc > 0 ? (size_t)nc * hca::kPpSlots * hca::kPpSlotStride : 0;
-}
-
 extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v, const void* kc, const void* vc,
-                                    void* out, float* lse, void* workspace, size_t ws_bytes,
+                                    void* out, float* lse,
                                     int B, int T, int Hq, int Hkv, int d, int dv, int blk,
                                     int W, float scale, unsigned flags, hca_stream_t stream) {
     using namespace hca;
@@ -396,7 +385,6 @@ extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v,
     PrefillParams p;
     p.out = out;
     p.lse = want_lse ? lse : nullptr;
-    p.scratch = static_cast<uint8_t*>(workspace);
     p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.tpt = 128 / G; p.blk = blk; p.W = W; p.Nc = Nc;
     p.ntile_t = (T + p.tpt - 1) / p.tpt;
     p.flags = (int)flags;
@@ -428,7 +416,7 @@ extern "C" hca_status_t hca_prefill(const void* q, const void* k, const void* v,
     const int es = (flags & HCA_OUT_F32) ? 4 : 2;
     if (!make_tmap_4d_plain(&tout, out, es, D, Hq, T, B, D, D * Hq, D * Hq * T, 128 / es, bh, bt, 1))
         return HCA_ERR_CUDA;
-    return launch_prefill_pair(p, tq, tk, tv, tkc, tvc, tout, ws_bytes, s);
+    return launch_prefill_pair(p, tq, tk, tv, tkc, tvc, tout, s);
 }
 
 

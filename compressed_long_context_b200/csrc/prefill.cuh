@@ -56,7 +56,6 @@ struct PfCfg {
 struct PrefillParams {
     void* out;          // [B, T, Hq, dv] bf16 or fp32
     float* lse;         // [B, Hq, T] or null
-    uint8_t* scratch;   // pair kernel: 2 P slots of 64 KB per CTA pair (caller's workspace)
     int B, T, Hq, Hkv, G, tpt, blk, W, Nc, ntile_t, flags;
     long long items;
     float scale_log2;

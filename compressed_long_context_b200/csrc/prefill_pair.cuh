@@ -56,7 +56,6 @@ constexpr uint32_t kPpUnit = 32768;              // K: 256 keys x 64 ch; V: 64 k
 constexpr uint32_t kPpVSub = 8192;               // V unit = 4 channel slabs of 64 keys x 64 ch
 constexpr uint32_t kPpPBuf = 32768;              // P unit: 128 rows x 128 keys, 16 key chunks of 2 KB
 constexpr uint32_t kPpHdrBytes = 528;            // per P unit: alpha[128], flag[4]
-constexpr uint32_t kPpSlotStride = kPpPBuf + 512; // global slot: P unit, then l[128] after an item's last unit
 // shared-memory layout (offsets from a 1024-aligned base); the two ranks reuse offsets
 constexpr uint32_t kPpSmQ = 0;                   // S-CTA: Q, 8 slabs (128 KB)
 constexpr uint32_t kPpSmP = 0;                   // O-CTA: P, 3 units (96 KB)
@@ -73,7 +72,6 @@ constexpr uint32_t kPpSmem = kPpSmMisc + 16;
 static_assert(kPpSmem <= 232448, "pair prefill shared memory exceeds the 227 KB per-block limit");
 static_assert(kPpSmHdr % 16 == 0 && kPpSmBar % 8 == 0 && kPpSmMisc % 16 == 0,
               "header 16-aligned, barriers 8-aligned");
-static_assert(kPpSlotStride % 128 == 0, "global slots 128-aligned");
 static_assert(kPpKeys == 2 * kPpUKeys, "an S tile is two P units");
 static_assert(kPpSmStage + 4 * kPpStageWarp <= kPpSmRing, "output staging fits below the ring");
 
@@ -81,7 +79,7 @@ static_assert(kPpSmStage + 4 * kPpStageWarp <= kPpSmRing, "output staging fits b
 enum : int {
     kBarKFull = 0, kBarKEmpty = 3, kBarQFull = 6, kBarQEmpty = 7, kBarSFull = 8, kBarSEmpty = 10,
     kBarPEmpty = 12,                                                       // S-CTA (+ [4])
-    kBarVFull = 16, kBarVEmpty = 19, kBarPFull = 22, kBarCorr = 26, kBarPCons = 30, kBarPLoaded = 34,
+    kBarVFull = 16, kBarVEmpty = 19, kBarPFull = 22, kBarCorr = 26, kBarPCons = 30,
     kBarOFull = 38, kBarOEmpty = 39,                                       // O-CTA
     kBarDrain = 40
 };
@@ -169,14 +167,7 @@ __device__ __forceinline__ void pp_bulk_wait_all() { asm volatile("cp.async.bulk
 __device__ __forceinline__ void pp_st_cluster_u32(uint32_t raddr, uint32_t v) {
     asm volatile("st.shared::cluster.b32 [%0], %1;" :: "r"(raddr), "r"(v) : "memory");
 }
-__device__ __forceinline__ void pp_fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-// bulk copy global -> this CTA's shared memory, completion counted in bytes on `bar`
-__device__ __forceinline__ void pp_bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
+
 // try_wait with acquire at cluster scope: for barriers the peer CTA arrives on
 __device__ __forceinline__ bool pp_try_wait_cl(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
@@ -277,7 +268,6 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
             mbar_init(&bars[kBarPFull + i], 4);        // armed by each TMEM lane quarter
             mbar_init(&bars[kBarCorr + i], 4);
             mbar_init(&bars[kBarPCons + i], 1);
-            mbar_init(&bars[kBarPLoaded + i], 1);
         }
         mbar_init(&bars[kBarOFull], 1);
         mbar_init(&bars[kBarOEmpty], 4);

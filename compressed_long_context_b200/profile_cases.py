@@ -16,7 +16,7 @@ import math
 
 import torch
 
-from . import compress, decode, decode_workspace_size, get_device_error, prefill, prefill_workspace_size
+from . import compress, decode, decode_workspace_size, get_device_error, prefill
 from . import workloads as wl
 
 
@@ -76,10 +76,8 @@ def run(case: str, reps: int, B_override: int = 0, L_override: int = 0) -> dict:
         inp = wl.prefill_inputs(cfg, dev)
         kc, vc = compress(inp["k"], inp["v"], inp["w"], 128)
         out = torch.empty((1, cfg.T, cfg.Hq, cfg.dv), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(max(1, prefill_workspace_size(1, cfg.T, cfg.Hq, cfg.Hkv, cfg.d, cfg.dv)), dtype=torch.uint8,
-                         device=dev)
         fn = lambda: prefill(inp["q"], inp["k"], inp["v"], kc, vc, 128, cfg.W, 1 / math.sqrt(cfg.d),  # noqa: E731
-                             out=out, workspace=ws)
+                             out=out)
         keys = sum(max(0, (t - cfg.W + 1) // 128) + min(cfg.W, t + 1) for t in range(cfg.T))
         nbytes = None
         flops = 2.0 * cfg.Hq * keys * (cfg.d + cfg.dv)

@@ -88,14 +88,6 @@ hca_status_t hca_compress(const void* k, const void* v, const float* w,
                           hca_stream_t stream);
 
 /*
- * hca_prefill_workspace_size -- bytes of device workspace hca_prefill needs on the CURRENT
- * device: four hand-off slots of 32.5 KB per pair of SMs for d == dv == 512 (the
- * probabilities of 128 keys pass from the SM that computes them to the SM that holds the
- * output accumulator), 0 when no workspace is needed (d == dv == 64) or the sizes are invalid.
- */
-size_t hca_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d, int dv);
-
-/*
  * hca_prefill -- causal HCA attention for every position of B sequences of T tokens
  * (official blog, section 2.1; Zhidx article, section 1).
  *   q  [B,T,Hq,d]    bf16
@@ -106,16 +98,13 @@ size_t hca_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d, int dv);
  *   out [B,T,Hq,dv]  bf16, or fp32 with HCA_OUT_F32
  *   lse [B,Hq,T]     fp32 natural-log sum-exp of the logits, written iff HCA_WRITE_LSE
  *                    (may be NULL otherwise)
- *   workspace, ws_bytes  device scratch of at least hca_prefill_workspace_size(...) bytes,
- *                    128-byte aligned, owned by the caller, no initialisation needed (NULL/0
- *                    when that size is 0); calls that overlap on the GPU need separate ones
  *   scale            logit scale (typically 1/sqrt(d))
  * Supported: d == dv in {64, 512}; Hq % Hkv == 0 with Hq / Hkv a power of two <= 128;
  * 1 <= blk <= 128; W >= 1; flags among HCA_WRITE_LSE | HCA_OUT_F32.
  */
 hca_status_t hca_prefill(const void* q, const void* k, const void* v,
                          const void* kc, const void* vc,
-                         void* out, float* lse, void* workspace, size_t ws_bytes,
+                         void* out, float* lse,
                          int B, int T, int Hq, int Hkv, int d, int dv, int blk, int W,
                          float scale, unsigned flags, hca_stream_t stream);
 

@@ -75,30 +75,27 @@ def test_compress_rejects_before_launch(libhca):
 
 def test_prefill_rejects_before_launch(libhca):
     p = ctypes.c_void_p(16)
-    # (q, k, v, kc, vc, out, lse, workspace, ws_bytes, B, T, Hq, Hkv, d, dv, blk, W, scale, flags, stream)
+    # (q, k, v, kc, vc, out, lse, B, T, Hq, Hkv, d, dv, blk, W, scale, flags, stream)
     # unsupported head dims, block, group size, flags
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 96, 96, 128, 128, 0.1, 0,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 4, 1, 96, 96, 128, 128, 0.1, 0,
                               None) == _lib.HCA_ERR_UNSUPPORTED
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 64, 512, 128, 128, 0.1, 0,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 4, 1, 64, 512, 128, 128, 0.1, 0,
                               None) == _lib.HCA_ERR_UNSUPPORTED
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 64, 64, 129, 128, 0.1, 0,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 4, 1, 64, 64, 129, 128, 0.1, 0,
                               None) == _lib.HCA_ERR_UNSUPPORTED
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 6, 2, 64, 64, 128, 128, 0.1, 0,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 6, 2, 64, 64, 128, 128, 0.1, 0,
                               None) == _lib.HCA_ERR_UNSUPPORTED
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 64, 64, 128, 128, 0.1, 1 << 8,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 4, 1, 64, 64, 128, 128, 0.1, 1 << 8,
                               None) == _lib.HCA_ERR_UNSUPPORTED
     # null pointers, bad sizes, NaN scale, LSE requested without a buffer
-    assert libhca.hca_prefill(None, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 64, 64, 128, 128, 0.1, 0,
+    assert libhca.hca_prefill(None, p, p, p, p, p, None, 1, 256, 4, 1, 64, 64, 128, 128, 0.1, 0,
                               None) == _lib.HCA_ERR_INVALID_ARG
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 64, 64, 128, 0, 0.1, 0,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 4, 1, 64, 64, 128, 0, 0.1, 0,
                               None) == _lib.HCA_ERR_INVALID_ARG
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 64, 64, 128, 128, float("nan"), 0,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 4, 1, 64, 64, 128, 128, float("nan"), 0,
                               None) == _lib.HCA_ERR_INVALID_ARG
-    assert libhca.hca_prefill(p, p, p, p, p, p, None, None, 0, 1, 256, 4, 1, 64, 64, 128, 128, 0.1,
+    assert libhca.hca_prefill(p, p, p, p, p, p, None, 1, 256, 4, 1, 64, 64, 128, 128, 0.1,
                               _lib.HCA_WRITE_LSE, None) == _lib.HCA_ERR_INVALID_ARG
     # nothing to do: no launch, OK
-    assert libhca.hca_prefill(None, None, None, None, None, None, None, None, 0, 0, 256, 4, 1, 512, 512, 128, 128,
+    assert libhca.hca_prefill(None, None, None, None, None, None, None, 0, 256, 4, 1, 512, 512, 128, 128,
                               0.1, 0, None) == _lib.HCA_OK
-    # the 64-dim kernel needs no workspace
-    assert libhca.hca_prefill_workspace_size(1, 256, 4, 1, 64, 64) == 0
-    assert libhca.hca_prefill_workspace_size(1, 256, 4, 1, 64, 96) == 0

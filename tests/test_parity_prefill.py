@@ -177,20 +177,3 @@ def test_prefill_128k_workload_sampled(cuda_device, libhca):
     del inp, kc, vc, out, lse
     torch.cuda.empty_cache()
 
-
-def test_prefill_workspace_checked(cuda_device, libhca):
-    """A 512-dim prefill without (enough) workspace is rejected before launch."""
-    dev = cuda_device
-    q = torch.zeros((1, 256, 64, 512), dtype=torch.bfloat16, device=dev)
-    k = torch.zeros((1, 256, 1, 512), dtype=torch.bfloat16, device=dev)
-    kc = torch.zeros((1, 2, 1, 512), dtype=torch.bfloat16, device=dev)
-    need = hca.prefill_workspace_size(1, 256, 64, 1, 512, 512)
-    assert need > 0 and need % 128 == 0
-    small = torch.empty(need // 2, dtype=torch.uint8, device=dev)
-    with pytest.raises(hca.HCAError):
-        hca.prefill(q, k, k, kc, kc, 128, 128, 0.05, workspace=small)
-    ok = torch.empty(need, dtype=torch.uint8, device=dev)
-    out = hca.prefill(q, k, k, kc, kc, 128, 128, 0.05, workspace=ok)
-    torch.cuda.synchronize()
-    hca.get_device_error()
-    assert torch.isfinite(out.float()).all()
