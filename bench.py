@@ -81,30 +81,55 @@ def prefill_flops(B, T, Hq, d, dv, blk, W):
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of this process's GPU, sampled every 20 ms while the
+    timed regions run (NVML; nvidia-smi at 200 ms if NVML is unavailable).  Reads only."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index):
-        self.index = index
-        self.samples = []
+    def __init__(self, device_index):
+        self.device_index = device_index
+        self.samples = []          # (sm_mhz, max_mhz, reason bits)
         self._stop = threading.Event()
         self._t = None
+        self._nvml = None
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            prop = torch.cuda.get_device_properties(device_index)
+            bus = "%08X:%02X:%02X.0" % (getattr(prop, "pci_domain_id", 0), prop.pci_bus_id, prop.pci_device_id)
+            self._handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nvml = pynvml
+        except Exception:
+            self._nvml = None
+
+    def _sample_nvml(self):
+        n = self._nvml
+        sm = n.nvmlDeviceGetClockInfo(self._handle, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(self._handle, n.NVML_CLOCK_SM)
+        try:
+            bits = n.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+        except Exception:
+            bits = n.nvmlDeviceGetCurrentClocksThrottleReasons(self._handle)
+        return float(sm), float(mx), int(bits)
+
+    def _sample_smi(self):
+        out = subprocess.run(["nvidia-smi", "-i", str(self.device_index), "--query-gpu=clocks.sm,clocks.max.sm,"
+                              "clocks_event_reasons.active", "--format=csv,noheader,nounits"],
+                             capture_output=True, text=True, timeout=5).stdout.strip().split(",")
+        return float(out[0]), float(out[1]), int(out[2].strip(), 16)
 
     def _run(self):
+        period = 0.02 if self._nvml else 0.2
         while not self._stop.is_set():
             try:
-                out = subprocess.run(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                                     timeout=5).stdout.strip()
-                if out:
-                    self.samples.append([x.strip() for x in out.split(",")])
+                self.samples.append(self._sample_nvml() if self._nvml else self._sample_smi())
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(period)
 
     def __enter__(self):
+        self._stop.clear()
         self._t = threading.Thread(target=self._run, daemon=True)
         self._t.start()
         return self
@@ -114,13 +139,11 @@ class ClockSampler:
         self._t.join(timeout=10)
 
     def summary(self):
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if len(s) > 2 + i and s[2 + i].lower().startswith("active")})
+        sm = [x[0] for x in self.samples]
+        mx = [x[1] for x in self.samples]
+        reasons = sorted({name for _, _, bits in self.samples for b, name in self.REASONS.items() if bits & b})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml" if self._nvml else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------- helpers
@@ -231,24 +254,32 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_sample():
-    """The oracle as it stands, on this host, for a bounded sample: 2 sequences of the workload."""
+def cpu_baseline_sample(target_s=10.0):
+    """The oracle as it stands, on this host, for a bounded sample of the workload: batches of
+    2 sequences (compress of their raw K/V + decode of their queries), repeated for about
+    ``target_s`` seconds."""
     import oracle
     from compressed_long_context_b200 import workloads as wl
     cfg = wl.DECODE_128K
     n = 2
     inp = wl.decode_inputs(cfg.scaled(B=n), "cpu")
     kb, vb = oracle.bf16_bits(inp["k"]), oracle.bf16_bits(inp["v"])
+    w = inp["w"].numpy()
+    qb, kwb, vwb = oracle.bf16_bits(inp["q"]), oracle.bf16_bits(inp["kw"]), oracle.bf16_bits(inp["vw"])
+    seq = inp["seqlens"].numpy()
     scale = 1.0 / np.sqrt(cfg.d)
+    reps = 0
     t0 = time.perf_counter()
-    kc, vc = oracle.compress(kb, vb, inp["w"].numpy(), cfg.blk)
-    oracle.decode(oracle.bf16_bits(inp["q"]), oracle.round_bf16(kc), oracle.round_bf16(vc),
-                  oracle.bf16_bits(inp["kw"]), oracle.bf16_bits(inp["vw"]), inp["seqlens"].numpy(), cfg.blk,
-                  cfg.W, scale)
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "queries/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "%d sequences of the workload: oracle fp64 compress (131072 raw tokens, K and V) + decode "
-                      "(64 heads, 1023 entries + 128 window), %.1f s" % (n, dt)}
+    while True:
+        kc, vc = oracle.compress(kb, vb, w, cfg.blk)
+        oracle.decode(qb, oracle.round_bf16(kc), oracle.round_bf16(vc), kwb, vwb, seq, cfg.blk, cfg.W, scale)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s:
+            break
+    return {"value": n * reps / dt, "unit": "queries/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d passes over 2 sequences of the workload (oracle fp64 compress of 131072 raw tokens, K and "
+                      "V, + decode of 64 heads over 1023 entries + 128 window tokens), %.1f s" % (reps, dt)}
 
 
 # ---------------------------------------------------------------- our arm
@@ -328,14 +359,15 @@ def main():
     # the events then bracket device work only, not host launch overhead.
     dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
-    torch.cuda._sleep(int(2e8))
-    for i in range(args.steps):
-        flush.zero_()
-        a, b = dev_ev[i]
-        a.record(stream)
-        hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
-        b.record(stream)
-    torch.cuda.synchronize()
+    with sampler:
+        torch.cuda._sleep(int(2e8))
+        for i in range(args.steps):
+            flush.zero_()
+            a, b = dev_ev[i]
+            a.record(stream)
+            hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
+            b.record(stream)
+        torch.cuda.synchronize()
     d_ms = [a.elapsed_time(b) for a, b in dev_ev]
     d_avg = max_over_ranks(sum(d_ms) / len(d_ms) / 1e3, world)
     dbytes = decode_bytes(B, L, cfg.Hq, 1, cfg.d, cfg.dv, cfg.blk, cfg.W)
@@ -407,15 +439,16 @@ def main():
         np_steps = max(2, min(args.steps, 5))
         pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
                 torch.cuda.Event(enable_timing=True)) for _ in range(np_steps)]
-        for i in range(np_steps):
-            flush.zero_()
-            a, m, b = pev[i]
-            a.record(stream)
-            hca.compress(pin["k"], pin["v"], pin["w"], pc.blk, kc=pkc, vc=pvc)
-            m.record(stream)
-            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
-            b.record(stream)
-        torch.cuda.synchronize()
+        with sampler:
+            for i in range(np_steps):
+                flush.zero_()
+                a, m, b = pev[i]
+                a.record(stream)
+                hca.compress(pin["k"], pin["v"], pin["w"], pc.blk, kc=pkc, vc=pvc)
+                m.record(stream)
+                hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
+                b.record(stream)
+            torch.cuda.synchronize()
         hca.get_device_error()
         p_ms = max_over_ranks(statistics.median([m.elapsed_time(b) for _, m, b in pev]), world)
         c3_ms = statistics.median([a.elapsed_time(m) for a, m, _ in pev])
@@ -424,12 +457,13 @@ def main():
         peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
         prefill_part = {"workload": pc.name, "tflops": tf, "ms": p_ms, "compress_ms": c3_ms,
                         "algorithmic_flops": flops, "keys_per_head": keys,
-                        "roofline": {"bound": "tensor", "kernel": "prefill_kernel<512>", "achieved": tf,
+                        "roofline": {"bound": "tensor", "kernel": "prefill_pair_kernel", "achieved": tf,
                                      "peak": peak_tf, "unit": "TFLOP/s", "frac": tf / peak_tf,
                                      "peak_kind": pk_kind + " (bf16_tflops_sustained)",
                                      "frac_of_burst": tf / pk["bf16_tflops"],
                                      "traffic": traffic_for("prefill_T131072",
-                                                            ["compressed_long_context_b200/csrc/prefill.cuh"])}}
+                                                            ["compressed_long_context_b200/csrc/prefill.cuh",
+                                                             "compressed_long_context_b200/csrc/prefill_pair.cuh"])}}
         del pin, pkc, pvc, pout
         torch.cuda.empty_cache()
 

@@ -27,7 +27,7 @@ def _events():
     return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
 
-def run(case: str, reps: int, B_override: int = 0, L_override: int = 0) -> dict:
+def run(case: str, reps: int, B_override: int = 0, L_override: int = 0, T_override: int = 0) -> dict:
     dev = torch.device("cuda", torch.cuda.current_device())
     g = torch.Generator(device=dev).manual_seed(123)
     if case == "compress":
@@ -71,8 +71,8 @@ def run(case: str, reps: int, B_override: int = 0, L_override: int = 0) -> dict:
                                 page_size=ps, gq=gq, gk=gk, gate=gate, out=out, workspace=ws)
         nbytes = B * (Hq * d * 2 + (nc + W) * 2 * d * 2 + Hq * d * 4)
     elif case == "prefill":
-        # T = 16384 tokens, 64 heads of 512: 1 GB of Q, 1 GB of output
-        cfg = wl.PREFILL_128K.scaled(T=16384)
+        # default T = 16384 tokens, 64 heads of 512: 1 GB of Q, 1 GB of output
+        cfg = wl.PREFILL_128K.scaled(T=T_override or 16384)
         inp = wl.prefill_inputs(cfg, dev)
         kc, vc = compress(inp["k"], inp["v"], inp["w"], 128)
         out = torch.empty((1, cfg.T, cfg.Hq, cfg.dv), dtype=torch.bfloat16, device=dev)
@@ -102,6 +102,7 @@ def run(case: str, reps: int, B_override: int = 0, L_override: int = 0) -> dict:
         res["bytes"] = nbytes
         res["GB_per_s"] = nbytes / (ms / 1e3) / 1e9
     if case == "prefill":
+        res["T"] = cfg.T
         res["TFLOP_per_s"] = flops / (ms / 1e3) / 1e12
     return res
 
@@ -110,7 +111,7 @@ def run_flushed(args) -> dict:
     """Per-launch device time with L2 flushed before every launch (a GPU spin is queued first
     so that launches are enqueued ahead of the GPU)."""
     import statistics
-    res = run(args.case, 1, args.B, args.L)
+    res = run(args.case, 1, args.B, args.L, args.T)
     fn = _last_fn[0]
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
     buf = torch.empty(2 * l2, dtype=torch.uint8, device="cuda")
@@ -136,9 +137,10 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--B", type=int, default=0, help="decode batch (default 64)")
     ap.add_argument("--L", type=int, default=0, help="decode context length (default 131072)")
+    ap.add_argument("--T", type=int, default=0, help="prefill tokens (default 16384)")
     ap.add_argument("--flush", action="store_true", help="flush L2 before every launch (events per launch)")
     args = ap.parse_args()
-    print(json.dumps(run(args.case, args.reps, args.B, args.L) if not args.flush else run_flushed(args)))
+    print(json.dumps(run(args.case, args.reps, args.B, args.L, args.T) if not args.flush else run_flushed(args)))
 
 
 if __name__ == "__main__":
