@@ -37,8 +37,8 @@ constexpr int kDecD = 512;                 // head dim (d == dv)
 constexpr int kDecSlabs = kDecD / 64;      // 64-channel slabs per key row
 constexpr int kDecTile = 128;              // keys per tile (MMA M of S^T)
 constexpr int kDecHeads = 64;              // MMA N: query heads of one KV group (padded)
-constexpr int kDecRingK = 3;               // K slab slots
-constexpr int kDecRingV = 6;               // V slab slots (even: V^T operands are slab pairs)
+constexpr int kDecRingK = 4;               // K slab slots
+constexpr int kDecRingV = 4;               // V slab slots (even: V^T operands are slab pairs)
 constexpr int kDecPBufs = 1;               // P^T buffers
 constexpr int kDecThreads = 224;           // 7 warps
 constexpr uint32_t kSlabBytes = 128 * 128;                 // 128 rows x 128 B
