@@ -333,11 +333,22 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         prefetch_tmap(&tm_vw);
     }
 
-    // ---- this CTA's tile range [ts, te) of the batch, and the unit holding tile ts
+    // ---- this CTA's tile range [ts, te) of the batch, and the unit holding tile ts.
+    // With at most one unit per thread, each thread reads its unit's length once.
+    const bool small_batch = U <= kDecThreads;
+    int my_n = 0;
+    if (small_batch && threadIdx.x < U) {
+        UnitTiles t = unit_tiles(p, threadIdx.x, true);
+        my_n = t.nct + t.nwt;
+    }
     long long total = 0;
-    for (int u = threadIdx.x; u < U; u += kDecThreads) {
-        UnitTiles t = unit_tiles(p, u, true);
-        total += t.nct + t.nwt;
+    if (small_batch) {
+        total = my_n;
+    } else {
+        for (int u = threadIdx.x; u < U; u += kDecThreads) {
+            UnitTiles t = unit_tiles(p, u, true);
+            total += t.nct + t.nwt;
+        }
     }
     {
 #pragma unroll
@@ -349,24 +360,61 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         for (int w = 0; w < kDecThreads / 32; ++w) total += wt[w];
         __syncthreads();
     }
-    // equal ranges of ceil(total / nsplit) tiles (the last CTAs may get fewer or none); a
-    // range may hold the tail of one unit and the head of the next
+    // Two ways to cut the batch's tiles into one range per CTA:
+    //  - unit-aligned, when the batch has no more units than CTAs: unit u gets
+    //    n_u = clamp(floor(tiles_u * nsplit / total), 1, tiles_u) CTAs, its tiles split evenly
+    //    among them, so every CTA holds exactly one piece (no second query load, record and
+    //    pipeline refill inside a CTA);
+    //  - otherwise equal ranges of ceil(total / nsplit) tiles (the last CTAs may get fewer or
+    //    none); a range may hold the tail of one unit and the head of the next.
     const long long tpc = (total + p.nsplit - 1) / p.nsplit;
     long long* sched64 = reinterpret_cast<long long*>(red + 64);   // [0] ts, [1] te, [2] p_first
+    int* wsum = reinterpret_cast<int*>(red);
+    int sum_n = 0;
+    const int my_k = (small_batch && threadIdx.x < U && total > 0)
+                         ? max(1, min(my_n, (int)((long long)my_n * p.nsplit / total))) : 0;
+    if (small_batch && U <= p.nsplit && total > 0) {
+        int local = my_k;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xffffffffu, local, off);
+        if (lane == 0) wsum[warp] = local;
+        __syncthreads();
+        for (int w = 0; w < kDecThreads / 32; ++w) sum_n += wsum[w];
+        __syncthreads();
+    }
+    const bool aligned = small_batch && U <= p.nsplit && total > 0 && sum_n <= p.nsplit;
     if (threadIdx.x == 0) {
         sched[0] = -1;
-        sched64[0] = min(total, tpc * cta);
-        sched64[1] = min(total, tpc * (cta + 1));
+        sched64[0] = aligned ? 0 : min(total, tpc * cta);
+        sched64[1] = aligned ? 0 : min(total, tpc * (cta + 1));
     }
     __syncthreads();
-    {
+    if (aligned) {
+        // the unit whose block of CTAs holds this CTA (block-wide scans over units, one
+        // unit per thread)
+        int tot_t, tot_c;
+        const int incl_t = block_scan_incl(my_n, sched + 2, &tot_t);
+        const int incl_c = block_scan_incl(my_k, sched + 2, &tot_c);
+        const long long pu = incl_t - my_n;
+        const int cu = incl_c - my_k;
+        if (threadIdx.x < U && cu <= cta && cta < cu + my_k) {
+            const int i = cta - cu;
+            sched[0] = threadIdx.x;
+            sched64[2] = pu;
+            sched64[0] = pu + (long long)my_n * i / my_k;
+            sched64[1] = pu + (long long)my_n * (i + 1) / my_k;
+        }
+        __syncthreads();
+    } else {
         // the unit holding tile ts (block-wide scan over units)
         const long long ts0 = sched64[0];
         long long base = 0;
         for (int c0 = 0; c0 < U; c0 += kDecThreads) {
             const int u = c0 + threadIdx.x;
             int n = 0;
-            if (u < U) {
+            if (small_batch) {
+                n = my_n;
+            } else if (u < U) {
                 UnitTiles t = unit_tiles(p, u, false);
                 n = t.nct + t.nwt;
             }

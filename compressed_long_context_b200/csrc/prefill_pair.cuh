@@ -48,9 +48,16 @@ constexpr int kPpThreads = 320;
 constexpr int kPpSoftWarps = 8;                 // S-CTA softmax warps (2..9)
 constexpr int kPpKeys = 256;                     // keys per S tile (MMA N of S)
 constexpr int kPpUKeys = 128;                    // keys per P unit (the hand-off granule)
-constexpr int kPpSlots = 3;                      // P units in flight between the two CTAs
+#ifndef HCA_PP_SLOTS
+#define HCA_PP_SLOTS 3
+#endif
+#ifndef HCA_PP_VRING
+#define HCA_PP_VRING 3
+#endif
+constexpr int kPpSlots = HCA_PP_SLOTS;           // P units in flight between the two CTAs
 constexpr int kPpD = 512;
-constexpr int kPpRing = 3;                       // K units (S-CTA) / V units (O-CTA)
+constexpr int kPpRingK = 3;                      // K units in flight (S-CTA)
+constexpr int kPpRingV = HCA_PP_VRING;           // V units in flight (O-CTA)
 constexpr uint32_t kPpQSlab = 128 * 128;         // Q: 128 rows x 64 channels
 constexpr uint32_t kPpUnit = 32768;              // K: 256 keys x 64 ch; V: 64 keys x 256 ch
 constexpr uint32_t kPpVSub = 8192;               // V unit = 4 channel slabs of 64 keys x 64 ch
@@ -58,11 +65,12 @@ constexpr uint32_t kPpPBuf = 32768;              // P unit: 128 rows x 128 keys,
 constexpr uint32_t kPpHdrBytes = 528;            // per P unit: alpha[128], flag[4]
 // shared-memory layout (offsets from a 1024-aligned base); the two ranks reuse offsets
 constexpr uint32_t kPpSmQ = 0;                   // S-CTA: Q, 8 slabs (128 KB)
-constexpr uint32_t kPpSmP = 0;                   // O-CTA: P, 3 units (96 KB)
+constexpr uint32_t kPpSmP = 0;                   // O-CTA: P units
 constexpr uint32_t kPpSmStage = kPpSmP + kPpSlots * kPpPBuf;   // O-CTA: output staging, 4 warps x 8 KB
 constexpr uint32_t kPpStageWarp = 8192;          // 2 pieces of 4 KB: 32 rows x 64 bf16 or 32 fp32 columns
-constexpr uint32_t kPpSmRing = 131072;           // both: ring of 3 units (96 KB)
-constexpr uint32_t kPpSmHdr = kPpSmRing + kPpRing * kPpUnit;     // O-CTA: unit headers
+constexpr uint32_t kPpSmRing = 131072;           // S-CTA: K ring (after Q)
+constexpr uint32_t kPpSmVRing = kPpSmStage + 4 * kPpStageWarp;  // O-CTA: V ring (after staging)
+constexpr uint32_t kPpSmHdr = kPpSmRing + kPpRingK * kPpUnit;    // O-CTA: unit headers
 constexpr uint32_t kPpSmXch = kPpSmHdr;          // S-CTA: softmax exchange, 2 x 2 x 128 floats
 constexpr uint32_t kPpHdrArea = kPpSlots * kPpHdrBytes > 2048 ? kPpSlots * kPpHdrBytes : 2048;
 constexpr uint32_t kPpSmBar = kPpSmHdr + kPpHdrArea;
@@ -73,15 +81,17 @@ static_assert(kPpSmem <= 232448, "pair prefill shared memory exceeds the 227 KB 
 static_assert(kPpSmHdr % 16 == 0 && kPpSmBar % 8 == 0 && kPpSmMisc % 16 == 0,
               "header 16-aligned, barriers 8-aligned");
 static_assert(kPpKeys == 2 * kPpUKeys, "an S tile is two P units");
-static_assert(kPpSmStage + 4 * kPpStageWarp <= kPpSmRing, "output staging fits below the ring");
+static_assert(kPpSlots <= 4 && kPpRingV <= 4 && kPpRingK == 3, "barrier index ranges");
+static_assert(kPpSmVRing + kPpRingV * kPpUnit <= kPpSmHdr, "O-CTA: P, staging and the V ring fit");
+static_assert(kPpSmVRing % 1024 == 0, "V units 1024-aligned");
 
 // barrier indices (both ranks initialise all of them; each rank uses its own)
 enum : int {
     kBarKFull = 0, kBarKEmpty = 3, kBarQFull = 6, kBarQEmpty = 7, kBarSFull = 8, kBarSEmpty = 10,
-    kBarPEmpty = 12,                                                       // S-CTA (+ [4])
-    kBarVFull = 16, kBarVEmpty = 19, kBarPFull = 22, kBarCorr = 26, kBarPCons = 30,
-    kBarOFull = 38, kBarOEmpty = 39,                                       // O-CTA
-    kBarDrain = 40
+    kBarPEmpty = 12,                                                       // S-CTA (+ [<= 4])
+    kBarVFull = 16, kBarVEmpty = 20, kBarPFull = 24, kBarCorr = 28, kBarPCons = 32,
+    kBarOFull = 36, kBarOEmpty = 37,                                       // O-CTA
+    kBarDrain = 38
 };
 
 struct PpItem {
@@ -226,9 +236,9 @@ __device__ __forceinline__ uint32_t pp_ld_cluster_u32(uint32_t raddr) {
 }
 
 // Producer-side drain: wait until the last load issued into every slot of a ring has landed.
-__device__ __forceinline__ void pp_drain_ring(uint64_t* full, uint32_t issued) {
-    for (uint32_t st = 0; st < (uint32_t)kPpRing; ++st)
-        if (issued > st) pp_drain_wait(&full[st], ((issued - 1 - st) / kPpRing) & 1);
+__device__ __forceinline__ void pp_drain_ring(uint64_t* full, uint32_t issued, uint32_t ring) {
+    for (uint32_t st = 0; st < ring; ++st)
+        if (issued > st) pp_drain_wait(&full[st], ((issued - 1 - st) / ring) & 1);
 }
 
 __global__ void __launch_bounds__(kPpThreads, 1)   // 10 warps: at most 168 registers (3 warps per SMSP)
@@ -251,9 +261,11 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         misc[2] = aligned ? 1 : 0;
-        for (int i = 0; i < kPpRing; ++i) {
+        for (int i = 0; i < kPpRingK; ++i) {
             mbar_init(&bars[kBarKFull + i], 1);
             mbar_init(&bars[kBarKEmpty + i], 1);
+        }
+        for (int i = 0; i < kPpRingV; ++i) {
             mbar_init(&bars[kBarVFull + i], 1);
             mbar_init(&bars[kBarVEmpty + i], 1);
         }
@@ -312,8 +324,8 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                     const bool comp = j < it.nct;
                     const int row = pp_tile_row(it, j);
                     for (int s = 0; s < 8; ++s) {
-                        const uint32_t st = kr % kPpRing;
-                        if (!mbar_wait(&bars[kBarKEmpty + st], ((kr / kPpRing) & 1) ^ 1, abort_flag)) {
+                        const uint32_t st = kr % kPpRingK;
+                        if (!mbar_wait(&bars[kBarKEmpty + st], ((kr / kPpRingK) & 1) ^ 1, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -324,7 +336,7 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                     }
                 }
             }
-            pp_drain_ring(&bars[kBarKFull], kr);
+            pp_drain_ring(&bars[kBarKFull], kr, kPpRingK);
             if (qn) pp_drain_wait(&bars[kBarQFull], (qn - 1) & 1);
         }
     } else if (s_cta && warp == 1) {
@@ -349,8 +361,8 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                     const uint32_t id = idesc_bf16(128, N, 0, 0);
                     const uint32_t dst = tmem + sb * kPpKeys;
                     for (int s = 0; s < 8; ++s) {
-                        const uint32_t st = kr % kPpRing;
-                        if (!warp_wait(&bars[kBarKFull + st], (kr / kPpRing) & 1, abort_flag)) {
+                        const uint32_t st = kr % kPpRingK;
+                        if (!warp_wait(&bars[kBarKFull + st], (kr / kPpRingK) & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -607,14 +619,14 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                         const int nv = (pp_unit_keys(nk, hh) + 63) >> 6;
                         for (int h = 0; ok && h < 2; ++h)
                             for (int u = 0; u < nv; ++u) {
-                                const uint32_t st = vr % kPpRing;
-                                if (!mbar_wait(&bars[kBarVEmpty + st], ((vr / kPpRing) & 1) ^ 1, abort_flag)) {
+                                const uint32_t st = vr % kPpRingV;
+                                if (!mbar_wait(&bars[kBarVEmpty + st], ((vr / kPpRingV) & 1) ^ 1, abort_flag)) {
                                     ok = false;
                                     break;
                                 }
                                 mbar_arrive_expect_tx(&bars[kBarVFull + st], kPpUnit);
                                 for (int c = 0; c < 4; ++c)
-                                    tma_load_4d(sm + kPpSmRing + st * kPpUnit + c * kPpVSub, comp ? &tm_vc : &tm_v,
+                                    tma_load_4d(sm + kPpSmVRing + st * kPpUnit + c * kPpVSub, comp ? &tm_vc : &tm_v,
                                                 &bars[kBarVFull + st], 256 * h + 64 * c, it.g,
                                                 row + kPpUKeys * hh + 64 * u, it.b);
                                 ++vr;
@@ -622,7 +634,7 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                     }
                 }
             }
-            pp_drain_ring(&bars[kBarVFull], vr);
+            pp_drain_ring(&bars[kBarVFull], vr, kPpRingV);
         }
     } else if (!s_cta && warp == 1) {
         // ===================================================== O-CTA: O += P V
@@ -654,14 +666,14 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                         const int nv = (nku + 63) >> 6;
                         for (int h = 0; ok && h < 2; ++h)
                             for (int u = 0; u < nv; ++u) {
-                                const uint32_t st = vr % kPpRing;
-                                if (!warp_wait(&bars[kBarVFull + st], (vr / kPpRing) & 1, abort_flag)) {
+                                const uint32_t st = vr % kPpRingV;
+                                if (!warp_wait(&bars[kBarVFull + st], (vr / kPpRingV) & 1, abort_flag)) {
                                     ok = false;
                                     break;
                                 }
                                 tc_fence_after();
                                 if (lane == 0) {
-                                    const uint32_t vb = smem_u32(sm + kPpSmRing + st * kPpUnit);
+                                    const uint32_t vb = smem_u32(sm + kPpSmVRing + st * kPpUnit);
                                     const uint32_t pa = p_base + us * kPpPBuf + u * 16384;   // 16 keys = 4 KB
 #pragma unroll
                                     for (int kk = 0; kk < 4; ++kk)
