@@ -836,9 +836,12 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 // Grid (units, heads / 4), 128 threads; a thread owns 4 heads x 4 channels.  All the
 // (m, l, O) values of a chunk of records are loaded before any is used, so a merge costs
 // about two memory round trips, and the grid fits in one wave.
-constexpr int kMergeChunk = 4;
 constexpr int kMergeHeads = 4;
 
+// kMergeChunk records are loaded per round: 4 when units have many pieces (few long
+// sequences), 2 otherwise -- the smaller chunk keeps registers low enough for the whole grid
+// to fit one wave.
+template <int kMergeChunk>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int u = blockIdx.x;

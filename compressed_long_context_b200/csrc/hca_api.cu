@@ -277,7 +277,10 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel, p) != cudaSuccess) {
+    // many pieces per unit (nsplit >= 3 U): load 4 records per round, else 2
+    const cudaError_t e = (long long)nsplit >= 3 * U ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<4>, p)
+                                                      : cudaLaunchKernelEx(&cfg, decode_combine_kernel<2>, p);
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return HCA_ERR_CUDA;
     }
