@@ -360,29 +360,46 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         for (int w = 0; w < kDecThreads / 32; ++w) total += wt[w];
         __syncthreads();
     }
-    // Two ways to cut the batch's tiles into one range per CTA:
+    // Two ways to cut the batch's tiles into one range per CTA (tpc = ceil(total / nsplit)):
     //  - unit-aligned, when the batch has no more units than CTAs: unit u gets
-    //    n_u = clamp(floor(tiles_u * nsplit / total), 1, tiles_u) CTAs, its tiles split evenly
-    //    among them, so every CTA holds exactly one piece (no second query load, record and
-    //    pipeline refill inside a CTA);
-    //  - otherwise equal ranges of ceil(total / nsplit) tiles (the last CTAs may get fewer or
-    //    none); a range may hold the tail of one unit and the head of the next.
+    //    k_u = clamp(max(floor(tiles_u * nsplit / total), ceil(tiles_u / T)), 1, tiles_u) CTAs
+    //    and its tiles are split evenly among them, for the smallest T in tpc .. tpc + 3 whose
+    //    counts fit the grid.  Every CTA then holds exactly one piece (no second query load,
+    //    record and pipeline refill inside a CTA) of at most T tiles;
+    //  - otherwise (no such T: a ragged batch whose long units cannot be cut finely enough)
+    //    equal ranges of tpc tiles (the last CTAs may get fewer or none); a range may hold the
+    //    tail of one unit and the head of the next.
     const long long tpc = (total + p.nsplit - 1) / p.nsplit;
     long long* sched64 = reinterpret_cast<long long*>(red + 64);   // [0] ts, [1] te, [2] p_first
-    int* wsum = reinterpret_cast<int*>(red);
-    int sum_n = 0;
-    const int my_k = (small_batch && threadIdx.x < U && total > 0)
-                         ? max(1, min(my_n, (int)((long long)my_n * p.nsplit / total))) : 0;
-    if (small_batch && U <= p.nsplit && total > 0) {
-        int local = my_k;
+    // the four candidate counts are summed in one reduction, as 16-bit fields of a 64-bit
+    // word: k_u <= nsplit * tiles_u / total + 1, so each sum is at most nsplit + U < 2^16
+    unsigned long long* wsum = reinterpret_cast<unsigned long long*>(red);   // [warp]
+    int my_k = 0;
+    bool aligned = false;
+    if (small_batch && U <= p.nsplit && p.nsplit < 0x8000 && total > 0 && total <= 0x3fffffffll) {
+        const unsigned n32 = (unsigned)my_n;
+        const unsigned fl = threadIdx.x < U ? (unsigned)((long long)my_n * p.nsplit / total) : 0u;
+        unsigned long long packed = 0;
+        if (threadIdx.x < U)
+#pragma unroll 1
+            for (unsigned w = 0; w < 4; ++w) {
+                const unsigned T = (unsigned)tpc + w;
+                packed |= (unsigned long long)max(1u, min(n32, max(fl, (n32 + T - 1u) / T))) << (16 * w);
+            }
+        unsigned long long sum = packed;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xffffffffu, local, off);
-        if (lane == 0) wsum[warp] = local;
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0) wsum[warp] = sum;
         __syncthreads();
-        for (int w = 0; w < kDecThreads / 32; ++w) sum_n += wsum[w];
+        sum = 0;
+        for (int v = 0; v < kDecThreads / 32; ++v) sum += wsum[v];
         __syncthreads();
+        for (int w = 3; w >= 0; --w)
+            if ((int)((sum >> (16 * w)) & 0xffffu) <= p.nsplit) {
+                aligned = true;
+                my_k = (int)((packed >> (16 * w)) & 0xffffu);
+            }
     }
-    const bool aligned = small_batch && U <= p.nsplit && total > 0 && sum_n <= p.nsplit;
     if (threadIdx.x == 0) {
         sched[0] = -1;
         sched64[0] = aligned ? 0 : min(total, tpc * cta);
@@ -451,19 +468,36 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             bool q_issued = false;
             uint64_t t_prog = globaltimer_ns();
             uint32_t idle = 0;
+            // Page ids of the two 64-entry halves of the current compressed K (V) tile, read
+            // from the page table once per tile, as soon as the iterator reaches the tile
+            // (its last slab's neighbour is still in flight, so the load's latency hides
+            // behind it): each read is a dependent global load in this one thread, and one
+            // per slab costs as much as streaming the tile.  A page id outside the pool is
+            // reported and clamped into it, so every load stays inside the pool.
+            int kpg[2] = {0, 0}, vpg[2] = {0, 0};
+            auto pages_of = [&](const TileIter& it, int* pg) {
+                if (!paged || it.done || !it.comp()) return;
+                const int j0 = it.tile * kDecTile;
+                const int* row = p.page_table + (size_t)it.t.b * p.max_pages;
+                pg[0] = __ldg(row + j0 / p.page_size);
+                pg[1] = j0 + 64 < it.t.nc ? __ldg(row + (j0 + 64) / p.page_size) : pg[0];
+                if (min(pg[0], pg[1]) < 0 || max(pg[0], pg[1]) >= p.num_pages) {
+                    record_error(HCA_ERR_DEVICE_INPUT);
+                    pg[0] = min(max(pg[0], 0), p.num_pages - 1);
+                    pg[1] = min(max(pg[1], 0), p.num_pages - 1);
+                }
+            };
+            pages_of(ki, kpg);
+            pages_of(vi, vpg);
             // One slab of the current tile of iterator `it` (K or V) into slot `dst`.
-            auto issue = [&](const TileIter& it, int s, bool is_v, uint8_t* dst, uint64_t* bar) {
+            auto issue = [&](const TileIter& it, const int* pg, int s, bool is_v, uint8_t* dst, uint64_t* bar) {
                 const CUtensorMap* m = it.comp() ? (is_v ? &tm_v : &tm_k) : (is_v ? &tm_vw : &tm_kw);
                 if (it.comp() && paged) {
                     const int j0 = it.tile * kDecTile;
                     const bool h1 = j0 + 64 < it.t.nc;
                     mbar_arrive_expect_tx(bar, h1 ? 2 * 8192 : 8192);
-                    for (int h = 0; h < (h1 ? 2 : 1); ++h) {
-                        const int j = j0 + 64 * h;
-                        const int pg = __ldg(p.page_table + (size_t)it.t.b * p.max_pages + j / p.page_size);
-                        if (pg < 0 || pg >= p.num_pages) record_error(HCA_ERR_DEVICE_INPUT);
-                        tma_load_4d(dst + h * 8192, m, bar, 64 * s, it.t.g, j % p.page_size, pg);
-                    }
+                    for (int h = 0; h < (h1 ? 2 : 1); ++h)
+                        tma_load_4d(dst + h * 8192, m, bar, 64 * s, it.t.g, (j0 + 64 * h) % p.page_size, pg[h]);
                 } else {
                     mbar_arrive_expect_tx(bar, kSlabBytes);
                     const int row = it.comp() ? it.tile * kDecTile : it.t.s0 + (it.tile - it.t.nct) * kDecTile;
@@ -486,12 +520,13 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     } else {
                         const uint32_t st = kring % kDecRingK;
                         if (mbar_test(&kempty[st], ((kring / kDecRingK) & 1) ^ 1)) {
-                            issue(ki, ks, false, sm + kSmRingK + st * kSlabBytes, &kfull[st]);
+                            issue(ki, kpg, ks, false, sm + kSmRingK + st * kSlabBytes, &kfull[st]);
                             ++kring;
                             prog = true;
                             if (++ks == kDecSlabs) {
                                 ks = 0;
                                 ki.next();
+                                pages_of(ki, kpg);
                                 ++kdone;
                                 q_issued = false;
                             }
@@ -502,12 +537,13 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 if (!vi.done && (vdone < kdone || ks > 0)) {
                     const uint32_t st = vring % kDecRingV;
                     if (mbar_test(&vempty[st], ((vring / kDecRingV) & 1) ^ 1)) {
-                        issue(vi, vs, true, sm + kSmRingV + st * kSlabBytes, &vfull[st]);
+                        issue(vi, vpg, vs, true, sm + kSmRingV + st * kSlabBytes, &vfull[st]);
                         ++vring;
                         prog = true;
                         if (++vs == kDecSlabs) {
                             vs = 0;
                             vi.next();
+                            pages_of(vi, vpg);
                             ++vdone;
                         }
                     }

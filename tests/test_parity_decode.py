@@ -158,6 +158,28 @@ def test_decode_device_input_error(cuda_device, libhca):
     hca.get_device_error()     # cleared
 
 
+def test_decode_bad_page_id_reported(cuda_device, libhca):
+    """A page id outside the pool is reported as a device-input error; the loads are
+    clamped into the pool, so nothing is read outside it."""
+    c = direct_case(cuda_device, 95, [9000, 3000], paged_ps=64)
+    c["page_table"][0, 1] = c["kc"].shape[0]          # one past the last page (entries 64..68)
+    hca.decode(c["q"], c["kc"], c["vc"], c["kw"], c["vw"], c["seqlens"], 128, 128, 0.05,
+               page_table=c["page_table"], page_size=64)
+    with pytest.raises(hca.HCAError) as e:
+        hca.get_device_error()
+    assert e.value.code == 5
+    hca.get_device_error()     # cleared
+
+
+def test_decode_ragged_long_and_short(cuda_device, libhca):
+    """Few long sequences among many short ones: the per-sequence CTA counts cannot hold
+    every CTA near the even share of tiles, so the batch is cut into equal ranges that
+    cross sequence boundaries."""
+    lengths = [60000 if i % 2 == 0 else 1000 for i in range(100)]    # 350 tiles over 148 CTAs
+    out, ref = run_both(direct_case(cuda_device, 96, lengths, paged_ps=128, norm=True))
+    check(out, ref)
+
+
 # ------------------------------------------------------------ full-size workloads (sampled)
 
 def _oracle_decode_from_raw(k, v, w, q, L, W, blk, scale):
