@@ -837,8 +837,11 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 if (!group_wait(o_full, it.item & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 float* orec = p.rec_o + (size_t)rec * 64 * kDecD;
+                // rolled: the code of a launch's last tile is fetched cold, and a smaller loop
+                // costs less fetch than the unrolling saves
+#pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
-#pragma unroll
+#pragma unroll 1
                     for (int c16 = 0; c16 < 64; c16 += 16) {
                         float o[16];
                         tmem_ld16(tmem + lane_off + kTmO + 64 * c + c16, o);
