@@ -882,11 +882,20 @@ constexpr int kMergeHeads = 4;
 // to fit one wave.
 template <int kMergeChunk>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int u = blockIdx.x;
     const int h0 = blockIdx.y * kMergeHeads;
     const int c = 4 * threadIdx.x;                // channels c .. c+3
     const int b = u / p.Hkv, g = u - (u / p.Hkv) * p.Hkv;
+    // the gate logits are an input, not a product of the split kernel: they are read before
+    // waiting for it, so their DRAM latency overlaps the records' loads
+    uint2 gv[kMergeHeads];
+#pragma unroll
+    for (int j = 0; j < kMergeHeads; ++j) {
+        const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h0 + j) * kDecD + c;
+        gv[j] = ((p.flags & HCA_OUT_GATE) && h0 + j < p.G)
+                    ? __ldg(reinterpret_cast<const uint2*>(p.gate + orow)) : make_uint2(0u, 0u);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int first = __ldg(p.meta + 2 * u), last = __ldg(p.meta + 2 * u + 1);
     if (first < 0 || last < first || last >= p.nsplit) {
         if (threadIdx.x == 0 && blockIdx.y == 0) record_error(HCA_ERR_DEVICE_INPUT);
@@ -946,11 +955,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
         float4 r = make_float4(acc[j].x * inv, acc[j].y * inv, acc[j].z * inv, acc[j].w * inv);
         const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h) * kDecD + c;
         if (p.flags & HCA_OUT_GATE) {
-            const uint2 gv = __ldg(reinterpret_cast<const uint2*>(p.gate + orow));
-            r.x *= 1.f / (1.f + __expf(-bf16lo(gv.x)));
-            r.y *= 1.f / (1.f + __expf(-bf16hi(gv.x)));
-            r.z *= 1.f / (1.f + __expf(-bf16lo(gv.y)));
-            r.w *= 1.f / (1.f + __expf(-bf16hi(gv.y)));
+            r.x *= 1.f / (1.f + __expf(-bf16lo(gv[j].x)));
+            r.y *= 1.f / (1.f + __expf(-bf16hi(gv[j].x)));
+            r.z *= 1.f / (1.f + __expf(-bf16lo(gv[j].y)));
+            r.w *= 1.f / (1.f + __expf(-bf16hi(gv[j].y)));
         }
         *reinterpret_cast<float4*>(p.out + orow) = r;
     }
