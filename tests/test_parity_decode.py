@@ -88,6 +88,7 @@ def run_both(c, scale=None):
     ([128 * 9 + 77] * 7, 128),
     ([4096 + 5, 70, 20000], 256),                # two window tiles
     ([60000, 3], 200),
+    ([128, 129, 255, 256, 257, 2], 128),   # around the window size and the first complete block
 ])
 def test_decode_contiguous(cuda_device, libhca, lengths, W):
     c = direct_case(cuda_device, 11 + len(lengths), lengths, W=W)

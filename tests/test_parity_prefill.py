@@ -115,6 +115,35 @@ def test_prefill_d512(cuda_device, libhca, B, T, Hq, Hkv, blk, W):
     run_case(cuda_device, B, T, Hq, Hkv, 512, blk, W, seed=T + 7 * Hq, out_f32=(Hq == 16))   # bf16 path too
 
 
+@pytest.mark.parametrize("B,T,Hq,Hkv,blk,W,wstd", [
+    (1, 1, 64, 1, 128, 128, 0.5),     # a single token: it sees only itself
+    (1, 100, 64, 1, 128, 50, 0.5),    # shorter than a block: no compressed entry exists
+    (1, 256, 64, 1, 128, 128, 0.5),   # T on a block boundary: the last row sees exactly one entry
+    (2, 640, 64, 1, 128, 128, 0.0),   # zero pooling weights: the cache is the block mean
+])
+def test_prefill_d512_edges(cuda_device, libhca, B, T, Hq, Hkv, blk, W, wstd):
+    run_case(cuda_device, B, T, Hq, Hkv, 512, blk, W, seed=11 * T + B, wstd=wstd, out_f32=False)
+
+
+def test_empty_inputs_are_noops(cuda_device, libhca):
+    """T = 0 or B = 0: every entry point returns at once with empty outputs."""
+    dev = cuda_device
+    k = torch.empty((1, 0, 1, 512), dtype=torch.bfloat16, device=dev)
+    kc, vc = hca.compress(k, k, None, 128)
+    assert kc.shape == (1, 0, 1, 512) and vc.shape == (1, 0, 1, 512)
+    q = torch.empty((1, 0, 64, 512), dtype=torch.bfloat16, device=dev)
+    out = hca.prefill(q, k, k, kc, vc, 128, 128, 0.05)
+    assert out.shape == (1, 0, 64, 512)
+    qd = torch.empty((0, 64, 512), dtype=torch.bfloat16, device=dev)
+    kcd = torch.empty((0, 4, 1, 512), dtype=torch.bfloat16, device=dev)
+    kw = torch.empty((0, 128, 1, 512), dtype=torch.bfloat16, device=dev)
+    seq = torch.empty((0,), dtype=torch.int32, device=dev)
+    od = hca.decode(qd, kcd, kcd, kw, kw, seq, 128, 128, 0.05)
+    assert od.shape == (0, 64, 512)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+
+
 def test_prefill_d512_long_sampled(cuda_device, libhca):
     T = 6000
     rs = np.random.RandomState(1)
