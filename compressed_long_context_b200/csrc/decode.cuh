@@ -886,19 +886,26 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     const int h0 = blockIdx.y * kMergeHeads;
     const int c = 4 * threadIdx.x;                // channels c .. c+3
     const int b = u / p.Hkv, g = u - (u / p.Hkv) * p.Hkv;
-    // the gate logits are an input, not a product of the split kernel: they are read before
-    // waiting for it, so their DRAM latency overlaps the records' loads
-    uint2 gv[kMergeHeads];
+    // the gate logits are an input, not a product of the split kernel: each thread copies its
+    // own into shared memory before waiting for it (cp.async: no registers held), so their
+    // DRAM latency overlaps the records' loads
+    __shared__ __align__(16) uint2 gsm[kMergeHeads][128];
+    const bool gated = (p.flags & HCA_OUT_GATE) != 0;
+    if (gated) {
 #pragma unroll
-    for (int j = 0; j < kMergeHeads; ++j) {
-        const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h0 + j) * kDecD + c;
-        gv[j] = ((p.flags & HCA_OUT_GATE) && h0 + j < p.G)
-                    ? __ldg(reinterpret_cast<const uint2*>(p.gate + orow)) : make_uint2(0u, 0u);
+        for (int j = 0; j < kMergeHeads; ++j)
+            if (h0 + j < p.G) {
+                const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h0 + j) * kDecD + c;
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 8;"
+                             :: "r"(smem_u32(&gsm[j][threadIdx.x])), "l"(p.gate + orow) : "memory");
+            }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int first = __ldg(p.meta + 2 * u), last = __ldg(p.meta + 2 * u + 1);
     if (first < 0 || last < first || last >= p.nsplit) {
         if (threadIdx.x == 0 && blockIdx.y == 0) record_error(HCA_ERR_DEVICE_INPUT);
+        if (gated) asm volatile("cp.async.wait_all;" ::: "memory");
         return;
     }
     float M[kMergeHeads], L[kMergeHeads];
@@ -947,6 +954,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
             M[j] = Mn;
         }
     }
+    if (gated) asm volatile("cp.async.wait_all;" ::: "memory");     // this thread's own copies
 #pragma unroll
     for (int j = 0; j < kMergeHeads; ++j) {
         const int h = h0 + j;
@@ -954,11 +962,12 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
         const float inv = 1.f / L[j];
         float4 r = make_float4(acc[j].x * inv, acc[j].y * inv, acc[j].z * inv, acc[j].w * inv);
         const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h) * kDecD + c;
-        if (p.flags & HCA_OUT_GATE) {
-            r.x *= 1.f / (1.f + __expf(-bf16lo(gv[j].x)));
-            r.y *= 1.f / (1.f + __expf(-bf16hi(gv[j].x)));
-            r.z *= 1.f / (1.f + __expf(-bf16lo(gv[j].y)));
-            r.w *= 1.f / (1.f + __expf(-bf16hi(gv[j].y)));
+        if (gated) {
+            const uint2 gv = gsm[j][threadIdx.x];
+            r.x *= 1.f / (1.f + __expf(-bf16lo(gv.x)));
+            r.y *= 1.f / (1.f + __expf(-bf16hi(gv.x)));
+            r.z *= 1.f / (1.f + __expf(-bf16lo(gv.y)));
+            r.w *= 1.f / (1.f + __expf(-bf16hi(gv.y)));
         }
         *reinterpret_cast<float4*>(p.out + orow) = r;
     }
