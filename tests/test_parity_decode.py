@@ -140,6 +140,19 @@ def test_decode_large_logits_rescale(cuda_device, libhca):
     check(*run_both(c))
 
 
+@pytest.mark.parametrize("boost", [12.0, 40.0])
+def test_decode_first_key_far_below(cuda_device, libhca, boost):
+    """Entry 0 (the first key of every piece that starts a sequence) is zero and the other
+    entries are scaled up, so the reference seeded from the first key lies far below the
+    tile maximum and must be raised inside the first tile; with the larger scale the logits
+    span hundreds of binary orders of magnitude."""
+    c = direct_case(cuda_device, 73, [40000, 20000, 9000])
+    kc = c["kc"].float() * boost
+    kc[:, 0] = 0.0
+    c["kc"] = kc.to(torch.bfloat16)
+    check(*run_both(c))
+
+
 def test_decode_repeatable_and_workspace_reuse(cuda_device, libhca):
     c = direct_case(cuda_device, 81, [20000, 100, 7000])
     ws = torch.empty(hca.decode_workspace_size(3, 64, 1, 512), dtype=torch.uint8, device=cuda_device)
