@@ -74,7 +74,7 @@ constexpr uint32_t kPpSmHdr = kPpSmRing + kPpRingK * kPpUnit;    // O-CTA: unit 
 constexpr uint32_t kPpSmXch = kPpSmHdr;          // S-CTA: softmax exchange, 2 x 2 x 128 floats
 constexpr uint32_t kPpHdrArea = kPpSlots * kPpHdrBytes > 2048 ? kPpSlots * kPpHdrBytes : 2048;
 constexpr uint32_t kPpSmBar = kPpSmHdr + kPpHdrArea;
-constexpr int kPpNumBars = 42;                  // 41 used; even count keeps misc 16-aligned
+constexpr int kPpNumBars = 56;                  // 56 used; even count keeps misc 16-aligned
 constexpr uint32_t kPpSmMisc = kPpSmBar + kPpNumBars * 8;
 constexpr uint32_t kPpSmem = kPpSmMisc + 16;
 static_assert(kPpSmem <= 232448, "pair prefill shared memory exceeds the 227 KB per-block limit");
@@ -87,11 +87,12 @@ static_assert(kPpSmVRing % 1024 == 0, "V units 1024-aligned");
 
 // barrier indices (both ranks initialise all of them; each rank uses its own)
 enum : int {
-    kBarKFull = 0, kBarKEmpty = 3, kBarQFull = 6, kBarQEmpty = 7, kBarSFull = 8, kBarSEmpty = 10,
+    kBarKFull = 0, kBarKEmpty = 3, kBarSFull = 8, kBarSEmpty = 10,      // (6, 7 unused)
     kBarPEmpty = 12,                                                       // S-CTA (+ [<= 4])
     kBarVFull = 16, kBarVEmpty = 20, kBarPFull = 24, kBarCorr = 28, kBarPCons = 32,
     kBarOFull = 36, kBarOEmpty = 37,                                       // O-CTA
-    kBarDrain = 38
+    kBarDrain = 38,
+    kBarQSFull = 40, kBarQSEmpty = 48                                      // S-CTA: per Q slab [8]
 };
 
 struct PpItem {
@@ -269,8 +270,10 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
             mbar_init(&bars[kBarVFull + i], 1);
             mbar_init(&bars[kBarVEmpty + i], 1);
         }
-        mbar_init(&bars[kBarQFull], 1);
-        mbar_init(&bars[kBarQEmpty], 1);
+        for (int i = 0; i < 8; ++i) {
+            mbar_init(&bars[kBarQSFull + i], 1);
+            mbar_init(&bars[kBarQSEmpty + i], 1);
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars[kBarSFull + i], 1);
             mbar_init(&bars[kBarSEmpty + i], kPpSoftWarps);
@@ -314,16 +317,22 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
             bool ok = true;
             for (long long i = pair; ok && i < p.items; i += npairs) {
                 const PpItem it = pp_item(p, i);
-                if (!mbar_wait(&bars[kBarQEmpty], (qn & 1) ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&bars[kBarQFull], 8 * kPpQSlab);
-                for (int s = 0; s < 8; ++s)
-                    tma_load_4d(sm + kPpSmQ + s * kPpQSlab, &tm_q, &bars[kBarQFull], 64 * s, it.g * p.G, it.t0, it.b);
-                ++qn;
                 const int nt = it.nct + it.nwt;
                 for (int j = 0; ok && j < nt; ++j) {
                     const bool comp = j < it.nct;
                     const int row = pp_tile_row(it, j);
                     for (int s = 0; s < 8; ++s) {
+                        if (j == 0) {
+                            // Q slab s of this row tile, as soon as the previous row tile's last
+                            // MMAs on slab s have completed (not after its whole last tile)
+                            if (!mbar_wait(&bars[kBarQSEmpty + s], (qn & 1) ^ 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(&bars[kBarQSFull + s], kPpQSlab);
+                            tma_load_4d(sm + kPpSmQ + s * kPpQSlab, &tm_q, &bars[kBarQSFull + s], 64 * s,
+                                        it.g * p.G, it.t0, it.b);
+                        }
                         const uint32_t st = kr % kPpRingK;
                         if (!mbar_wait(&bars[kBarKEmpty + st], ((kr / kPpRingK) & 1) ^ 1, abort_flag)) {
                             ok = false;
@@ -335,9 +344,11 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                         ++kr;
                     }
                 }
+                ++qn;
             }
             pp_drain_ring(&bars[kBarKFull], kr, kPpRingK);
-            if (qn) pp_drain_wait(&bars[kBarQFull], (qn - 1) & 1);
+            if (qn)
+                for (int s = 0; s < 8; ++s) pp_drain_wait(&bars[kBarQSFull + s], (qn - 1) & 1);
         }
     } else if (s_cta && warp == 1) {
         // ===================================================== S-CTA: S = Q K^T
@@ -349,7 +360,6 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
             for (long long i = pair; ok && i < p.items; i += npairs, ++item_n) {
                 const PpItem it = pp_item(p, i);
                 const int nt = it.nct + it.nwt;
-                if (!warp_wait(&bars[kBarQFull], item_n & 1, abort_flag)) break;
                 for (int j = 0; ok && j < nt; ++j, ++n) {
                     const int sb = n & 1;
                     if (!warp_wait(&bars[kBarSEmpty + sb], ((n >> 1) & 1) ^ 1, abort_flag)) {
@@ -362,7 +372,9 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                     const uint32_t dst = tmem + sb * kPpKeys;
                     for (int s = 0; s < 8; ++s) {
                         const uint32_t st = kr % kPpRingK;
-                        if (!warp_wait(&bars[kBarKFull + st], (kr / kPpRingK) & 1, abort_flag)) {
+                        // Q slab s of this row tile (landed once per item, used by every tile)
+                        if ((j == 0 && !warp_wait(&bars[kBarQSFull + s], item_n & 1, abort_flag)) ||
+                            !warp_wait(&bars[kBarKFull + st], (kr / kPpRingK) & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -375,15 +387,15 @@ prefill_pair_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap t
                                 mma_ss(dst, smem_desc_sw128(qa + kk * 32, 16, 1024),
                                        smem_desc_sw128(kb + kk * 32, 16, 1024), id, (s | kk) ? 1u : 0u);
                             mma_commit(&bars[kBarKEmpty + st]);
+                            // the row tile's last use of Q slab s: the next row tile's slab s
+                            // may land once these MMAs have completed
+                            if (j == nt - 1) mma_commit(&bars[kBarQSEmpty + s]);
                         }
                         __syncwarp();
                         ++kr;
                     }
                     if (!ok) break;
-                    if (lane == 0) {
-                        mma_commit(&bars[kBarSFull + sb]);
-                        if (j == nt - 1) mma_commit(&bars[kBarQEmpty]);
-                    }
+                    if (lane == 0) mma_commit(&bars[kBarSFull + sb]);
                     __syncwarp();
                 }
             }
