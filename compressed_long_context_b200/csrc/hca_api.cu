@@ -217,7 +217,7 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     }
     if (norm && (!gq || !gk || (reinterpret_cast<uintptr_t>(gq) & 3) || (reinterpret_cast<uintptr_t>(gk) & 3)))
         return HCA_ERR_INVALID_ARG;
-    if (gated && (!gate || (reinterpret_cast<uintptr_t>(gate) & 3))) return HCA_ERR_INVALID_ARG;
+    if (gated && (!gate || !aligned16(gate))) return HCA_ERR_INVALID_ARG;   // read 8 bytes per thread
     const int nsplit = num_sms();
     if (nsplit <= 0) return HCA_ERR_CUDA;
     const long long U = (long long)B * Hkv;

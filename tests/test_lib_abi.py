@@ -99,3 +99,38 @@ def test_prefill_rejects_before_launch(libhca):
     # nothing to do: no launch, OK
     assert libhca.hca_prefill(None, None, None, None, None, None, None, 0, 256, 4, 1, 512, 512, 128, 128,
                               0.1, 0, None) == _lib.HCA_OK
+
+
+def test_decode_rejects_before_launch(libhca):
+    p = ctypes.c_void_p(16)
+    f = ctypes.c_void_p(32)
+
+    def call(q=p, kc=p, vc=p, table=None, ps=0, maxp=0, npages=0, kw=p, vw=p, seq=p, gq=None, gk=None,
+             eps=1e-6, gate=None, out=p, ws=p, ws_bytes=1 << 20, B=1, Hq=64, Hkv=1, d=512, dv=512, blk=128,
+             W=128, Nmax=8, scale=0.05, flags=0):
+        return libhca.hca_decode(q, kc, vc, table, ps, maxp, npages, kw, vw, seq, gq, gk, eps, gate, out, ws,
+                                 ws_bytes, B, Hq, Hkv, d, dv, blk, W, Nmax, scale, flags, None)
+
+    # unsupported head dim, group larger than 64, block larger than 128, unknown flag
+    assert call(d=64, dv=64) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(Hq=128) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(blk=129) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(flags=1 << 8) == _lib.HCA_ERR_UNSUPPORTED
+    # null or misaligned pointers, bad sizes
+    assert call(q=None) == _lib.HCA_ERR_INVALID_ARG
+    assert call(kw=ctypes.c_void_p(24)) == _lib.HCA_ERR_INVALID_ARG
+    assert call(B=-1) == _lib.HCA_ERR_INVALID_ARG
+    assert call(W=0) == _lib.HCA_ERR_INVALID_ARG
+    assert call(eps=-1.0) == _lib.HCA_ERR_INVALID_ARG
+    # QK normalisation without gains; a gate that is NULL or not 16-byte aligned (read 8 bytes
+    # at a time on the device, so a 4-byte-aligned gate must be refused, not faulted on)
+    assert call(flags=_lib.HCA_QK_NORM) == _lib.HCA_ERR_INVALID_ARG
+    assert call(flags=_lib.HCA_OUT_GATE) == _lib.HCA_ERR_INVALID_ARG
+    assert call(flags=_lib.HCA_OUT_GATE, gate=ctypes.c_void_p(20)) == _lib.HCA_ERR_INVALID_ARG
+    assert call(flags=_lib.HCA_OUT_GATE, gate=ctypes.c_void_p(24)) == _lib.HCA_ERR_INVALID_ARG
+    # paged without a table, a page size that is not a multiple of 64
+    assert call(flags=_lib.HCA_PAGED) == _lib.HCA_ERR_INVALID_ARG
+    assert call(flags=_lib.HCA_PAGED, table=f, ps=100, maxp=4, npages=4) == _lib.HCA_ERR_INVALID_ARG
+    # nothing to do: no launch, OK
+    assert call(q=None, kc=None, vc=None, kw=None, vw=None, seq=None, out=None, ws=None, B=0) == _lib.HCA_OK
+
