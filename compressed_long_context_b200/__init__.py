@@ -14,10 +14,10 @@ import torch
 
 from . import _lib
 from ._lib import (HCA_OUT_F32, HCA_OUT_GATE, HCA_PAGED, HCA_QK_NORM,  # noqa: F401
-                   HCA_WRITE_LSE)
+                   HCA_WINDOW_RING, HCA_WRITE_LSE)
 
-__all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "get_device_error",
-           "status_string"]
+__all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "append", "append_state_size",
+           "get_device_error", "status_string"]
 
 
 class HCAError(RuntimeError):
@@ -110,7 +110,7 @@ def decode_workspace_size(B, Hq, Hkv, dv) -> int:
 
 
 def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size=0,
-           gq=None, gk=None, eps=1e-6, gate=None, out=None, workspace=None):
+           gq=None, gk=None, eps=1e-6, gate=None, out=None, workspace=None, window_ring=False):
     """One query per sequence at position seqlens[b]-1 over its compressed cache + raw window.
 
     q [B,Hq,d] bf16; kc/vc contiguous [B,Nmax,Hkv,d|dv] or page pools [P,page_size,Hkv,d|dv]
@@ -141,6 +141,8 @@ def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size
     if gate is not None:
         _need(gate, torch.bfloat16, "gate", dev)
         flags |= HCA_OUT_GATE
+    if window_ring:
+        flags |= HCA_WINDOW_RING
     if out is None:
         out = torch.empty((B, Hq, dv), dtype=torch.float32, device=dev)
     _need(out, torch.float32, "out", dev)
@@ -154,3 +156,49 @@ def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size
                                 float(scale), flags, _stream(dev))
     _check(rc, "hca_decode")
     return out
+
+
+def append_state_size(B, Hkv, d, dv) -> int:
+    """Bytes of pooling state ``append`` keeps for a batch (zero it before a sequence starts)."""
+    return int(_lib.load().hca_append_state_size(B, Hkv, d, dv))
+
+
+def append(k_new, v_new, w_new, seqlens, kw, vw, kc, vc, state, blk, page_table=None):
+    """One decode step's cache update: the newest token of each sequence enters the window
+    ring (slot (L-1) % W), and a block it completes is pooled into the compressed cache.
+
+    k_new [B,Hkv,d], v_new [B,Hkv,dv] bf16; w_new [B] fp32 or None; seqlens [B] int32 (length
+    including the new token); kw/vw [B,W,Hkv,d|dv] bf16 rings; kc/vc contiguous
+    [B,Nmax,Hkv,d|dv] or page pools with page_table [B,max_pages] int32; state: a uint8 or
+    float32 tensor of ``append_state_size`` bytes, zero for an empty block.
+    """
+    _need(k_new, torch.bfloat16, "k_new")
+    dev = k_new.device
+    _need(v_new, torch.bfloat16, "v_new", dev)
+    for name, t in (("kw", kw), ("vw", vw), ("kc", kc), ("vc", vc)):
+        _need(t, torch.bfloat16, name, dev)
+    _need(seqlens, torch.int32, "seqlens", dev)
+    if w_new is not None:
+        _need(w_new, torch.float32, "w_new", dev)
+    if state.dtype not in (torch.uint8, torch.float32) or not state.is_cuda or not state.is_contiguous():
+        raise ValueError("state must be a contiguous uint8 or float32 CUDA tensor")
+    B, Hkv, d = k_new.shape
+    dv = v_new.shape[2]
+    W = kw.shape[1]
+    if state.numel() * state.element_size() < append_state_size(B, Hkv, d, dv):
+        raise ValueError("state is smaller than append_state_size()")
+    flags = 0
+    max_pages = num_pages = page_size = 0
+    Nmax = kc.shape[1]
+    if page_table is not None:
+        _need(page_table, torch.int32, "page_table", dev)
+        flags |= HCA_PAGED
+        max_pages = page_table.shape[1]
+        num_pages = kc.shape[0]
+        page_size = kc.shape[1]
+        Nmax = 0
+    rc = _lib.load().hca_append(_p(k_new), _p(v_new), _p(w_new), _p(seqlens), _p(kw), _p(vw), _p(kc), _p(vc),
+                                _p(page_table), int(page_size), int(max_pages), int(num_pages), _p(state),
+                                B, Hkv, d, dv, int(blk), int(W), int(Nmax), flags, _stream(dev))
+    _check(rc, "hca_append")
+

@@ -114,7 +114,9 @@ __device__ __forceinline__ UnitTiles unit_tiles(const DecodeParams& p, int u, bo
     t.nw = L < p.W ? L : p.W;
     t.nct = (t.nc + kDecTile - 1) / kDecTile;
     t.nwt = (t.nw + kDecTile - 1) / kDecTile;
-    t.s0 = p.W - t.nw;
+    // oldest-first window: the nw valid slots are the last ones; ring (slot = position % W):
+    // before the ring wraps, positions 0 .. L-1 sit in slots 0 .. L-1
+    t.s0 = (p.flags & HCA_WINDOW_RING) ? 0 : p.W - t.nw;
     return t;
 }
 
@@ -234,7 +236,7 @@ struct TileIter {
     // keys of the current tile that belong to the sequence
     __device__ int nvalid() const {
         return comp() ? min(kDecTile, t.nc - tile * kDecTile)
-                      : min(kDecTile, p->W - (t.s0 + (tile - t.nct) * kDecTile));
+                      : min(kDecTile, t.nw - (tile - t.nct) * kDecTile);     // slots s0 .. s0 + nw - 1
     }
     __device__ void next() {
         if (++tile < tend) return;

@@ -6,6 +6,7 @@
 
 #include <mutex>
 
+#include "append.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "decode.cuh"
@@ -156,6 +157,53 @@ hca_status_t hca_compress(const void* k, const void* v, const float* w, void* kc
     return HCA_ERR_UNSUPPORTED;
 }
 
+size_t hca_append_state_size(int B, int Hkv, int d, int dv) {
+    if (B < 0 || Hkv < 1 || d < 0 || dv < 0) return 0;
+    return (size_t)B * Hkv * (size_t)(hca::kAppendHeader + d + dv) * sizeof(float);
+}
+
+hca_status_t hca_append(const void* k_new, const void* v_new, const float* w_new, const int* seqlens, void* kw,
+                        void* vw, void* kc, void* vc, const int* page_table, int page_size, int max_pages,
+                        int num_pages, void* state, int B, int Hkv, int d, int dv, int blk, int W, int Nmax,
+                        unsigned flags, hca_stream_t stream) {
+    if (B < 0 || Hkv < 1 || blk < 1 || W < 1) return HCA_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)HCA_PAGED) return HCA_ERR_UNSUPPORTED;
+    auto ok_dim = [](int x) { return x == 64 || x == 128 || x == 256 || x == 512; };
+    if (!ok_dim(d) || !ok_dim(dv) || blk > 128) return HCA_ERR_UNSUPPORTED;
+    if (B == 0) return HCA_OK;
+    if ((long long)B * Hkv > 0x7fffffffLL) return HCA_ERR_INVALID_ARG;
+    const bool paged = flags & HCA_PAGED;
+    if (!k_new || !v_new || !seqlens || !kw || !vw || !kc || !vc || !state) return HCA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kw) || !aligned16(vw) || !aligned16(kc) ||
+        !aligned16(vc) || !aligned16(state) || (reinterpret_cast<uintptr_t>(seqlens) & 3) ||
+        (w_new && (reinterpret_cast<uintptr_t>(w_new) & 3)))
+        return HCA_ERR_INVALID_ARG;
+    if (paged) {
+        if (!page_table || page_size < 64 || page_size % 64 || max_pages < 1 || num_pages < 1 ||
+            (reinterpret_cast<uintptr_t>(page_table) & 3))
+            return HCA_ERR_INVALID_ARG;
+    } else if (Nmax < 1) {
+        return HCA_ERR_INVALID_ARG;
+    }
+    hca::AppendParams p;
+    p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    p.w = w_new;
+    p.seqlens = seqlens;
+    p.kw = static_cast<__nv_bfloat16*>(kw);
+    p.vw = static_cast<__nv_bfloat16*>(vw);
+    p.kc = static_cast<__nv_bfloat16*>(kc);
+    p.vc = static_cast<__nv_bfloat16*>(vc);
+    p.page_table = paged ? page_table : nullptr;
+    p.state = static_cast<float*>(state);
+    p.B = B; p.Hkv = Hkv; p.d = d; p.dv = dv; p.blk = blk; p.W = W;
+    p.Nmax = paged ? 0 : Nmax;
+    p.page_size = paged ? page_size : 0; p.max_pages = paged ? max_pages : 0; p.num_pages = paged ? num_pages : 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    hca::append_kernel<<<(unsigned)(B * Hkv), hca::kAppendThreads, 0, s>>>(p);
+    return launch_status();
+}
+
 }  // extern "C"
 
 namespace {
@@ -196,7 +244,7 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
                         int Nmax, float scale, unsigned flags, hca_stream_t stream) {
     using namespace hca;
     if (B < 0 || Hq < 1 || Hkv < 1 || blk < 1 || W < 1) return HCA_ERR_INVALID_ARG;
-    if (flags & ~(unsigned)(HCA_QK_NORM | HCA_OUT_GATE | HCA_PAGED)) return HCA_ERR_UNSUPPORTED;
+    if (flags & ~(unsigned)(HCA_QK_NORM | HCA_OUT_GATE | HCA_PAGED | HCA_WINDOW_RING)) return HCA_ERR_UNSUPPORTED;
     if (d != kDecD || dv != kDecD || Hq % Hkv != 0 || Hq / Hkv > kDecHeads || blk > 128)
         return HCA_ERR_UNSUPPORTED;
     if (!(scale == scale) || !(eps >= 0.f)) return HCA_ERR_INVALID_ARG;

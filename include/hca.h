@@ -67,7 +67,8 @@ enum {
     HCA_OUT_GATE = 2,   /* decode: multiply the output by sigmoid(gate) */
     HCA_PAGED = 4,      /* decode: compressed cache is a page pool addressed by page_table */
     HCA_WRITE_LSE = 8,  /* prefill: also write the natural-log sum-exp of the logits */
-    HCA_OUT_F32 = 16    /* prefill: output in fp32 instead of bf16 */
+    HCA_OUT_F32 = 16,   /* prefill: output in fp32 instead of bf16 */
+    HCA_WINDOW_RING = 32 /* decode: the raw window is a ring, slot p % W holds position p */
 };
 
 /*
@@ -125,9 +126,12 @@ size_t hca_decode_workspace_size(int B, int Hq, int Hkv, int dv);
  *            pool[page_table[b*max_pages + j/page_size], j % page_size]
  *   page_table [B,max_pages] int32 (HCA_PAGED only, else NULL); num_pages = P, the
  *            number of pages in the pools (entries outside [0, P) are reported as
- *            HCA_ERR_DEVICE_INPUT and read as zeros)
+ *            HCA_ERR_DEVICE_INPUT and clamped into the pool; the output is then unspecified)
  *   kw, vw   [B,W,Hkv,d|dv] bf16  raw window: slot i holds position seqlens[b] - W + i;
- *            slots with a negative position are ignored
+ *            slots with a negative position are ignored.  With HCA_WINDOW_RING (the
+ *            layout hca_append maintains) slot p % W holds position p instead; attention
+ *            over the window does not depend on the order of its keys, so only which
+ *            slots are valid changes (slots 0 .. L_b - 1 while L_b < W)
  *   seqlens  [B] int32            context length L_b >= 1 including the new token; the
  *            visible entry count n_c(L_b - 1) must not exceed Nmax (or the pages)
  *   gq, gk   [d] fp32 gains, eps  (HCA_QK_NORM only, else NULL)
@@ -180,6 +184,42 @@ hca_status_t hca_decode_noalloc(const void* q, const void* kc, const void* vc,
                                 const void* gate, float* out,
                                 int B, int Hq, int Hkv, int d, int dv, int blk, int W, int Nmax,
                                 float scale, unsigned flags, hca_stream_t stream);
+
+/*
+ * hca_append_state_size -- bytes of pooling state hca_append keeps per batch:
+ * B * Hkv * (4 + d + dv) floats.  Returns 0 for invalid sizes.
+ */
+size_t hca_append_state_size(int B, int Hkv, int d, int dv);
+
+/*
+ * hca_append -- one decode step's cache update: the newest token of every sequence enters
+ * the raw window, and a block of blk tokens that it completes becomes one compressed entry
+ * (official blog, section 2.1: every 128 tokens are compressed into a single cached entry).
+ * The entry is the compressor's softmax-weighted mean of the block (hca_compress), computed
+ * online: no raw token has to stay resident after it leaves the window.
+ *   k_new, v_new [B,Hkv,d|dv] bf16  the newest token of each sequence, at position
+ *                seqlens[b] - 1
+ *   w_new    [B] fp32 pooling weight of that token (NULL = 0, i.e. the mean)
+ *   seqlens  [B] int32 length L_b >= 1 INCLUDING the new token
+ *   kw, vw   [B,W,Hkv,d|dv] bf16 window rings, written at slot (L_b - 1) % W; read them
+ *            with hca_decode(..., HCA_WINDOW_RING)
+ *   kc, vc   the compressed cache, laid out as for hca_decode (contiguous [B,Nmax,...], or
+ *            page pools with HCA_PAGED); entry (L_b / blk) - 1 is written when
+ *            L_b % blk == 0.  An entry outside the cache (or its pages) is reported as
+ *            HCA_ERR_DEVICE_INPUT and not written
+ *   state    hca_append_state_size(B, Hkv, d, dv) bytes of fp32 owned by the caller: the
+ *            running pool of each (sequence, KV head)'s current block.  All zero means an
+ *            empty block; set a sequence's state to zero before its first token (a call
+ *            that completes a block leaves it zero).  Tokens must be appended in order,
+ *            one call per position
+ * Supported: d, dv in {64, 128, 256, 512}; 1 <= blk <= 128; W >= 1; flags 0 or HCA_PAGED
+ * (page_size a multiple of 64).  One CTA per (sequence, KV head); the call only queues it.
+ */
+hca_status_t hca_append(const void* k_new, const void* v_new, const float* w_new, const int* seqlens,
+                        void* kw, void* vw, void* kc, void* vc,
+                        const int* page_table, int page_size, int max_pages, int num_pages,
+                        void* state, int B, int Hkv, int d, int dv, int blk, int W, int Nmax,
+                        unsigned flags, hca_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* hca_status_string(hca_status_t status);

@@ -134,3 +134,29 @@ def test_decode_rejects_before_launch(libhca):
     # nothing to do: no launch, OK
     assert call(q=None, kc=None, vc=None, kw=None, vw=None, seq=None, out=None, ws=None, B=0) == _lib.HCA_OK
 
+
+def test_append_rejects_before_launch(libhca):
+    p = ctypes.c_void_p(16)
+
+    def call(k=p, v=p, w=None, seq=p, kw=p, vw=p, kc=p, vc=p, table=None, ps=0, maxp=0, npages=0, state=p,
+             B=1, Hkv=1, d=512, dv=512, blk=128, W=128, Nmax=8, flags=0):
+        return libhca.hca_append(k, v, w, seq, kw, vw, kc, vc, table, ps, maxp, npages, state, B, Hkv, d, dv,
+                                 blk, W, Nmax, flags, None)
+
+    assert libhca.hca_append_state_size(2, 3, 512, 512) == 2 * 3 * (4 + 1024) * 4
+    assert libhca.hca_append_state_size(-1, 1, 64, 64) == 0
+    # unsupported head dims, block, flags
+    assert call(d=96) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(blk=129) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(flags=_lib.HCA_QK_NORM) == _lib.HCA_ERR_UNSUPPORTED
+    # null / misaligned pointers, bad sizes, no cache rows
+    assert call(k=None) == _lib.HCA_ERR_INVALID_ARG
+    assert call(state=ctypes.c_void_p(24)) == _lib.HCA_ERR_INVALID_ARG
+    assert call(seq=ctypes.c_void_p(18)) == _lib.HCA_ERR_INVALID_ARG
+    assert call(W=0) == _lib.HCA_ERR_INVALID_ARG
+    assert call(Nmax=0) == _lib.HCA_ERR_INVALID_ARG
+    assert call(flags=_lib.HCA_PAGED) == _lib.HCA_ERR_INVALID_ARG
+    assert call(flags=_lib.HCA_PAGED, table=p, ps=96, maxp=2, npages=2) == _lib.HCA_ERR_INVALID_ARG
+    # nothing to do: no launch, OK
+    assert call(k=None, v=None, seq=None, kw=None, vw=None, kc=None, vc=None, state=None, B=0) == _lib.HCA_OK
+
