@@ -70,6 +70,13 @@ def decode_bytes(B, L, Hq, Hkv, d, dv, blk, W):
     return B * per
 
 
+def append_bytes(B, Hkv, d, dv):
+    """hca_append when every sequence completes a block: new token read, pooling state read and
+    written, ring slot written, entry written (bytes per call)."""
+    state = (4 + d + dv) * 4
+    return B * Hkv * ((d + dv) * 2 + 2 * state + (d + dv) * 2 + (d + dv) * 2) + B * 8
+
+
 def prefill_flops(B, T, Hq, d, dv, blk, W):
     t = np.arange(T, dtype=np.int64)
     a = t - W + 1
@@ -381,6 +388,43 @@ def main():
                    "median_us_per_call": statistics.median(d_ms) * 1e3,
                    "decode_in_step_us": statistics.median(dec_in_step_ms) * 1e3}
 
+    # ---- one serving step: hca_append of every sequence's newest token (window ring write +
+    # online pooling; at L = 131072 every sequence completes a block, so an entry is written
+    # too), then hca_decode over the ring.  L2 flushed before each step.
+    kn, vn = k[:, L - 1].contiguous(), v[:, L - 1].contiguous()
+    wn = w[:, L - 1].contiguous()
+    state = torch.zeros(hca.append_state_size(B, 1, cfg.d, cfg.dv), dtype=torch.uint8, device=dev)
+
+    def serve(decode_too):
+        hca.append(kn, vn, wn, seq, kw, vw, kc, vc, state, cfg.blk)
+        if decode_too:
+            hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws, window_ring=True)
+
+    serve_part = {}
+    for name, dec in (("append_us", False), ("append_plus_decode_us", True)):
+        for _ in range(3):
+            serve(dec)
+        sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        with sampler:
+            torch.cuda._sleep(int(2e8))
+            for i in range(args.steps):
+                flush.zero_()
+                a, b = sev[i]
+                a.record(stream)
+                serve(dec)
+                b.record(stream)
+            torch.cuda.synchronize()
+        serve_part[name] = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in sev]) / 1e3,
+                                          world) * 1e6
+    hca.get_device_error()
+    abytes = append_bytes(B, 1, cfg.d, cfg.dv)
+    serve_part.update({"workload": "append + ring decode, %s" % cfg.name,
+                       "append_algorithmic_bytes": abytes,
+                       "append_frac_of_hbm": abytes / (serve_part["append_us"] / 1e6) / 1e9 / pk["hbm_gbs"],
+                       "append_bound": "latency (one small CTA per sequence; %d KB moved)" % (abytes // 1024)})
+    del state
+
     # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
     if not args.no_e2e:
@@ -481,7 +525,7 @@ def main():
                            "blk": cfg.blk, "W": cfg.W, "step": "hca_compress(raw K/V) + hca_decode",
                            "l2": "flushed (2x L2 memset) before every timed step; raw K/V 17.2 GB > L2",
                            "parallelism": "dp%d (independent batches, no collective)" % world},
-                "roofline": roof, "decode": decode_part, "prefill": prefill_part,
+                "roofline": roof, "decode": decode_part, "serving_step": serve_part, "prefill": prefill_part,
                 "cpu_baseline": cpu_base, "e2e": e2e,
                 "gpu_launches": 3 * args.steps, "clocks": clocks,
                 "libhca": os.path.relpath(_lib.LIB_PATH, ROOT)}

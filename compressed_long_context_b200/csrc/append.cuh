@@ -39,14 +39,12 @@ struct AppendParams {
     int B, Hkv, d, dv, blk, W, Nmax, page_size, max_pages, num_pages;
 };
 
-// Channels c .. c+3 of one tensor (K or V) for the current (b, g): ring write, state update
-// and, when the block completes, the entry.
-__device__ __forceinline__ void append_channels(const __nv_bfloat16* src, __nv_bfloat16* ring,
-                                                float* acc, __nv_bfloat16* entry, int c, float a,
-                                                float e, float inv_s, bool complete) {
-    const uint2 x = *reinterpret_cast<const uint2*>(src + c);
+// Channels c .. c+3 of one tensor (K or V), already loaded: ring write, state update and,
+// when the block completes, the entry.
+__device__ __forceinline__ void append_channels(uint2 x, float4 t, __nv_bfloat16* ring, float* acc,
+                                                __nv_bfloat16* entry, int c, float a, float e, float inv_s,
+                                                bool complete) {
     *reinterpret_cast<uint2*>(ring + c) = x;
-    float4 t = *reinterpret_cast<const float4*>(acc + c);
     t.x = fmaf(e, bf16lo(x.x), t.x * a);
     t.y = fmaf(e, bf16hi(x.x), t.y * a);
     t.z = fmaf(e, bf16lo(x.y), t.z * a);
@@ -60,20 +58,32 @@ __device__ __forceinline__ void append_channels(const __nv_bfloat16* src, __nv_b
     *reinterpret_cast<float4*>(acc + c) = t;
 }
 
-// One CTA per (sequence, KV head).
+// One CTA per (sequence, KV head); thread i owns channels 4i .. 4i+3 of K and of V (d, dv <=
+// 512).  Every load is issued before any result is needed -- the new token, the pooling
+// state, the weight and the length do not depend on one another -- so a call costs one
+// memory round trip after launch.
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendParams p) {
     const int u = blockIdx.x;
     const int b = u / p.Hkv, g = u - b * p.Hkv;
+    const int c = 4 * threadIdx.x;
+    const bool hk = c < p.d, hv = c < p.dv;
+    float* st = p.state + (size_t)u * (kAppendHeader + p.d + p.dv);
+    float* acc_k = st + kAppendHeader;
+    float* acc_v = st + kAppendHeader + p.d;
     const int L = __ldg(p.seqlens + b);
+    const float w = p.w ? __ldg(p.w + b) : 0.f;
+    const float2 ms = *reinterpret_cast<const float2*>(st);
+    const uint2 xk = hk ? *reinterpret_cast<const uint2*>(p.k_new + (size_t)u * p.d + c) : make_uint2(0u, 0u);
+    const uint2 xv = hv ? *reinterpret_cast<const uint2*>(p.v_new + (size_t)u * p.dv + c) : make_uint2(0u, 0u);
+    const float4 tk = hk ? *reinterpret_cast<const float4*>(acc_k + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 tv = hv ? *reinterpret_cast<const float4*>(acc_v + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     if (L < 1) {
         if (threadIdx.x == 0) record_error(HCA_ERR_DEVICE_INPUT);
         return;
     }
     const long long pos = (long long)L - 1;
     const int slot = (int)(pos % p.W);
-    float* st = p.state + (size_t)u * (kAppendHeader + p.d + p.dv);
-    const float w = p.w ? __ldg(p.w + b) : 0.f;
-    const float m_old = st[0], s_old = st[1];
+    const float m_old = ms.x, s_old = ms.y;
     const bool empty = !(s_old > 0.f);
     const float m_new = empty ? w : fmaxf(m_old, w);
     const float a = empty ? 0.f : expf(m_old - m_new);
@@ -103,17 +113,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendPara
     }
     const float inv_s = 1.f / s_new;
     const size_t ring_row = (size_t)b * p.W + slot;
-    for (int c = 4 * threadIdx.x; c < p.d; c += 4 * kAppendThreads)
-        append_channels(p.k_new + (size_t)u * p.d, p.kw + (ring_row * p.Hkv + g) * p.d, st + kAppendHeader, ek, c,
-                        a, e, inv_s, complete);
-    for (int c = 4 * threadIdx.x; c < p.dv; c += 4 * kAppendThreads)
-        append_channels(p.v_new + (size_t)u * p.dv, p.vw + (ring_row * p.Hkv + g) * p.dv,
-                        st + kAppendHeader + p.d, ev, c, a, e, inv_s, complete);
+    if (hk) append_channels(xk, tk, p.kw + (ring_row * p.Hkv + g) * p.d, acc_k, ek, c, a, e, inv_s, complete);
+    if (hv) append_channels(xv, tv, p.vw + (ring_row * p.Hkv + g) * p.dv, acc_v, ev, c, a, e, inv_s, complete);
     __syncthreads();      // every thread has read m and s
-    if (threadIdx.x == 0) {
-        st[0] = complete ? 0.f : m_new;
-        st[1] = complete ? 0.f : s_new;
-    }
+    if (threadIdx.x == 0) *reinterpret_cast<float2*>(st) = complete ? make_float2(0.f, 0.f) : make_float2(m_new, s_new);
 }
 
 }  // namespace hca
