@@ -6,5 +6,5 @@ the CUDA library in ``compressed_long_context_b200``.
 """
 from .oracle import (  # noqa: F401
     compress, round_bf16, visible_entries, prefill_rows, decode, num_threads,
-    bf16_bits, bits_to_f64,
+    bf16_bits, bits_to_f64, vha,
 )

@@ -171,3 +171,21 @@ def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size
     if rc:
         raise ValueError("oracle_decode rejected its arguments (%d)" % rc)
     return (out, lse) if want_lse else out
+
+
+def vha(out, U, V):
+    """Virtual Head Attention, the reading of the pages' "cross-head low-rank mixing with an
+    identity skip" (official blog, section 2.1; Zhidx article, section "1. Latent-Gated
+    Sparse Attention"): per token and per channel c, o'[:, c] = (I + U V^T) o[:, c] over the
+    token's Hq heads, with U, V of shape [Hq, r].  Applied to the final attention output.
+
+    out [n, Hq, dv] (any float), U, V [Hq, r] float32.  Returns fp64 [n, Hq, dv].
+    Plain numpy in fp64: t = V^T o (r values per channel), then o + U t.
+    """
+    o = np.asarray(out, dtype=np.float64)
+    U = np.asarray(U, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    assert o.ndim == 3 and U.shape == V.shape and U.shape[0] == o.shape[1]
+    t = np.einsum("hk,nhc->nkc", V, o)
+    return o + np.einsum("hk,nkc->nhc", U, t)
+

@@ -392,3 +392,50 @@ def test_decode_rejects_short_cache():
     q, kc, vc, kw, vw, seq = _small_decode_case(120)
     with pytest.raises(ValueError):
         oracle.decode(q, kc[:, :3], vc[:, :3], kw, vw, seq, 128, 64, 0.125)
+
+
+# ------------------------------------------------------------------ VHA (cross-head mixing)
+
+def test_vha_zero_factor_is_identity():
+    rs = np.random.RandomState(0)
+    o = rs.randn(3, 8, 16)
+    U = rs.randn(8, 2).astype(np.float32)
+    np.testing.assert_array_equal(oracle.vha(o, U, np.zeros_like(U)), o)
+    np.testing.assert_array_equal(oracle.vha(o, np.zeros_like(U), U), o)
+
+
+def test_vha_rank_one_closed_form():
+    """U = e_i, V = e_j: head i gains head j's output, every other head is unchanged."""
+    rs = np.random.RandomState(1)
+    o = rs.randn(2, 6, 5)
+    U = np.zeros((6, 1), np.float32)
+    V = np.zeros((6, 1), np.float32)
+    U[4, 0] = 1.0
+    V[1, 0] = 1.0
+    got = oracle.vha(o, U, V)
+    want = o.copy()
+    want[:, 4] += o[:, 1]
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+
+
+def test_vha_factor_gauge_invariance():
+    """(U A, V A^-T) is the same mixing matrix as (U, V) for any invertible A."""
+    rs = np.random.RandomState(2)
+    o = rs.randn(4, 16, 7)
+    U = rs.randn(16, 3)
+    V = rs.randn(16, 3)
+    A = rs.randn(3, 3) + 3 * np.eye(3)
+    got = oracle.vha(o, U @ A, V @ np.linalg.inv(A).T)
+    np.testing.assert_allclose(got, oracle.vha(o, U, V), rtol=1e-11, atol=1e-11)
+
+
+def test_vha_equals_dense_mixing_matrix():
+    """Channel by channel, the result is the dense (I + U V^T) applied to the head vector."""
+    rs = np.random.RandomState(3)
+    o = rs.randn(2, 12, 9)
+    U = rs.randn(12, 4).astype(np.float32)
+    V = rs.randn(12, 4).astype(np.float32)
+    M = np.eye(12) + U.astype(np.float64) @ V.astype(np.float64).T
+    want = np.stack([np.stack([M @ o[n, :, c] for c in range(9)], axis=1) for n in range(2)])
+    np.testing.assert_allclose(oracle.vha(o, U, V), want, rtol=1e-12, atol=1e-12)
+
