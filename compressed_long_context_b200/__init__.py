@@ -17,7 +17,7 @@ from ._lib import (HCA_OUT_F32, HCA_OUT_GATE, HCA_PAGED, HCA_QK_NORM,  # noqa: F
                    HCA_WINDOW_RING, HCA_WRITE_LSE)
 
 __all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "append", "append_state_size",
-           "get_device_error", "status_string"]
+           "vha", "get_device_error", "status_string"]
 
 
 class HCAError(RuntimeError):
@@ -201,4 +201,23 @@ def append(k_new, v_new, w_new, seqlens, kw, vw, kc, vc, state, blk, page_table=
                                 _p(page_table), int(page_size), int(max_pages), int(num_pages), _p(state),
                                 B, Hkv, d, dv, int(blk), int(W), int(Nmax), flags, _stream(dev))
     _check(rc, "hca_append")
+
+
+def vha(out, U, V):
+    """Virtual Head Attention in place on an attention output ``out`` [..., Hq, dv] (bf16 or
+    fp32): per token and channel, out[:, c] <- (I + U V^T) out[:, c] over the heads.
+    U, V [Hq, r] fp32.  Returns ``out``."""
+    if out.dtype not in (torch.bfloat16, torch.float32) or not out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 or fp32 CUDA tensor")
+    dev = out.device
+    _need(U, torch.float32, "U", dev)
+    _need(V, torch.float32, "V", dev)
+    Hq, dv = out.shape[-2], out.shape[-1]
+    n = out.numel() // (Hq * dv)
+    r = U.shape[1]
+    if U.shape != (Hq, r) or V.shape != (Hq, r):
+        raise ValueError("U and V must both be [Hq, r]")
+    flags = HCA_OUT_F32 if out.dtype == torch.float32 else 0
+    _check(_lib.load().hca_vha(_p(out), _p(U), _p(V), int(n), Hq, dv, r, flags, _stream(dev)), "hca_vha")
+    return out
 

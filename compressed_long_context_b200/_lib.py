@@ -22,7 +22,7 @@ HCA_WINDOW_RING = 32
 
 # Names of every entry point declared in include/hca.h.
 EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_decode", "hca_decode_noalloc",
-           "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error")
+           "hca_vha", "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error")
 
 _lib = None
 
@@ -58,6 +58,8 @@ def load():
     lib.hca_decode_noalloc.restype = _i
     lib.hca_decode_noalloc.argtypes = ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp]
                                        + [_i] * 8 + [_f, _u, _vp])
+    lib.hca_vha.restype = _i
+    lib.hca_vha.argtypes = [_vp, _vp, _vp, ctypes.c_longlong, _i, _i, _i, _u, _vp]
     lib.hca_append_state_size.restype = _sz
     lib.hca_append_state_size.argtypes = [_i] * 4
     lib.hca_append.restype = _i

@@ -12,6 +12,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "prefill_pair.cuh"
+#include "vha.cuh"
 
 namespace {
 
@@ -155,6 +156,27 @@ hca_status_t hca_compress(const void* k, const void* v, const float* w, void* kc
 #undef HCA_COMPRESS_ROW
 #undef HCA_COMPRESS_CASE
     return HCA_ERR_UNSUPPORTED;
+}
+
+hca_status_t hca_vha(void* out, const float* U, const float* V, long long n, int Hq, int dv, int r,
+                     unsigned flags, hca_stream_t stream) {
+    if (n < 0 || Hq < 1 || dv < 1 || r < 1) return HCA_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)HCA_OUT_F32) return HCA_ERR_UNSUPPORTED;
+    if (Hq > hca::kVhaMaxHeads || r > hca::kVhaMaxRank || dv % hca::kVhaCh) return HCA_ERR_UNSUPPORTED;
+    if (n == 0) return HCA_OK;
+    const long long blocks = n * (dv / hca::kVhaCh);
+    if (blocks > 0x7fffffffLL) return HCA_ERR_INVALID_ARG;
+    if (!out || !U || !V || !aligned16(out) || (reinterpret_cast<uintptr_t>(U) & 3) ||
+        (reinterpret_cast<uintptr_t>(V) & 3))
+        return HCA_ERR_INVALID_ARG;
+    hca::VhaParams p;
+    p.out = out; p.U = U; p.V = V; p.n = n; p.Hq = Hq; p.dv = dv; p.r = r;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (flags & HCA_OUT_F32)
+        hca::vha_kernel<true><<<(unsigned)blocks, hca::kVhaThreads, 0, s>>>(p);
+    else
+        hca::vha_kernel<false><<<(unsigned)blocks, hca::kVhaThreads, 0, s>>>(p);
+    return launch_status();
 }
 
 size_t hca_append_state_size(int B, int Hkv, int d, int dv) {

@@ -186,6 +186,20 @@ hca_status_t hca_decode_noalloc(const void* q, const void* kc, const void* vc,
                                 float scale, unsigned flags, hca_stream_t stream);
 
 /*
+ * hca_vha -- Virtual Head Attention on an attention output, in place (official blog, section
+ * 2.1, and the Zhidx article, section "1. Latent-Gated Sparse Attention": a lightweight
+ * cross-head low-rank mixing with an identity skip after the attention).  Per token and per
+ * channel c: out[:, c] <- (I + U V^T) out[:, c] over the token's Hq heads.
+ *   out    [n,Hq,dv] bf16, or fp32 with HCA_OUT_F32 (a prefill output is n = B*T tokens, a
+ *          decode output n = B); applied after the decode gate, to the final output
+ *   U, V   [Hq,r] fp32 mixing factors (4-byte aligned)
+ * Supported: Hq <= 64, 1 <= r <= 32, dv a multiple of 64; flags 0 or HCA_OUT_F32.  The
+ * kernel reads and writes the output once.
+ */
+hca_status_t hca_vha(void* out, const float* U, const float* V, long long n, int Hq, int dv, int r,
+                     unsigned flags, hca_stream_t stream);
+
+/*
  * hca_append_state_size -- bytes of pooling state hca_append keeps per batch:
  * B * Hkv * (4 + d + dv) floats.  Returns 0 for invalid sizes.
  */

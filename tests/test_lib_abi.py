@@ -160,3 +160,16 @@ def test_append_rejects_before_launch(libhca):
     # nothing to do: no launch, OK
     assert call(k=None, v=None, seq=None, kw=None, vw=None, kc=None, vc=None, state=None, B=0) == _lib.HCA_OK
 
+
+def test_vha_rejects_before_launch(libhca):
+    p = ctypes.c_void_p(16)
+    # (out, U, V, n, Hq, dv, r, flags, stream)
+    assert libhca.hca_vha(p, p, p, 4, 65, 512, 4, 0, None) == _lib.HCA_ERR_UNSUPPORTED     # more than 64 heads
+    assert libhca.hca_vha(p, p, p, 4, 64, 512, 33, 0, None) == _lib.HCA_ERR_UNSUPPORTED    # rank above 32
+    assert libhca.hca_vha(p, p, p, 4, 64, 96, 4, 0, None) == _lib.HCA_ERR_UNSUPPORTED      # dv not a multiple of 64
+    assert libhca.hca_vha(p, p, p, 4, 64, 512, 4, 1 << 8, None) == _lib.HCA_ERR_UNSUPPORTED
+    assert libhca.hca_vha(None, p, p, 4, 64, 512, 4, 0, None) == _lib.HCA_ERR_INVALID_ARG
+    assert libhca.hca_vha(ctypes.c_void_p(24), p, p, 4, 64, 512, 4, 0, None) == _lib.HCA_ERR_INVALID_ARG
+    assert libhca.hca_vha(p, p, p, 4, 64, 512, 0, 0, None) == _lib.HCA_ERR_INVALID_ARG
+    assert libhca.hca_vha(None, None, None, 0, 64, 512, 4, 0, None) == _lib.HCA_OK          # nothing to do
+

@@ -1,0 +1,112 @@
+"""GPU parity of hca_vha (Virtual Head Attention on an attention output) against the fp64
+oracle.
+
+ - After attention: the oracle's attention output (prefill rows or decode, gate included)
+   followed by the oracle's cross-head mixing; fp32 outputs, bar max abs 1e-2 and mean abs
+   1e-3.
+ - The bf16 path on its own: seeded bf16 inputs (not from the CUDA path), each result
+   within one bf16 rounding of the fp64 mixing of the same values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import compressed_long_context_b200 as hca
+import oracle
+
+pytestmark = pytest.mark.gpu
+MAX_TOL, MEAN_TOL = 1e-2, 1e-3
+
+
+def bits(t):
+    return oracle.bf16_bits(t)
+
+
+def check(got, ref):
+    g = got.detach().float().cpu().numpy().astype(np.float64)
+    assert g.shape == ref.shape and np.isfinite(g).all()
+    err = np.abs(g - ref)
+    assert err.max() <= MAX_TOL, ("max", err.max())
+    assert err.mean() <= MEAN_TOL, ("mean", err.mean())
+
+
+def factors(dev, Hq, r, seed, std=0.1):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    U = torch.randn((Hq, r), generator=g, device=dev) * std
+    V = torch.randn((Hq, r), generator=g, device=dev) * std
+    return U, V
+
+
+@pytest.mark.parametrize("r", [1, 8, 32])
+def test_vha_after_gated_decode(cuda_device, libhca, r):
+    dev = cuda_device
+    g = torch.Generator(device=dev).manual_seed(40 + r)
+    B, Hq, W, blk = 4, 64, 128, 128
+    lengths = [9000, 130, 20000, 700]
+    Nmax = max(oracle.visible_entries(L - 1, W, blk) for L in lengths)
+    q = torch.randn((B, Hq, 512), generator=g, device=dev).to(torch.bfloat16)
+    kc = torch.randn((B, Nmax, 1, 512), generator=g, device=dev).to(torch.bfloat16)
+    vc = torch.randn((B, Nmax, 1, 512), generator=g, device=dev).to(torch.bfloat16)
+    kw = torch.randn((B, W, 1, 512), generator=g, device=dev).to(torch.bfloat16)
+    vw = torch.randn((B, W, 1, 512), generator=g, device=dev).to(torch.bfloat16)
+    gate = torch.randn((B, Hq, 512), generator=g, device=dev).to(torch.bfloat16)
+    seq = torch.tensor(lengths, dtype=torch.int32, device=dev)
+    U, V = factors(dev, Hq, r, 50 + r)
+    scale = 1.0 / np.sqrt(512)
+    out = hca.decode(q, kc, vc, kw, vw, seq, blk, W, scale, gate=gate)
+    hca.vha(out, U, V)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    ref = oracle.decode(bits(q), bits(kc), bits(vc), bits(kw), bits(vw), seq.cpu().numpy(), blk, W, scale,
+                        gate=bits(gate))
+    check(out, oracle.vha(ref, U.cpu().numpy(), V.cpu().numpy()))
+
+
+@pytest.mark.parametrize("d,Hq,r", [(512, 64, 4), (512, 64, 16), (64, 8, 2), (64, 32, 32)])
+def test_vha_after_prefill(cuda_device, libhca, d, Hq, r):
+    dev = cuda_device
+    g = torch.Generator(device=dev).manual_seed(60 + d + Hq + r)
+    B, T, blk, W = 1, 400, 128, 128
+    q = torch.randn((B, T, Hq, d), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((B, T, 1, d), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((B, T, 1, d), generator=g, device=dev).to(torch.bfloat16)
+    w = torch.randn((B, T), generator=g, device=dev) * 0.5
+    U, V = factors(dev, Hq, r, 70 + r)
+    scale = 1.0 / np.sqrt(d)
+    kc, vc = hca.compress(k, v, w, blk)
+    out = hca.prefill(q, k, v, kc, vc, blk, W, scale, out_f32=True)
+    hca.vha(out, U, V)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    okc, ovc = oracle.compress(bits(k), bits(v), w.cpu().numpy(), blk)
+    rows = [(0, t) for t in range(T)]
+    ref = oracle.prefill_rows(bits(q), bits(k), bits(v), oracle.round_bf16(okc), oracle.round_bf16(ovc), blk, W,
+                              scale, rows)
+    check(out[0], oracle.vha(ref, U.cpu().numpy(), V.cpu().numpy()))
+
+
+@pytest.mark.parametrize("n,Hq,dv,r", [(300, 64, 512, 8), (7, 16, 64, 32), (50, 64, 128, 1)])
+def test_vha_bf16_within_one_rounding(cuda_device, libhca, n, Hq, dv, r):
+    dev = cuda_device
+    g = torch.Generator(device=dev).manual_seed(80 + n + r)
+    x = (torch.randn((n, Hq, dv), generator=g, device=dev) * 2.0).to(torch.bfloat16)
+    U, V = factors(dev, Hq, r, 90 + r, std=0.2)
+    ref = oracle.vha(oracle.bits_to_f64(bits(x)), U.cpu().numpy(), V.cpu().numpy())
+    y = x.clone()
+    hca.vha(y, U, V)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    got = y.float().cpu().numpy().astype(np.float64)
+    # bf16 keeps 8 significant bits: a correctly rounded value is within 2^-9 |ref| (plus the
+    # fp32 arithmetic's own error, far smaller), so 2^-8 |ref| + 1e-6 allows one ulp
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
+
+
+def test_vha_zero_factor_leaves_output_unchanged(cuda_device, libhca):
+    dev = cuda_device
+    x = torch.randn((5, 16, 128), device=dev).to(torch.bfloat16)
+    y = x.clone()
+    U = torch.randn((16, 3), device=dev)
+    hca.vha(y, U, torch.zeros_like(U))
+    torch.cuda.synchronize()
+    assert torch.equal(x, y)
