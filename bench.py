@@ -508,6 +508,27 @@ def main():
                                      "traffic": traffic_for("prefill_T131072",
                                                             ["compressed_long_context_b200/csrc/prefill.cuh",
                                                              "compressed_long_context_b200/csrc/prefill_pair.cuh"])}}
+        # Virtual Head Attention on the prefill output (in place, bf16): one read and one write
+        # of the 8.6 GB output, HBM-bound; synthetic rank-8 factors
+        gv = torch.Generator(device=dev).manual_seed(5)
+        vu = torch.randn((pc.Hq, 8), generator=gv, device=dev) * 0.1
+        vv = torch.randn((pc.Hq, 8), generator=gv, device=dev) * 0.1
+        hca.vha(pout, vu, vv)
+        vev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(np_steps)]
+        with sampler:
+            for i in range(np_steps):
+                a, b = vev[i]
+                a.record(stream)
+                hca.vha(pout, vu, vv)
+                b.record(stream)
+            torch.cuda.synchronize()
+        hca.get_device_error()
+        v_ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in vev]), world)
+        vbytes = 2 * pout.numel() * pout.element_size() + 2 * vu.numel() * 4
+        prefill_part["vha"] = {"ms": v_ms, "rank": 8, "algorithmic_bytes": vbytes, "bound": "hbm",
+                               "achieved_gbs": vbytes / (v_ms / 1e3) / 1e9,
+                               "frac": vbytes / (v_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                               "peak_kind": pk_kind + " (hbm_gbs)"}
         del pin, pkc, pvc, pout
         torch.cuda.empty_cache()
 

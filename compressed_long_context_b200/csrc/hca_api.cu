@@ -158,26 +158,48 @@ hca_status_t hca_compress(const void* k, const void* v, const float* w, void* kc
     return HCA_ERR_UNSUPPORTED;
 }
 
-hca_status_t hca_vha(void* out, const float* U, const float* V, long long n, int Hq, int dv, int r,
-                     unsigned flags, hca_stream_t stream) {
+}  // extern "C"
+
+namespace {
+template <bool F32, int RP>
+hca_status_t vha_launch(const hca::VhaParams& p, cudaStream_t s) {
+    const auto kern = hca::vha_kernel<F32, RP>;
+    const int smem = hca::vha_smem_bytes(p.Hq, RP, F32);      // <= 32 KB: no opt-in needed
+    const int sms = hca::num_sms();
+    int per_sm = 0;
+    if (sms <= 0 || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hca::kVhaThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        return HCA_ERR_CUDA;
+    // persistent: every resident CTA slot filled once, warps stride over the work items
+    const long long items = p.n * (p.dv / (F32 ? 32 : 64));
+    const long long need = (items + hca::kVhaThreads / 32 - 1) / (hca::kVhaThreads / 32);
+    const long long grid = std::min<long long>(need, (long long)sms * per_sm);
+    kern<<<(unsigned)grid, hca::kVhaThreads, smem, s>>>(p);
+    return launch_status();
+}
+}  // namespace
+
+extern "C" hca_status_t hca_vha(void* out, const float* U, const float* V, long long n, int Hq, int dv, int r,
+                                unsigned flags, hca_stream_t stream) {
     if (n < 0 || Hq < 1 || dv < 1 || r < 1) return HCA_ERR_INVALID_ARG;
     if (flags & ~(unsigned)HCA_OUT_F32) return HCA_ERR_UNSUPPORTED;
     if (Hq > hca::kVhaMaxHeads || r > hca::kVhaMaxRank || dv % hca::kVhaCh) return HCA_ERR_UNSUPPORTED;
     if (n == 0) return HCA_OK;
-    const long long blocks = n * (dv / hca::kVhaCh);
-    if (blocks > 0x7fffffffLL) return HCA_ERR_INVALID_ARG;
     if (!out || !U || !V || !aligned16(out) || (reinterpret_cast<uintptr_t>(U) & 3) ||
         (reinterpret_cast<uintptr_t>(V) & 3))
         return HCA_ERR_INVALID_ARG;
     hca::VhaParams p;
     p.out = out; p.U = U; p.V = V; p.n = n; p.Hq = Hq; p.dv = dv; p.r = r;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (flags & HCA_OUT_F32)
-        hca::vha_kernel<true><<<(unsigned)blocks, hca::kVhaThreads, 0, s>>>(p);
-    else
-        hca::vha_kernel<false><<<(unsigned)blocks, hca::kVhaThreads, 0, s>>>(p);
-    return launch_status();
+    const bool f32 = flags & HCA_OUT_F32;
+    // rank padded with zero factors to the next of 4, 8, 16, 32
+    if (r <= 4) return f32 ? vha_launch<true, 4>(p, s) : vha_launch<false, 4>(p, s);
+    if (r <= 8) return f32 ? vha_launch<true, 8>(p, s) : vha_launch<false, 8>(p, s);
+    if (r <= 16) return f32 ? vha_launch<true, 16>(p, s) : vha_launch<false, 16>(p, s);
+    return f32 ? vha_launch<true, 32>(p, s) : vha_launch<false, 32>(p, s);
 }
+
+extern "C" {
 
 size_t hca_append_state_size(int B, int Hkv, int d, int dv) {
     if (B < 0 || Hkv < 1 || d < 0 || dv < 0) return 0;

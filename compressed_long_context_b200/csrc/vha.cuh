@@ -4,18 +4,23 @@
 // attention).  Reading: per token and per channel c, o'[:, c] = (I + U V^T) o[:, c] over the
 // token's Hq heads, with U, V of shape [Hq, r].
 //
-// In place on out [n, Hq, dv] (bf16 or fp32).  One CTA per (token, 64-channel slice): the
-// slice's Hq x 64 values go to shared memory with 16-byte loads, t = V^T o (r x 64) is
-// reduced over the heads, and o + U t is written back.  The kernel reads and writes the
-// output once: it is bound by HBM bandwidth.
+// In place on out [n, Hq, dv] (bf16 or fp32).  Work item = (token, slice of 64 bf16 or 32
+// fp32 channels), one warp each: lane l holds one 32-bit word of every head row (two bf16
+// channels, or one fp32 channel) in registers, so the reduction over heads, t = V^T o
+// (r values per channel), runs inside the lane with no shared-memory traffic for the data;
+// o + U t is written back over the same words.  U and V sit in shared memory, padded with
+// zeros to a power-of-two rank RP >= 4 (zero terms add nothing), and are read as broadcasts.  Both
+// products use the two-wide fp32 FMA, each lane of which rounds like fmaf.  The output is
+// read and written once: HBM-bound when the FMA work per byte is small (2 Hq r FMAs per
+// channel; at Hq 64 the rank-8 mixing is about 1000 FMAs per 2-byte channel).
 #pragma once
 
 #include "common.cuh"
 
 namespace hca {
 
-constexpr int kVhaThreads = 256;
-constexpr int kVhaCh = 64;          // channels per CTA
+constexpr int kVhaThreads = 128;    // 4 warps, each its own work item
+constexpr int kVhaCh = 64;          // dv must be a multiple of this
 constexpr int kVhaMaxHeads = 64;
 constexpr int kVhaMaxRank = 32;
 
@@ -27,66 +32,111 @@ struct VhaParams {
     int Hq, dv, r;
 };
 
-template <bool F32>
+// Factor copies in shared memory: [Hq][RP] each, and for bf16 every value twice, so that one
+// 16-byte broadcast load yields the (u, u) pairs the two-channel FMA takes.
+__host__ __device__ inline int vha_smem_bytes(int Hq, int rp, bool f32) { return 2 * Hq * rp * (f32 ? 1 : 2) * 4; }
+
+// 16-byte shared-memory load kept where it is written: the factors are loop-invariant, and a
+// compiler that hoists their Hq * RP values out of the work-item loop spills.
+__device__ __forceinline__ float4 vha_lds4(uint32_t addr) {
+    float4 f;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(addr));
+    return f;
+}
+
+template <bool F32, int RP>
 __global__ void __launch_bounds__(kVhaThreads) vha_kernel(const VhaParams p) {
-    __shared__ __align__(16) float o_s[kVhaMaxHeads * kVhaCh];
-    __shared__ float t_s[kVhaMaxRank * kVhaCh];
-    __shared__ float u_s[kVhaMaxHeads * kVhaMaxRank];
-    __shared__ float v_s[kVhaMaxHeads * kVhaMaxRank];
-    const int slices = p.dv / kVhaCh;
-    const long long tok = blockIdx.x / slices;
-    const int c0 = (int)(blockIdx.x - tok * slices) * kVhaCh;
-    const int tid = threadIdx.x;
-    const int hr = p.Hq * p.r;
-    for (int i = tid; i < hr; i += kVhaThreads) {
-        u_s[i] = __ldg(p.U + i);
-        v_s[i] = __ldg(p.V + i);
-    }
-    // the slice: head h, channels c0 .. c0+63, 16 bytes per load
-    const size_t base = (size_t)tok * p.Hq * p.dv + c0;
-    constexpr int vec = F32 ? 4 : 8;                  // channels per 16-byte load
-    constexpr int per_row = kVhaCh / vec;
-    for (int i = tid; i < p.Hq * per_row; i += kVhaThreads) {
-        const int h = i / per_row, c = (i - h * per_row) * vec;
-        if constexpr (F32) {
-            const float4 x = *reinterpret_cast<const float4*>(static_cast<const float*>(p.out) + base +
-                                                              (size_t)h * p.dv + c);
-            *reinterpret_cast<float4*>(o_s + h * kVhaCh + c) = x;
-        } else {
-            const uint4 x = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.out) + base +
-                                                            (size_t)h * p.dv + c);
-            float* d = o_s + h * kVhaCh + c;
-            d[0] = bf16lo(x.x); d[1] = bf16hi(x.x); d[2] = bf16lo(x.y); d[3] = bf16hi(x.y);
-            d[4] = bf16lo(x.z); d[5] = bf16hi(x.z); d[6] = bf16lo(x.w); d[7] = bf16hi(x.w);
+    // RP * kS a multiple of 4: whole 16-byte loads per head row, and v_s (after Hq rows of
+    // u_s) 16-byte aligned for any Hq
+    static_assert(RP >= 4 && RP % 4 == 0, "rank padded to a multiple of 4");
+    constexpr int kS = F32 ? 1 : 2;                  // stored copies of each factor value
+    constexpr int kQ = RP * kS / 4;                  // float4 loads per head row of a factor
+    constexpr int kT = F32 ? RP / 2 : RP;            // float2 accumulators of t per lane
+    extern __shared__ __align__(16) float vsm[];
+    float* u_s = vsm;
+    float* v_s = vsm + p.Hq * RP * kS;
+    for (int i = threadIdx.x; i < p.Hq * RP; i += kVhaThreads) {
+        const int h = i / RP, k = i - h * RP;
+        const float u = k < p.r ? __ldg(p.U + h * p.r + k) : 0.f;
+        const float v = k < p.r ? __ldg(p.V + h * p.r + k) : 0.f;
+#pragma unroll
+        for (int e = 0; e < kS; ++e) {
+            u_s[i * kS + e] = u;
+            v_s[i * kS + e] = v;
         }
     }
     __syncthreads();
-    // t[k][c] = sum_h V[h][k] o[h][c]
-    for (int i = tid; i < p.r * kVhaCh; i += kVhaThreads) {
-        const int k = i / kVhaCh, c = i - k * kVhaCh;
-        float acc = 0.f;
-        for (int h = 0; h < p.Hq; ++h) acc = fmaf(v_s[h * p.r + k], o_s[h * kVhaCh + c], acc);
-        t_s[i] = acc;
-    }
-    __syncthreads();
-    // o'[h][c] = o[h][c] + sum_k U[h][k] t[k][c], written back in the output's type
-    for (int i = tid; i < p.Hq * per_row; i += kVhaThreads) {
-        const int h = i / per_row, c = (i - h * per_row) * vec;
-        float y[vec];
+    const int lane = threadIdx.x & 31;
+    const int slices = p.dv / (F32 ? 32 : 64);
+    const long long items = p.n * slices;
+    const long long stride = (long long)gridDim.x * (kVhaThreads / 32);
+    const int row_words = F32 ? p.dv : p.dv / 2;     // 32-bit words per head row
+    uint32_t* out = static_cast<uint32_t*>(p.out);
+    for (long long item = (long long)blockIdx.x * (kVhaThreads / 32) + (threadIdx.x >> 5); item < items;
+         item += stride) {
+        // factor bases re-derived per item (opaque to the compiler), so that their per-head
+        // addresses are not hoisted out of the loop and kept live in registers
+        uint32_t vb = smem_u32(v_s), ub = smem_u32(u_s);
+        asm volatile("" : "+r"(vb), "+r"(ub));
+        const long long tok = item / slices;
+        uint32_t* row = out + tok * p.Hq * row_words + (item - tok * slices) * 32 + lane;
+        uint32_t x[kVhaMaxHeads];
+        {
+            const uint32_t* src = row;
 #pragma unroll
-        for (int e = 0; e < vec; ++e) y[e] = o_s[h * kVhaCh + c + e];
-        for (int k = 0; k < p.r; ++k) {
-            const float u = u_s[h * p.r + k];
-#pragma unroll
-            for (int e = 0; e < vec; ++e) y[e] = fmaf(u, t_s[k * kVhaCh + c + e], y[e]);
+            for (int h = 0; h < kVhaMaxHeads; ++h) {
+                if (h < p.Hq) x[h] = *src;
+                src += row_words;
+                asm volatile("" : "+l"(src));      // one live address: the chain is not unrolled into 64
+
+            }
         }
-        if constexpr (F32) {
-            *reinterpret_cast<float4*>(static_cast<float*>(p.out) + base + (size_t)h * p.dv + c) =
-                make_float4(y[0], y[1], y[2], y[3]);
-        } else {
-            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + base + (size_t)h * p.dv + c) =
-                make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                           pack_bf16x2(y[6], y[7]));
+        // t = V^T o.  bf16: t[k] = (t_k at channel 2l, at 2l+1); fp32: t[j] = (t_2j, t_2j+1).
+        float2 t[kT];
+#pragma unroll
+        for (int j = 0; j < kT; ++j) t[j] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < kVhaMaxHeads; ++h) {
+            if (h < p.Hq) {
+                const uint32_t vh = vb + h * RP * kS * 4;
+                const float2 xx = F32 ? make_float2(__uint_as_float(x[h]), __uint_as_float(x[h]))
+                                      : make_float2(__uint_as_float(x[h] << 16), __uint_as_float(x[h] & 0xffff0000u));
+#pragma unroll
+                for (int q = 0; q < kQ; ++q) {
+                    const float4 f = vha_lds4(vh + 16 * q);
+                    t[2 * q] = __ffma2_rn(make_float2(f.x, f.y), xx, t[2 * q]);
+                    t[2 * q + 1] = __ffma2_rn(make_float2(f.z, f.w), xx, t[2 * q + 1]);
+                }
+            }
+        }
+        // o' = o + U t, over the words just read
+        uint32_t* dst = row;
+#pragma unroll
+        for (int h = 0; h < kVhaMaxHeads; ++h) {
+            if (h < p.Hq) {
+                const uint32_t uh = ub + h * RP * kS * 4;
+                if constexpr (F32) {
+                    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int q = 0; q < kQ; ++q) {
+                        const float4 f = vha_lds4(uh + 16 * q);
+                        acc = __ffma2_rn(make_float2(f.x, f.y), t[2 * q], acc);
+                        acc = __ffma2_rn(make_float2(f.z, f.w), t[2 * q + 1], acc);
+                    }
+                    *dst = __float_as_uint(__uint_as_float(x[h]) + (acc.x + acc.y));
+                } else {
+                    float2 y = make_float2(__uint_as_float(x[h] << 16), __uint_as_float(x[h] & 0xffff0000u));
+#pragma unroll
+                    for (int q = 0; q < kQ; ++q) {
+                        const float4 f = vha_lds4(uh + 16 * q);
+                        y = __ffma2_rn(make_float2(f.x, f.y), t[2 * q], y);
+                        y = __ffma2_rn(make_float2(f.z, f.w), t[2 * q + 1], y);
+                    }
+                    *dst = pack_bf16x2(y.x, y.y);
+                }
+            }
+            dst += row_words;
+            asm volatile("" : "+l"(dst));
         }
     }
 }

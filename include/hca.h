@@ -190,11 +190,15 @@ hca_status_t hca_decode_noalloc(const void* q, const void* kc, const void* vc,
  * 2.1, and the Zhidx article, section "1. Latent-Gated Sparse Attention": a lightweight
  * cross-head low-rank mixing with an identity skip after the attention).  Per token and per
  * channel c: out[:, c] <- (I + U V^T) out[:, c] over the token's Hq heads.
- *   out    [n,Hq,dv] bf16, or fp32 with HCA_OUT_F32 (a prefill output is n = B*T tokens, a
- *          decode output n = B); applied after the decode gate, to the final output
+ *   out    [n,Hq,dv] bf16, or fp32 with HCA_OUT_F32, 16-byte aligned (a prefill output is
+ *          n = B*T tokens, a decode output n = B); applied after the decode gate, to the final
+ *          output
  *   U, V   [Hq,r] fp32 mixing factors (4-byte aligned)
  * Supported: Hq <= 64, 1 <= r <= 32, dv a multiple of 64; flags 0 or HCA_OUT_F32.  The
- * kernel reads and writes the output once.
+ * kernel reads and writes the output once; it computes in fp32 (the rank padded with zero
+ * factors to 4, 8, 16 or 32) and rounds once to the output type.  Errors (nothing launched):
+ * HCA_ERR_INVALID_ARG for null or misaligned pointers and negative sizes,
+ * HCA_ERR_UNSUPPORTED outside the supported shapes or for other flags.
  */
 hca_status_t hca_vha(void* out, const float* U, const float* V, long long n, int Hq, int dv, int r,
                      unsigned flags, hca_stream_t stream);
