@@ -80,6 +80,17 @@ __global__ void __launch_bounds__(kVhaThreads) vha_kernel(const VhaParams p) {
         asm volatile("" : "+r"(vb), "+r"(ub));
         const long long tok = item / slices;
         uint32_t* row = out + tok * p.Hq * row_words + (item - tok * slices) * 32 + lane;
+        // fp32: the warp's next item into L2 (lane l: head rows l and l + 32, 128 bytes each),
+        // so its DRAM latency overlaps this item's arithmetic without holding registers.  An
+        // fp32 item is half as many channels per byte as a bf16 one; for bf16 the prefetch
+        // measured slower (its items are already long enough to hide the loads).
+        if (F32 && item + stride < items) {
+            const long long nt = (item + stride) / slices;
+            const uint32_t* nrow = out + nt * p.Hq * row_words + (item + stride - nt * slices) * 32;
+#pragma unroll
+            for (int h = lane; h < kVhaMaxHeads; h += 32)
+                if (h < p.Hq) asm volatile("prefetch.global.L2 [%0];" :: "l"(nrow + (size_t)h * row_words));
+        }
         uint32_t x[kVhaMaxHeads];
         {
             const uint32_t* src = row;
