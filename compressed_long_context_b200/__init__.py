@@ -56,6 +56,13 @@ def _need(t, dtype, name, device=None):
         raise ValueError("%s must be contiguous" % name)
 
 
+def _room(t, n, name):
+    """The kernels address a buffer from the sizes they are given: refuse one that holds fewer
+    elements than that footprint (it would be read or written out of bounds)."""
+    if t is not None and t.numel() < n:
+        raise ValueError("%s holds %d elements, the call addresses %d" % (name, t.numel(), n))
+
+
 def get_device_error(device=None) -> None:
     """Synchronise the current stream and raise if a kernel recorded a device-side error."""
     device = device or torch.device("cuda", torch.cuda.current_device())
@@ -81,6 +88,10 @@ def compress(k, v, w=None, blk=128, kc=None, vc=None):
         vc = torch.empty((B, Nc, Hkv, dv), dtype=torch.bfloat16, device=k.device)
     _need(kc, torch.bfloat16, "kc", k.device)
     _need(vc, torch.bfloat16, "vc", k.device)
+    _room(v, B * T * Hkv * dv, "v")
+    _room(w, B * T, "w")
+    _room(kc, B * Nc * Hkv * d, "kc")
+    _room(vc, B * Nc * Hkv * dv, "vc")
     rc = _lib.load().hca_compress(_p(k), _p(v), _p(w), _p(kc), _p(vc), B, T, Hkv, d, dv, blk, _stream(k.device))
     _check(rc, "hca_compress")
     return kc, vc
@@ -96,6 +107,12 @@ def prefill(q, k, v, kc, vc, blk, W, scale, out=None, want_lse=False, out_f32=Fa
     if out is None:
         out = torch.empty((B, T, Hq, dv), dtype=torch.float32 if out_f32 else torch.bfloat16, device=q.device)
     _need(out, torch.float32 if out_f32 else torch.bfloat16, "out", q.device)
+    Nc = T // blk if blk > 0 else 0
+    _room(k, B * T * Hkv * d, "k")
+    _room(v, B * T * Hkv * dv, "v")
+    _room(kc, B * Nc * Hkv * d, "kc")
+    _room(vc, B * Nc * Hkv * dv, "vc")
+    _room(out, B * T * Hq * dv, "out")
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device) if want_lse else None
     flags = (HCA_WRITE_LSE if want_lse else 0) | (HCA_OUT_F32 if out_f32 else 0)
     rc = _lib.load().hca_prefill(_p(q), _p(k), _p(v), _p(kc), _p(vc), _p(out), _p(lse), B, T, Hq, Hkv, d, dv,
@@ -146,6 +163,17 @@ def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size
     if out is None:
         out = torch.empty((B, Hq, dv), dtype=torch.float32, device=dev)
     _need(out, torch.float32, "out", dev)
+    rows = num_pages * page_size if page_table is not None else B * Nmax
+    _room(kc, rows * Hkv * d, "kc")
+    _room(vc, rows * Hkv * dv, "vc")
+    _room(page_table, B * max_pages, "page_table")
+    _room(kw, B * W * Hkv * d, "kw")
+    _room(vw, B * W * Hkv * dv, "vw")
+    _room(seqlens, B, "seqlens")
+    _room(gq, d, "gq")
+    _room(gk, d, "gk")
+    _room(gate, B * Hq * dv, "gate")
+    _room(out, B * Hq * dv, "out")
     ws_bytes = decode_workspace_size(B, Hq, Hkv, dv)
     if workspace is None:
         workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
@@ -180,8 +208,9 @@ def append(k_new, v_new, w_new, seqlens, kw, vw, kc, vc, state, blk, page_table=
     _need(seqlens, torch.int32, "seqlens", dev)
     if w_new is not None:
         _need(w_new, torch.float32, "w_new", dev)
-    if state.dtype not in (torch.uint8, torch.float32) or not state.is_cuda or not state.is_contiguous():
-        raise ValueError("state must be a contiguous uint8 or float32 CUDA tensor")
+    if not isinstance(state, torch.Tensor) or state.dtype not in (torch.uint8, torch.float32):
+        raise TypeError("state must be a uint8 or float32 torch.Tensor")
+    _need(state, state.dtype, "state", dev)
     B, Hkv, d = k_new.shape
     dv = v_new.shape[2]
     W = kw.shape[1]
@@ -197,6 +226,15 @@ def append(k_new, v_new, w_new, seqlens, kw, vw, kc, vc, state, blk, page_table=
         num_pages = kc.shape[0]
         page_size = kc.shape[1]
         Nmax = 0
+    rows = num_pages * page_size if page_table is not None else B * Nmax
+    _room(v_new, B * Hkv * dv, "v_new")
+    _room(w_new, B, "w_new")
+    _room(seqlens, B, "seqlens")
+    _room(kw, B * W * Hkv * d, "kw")
+    _room(vw, B * W * Hkv * dv, "vw")
+    _room(kc, rows * Hkv * d, "kc")
+    _room(vc, rows * Hkv * dv, "vc")
+    _room(page_table, B * max_pages, "page_table")
     rc = _lib.load().hca_append(_p(k_new), _p(v_new), _p(w_new), _p(seqlens), _p(kw), _p(vw), _p(kc), _p(vc),
                                 _p(page_table), int(page_size), int(max_pages), int(num_pages), _p(state),
                                 B, Hkv, d, dv, int(blk), int(W), int(Nmax), flags, _stream(dev))
@@ -207,8 +245,9 @@ def vha(out, U, V):
     """Virtual Head Attention in place on an attention output ``out`` [..., Hq, dv] (bf16 or
     fp32): per token and channel, out[:, c] <- (I + U V^T) out[:, c] over the heads.
     U, V [Hq, r] fp32.  Returns ``out``."""
-    if out.dtype not in (torch.bfloat16, torch.float32) or not out.is_cuda or not out.is_contiguous():
-        raise ValueError("out must be a contiguous bf16 or fp32 CUDA tensor")
+    if not isinstance(out, torch.Tensor) or out.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be a bf16 or fp32 torch.Tensor")
+    _need(out, out.dtype, "out")
     dev = out.device
     _need(U, torch.float32, "U", dev)
     _need(V, torch.float32, "V", dev)
