@@ -81,3 +81,65 @@ def test_pins_catch_mutant(name):
 
 def test_unmutated_oracle_passes_all_checks():
     assert not _caught(oracle_mod._load())
+
+
+# ---- the backward oracle (oracle/backward.py, numpy): same idea, one textual change per
+# mutant, the mutated module swapped in for the backward pins
+
+BACKWARD_MUTANTS = {
+    "dS misses rowsum(dO*O)": ("ds = p * (dp - (do * o).sum(axis=1, keepdims=True))", "ds = p * dp"),
+    "pooling path of dK dropped": ("return dq, dk_raw + dk_pool, dv_raw + dv_pool, dw",
+                                   "return dq, dk_raw, dv_raw + dv_pool, dw"),
+    "weight softmax Jacobian dropped": ("dwb = a * (dal - (a * dal).sum(axis=2, keepdims=True))", "dwb = a * dal"),
+    "entry boundary moved by one": ("n_c = np.maximum(0, (t - W + 1) // blk)", "n_c = np.maximum(0, (t - W + 2) // blk)"),
+    "dq without the scale": ("dq[b, :, h] = scale * (ds @ keys)", "dq[b, :, h] = ds @ keys"),
+    "gradient to the wrong kv head": ("            g = h * Hkv // Hq\n            keys, vals = _keys(k, v, kc, vc, b, g)",
+                                      "            g = h % Hkv\n            keys, vals = _keys(k, v, kc, vc, b, g)"),
+    "dV from dS": ("dvals = p.T @ do", "dvals = ds.T @ do"),
+}
+
+
+def _backward_checks(tb):
+    return [
+        lambda: tb.test_backward_matches_finite_differences(11, 2, 1, 2, 3),
+        lambda: tb.test_backward_matches_finite_differences(13, 4, 2, 3, 4),
+        tb.test_pool_backward_matches_finite_differences,
+        lambda: tb.test_one_token_blocks_are_causal_attention(4, 2),
+        tb.test_window_covering_the_sequence_is_causal_attention,
+        tb.test_weight_gradients_sum_to_zero_per_block,
+        tb.test_value_gradients_sum_to_output_gradients,
+        tb.test_query_with_only_itself_has_zero_gradient,
+        tb.test_dense_forward_matches_c_oracle,
+    ]
+
+
+def _backward_caught(module):
+    from tests import test_oracle_backward as tb
+    saved = tb.ob
+    tb.ob = module
+    try:
+        for check in _backward_checks(tb):
+            try:
+                check()
+            except AssertionError:
+                return True
+        return False
+    finally:
+        tb.ob = saved
+
+
+@pytest.mark.parametrize("name", sorted(BACKWARD_MUTANTS))
+def test_backward_pins_catch_mutant(name):
+    import types
+    from oracle import backward
+    src = open(backward.__file__).read()
+    old, new = BACKWARD_MUTANTS[name]
+    assert src.count(old) == 1, "mutation anchor not found: " + name
+    mutant = types.ModuleType("backward_mutant")
+    exec(compile(src.replace(old, new), "backward_mutant.py", "exec"), mutant.__dict__)
+    assert _backward_caught(mutant), "no pin caught the planted mistake: " + name
+
+
+def test_unmutated_backward_passes_all_checks():
+    from oracle import backward
+    assert not _backward_caught(backward)
