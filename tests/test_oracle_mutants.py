@@ -143,3 +143,45 @@ def test_backward_pins_catch_mutant(name):
 def test_unmutated_backward_passes_all_checks():
     from oracle import backward
     assert not _backward_caught(backward)
+
+
+# ---- the VHA oracle (numpy): the function's source with one change, swapped in for its pins
+
+VHA_MUTANTS = {
+    "identity skip dropped": ('return o + np.einsum("hk,nkc->nhc", U, t)', 'return np.einsum("hk,nkc->nhc", U, t)'),
+    "factors swapped": ('t = np.einsum("hk,nhc->nkc", V, o)', 't = np.einsum("hk,nhc->nkc", U, o)'),
+    "mixing matrix transposed": ('t = np.einsum("hk,nhc->nkc", V, o)\n    return o + np.einsum("hk,nkc->nhc", U, t)',
+                                 't = np.einsum("hk,nhc->nkc", U, o)\n    return o + np.einsum("hk,nkc->nhc", V, t)'),
+}
+
+
+def _vha_caught(fn):
+    saved = oracle.vha
+    oracle.vha = fn
+    try:
+        for check in (pins.test_vha_zero_factor_is_identity, pins.test_vha_rank_one_closed_form,
+                      pins.test_vha_factor_gauge_invariance, pins.test_vha_equals_dense_mixing_matrix):
+            try:
+                check()
+            except AssertionError:
+                return True
+        return False
+    finally:
+        oracle.vha = saved
+
+
+@pytest.mark.parametrize("name", sorted(VHA_MUTANTS))
+def test_vha_pins_catch_mutant(name):
+    import inspect
+    import textwrap
+    import numpy as np
+    src = textwrap.dedent(inspect.getsource(oracle_mod.vha))
+    old, new = VHA_MUTANTS[name]
+    assert src.count(old) == 1, "mutation anchor not found: " + name
+    ns = {"np": np}
+    exec(compile(src.replace(old, new), "vha_mutant.py", "exec"), ns)
+    assert _vha_caught(ns["vha"]), "no pin caught the planted mistake: " + name
+
+
+def test_unmutated_vha_passes_all_checks():
+    assert not _vha_caught(oracle_mod.vha)
