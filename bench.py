@@ -77,6 +77,11 @@ def append_bytes(B, Hkv, d, dv):
     return B * Hkv * ((d + dv) * 2 + 2 * state + (d + dv) * 2 + (d + dv) * 2) + B * 8
 
 
+def vha_bytes(numel, esize, Hq, r):
+    """hca_vha in place: the output read and written once, plus the two fp32 factors."""
+    return 2 * numel * esize + 2 * Hq * r * 4
+
+
 def prefill_flops(B, T, Hq, d, dv, blk, W):
     t = np.arange(T, dtype=np.int64)
     a = t - W + 1
@@ -524,7 +529,7 @@ def main():
             torch.cuda.synchronize()
         hca.get_device_error()
         v_ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in vev]), world)
-        vbytes = 2 * pout.numel() * pout.element_size() + 2 * vu.numel() * 4
+        vbytes = vha_bytes(pout.numel(), pout.element_size(), pc.Hq, vu.shape[1])
         prefill_part["vha"] = {"ms": v_ms, "rank": 8, "algorithmic_bytes": vbytes, "bound": "hbm",
                                "achieved_gbs": vbytes / (v_ms / 1e3) / 1e9,
                                "frac": vbytes / (v_ms / 1e3) / 1e9 / pk["hbm_gbs"],

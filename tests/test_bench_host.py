@@ -35,6 +35,20 @@ def test_prefill_flops_128k():
     assert flops == 2.0 * 64 * keys * 1024
 
 
+def test_append_bytes_block_completing_step():
+    # per (sequence, KV head): the new token (2 KB), the pooling state read and written
+    # (2 x 4,112 B), the ring slot (2 KB) and the entry (2 KB); plus length and weight
+    per = 2048 + 2 * (4 + 1024) * 4 + 2048 + 2048
+    assert bench.append_bytes(64, 1, 512, 512) == 64 * per + 64 * 8 == 920064
+
+
+def test_vha_bytes_prefill_output():
+    # the 128K prefill output, bf16, read and written once; rank-8 factors
+    n = 131072 * 64 * 512
+    assert bench.vha_bytes(n, 2, 64, 8) == 2 * n * 2 + 2 * 64 * 8 * 4
+    assert abs(bench.vha_bytes(n, 2, 64, 8) - 17.18e9) < 0.01e9
+
+
 def test_weak_scaling_value():
     assert bench.weak_scaling_value(64 * 10, 4, 2.0) == 64 * 10 * 4 / 2.0
 
