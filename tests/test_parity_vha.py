@@ -110,3 +110,31 @@ def test_vha_zero_factor_leaves_output_unchanged(cuda_device, libhca):
     hca.vha(y, U, torch.zeros_like(U))
     torch.cuda.synchronize()
     assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("n,Hq,dv,r,f32", [
+    (33, 3, 64, 5, False),     # odd head count (factor rows not a multiple of 16 bytes apart), rank padded 5 -> 8
+    (33, 3, 64, 5, True),      # fp32: two 32-channel slices per token
+    (10, 1, 128, 1, False),    # one head: the mixing is a scalar 1 + u v per channel
+    (3, 64, 512, 32, True),    # every head, the largest rank, fp32
+    (257, 8, 192, 2, True),    # rank padded 2 -> 4, three slices per 64-wide channel block
+])
+def test_vha_odd_shapes(cuda_device, libhca, n, Hq, dv, r, f32):
+    dev = cuda_device
+    g = torch.Generator(device=dev).manual_seed(100 + n + Hq + r)
+    x = torch.randn((n, Hq, dv), generator=g, device=dev)
+    if not f32:
+        x = x.to(torch.bfloat16)
+    U, V = factors(dev, Hq, r, 110 + r, std=0.3)
+    ref = oracle.vha((oracle.bits_to_f64(bits(x)) if not f32 else x.double().cpu().numpy()), U.cpu().numpy(),
+                     V.cpu().numpy())
+    y = x.clone()
+    hca.vha(y, U, V)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    got = y.double().cpu().numpy()
+    if f32:
+        # fp32 arithmetic over at most 2 Hq r products per value: far inside 1e-4 at these magnitudes
+        assert np.abs(got - ref).max() <= 1e-4
+    else:
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
