@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for Heavily Compressed Attention (HCA).
+"""fp64 CPU oracle for Heavily Compressed Attention (HCA): the forward in plain C
+(compress, prefill rows, decode), Virtual Head Attention and the backward pass in numpy.
 
 TEST INFRASTRUCTURE ONLY.  Only tests/, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg may import this package.  It shares no code with
