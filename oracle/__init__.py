@@ -7,6 +7,6 @@ the CUDA library in ``compressed_long_context_b200``.
 """
 from .oracle import (  # noqa: F401
     compress, round_bf16, visible_entries, prefill_rows, decode, num_threads,
-    bf16_bits, bits_to_f64, vha,
+    bf16_bits, bits_to_f64, vha, gate_logits,
 )
 from . import backward  # noqa: F401  (fp64 gradients of the layer, numpy)

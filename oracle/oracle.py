@@ -189,3 +189,18 @@ def vha(out, U, V):
     t = np.einsum("hk,nhc->nkc", V, o)
     return o + np.einsum("hk,nkc->nhc", U, t)
 
+
+def gate_logits(cq, Wg):
+    """Low-Rank Gated Attention, the reading of the pages' gate (Zhidx article, section "1.
+    Latent-Gated Sparse Attention"; official blog, section 2.1): the output gate's logits come
+    from the attention layer's own query latent instead of the hidden state.  The latent is a
+    quarter of the hidden size, so the gate projection has a quarter of the weights.
+
+    cq [n, r_q] query latents, Wg [r_q, Hq, dv] gate projection.  Returns the logits
+    g[n, h, c] = sum_k cq[n, k] Wg[k, h, c] in fp64; the attention output is then scaled by
+    sigmoid(g), element-wise (the decode gate).  A plain contraction, written out with einsum.
+    """
+    cq = np.asarray(cq, dtype=np.float64)
+    Wg = np.asarray(Wg, dtype=np.float64)
+    assert cq.ndim == 2 and Wg.ndim == 3 and cq.shape[1] == Wg.shape[0]
+    return np.einsum("nk,khc->nhc", cq, Wg)

@@ -100,3 +100,27 @@ def test_compress_two_rows_fixture():
     # the weight ln 3 is rounded to fp32; alpha moves by at most ~1e-7 from 3/4
     np.testing.assert_allclose(kc[0, 0, 0], [float(x) for x in vals["kc"]], rtol=0, atol=1e-6)
     np.testing.assert_allclose(vc[0, 0, 0], [float(x) for x in vals["vc"]], rtol=0, atol=1e-6)
+
+
+def test_low_rank_gate_fixture():
+    """The gate projection maps the query latent (not the hidden state) to one logit per head
+    and channel; with the pages' dimensions that is 75% fewer weights."""
+    dims = {}
+    for ln in rows_of("low_rank_gate_dims.txt"):
+        key, val = ln.split(":")
+        dims[key] = int(val)
+    out_width = dims["heads"] * dims["head_dim"]
+    full = dims["hidden"] * out_width                 # a gate projected from the hidden state
+    low = dims["query_latent"] * out_width            # the low-rank gate
+    assert 100 * (full - low) // full == dims["fewer_weights_percent"]
+    # the oracle's gate has exactly the low-rank projection's shape and is linear in the latent:
+    # a one-hot latent selects one row of the projection
+    rs = np.random.RandomState(5)
+    Wg = rs.standard_normal((8, 4, 6))               # a small stand-in: r_q 8, 4 heads, 6 channels
+    cq = np.zeros((2, 8))
+    cq[0, 3] = 1.0
+    cq[1, 5] = -2.0
+    g = oracle.gate_logits(cq, Wg)
+    assert g.shape == (2, 4, 6)
+    np.testing.assert_array_equal(g[0], Wg[3])
+    np.testing.assert_array_equal(g[1], -2.0 * Wg[5])
