@@ -148,3 +148,79 @@ def backward(q, k, v, w, blk, W, scale, dout):
     dq, dk_raw, dv_raw, dkc, dvc = attend_backward_f64(q, k, v, kc, vc, blk, W, scale, dout)
     dk_pool, dv_pool, dw = pool_backward_f64(k, v, w, blk, dkc, dvc)
     return dq, dk_raw + dk_pool, dv_raw + dv_pool, dw
+
+
+def _row_keys(t, T, Nc, blk, W):
+    """Indices of the keys query t sees: entries j < n_c(t) and raw positions [t-W+1, t]."""
+    n_c = max(0, (t - W + 1) // blk)
+    return np.arange(min(n_c, Nc)), np.arange(max(0, t - W + 1), t + 1)
+
+
+def backward_sampled(q, k, v, w, blk, W, scale, dout, b, rows=(), raw=(), entries=()):
+    """Selected gradients of sequence b without the dense [T, Nc + T] matrices, for checks at
+    lengths where the dense form does not fit.
+
+    rows: query positions t -> dq[t] [Hq, d] (each needs only its own softmax row).
+    raw: positions u -> the total dk[u], dv[u] [Hkv, d|dv] (window path from the W queries
+    t in [u, u+W-1], plus the pooling path through u's block when it is complete) and dw[u].
+    entries: blocks j -> dkc[j], dvc[j] (from the queries t >= blk(j+1) + W - 1).
+    The cost is that of the queries involved: cheap for entries near the end of the
+    sequence. Returns a dict of dicts keyed by position / block.
+    """
+    # q and dout are read row by row (widened to fp64 per row), so that full-size inputs need
+    # no fp64 copy; sequence b's K and V are widened once
+    T, Hq = q.shape[1], q.shape[2]
+    Hkv = k.shape[2]
+    k, v = _f64(k[b:b + 1]), _f64(v[b:b + 1])
+    b_in, b = b, 0
+    kc, vc, a = pool_f64(k, v, None if w is None else _f64(w)[b_in:b_in + 1], blk)
+    kc, vc, a = kc[0], vc[0], a[0]
+    Nc = kc.shape[0]
+    blocks = sorted(set(entries) | {u // blk for u in raw if u // blk < Nc})
+    # the queries whose softmax rows are needed
+    need = set(rows)
+    for u in raw:
+        need.update(range(u, min(T, u + W)))
+    for j in blocks:
+        need.update(range(blk * (j + 1) + W - 1, T))
+    dq = {t: np.zeros((Hq, q.shape[3])) for t in rows}
+    dk_win = {u: np.zeros((Hkv, k.shape[3])) for u in raw}
+    dv_win = {u: np.zeros((Hkv, v.shape[3])) for u in raw}
+    dkc = {j: np.zeros((Hkv, kc.shape[2])) for j in blocks}
+    dvc = {j: np.zeros((Hkv, vc.shape[2])) for j in blocks}
+    for t in sorted(need):
+        ej, ru = _row_keys(t, T, Nc, blk, W)
+        for h in range(Hq):
+            g = h * Hkv // Hq
+            keys = np.concatenate([kc[ej, g], k[b, ru, g]])
+            vals = np.concatenate([vc[ej, g], v[b, ru, g]])
+            qh = _f64(q[b_in, t, h])
+            s = scale * (keys @ qh)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            do = _f64(dout[b_in, t, h])
+            dp = vals @ do
+            ds = p * (dp - do @ (p @ vals))
+            if t in dq:
+                dq[t][h] = scale * (ds @ keys)
+            for i, j in enumerate(ej):
+                if j in dkc:
+                    dkc[j][g] += scale * ds[i] * qh
+                    dvc[j][g] += p[i] * do
+            for i, u in enumerate(ru):
+                if u in dk_win:
+                    dk_win[u][g] += scale * ds[len(ej) + i] * qh
+                    dv_win[u][g] += p[len(ej) + i] * do
+    # pooling path of the requested raw positions, and their weight gradients
+    dk, dv, dw = {}, {}, {}
+    for u in raw:
+        j, i = divmod(u, blk)
+        dk[u], dv[u], dw[u] = dk_win[u].copy(), dv_win[u].copy(), 0.0
+        if j < Nc:
+            dk[u] += a[j, i] * dkc[j]
+            dv[u] += a[j, i] * dvc[j]
+            kb, vb = k[b, blk * j:blk * (j + 1)], v[b, blk * j:blk * (j + 1)]
+            dal = np.einsum("igc,gc->i", kb, dkc[j]) + np.einsum("igc,gc->i", vb, dvc[j])
+            dw[u] = float(a[j, i] * (dal[i] - (a[j] * dal).sum()))
+    return {"dq": dq, "dk": dk, "dv": dv, "dw": dw,
+            "dkc": {j: dkc[j] for j in entries}, "dvc": {j: dvc[j] for j in entries}}

@@ -146,3 +146,28 @@ def test_dense_forward_matches_c_oracle():
     pk, pv, _ = ob.pool_f64(k.double().numpy(), v.double().numpy(), w.double().numpy(), blk)
     np.testing.assert_allclose(pk, kc, rtol=0, atol=1e-13)
     np.testing.assert_allclose(pv, vc, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,blk,W", [(40, 4, 2, 4, 6), (37, 2, 1, 8, 3), (25, 3, 1, 1, 2)])
+def test_sampled_backward_equals_dense(T, Hq, Hkv, blk, W):
+    """The sampled form (only the queries that matter) gives the dense backward's values."""
+    q, k, v, w, dout = case(70 + T, B=2, T=T, Hq=Hq, Hkv=Hkv, d=5, dv=3)
+    scale = 0.6
+    dq, dk, dv, dw = ob.backward(q, k, v, w, blk, W, scale, dout)
+    kc, vc, _ = ob.pool_f64(k, v, w, blk)
+    _, _, _, dkc, dvc = ob.attend_backward_f64(q, k, v, kc, vc, blk, W, scale, dout)
+    Nc = T // blk
+    rows = [0, 1, T // 2, T - 1]
+    raw = sorted({0, blk - 1, blk, T // 2, T - 2, T - 1})
+    entries = sorted({0, Nc // 2, Nc - 1}) if Nc else []
+    for b in range(2):
+        got = ob.backward_sampled(q, k, v, w, blk, W, scale, dout, b, rows=rows, raw=raw, entries=entries)
+        for t in rows:
+            np.testing.assert_allclose(got["dq"][t], dq[b, t], rtol=1e-12, atol=1e-13)
+        for u in raw:
+            np.testing.assert_allclose(got["dk"][u], dk[b, u], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(got["dv"][u], dv[b, u], rtol=1e-12, atol=1e-13)
+            assert abs(got["dw"][u] - dw[b, u]) <= 1e-12 + 1e-12 * abs(dw[b, u])
+        for j in entries:
+            np.testing.assert_allclose(got["dkc"][j], dkc[b, j], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(got["dvc"][j], dvc[b, j], rtol=1e-12, atol=1e-13)
