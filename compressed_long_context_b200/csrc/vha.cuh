@@ -9,10 +9,11 @@
 // channels, or one fp32 channel) in registers, so the reduction over heads, t = V^T o
 // (r values per channel), runs inside the lane with no shared-memory traffic for the data;
 // o + U t is written back over the same words.  U and V sit in shared memory, padded with
-// zeros to a power-of-two rank RP >= 4 (zero terms add nothing), and are read as broadcasts.  Both
-// products use the two-wide fp32 FMA, each lane of which rounds like fmaf.  The output is
-// read and written once: HBM-bound when the FMA work per byte is small (2 Hq r FMAs per
-// channel; at Hq 64 the rank-8 mixing is about 1000 FMAs per 2-byte channel).
+// zeros to a power-of-two rank RP >= 4 (zero terms add nothing), and are read as
+// broadcasts.  Both products use the two-wide fp32 FMA, each lane of which rounds like
+// fmaf.  The output is read and written once: HBM-bound when the FMA work per byte is small
+// (2 Hq r FMAs per channel; at Hq 64 the rank-8 mixing is about 1000 FMAs per 2-byte
+// channel).  The fp32 path also prefetches each warp's next item into L2.
 #pragma once
 
 #include "common.cuh"
