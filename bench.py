@@ -259,7 +259,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "L": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
-                       "blk": cfg.blk, "W": cfg.W, "sample_sequences_per_step": 1},
+                       "blk": cfg.blk, "W": cfg.W, "step": "oracle compress(raw K/V) + oracle decode",
+                       "sample_sequences_per_step": 1},
             "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
