@@ -173,3 +173,23 @@ def test_vha_rejects_before_launch(libhca):
     assert libhca.hca_vha(p, p, p, 4, 64, 512, 0, 0, None) == _lib.HCA_ERR_INVALID_ARG
     assert libhca.hca_vha(None, None, None, 0, 64, 512, 4, 0, None) == _lib.HCA_OK          # nothing to do
 
+
+
+def test_header_compiles_as_c_and_links(tmp_path, libhca):
+    """include/hca.h is a plain C header: a C99 translation unit that includes it and takes the
+    address of every entry point compiles warning-free and links against libhca.so."""
+    import shutil
+    import subprocess
+    from compressed_long_context_b200 import _lib as L
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_hca.c"
+    names = sorted(L.EXPORTS)
+    body = "\n".join("    (void)&%s;" % n for n in names)
+    src.write_text('#include "hca.h"\n#include <stddef.h>\nint main(void) {\n%s\n    return 0;\n}\n' % body)
+    exe = tmp_path / "use_hca"
+    lib_dir = os.path.dirname(L.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-L", lib_dir, "-l:libhca.so", "-Wl,--unresolved-symbols=ignore-in-shared-libs",
+                        "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
