@@ -174,6 +174,8 @@ int oracle_prefill_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         int64_t blk, int64_t W, double scale,
                         const int64_t* rows, int64_t n_rows, int q_rows, double* out, double* lse) {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv || blk <= 0 || W <= 0) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)     /* every requested row inside the batch */
+        if (rows[2 * r] < 0 || rows[2 * r] >= B || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= T) return 1;
     int64_t Nc = T / blk, grp = Hq / Hkv;
     #pragma omp parallel
     {

@@ -439,3 +439,12 @@ def test_vha_equals_dense_mixing_matrix():
     want = np.stack([np.stack([M @ o[n, :, c] for c in range(9)], axis=1) for n in range(2)])
     np.testing.assert_allclose(oracle.vha(o, U, V), want, rtol=1e-12, atol=1e-12)
 
+
+
+def test_prefill_rows_rejects_rows_outside_the_batch():
+    z = np.zeros((1, 8, 1, 4), np.uint16)
+    zc = np.zeros((1, 2, 1, 4), np.uint16)
+    for bad in ([(1, 0)], [(0, 8)], [(-1, 3)], [(0, -1)]):
+        with pytest.raises(ValueError):
+            oracle.prefill_rows(z, z, z, zc, zc, 4, 2, 1.0, bad)
+    oracle.prefill_rows(z, z, z, zc, zc, 4, 2, 1.0, [(0, 7)])
