@@ -1,21 +1,26 @@
 """Benchmark of the HCA hot path on B200 (one JSON line on stdout).
 
-Workload (the decode configuration the headline metric is quoted on): 64 sequences of
-131072 tokens, Hq=64 query heads sharing one 512-dim KV head, blocks of 128, a raw
-window of 128 tokens; pooling weights ~N(0, 0.5); bf16 inputs ~N(0, 1); seed 1.
+Headline (`value`): HCA decode queries/s on the 128K decode workload -- 64 sequences of
+131072 tokens, Hq=64 query heads sharing one 512-dim KV head, blocks of 128, a raw window
+of 128 tokens (1023 compressed entries + 128 raw tokens per query); pooling weights
+~N(0, 0.5); bf16 inputs ~N(0, 1); seed 1.  One step = one `hca_decode` call (split kernel +
+combine kernel) over the whole batch, the compressed cache resident in HBM, L2 flushed
+before every timed call.  value = queries of all ranks / device time (max over ranks).
 
-One step = the whole path for one batch:
-    hca_compress  (raw K/V [64, 131072, 1, 512] -> 1024 cached entries per sequence)
-    hca_decode    (one query per sequence over 1023 entries + 128 raw tokens;
-                   split kernel + combine kernel)
-value = queries of all ranks / device time of the step (max over ranks).
-
-Also reported, measured in the same run: the decode kernels alone (cache resident,
-L2 flushed before each call) and the 128K prefill (T=131072, Hq=64, d=512, W=128,
-1% of raw keys x8; seed 2) in TFLOP/s.
+Every workload of the hot path is measured in the same run, one at a time (memory freed in
+between), under `configs`: its GPU time and rate, its roofline fraction, the algorithmic
+bytes or flops per unit, the fp64 CPU oracle's time on this host's cores and the max/mean
+absolute error of the GPU result against that oracle:
+  tiny_prefill       T=1024, Hq=4, d=64, mean pooling, fp32 output (compress + prefill)
+  decode_128k        the headline batch; compress of its raw K/V reported as its own GB/s
+  prefill_128k       T=131072, Hq=64, d=512, 1% of raw keys x8 (compress + prefill TFLOP/s,
+                     fraction of the burst bf16 peak); oracle on sampled rows
+  decode_1m          8 sequences of 1048576 tokens: compress GB/s + decode queries/s
+  ragged_paged       128 ragged sequences (4K..1M), paged cache, QK RMSNorm + sigmoid gate
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-Multi-GPU: torchrun, one rank per GPU, each rank a full batch (weak scaling).
+Multi-GPU: torchrun, one rank per GPU, each rank a full batch (weak scaling); the oracle
+checks run at N=1 only.
 """
 import argparse
 import hashlib
@@ -33,18 +38,21 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "HCA decode queries/s, prefill TFLOP/s, % of HBM/TC roofline (1 B200)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CONFIG_KEYS = ("tiny_prefill", "decode_128k", "prefill_128k", "decode_1m", "ragged_paged")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--no-oracle", action="store_true", help="skip the per-config oracle checks")
+    ap.add_argument("--configs", default=",".join(CONFIG_KEYS),
+                    help="comma-separated subset of %s (the headline config always runs)" % ",".join(CONFIG_KEYS))
+    return ap.parse_args(argv)
 
 
 def peaks():
@@ -59,15 +67,21 @@ def peaks():
 # ---------------------------------------------------------------- algorithmic work
 
 def compress_bytes(B, T, Hkv, d, dv, blk):
+    """Raw K/V and weights read, entries written."""
     Nc = T // blk
     return B * Nc * Hkv * (blk * (d + dv) * 2 + 2 * (d + dv)) + B * Nc * blk * 4
 
 
-def decode_bytes(B, L, Hq, Hkv, d, dv, blk, W):
+def decode_seq_bytes(L, Hq, Hkv, d, dv, blk, W, gate=False):
+    """One query: q read, visible entries + window keys/values read, fp32 output written,
+    the length read (+ the gate logits read)."""
     nc = max(0, (L - W) // blk)
     nw = min(W, L)
-    per = Hq * d * 2 + (nc + nw) * Hkv * (d + dv) * 2 + Hq * dv * 4 + 4
-    return B * per
+    return Hq * d * 2 + (nc + nw) * Hkv * (d + dv) * 2 + Hq * dv * 4 + 4 + (Hq * dv * 2 if gate else 0)
+
+
+def decode_bytes(B, L, Hq, Hkv, d, dv, blk, W):
+    return B * decode_seq_bytes(L, Hq, Hkv, d, dv, blk, W)
 
 
 def append_bytes(B, Hkv, d, dv):
@@ -83,6 +97,7 @@ def vha_bytes(numel, esize, Hq, r):
 
 
 def prefill_flops(B, T, Hq, d, dv, blk, W):
+    """2 * Hq * (d + dv) flops per (query row, visible key)."""
     t = np.arange(T, dtype=np.int64)
     a = t - W + 1
     nc = np.where(a > 0, a // blk, 0)
@@ -220,7 +235,66 @@ def traffic_for(kernel_key, source_files):
     return ent.get("dram_bytes_per_launch")
 
 
+def timed_calls(fn, n, stream, sampler, flush=None, spin=True):
+    """n calls of fn on `stream`, each bracketed by CUDA events (an L2 flush before each when
+    `flush` is given).  A GPU-side spin queued first keeps every timed call enqueued before the
+    GPU reaches it, so the events bracket device work only.  Returns the per-call ms."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    with sampler:
+        if spin:
+            torch.cuda._sleep(int(2e8))
+        for a, b in ev:
+            if flush is not None:
+                flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def err_stats(got, ref):
+    """Max and mean absolute error of a GPU result against an fp64 oracle array."""
+    g = got.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    e = np.abs(g - ref)
+    return {"max_abs_err": float(e.max()), "mean_abs_err": float(e.mean()), "finite": bool(np.isfinite(g).all()),
+            "outputs_compared": int(e.size)}
+
+
+def within(stats, max_tol=1e-2, mean_tol=1e-3):
+    return bool(stats["finite"] and stats["max_abs_err"] <= max_tol and stats["mean_abs_err"] <= mean_tol)
+
+
+class OracleTimer:
+    def __init__(self):
+        self.s = 0.0
+
+    def __call__(self, f, *a, **k):
+        t0 = time.perf_counter()
+        r = f(*a, **k)
+        self.s += time.perf_counter() - t0
+        return r
+
+
 # ---------------------------------------------------------------- reference arm (the CPU oracle)
+
+def reference_decode_inputs(cfg):
+    """Inputs of one decode step of `cfg` for the oracle: the query, a compressed cache with
+    the workload's shape and the raw window, drawn on the host with a seeded generator.  The
+    decode's work does not depend on the cache's values, so its entries are drawn directly
+    (N(0, 0.1^2), the spread of pooled N(0, 1) rows) instead of pooling 17 GB of raw history."""
+    import oracle
+    g = torch.Generator().manual_seed(cfg.seed)
+    B, Hkv, d = cfg.B, cfg.Hkv, cfg.d
+    Nc = cfg.T // cfg.blk
+    q = torch.randn((B, cfg.Hq, d), generator=g).to(torch.bfloat16)
+    kc = (torch.randn((B, Nc, Hkv, d), generator=g) * 0.1).to(torch.bfloat16)
+    vc = (torch.randn((B, Nc, Hkv, cfg.dv), generator=g) * 0.1).to(torch.bfloat16)
+    kw = torch.randn((B, cfg.W, Hkv, d), generator=g).to(torch.bfloat16)
+    vw = torch.randn((B, cfg.W, Hkv, cfg.dv), generator=g).to(torch.bfloat16)
+    seq = np.full((B,), cfg.T, np.int32)
+    return [oracle.bf16_bits(x) for x in (q, kc, vc, kw, vw)] + [seq]
+
 
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -231,330 +305,503 @@ def run_reference(args):
     import oracle
     from compressed_long_context_b200 import workloads as wl
     cfg = wl.DECODE_128K
-    one = cfg.scaled(B=1)
-    inp = wl.decode_inputs(one, "cpu")
-    kb, vb = oracle.bf16_bits(inp["k"]), oracle.bf16_bits(inp["v"])
-    wn, qb = inp["w"].numpy(), oracle.bf16_bits(inp["q"])
-    kwb, vwb = oracle.bf16_bits(inp["kw"]), oracle.bf16_bits(inp["vw"])
-    seq = inp["seqlens"].numpy()
+    qb, kcb, vcb, kwb, vwb, seq = reference_decode_inputs(cfg)
     scale = 1.0 / np.sqrt(cfg.d)
 
     def step():
-        kc, vc = oracle.compress(kb, vb, wn, cfg.blk)
-        out = oracle.decode(qb, oracle.round_bf16(kc), oracle.round_bf16(vc), kwb, vwb, seq, cfg.blk, cfg.W,
-                            scale)
-        return out
+        return oracle.decode(qb, kcb, vcb, kwb, vwb, seq, cfg.blk, cfg.W, scale)
 
-    for _ in range(args.warmup):
+    for _ in range(max(1, args.warmup)):
         step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
     dt = (time.perf_counter() - t0) / args.steps
-    qps = 1.0 / dt
+    qps = cfg.B / dt
     cores = oracle.num_threads()
-    sample = ("oracle fp64 compress of one 131072-token sequence (K and V, d=512) + decode of its query "
-              "(64 heads, 1023 entries + 128 window), per step")
+    sample = ("oracle fp64 decode of the whole batch per step: %d queries (64 heads each) over 1023 cached "
+              "entries + 128 window tokens; cache entries drawn directly with the workload's shape" % cfg.B)
     line = {"metric": METRIC, "value": qps, "unit": "queries/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "L": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
-                       "blk": cfg.blk, "W": cfg.W, "step": "oracle compress(raw K/V) + oracle decode",
-                       "sample_sequences_per_step": 1},
+                       "blk": cfg.blk, "W": cfg.W, "step": "oracle decode of the batch (cache resident)"},
             "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_sample(target_s=10.0):
-    """The oracle as it stands, on this host, for a bounded sample of the workload: batches of
-    2 sequences (compress of their raw K/V + decode of their queries), repeated for about
+# ---------------------------------------------------------------- our arm: one function per workload
+
+class Ctx:
+    def __init__(self, args, world, rank, local):
+        import compressed_long_context_b200 as hca
+        from compressed_long_context_b200 import workloads as wl
+        self.args, self.world, self.rank = args, world, rank
+        self.hca, self.wl = hca, wl
+        self.pk, self.pk_kind = peaks()
+        self.dev = torch.device("cuda", torch.cuda.current_device())
+        self.stream = torch.cuda.current_stream()
+        self.flush = l2_flush_buffer()
+        self.sampler = ClockSampler(local)
+        self.oracle_on = world == 1 and not args.no_oracle
+        self.launches = 0
+
+    def hbm_roof(self, kernel, nbytes, seconds, traffic=None):
+        gbs = nbytes / seconds / 1e9
+        return {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": self.pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / self.pk["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes, "traffic": traffic,
+                "peak_kind": self.pk_kind + " (hbm_gbs)"}
+
+    def median_s(self, ms):
+        return max_over_ranks(statistics.median(ms) / 1e3, self.world)
+
+    def mean_s(self, ms):
+        return max_over_ranks(sum(ms) / len(ms) / 1e3, self.world)
+
+
+def oracle_cache_of(oracle, k, v, w, blk, timer):
+    kc, vc = timer(oracle.compress, oracle.bf16_bits(k), oracle.bf16_bits(v),
+                   None if w is None else w.cpu().numpy(), blk)
+    return kc, vc, timer(oracle.round_bf16, kc), timer(oracle.round_bf16, vc)
+
+
+def bench_tiny_prefill(c):
+    hca, wl = c.hca, c.wl
+    cfg = wl.TINY_PREFILL
+    inp = wl.prefill_inputs(cfg, c.dev)
+    scale = 1.0 / np.sqrt(cfg.d)
+    kc = torch.empty((1, cfg.T // cfg.blk, 1, cfg.d), dtype=torch.bfloat16, device=c.dev)
+    vc = torch.empty_like(kc)
+    out = torch.empty((1, cfg.T, cfg.Hq, cfg.dv), dtype=torch.float32, device=c.dev)
+
+    def step():
+        hca.compress(inp["k"], inp["v"], inp["w"], cfg.blk, kc=kc, vc=vc)
+        hca.prefill(inp["q"], inp["k"], inp["v"], kc, vc, cfg.blk, cfg.W, scale, out=out, out_f32=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    ms = timed_calls(step, c.args.steps, c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    flops, keys = prefill_flops(1, cfg.T, cfg.Hq, cfg.d, cfg.dv, cfg.blk, cfg.W)
+    t = c.median_s(ms)
+    res = {"workload": cfg.name, "us": t * 1e6, "what": "hca_compress + hca_prefill (fp32 output)",
+           "algorithmic_flops": flops, "keys_per_head": keys, "tflops": flops / t / 1e12,
+           "bound": "launch latency (4 row tiles)"}
+    if c.oracle_on:
+        import oracle
+        tm = OracleTimer()
+        rk, rv, kcb, vcb = oracle_cache_of(oracle, inp["k"], inp["v"], inp["w"], cfg.blk, tm)
+        rows = [(0, t) for t in range(cfg.T)]
+        ro = tm(oracle.prefill_rows, oracle.bf16_bits(inp["q"]), oracle.bf16_bits(inp["k"]),
+                oracle.bf16_bits(inp["v"]), kcb, vcb, cfg.blk, cfg.W, scale, rows)
+        e = err_stats(out[0], ro)
+        ek = err_stats(kc, rk)
+        res["oracle"] = {"seconds": tm.s, "cores": oracle.num_threads(), "scope": "full (every row and head)"}
+        res["parity"] = dict(e, cache_max_abs_err=ek["max_abs_err"],
+                             within_tolerance=within(e) and ek["max_abs_err"] <= 4e-3)
+    return res
+
+
+def bench_decode_128k(c):
+    """The headline: decode alone (cache resident, L2 flushed before each call); compress of the
+    raw K/V timed separately (GB/s); serving step; e2e through host buffers; oracle parity."""
+    hca, wl = c.hca, c.wl
+    cfg = wl.DECODE_128K
+    scale = 1.0 / np.sqrt(cfg.d)
+    inp = wl.decode_inputs(cfg, c.dev)
+    k, v, w, q, kw, vw, seq = (inp[x] for x in ("k", "v", "w", "q", "kw", "vw", "seqlens"))
+    B, L = cfg.B, cfg.T
+    Nc = L // cfg.blk
+    kc = torch.empty((B, Nc, 1, cfg.d), dtype=torch.bfloat16, device=c.dev)
+    vc = torch.empty((B, Nc, 1, cfg.dv), dtype=torch.bfloat16, device=c.dev)
+    out = torch.empty((B, cfg.Hq, cfg.dv), dtype=torch.float32, device=c.dev)
+    ws = torch.empty(hca.decode_workspace_size(B, cfg.Hq, cfg.Hkv, cfg.dv), dtype=torch.uint8, device=c.dev)
+
+    def comp():
+        hca.compress(k, v, w, cfg.blk, kc=kc, vc=vc)
+
+    def dec():
+        hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
+
+    for _ in range(max(3, c.args.warmup)):
+        comp()
+        dec()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+
+    # ---- the headline: K timed decode calls
+    barrier(c.world)
+    torch.cuda.synchronize()
+    d_ms = timed_calls(dec, c.args.steps, c.stream, c.sampler, flush=c.flush)
+    barrier(c.world)
+    hca.get_device_error()
+    c.launches += 2 * c.args.steps
+    t_dec = c.mean_s(d_ms)
+    dbytes = decode_bytes(B, L, cfg.Hq, 1, cfg.d, cfg.dv, cfg.blk, cfg.W)
+    head = {"value": weak_scaling_value(B, c.world, t_dec), "ms_per_step": t_dec * 1e3,
+            "roofline": c.hbm_roof("decode_split_kernel + decode_combine_kernel", dbytes, t_dec,
+                                   traffic_for("decode_B64_L131072", ["compressed_long_context_b200/csrc/decode.cuh"]))}
+
+    # ---- compress of the raw history (17.35 GB), its own GB/s
+    c_ms = timed_calls(comp, max(3, min(c.args.steps, 10)), c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    cbytes = compress_bytes(B, L, 1, cfg.d, cfg.dv, cfg.blk)
+    t_c = c.mean_s(c_ms)
+    res = {"workload": cfg.name, "what": "hca_decode (split + combine), cache resident; compress separately",
+           "decode": {"us": t_dec * 1e6, "median_us": statistics.median(d_ms) * 1e3,
+                      "queries_per_s": B / t_dec, "algorithmic_bytes": dbytes,
+                      "bytes_per_query": dbytes // B, "roofline": head["roofline"]},
+           "compress": {"ms": t_c * 1e3, "gbs": cbytes / t_c / 1e9, "algorithmic_bytes": cbytes,
+                        "bytes_per_entry": cbytes // (B * Nc),
+                        "roofline": c.hbm_roof("compress_kernel<512,512>", cbytes, t_c,
+                                               traffic_for("compress_decode_B64_L131072",
+                                                           ["compressed_long_context_b200/csrc/compress.cuh"]))}}
+
+    # ---- one serving step: hca_append of every sequence's newest token, then hca_decode over the
+    # window ring (at L = 131072 every sequence completes a block, so an entry is written too)
+    kn, vn = k[:, L - 1].contiguous(), v[:, L - 1].contiguous()
+    wn = w[:, L - 1].contiguous()
+    state = torch.zeros(hca.append_state_size(B, 1, cfg.d, cfg.dv), dtype=torch.uint8, device=c.dev)
+    kc_s, vc_s = kc.clone(), vc.clone()
+    kw_s, vw_s = kw.clone(), vw.clone()
+
+    def serve(decode_too):
+        hca.append(kn, vn, wn, seq, kw_s, vw_s, kc_s, vc_s, state, cfg.blk)
+        if decode_too:
+            hca.decode(q, kc_s, vc_s, kw_s, vw_s, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws,
+                       window_ring=True)
+
+    serve_part = {}
+    for name, dflag in (("append_us", False), ("append_plus_decode_us", True)):
+        for _ in range(3):
+            serve(dflag)
+        sm = timed_calls(lambda: serve(dflag), c.args.steps, c.stream, c.sampler, flush=c.flush)
+        serve_part[name] = c.median_s(sm) * 1e6
+    hca.get_device_error()
+    abytes = append_bytes(B, 1, cfg.d, cfg.dv)
+    serve_part.update({"append_algorithmic_bytes": abytes,
+                       "append_frac_of_hbm": abytes / (serve_part["append_us"] / 1e6) / 1e9 / c.pk["hbm_gbs"],
+                       "append_bound": "latency (one small CTA per sequence; %d KB moved)" % (abytes // 1024)})
+    res["serving_step"] = serve_part
+    del state, kc_s, vc_s, kw_s, vw_s
+
+    # ---- parity of the benchmarked decode (and compress) against the oracle, every output
+    dec()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    ref_cache = None
+    if c.oracle_on:
+        import oracle
+        tm = OracleTimer()
+        rk, rv, kcb, vcb = oracle_cache_of(oracle, k, v, w, cfg.blk, tm)
+        t_comp = tm.s
+        ro = tm(oracle.decode, oracle.bf16_bits(q), kcb, vcb, oracle.bf16_bits(kw), oracle.bf16_bits(vw),
+                seq.cpu().numpy(), cfg.blk, cfg.W, scale)
+        e = err_stats(out, ro)
+        ek = err_stats(kc, rk)
+        ev = err_stats(vc, rv)
+        res["oracle"] = {"seconds": tm.s, "compress_seconds": t_comp, "decode_seconds": tm.s - t_comp,
+                         "cores": oracle.num_threads(), "scope": "full (every sequence, head and channel)"}
+        res["parity"] = dict(e, cache_max_abs_err=max(ek["max_abs_err"], ev["max_abs_err"]),
+                             within_tolerance=within(e) and max(ek["max_abs_err"], ev["max_abs_err"]) <= 4e-3)
+        ref_cache = (oracle.bf16_bits(q), kcb, vcb, oracle.bf16_bits(kw), oracle.bf16_bits(vw),
+                     seq.cpu().numpy(), cfg.blk, cfg.W, scale)
+        del rk, rv
+    del k, v, w, inp
+    torch.cuda.empty_cache()
+
+    # ---- e2e through the public API: the step's inputs copied from pinned host buffers, the
+    # result read back, both inside the timed region
+    e2e = None
+    if not c.args.no_e2e:
+        srcs = (q, kc, vc, kw, vw, seq)
+        hsrc = [x.cpu().pin_memory() for x in srcs]
+        dsts = [torch.empty_like(x) for x in srcs]
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(x.numel() * x.element_size() for x in hsrc)
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for hs, dd in zip(hsrc, dsts):
+                dd.copy_(hs, non_blocking=True)
+            hca.decode(dsts[0], dsts[1], dsts[2], dsts[3], dsts[4], dsts[5], cfg.blk, cfg.W, scale, out=out,
+                       workspace=ws)
+            hout.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ne = max(3, min(c.args.steps, 10))
+        barrier(c.world)
+        e_ms = timed_calls(e2e_step, ne, c.stream, c.sampler, flush=None, spin=False)
+        barrier(c.world)
+        hca.get_device_error()
+        te = c.mean_s(e_ms)
+        e2e = {"value": weak_scaling_value(B, c.world, te), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": ne,
+               "step": "pinned host -> device copies of q, cache, window and lengths; hca_decode; output read back"}
+        del hsrc, dsts, hout
+    del kc, vc, out, ws
+    torch.cuda.empty_cache()
+    return head, res, e2e, ref_cache
+
+
+def bench_prefill_128k(c):
+    hca, wl = c.hca, c.wl
+    pc = wl.PREFILL_128K
+    scale = 1.0 / np.sqrt(pc.d)
+    pin = wl.prefill_inputs(pc, c.dev)
+    pkc, pvc = hca.compress(pin["k"], pin["v"], pin["w"], pc.blk)
+    pout = torch.empty((1, pc.T, pc.Hq, pc.dv), dtype=torch.bfloat16, device=c.dev)
+
+    def pre():
+        hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, scale, out=pout)
+
+    def comp():
+        hca.compress(pin["k"], pin["v"], pin["w"], pc.blk, kc=pkc, vc=pvc)
+
+    for _ in range(2):
+        comp()
+        pre()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    n = max(3, min(c.args.steps, 6))
+    p_ms = timed_calls(pre, n, c.stream, c.sampler, flush=c.flush)
+    c_ms = timed_calls(comp, n, c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    flops, keys = prefill_flops(1, pc.T, pc.Hq, pc.d, pc.dv, pc.blk, pc.W)
+    tp = c.median_s(p_ms)
+    tf = flops / tp / 1e12
+    burst = c.pk["bf16_tflops"]
+    sust = c.pk.get("bf16_tflops_sustained", burst)
+    res = {"workload": pc.name, "what": "hca_prefill (bf16 output) after hca_compress of the raw K/V",
+           "ms": tp * 1e3, "compress_ms": c.median_s(c_ms) * 1e3, "tflops": tf, "algorithmic_flops": flops,
+           "flops_per_row_key": 2 * pc.Hq * (pc.d + pc.dv), "keys_per_head": keys,
+           "roofline": {"bound": "tensor", "kernel": "prefill_pair_kernel", "achieved": tf, "peak": burst,
+                        "unit": "TFLOP/s", "frac": tf / burst,
+                        "peak_kind": c.pk_kind + " (bf16_tflops, burst: each call is an isolated ~15 ms launch)",
+                        "frac_of_sustained": tf / sust,
+                        "traffic": traffic_for("prefill_T131072",
+                                               ["compressed_long_context_b200/csrc/prefill.cuh",
+                                                "compressed_long_context_b200/csrc/prefill_pair.cuh"])}}
+    # Virtual Head Attention on the prefill output (in place, bf16), synthetic rank-8 factors
+    gv = torch.Generator(device=c.dev).manual_seed(5)
+    vu = torch.randn((pc.Hq, 8), generator=gv, device=c.dev) * 0.1
+    vv = torch.randn((pc.Hq, 8), generator=gv, device=c.dev) * 0.1
+    vout = pout.clone()
+    hca.vha(vout, vu, vv)
+    v_ms = timed_calls(lambda: hca.vha(vout, vu, vv), n, c.stream, c.sampler)
+    hca.get_device_error()
+    tv = c.median_s(v_ms)
+    vbytes = vha_bytes(vout.numel(), vout.element_size(), pc.Hq, vu.shape[1])
+    res["vha"] = {"ms": tv * 1e3, "rank": 8, "algorithmic_bytes": vbytes,
+                  "roofline": c.hbm_roof("vha_kernel<false,8>", vbytes, tv)}
+    del vout
+    if c.oracle_on:
+        import oracle
+        T = pc.T
+        kmax = pin["k"][0, :, 0].float().abs().amax(dim=1)
+        boosted = torch.nonzero(kmax > 6.0).flatten().tolist()[:8]
+        rs = np.random.RandomState(2)
+        ts = set([0, 1, 127, 128, 129, 255, 256, T - 2, T - 1])
+        ts |= set(int(x) for x in rs.randint(0, T, 40))
+        ts |= set(min(T - 1, b + o) for b in boosted for o in (0, 127))
+        rows = [(0, t) for t in sorted(ts)]
+        tm = OracleTimer()
+        rk, rv, kcb, vcb = oracle_cache_of(oracle, pin["k"], pin["v"], pin["w"], pc.blk, tm)
+        t_comp = tm.s
+        qsel = oracle.bf16_bits(pin["q"][0, [t for _, t in rows]])
+        ro = tm(oracle.prefill_rows, qsel, oracle.bf16_bits(pin["k"]), oracle.bf16_bits(pin["v"]), kcb, vcb,
+                pc.blk, pc.W, scale, rows, q_rows=True)
+        t_rows = tm.s - t_comp
+        idx = torch.tensor([t for _, t in rows], device=c.dev)
+        got = pout[0, idx]
+        e = err_stats(got, ro)
+        # the bf16 output is the stored result: within the bar plus half a bf16 ulp of the reference
+        half_ulp = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(ro), 2.0 ** -126))).astype(np.int64) - 8)
+        g64 = got.float().cpu().numpy().astype(np.float64)
+        ok_bf16 = bool(np.all(np.abs(g64 - ro) <= 1e-2 + half_ulp))
+        ek = err_stats(pkc, rk)
+        sel_keys = sum(oracle.visible_entries(t, pc.W, pc.blk) + min(pc.W, t + 1) for _, t in rows)
+        res["oracle"] = {"seconds_sampled_rows": t_rows, "compress_seconds": t_comp, "rows": len(rows),
+                         "cores": oracle.num_threads(),
+                         "seconds_full_extrapolated": t_comp + t_rows * keys / sel_keys,
+                         "scope": "compress in full; %d sampled query rows x all 64 heads (the full fp64 "
+                                  "prefill is ~1.1e13 flop), extrapolated by visible keys" % len(rows)}
+        res["parity"] = dict(e, cache_max_abs_err=ek["max_abs_err"], bf16_within_bar_plus_half_ulp=ok_bf16,
+                             within_tolerance=ok_bf16 and e["mean_abs_err"] <= 1e-3 and ek["max_abs_err"] <= 4e-3)
+    del pin, pkc, pvc, pout
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode_1m(c):
+    hca, wl = c.hca, c.wl
+    cfg = wl.DECODE_1M
+    scale = 1.0 / np.sqrt(cfg.d)
+    inp = wl.decode_inputs(cfg, c.dev)
+    k, v, w, q, kw, vw, seq = (inp[x] for x in ("k", "v", "w", "q", "kw", "vw", "seqlens"))
+    B, L = cfg.B, cfg.T
+    Nc = L // cfg.blk
+    kc = torch.empty((B, Nc, 1, cfg.d), dtype=torch.bfloat16, device=c.dev)
+    vc = torch.empty((B, Nc, 1, cfg.dv), dtype=torch.bfloat16, device=c.dev)
+    out = torch.empty((B, cfg.Hq, cfg.dv), dtype=torch.float32, device=c.dev)
+    ws = torch.empty(hca.decode_workspace_size(B, cfg.Hq, cfg.Hkv, cfg.dv), dtype=torch.uint8, device=c.dev)
+
+    def comp():
+        hca.compress(k, v, w, cfg.blk, kc=kc, vc=vc)
+
+    def dec():
+        hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
+
+    for _ in range(3):
+        comp()
+        dec()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    c_ms = timed_calls(comp, max(3, min(c.args.steps, 10)), c.stream, c.sampler, flush=c.flush)
+    d_ms = timed_calls(dec, c.args.steps, c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    t_c, t_d = c.mean_s(c_ms), c.mean_s(d_ms)
+    cbytes = compress_bytes(B, L, 1, cfg.d, cfg.dv, cfg.blk)
+    dbytes = decode_bytes(B, L, cfg.Hq, 1, cfg.d, cfg.dv, cfg.blk, cfg.W)
+    res = {"workload": cfg.name, "what": "hca_compress (timed alone) then hca_decode (cache resident)",
+           "compress": {"ms": t_c * 1e3, "gbs": cbytes / t_c / 1e9, "algorithmic_bytes": cbytes,
+                        "roofline": c.hbm_roof("compress_kernel<512,512>", cbytes, t_c)},
+           "decode": {"us": t_d * 1e6, "median_us": statistics.median(d_ms) * 1e3, "queries_per_s": B / t_d,
+                      "algorithmic_bytes": dbytes, "bytes_per_query": dbytes // B,
+                      "roofline": c.hbm_roof("decode_split_kernel + decode_combine_kernel", dbytes, t_d)}}
+    dec()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    if c.oracle_on:
+        import oracle
+        tm = OracleTimer()
+        rk, rv, kcb, vcb = oracle_cache_of(oracle, k, v, w, cfg.blk, tm)
+        t_comp = tm.s
+        ro = tm(oracle.decode, oracle.bf16_bits(q), kcb, vcb, oracle.bf16_bits(kw), oracle.bf16_bits(vw),
+                seq.cpu().numpy(), cfg.blk, cfg.W, scale)
+        e = err_stats(out, ro)
+        ek = max(err_stats(kc, rk)["max_abs_err"], err_stats(vc, rv)["max_abs_err"])
+        res["oracle"] = {"seconds": tm.s, "compress_seconds": t_comp, "decode_seconds": tm.s - t_comp,
+                         "cores": oracle.num_threads(), "scope": "full (every sequence, head and channel)"}
+        res["parity"] = dict(e, cache_max_abs_err=ek, within_tolerance=within(e) and ek <= 4e-3)
+        del rk, rv, kcb, vcb
+    del inp, k, v, w, kc, vc, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_ragged_paged(c):
+    hca, wl = c.hca, c.wl
+    cfg = wl.RAGGED_PAGED
+    scale = 1.0 / np.sqrt(cfg.d)
+    inp = wl.paged_decode_inputs(cfg, c.dev)
+    B = cfg.B
+    out = torch.empty((B, cfg.Hq, cfg.dv), dtype=torch.float32, device=c.dev)
+    ws = torch.empty(hca.decode_workspace_size(B, cfg.Hq, cfg.Hkv, cfg.dv), dtype=torch.uint8, device=c.dev)
+
+    def dec():
+        hca.decode(inp["q"], inp["kc"], inp["vc"], inp["kw"], inp["vw"], inp["seqlens"], cfg.blk, cfg.W, scale,
+                   page_table=inp["page_table"], page_size=cfg.page_size, gq=inp["gq"], gk=inp["gk"],
+                   gate=inp["gate"], out=out, workspace=ws)
+
+    for _ in range(3):
+        dec()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    d_ms = timed_calls(dec, c.args.steps, c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    t = c.mean_s(d_ms)
+    lens = inp["seqlens"].cpu().tolist()
+    dbytes = sum(decode_seq_bytes(L, cfg.Hq, cfg.Hkv, cfg.d, cfg.dv, cfg.blk, cfg.W, gate=True) for L in lens)
+    res = {"workload": cfg.name, "what": "hca_decode, paged cache, QK RMSNorm + sigmoid gate",
+           "us": t * 1e6, "median_us": statistics.median(d_ms) * 1e3, "queries_per_s": B / t,
+           "algorithmic_bytes": dbytes, "mean_context": float(np.mean(lens)),
+           "roofline": c.hbm_roof("decode_split_kernel + decode_combine_kernel", dbytes, t)}
+    dec()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    if c.oracle_on:
+        import oracle
+        tm = OracleTimer()
+        b = oracle.bf16_bits
+        ro = tm(oracle.decode, b(inp["q"]), b(inp["kc"]), b(inp["vc"]), b(inp["kw"]), b(inp["vw"]),
+                inp["seqlens"].cpu().numpy(), cfg.blk, cfg.W, scale, page_table=inp["page_table"].cpu().numpy(),
+                page_size=cfg.page_size, gq=inp["gq"].cpu().numpy(), gk=inp["gk"].cpu().numpy(), eps=1e-6,
+                gate=b(inp["gate"]))
+        e = err_stats(out, ro)
+        res["oracle"] = {"seconds": tm.s, "cores": oracle.num_threads(),
+                         "scope": "full (every sequence, head and channel)"}
+        res["parity"] = dict(e, within_tolerance=within(e))
+    del inp, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline_sample(ref_cache, target_s=10.0):
+    """The oracle as it stands, on this host, for a bounded sample of the headline workload: the
+    oracle's decode of the whole 64-query batch over its own compressed cache, repeated for about
     ``target_s`` seconds."""
     import oracle
-    from compressed_long_context_b200 import workloads as wl
-    cfg = wl.DECODE_128K
-    n = 2
-    inp = wl.decode_inputs(cfg.scaled(B=n), "cpu")
-    kb, vb = oracle.bf16_bits(inp["k"]), oracle.bf16_bits(inp["v"])
-    w = inp["w"].numpy()
-    qb, kwb, vwb = oracle.bf16_bits(inp["q"]), oracle.bf16_bits(inp["kw"]), oracle.bf16_bits(inp["vw"])
-    seq = inp["seqlens"].numpy()
-    scale = 1.0 / np.sqrt(cfg.d)
+    B = ref_cache[0].shape[0]
     reps = 0
     t0 = time.perf_counter()
     while True:
-        kc, vc = oracle.compress(kb, vb, w, cfg.blk)
-        oracle.decode(qb, oracle.round_bf16(kc), oracle.round_bf16(vc), kwb, vwb, seq, cfg.blk, cfg.W, scale)
+        oracle.decode(*ref_cache)
         reps += 1
         dt = time.perf_counter() - t0
         if dt >= target_s:
             break
-    return {"value": n * reps / dt, "unit": "queries/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "%d passes over 2 sequences of the workload (oracle fp64 compress of 131072 raw tokens, K and "
-                      "V, + decode of 64 heads over 1023 entries + 128 window tokens), %.1f s" % (reps, dt)}
+    return {"value": B * reps / dt, "unit": "queries/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d oracle fp64 decodes of the whole batch (%d queries, 64 heads, 1023 entries + 128 window "
+                      "tokens each, over the oracle's own compressed cache), %.1f s" % (reps, B, dt)}
 
 
-# ---------------------------------------------------------------- our arm
-
-def main():
-    args = parse()
+def main(argv=None):
+    args = parse(argv)
     if args.impl == "reference":
         run_reference(args)
         return
     world, rank, local = dist_setup(args)
     sys.path.insert(0, ROOT)
-    import compressed_long_context_b200 as hca
-    from compressed_long_context_b200 import _lib, workloads as wl
+    from compressed_long_context_b200 import _lib
+    c = Ctx(args, world, rank, local)
+    want = set(x.strip() for x in args.configs.split(",") if x.strip())
+    unknown = want - set(CONFIG_KEYS)
+    if unknown:
+        raise SystemExit("unknown configs: %s" % ",".join(sorted(unknown)))
 
-    pk, pk_kind = peaks()
-    dev = torch.device("cuda", torch.cuda.current_device())
-    cfg = wl.DECODE_128K
-    scale = 1.0 / np.sqrt(cfg.d)
-    inp = wl.decode_inputs(cfg, dev)
-    k, v, w, q, kw, vw, seq = (inp[x] for x in ("k", "v", "w", "q", "kw", "vw", "seqlens"))
-    B, L = cfg.B, cfg.T
-    Nc = L // cfg.blk
-    kc = torch.empty((B, Nc, 1, cfg.d), dtype=torch.bfloat16, device=dev)
-    vc = torch.empty((B, Nc, 1, cfg.dv), dtype=torch.bfloat16, device=dev)
-    out = torch.empty((B, cfg.Hq, cfg.dv), dtype=torch.float32, device=dev)
-    ws = torch.empty(hca.decode_workspace_size(B, cfg.Hq, cfg.Hkv, cfg.dv), dtype=torch.uint8, device=dev)
-    flush = l2_flush_buffer()
-    stream = torch.cuda.current_stream()
-
-    def step():
-        hca.compress(k, v, w, cfg.blk, kc=kc, vc=vc)
-        hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-    hca.get_device_error()
-
-    # ---- timed region: K steps, each bracketed by events; L2 flushed between steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    with sampler:
-        torch.cuda._sleep(int(2e8))
-        for i in range(args.steps):
-            flush.zero_()
-            a, m, b = ev[i]
-            a.record(stream)
-            hca.compress(k, v, w, cfg.blk, kc=kc, vc=vc)
-            m.record(stream)
-            hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
-            b.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    step_ms = [a.elapsed_time(b) for a, _, b in ev]
-    comp_ms = [a.elapsed_time(m) for a, m, _ in ev]
-    dec_in_step_ms = [m.elapsed_time(b) for _, m, b in ev]
-    hca.get_device_error()
-    t_step = max_over_ranks(sum(step_ms) / 1e3, world)
-    ms_per_step = t_step * 1e3 / args.steps
-    value = weak_scaling_value(B * args.steps, world, t_step)
-
-    # compress roofline (dominant kernel of the step)
-    cbytes = compress_bytes(B, L, 1, cfg.d, cfg.dv, cfg.blk)
-    c_avg = sum(comp_ms) / len(comp_ms) / 1e3
-    c_gbs = cbytes / c_avg / 1e9
-    roof = {"bound": "hbm", "kernel": "compress_kernel<512,512>", "achieved": c_gbs, "peak": pk["hbm_gbs"],
-            "unit": "GB/s", "frac": c_gbs / pk["hbm_gbs"],
-            "traffic": traffic_for("compress_decode_B64_L131072",
-                                   ["compressed_long_context_b200/csrc/compress.cuh"]),
-            "algorithmic_bytes_per_launch": cbytes, "peak_kind": pk_kind + " (hbm_gbs)"}
-
-    # ---- decode alone: cache resident, L2 flushed before each call.  A GPU-side spin is
-    # queued first so that every timed call is already enqueued when the GPU reaches it:
-    # the events then bracket device work only, not host launch overhead.
-    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    with sampler:
-        torch.cuda._sleep(int(2e8))
-        for i in range(args.steps):
-            flush.zero_()
-            a, b = dev_ev[i]
-            a.record(stream)
-            hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws)
-            b.record(stream)
-        torch.cuda.synchronize()
-    d_ms = [a.elapsed_time(b) for a, b in dev_ev]
-    d_avg = max_over_ranks(sum(d_ms) / len(d_ms) / 1e3, world)
-    dbytes = decode_bytes(B, L, cfg.Hq, 1, cfg.d, cfg.dv, cfg.blk, cfg.W)
-    d_gbs = dbytes / d_avg / 1e9
-    decode_part = {"queries_per_s": world * B / d_avg, "us_per_call": d_avg * 1e6,
-                   "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + decode_combine_kernel",
-                                "achieved": d_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                "frac": d_gbs / pk["hbm_gbs"], "algorithmic_bytes_per_call": dbytes,
-                                "traffic": traffic_for("decode_B64_L131072",
-                                                       ["compressed_long_context_b200/csrc/decode.cuh"])},
-                   "median_us_per_call": statistics.median(d_ms) * 1e3,
-                   "decode_in_step_us": statistics.median(dec_in_step_ms) * 1e3}
-
-    # ---- one serving step: hca_append of every sequence's newest token (window ring write +
-    # online pooling; at L = 131072 every sequence completes a block, so an entry is written
-    # too), then hca_decode over the ring.  L2 flushed before each step.
-    kn, vn = k[:, L - 1].contiguous(), v[:, L - 1].contiguous()
-    wn = w[:, L - 1].contiguous()
-    state = torch.zeros(hca.append_state_size(B, 1, cfg.d, cfg.dv), dtype=torch.uint8, device=dev)
-
-    def serve(decode_too):
-        hca.append(kn, vn, wn, seq, kw, vw, kc, vc, state, cfg.blk)
-        if decode_too:
-            hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, out=out, workspace=ws, window_ring=True)
-
-    serve_part = {}
-    for name, dec in (("append_us", False), ("append_plus_decode_us", True)):
-        for _ in range(3):
-            serve(dec)
-        sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        with sampler:
-            torch.cuda._sleep(int(2e8))
-            for i in range(args.steps):
-                flush.zero_()
-                a, b = sev[i]
-                a.record(stream)
-                serve(dec)
-                b.record(stream)
-            torch.cuda.synchronize()
-        serve_part[name] = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in sev]) / 1e3,
-                                          world) * 1e6
-    hca.get_device_error()
-    abytes = append_bytes(B, 1, cfg.d, cfg.dv)
-    serve_part.update({"workload": "append + ring decode, %s" % cfg.name,
-                       "append_algorithmic_bytes": abytes,
-                       "append_frac_of_hbm": abytes / (serve_part["append_us"] / 1e6) / 1e9 / pk["hbm_gbs"],
-                       "append_bound": "latency (one small CTA per sequence; %d KB moved)" % (abytes // 1024)})
-    del state
-
-    # ---- e2e through the public API with host buffers (pinned), copies inside the timed region
-    e2e = None
-    if not args.no_e2e:
-        hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
-        hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
-        hk.copy_(k)
-        hv.copy_(v)
-        hw, hq, hkw, hvw, hs = (x.cpu().pin_memory() for x in (w, q, kw, vw, seq))
-        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        dk, dvv = torch.empty_like(k), torch.empty_like(v)
-        dw, dq, dkw, dvw, ds = (torch.empty_like(x) for x in (w, q, kw, vw, seq))
-        h2d = sum(x.numel() * x.element_size() for x in (hk, hv, hw, hq, hkw, hvw, hs))
-        d2h = hout.numel() * hout.element_size()
-        del k, v
-        torch.cuda.empty_cache()
-
-        def e2e_step():
-            for hsrc, ddst in ((hk, dk), (hv, dvv), (hw, dw), (hq, dq), (hkw, dkw), (hvw, dvw), (hs, ds)):
-                ddst.copy_(hsrc, non_blocking=True)
-            hca.compress(dk, dvv, dw, cfg.blk, kc=kc, vc=vc)
-            hca.decode(dq, kc, vc, dkw, dvw, ds, cfg.blk, cfg.W, scale, out=out, workspace=ws)
-            hout.copy_(out, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        ne = max(2, min(args.steps, 5))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(ne):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        te = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-        e2e = {"value": world * B * ne / te, "unit": "queries/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": ne}
-        del hk, hv, dk, dvv
-        torch.cuda.empty_cache()
-    else:
-        del k, v
-        torch.cuda.empty_cache()
-
-    # ---- prefill 128K (TFLOP/s)
-    prefill_part = None
-    if not args.no_prefill:
-        pc = wl.PREFILL_128K
-        pin = wl.prefill_inputs(pc, dev)
-        pkc, pvc = hca.compress(pin["k"], pin["v"], pin["w"], pc.blk)
-        pout = torch.empty((1, pc.T, pc.Hq, pc.dv), dtype=torch.bfloat16, device=dev)
-        for _ in range(2):
-            hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
-        torch.cuda.synchronize()
-        hca.get_device_error()
-        np_steps = max(2, min(args.steps, 5))
-        pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-                torch.cuda.Event(enable_timing=True)) for _ in range(np_steps)]
-        with sampler:
-            for i in range(np_steps):
-                flush.zero_()
-                a, m, b = pev[i]
-                a.record(stream)
-                hca.compress(pin["k"], pin["v"], pin["w"], pc.blk, kc=pkc, vc=pvc)
-                m.record(stream)
-                hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, 1.0 / np.sqrt(pc.d), out=pout)
-                b.record(stream)
-            torch.cuda.synchronize()
-        hca.get_device_error()
-        p_ms = max_over_ranks(statistics.median([m.elapsed_time(b) for _, m, b in pev]), world)
-        c3_ms = statistics.median([a.elapsed_time(m) for a, m, _ in pev])
-        flops, keys = prefill_flops(1, pc.T, pc.Hq, pc.d, pc.dv, pc.blk, pc.W)
-        tf = flops / (p_ms / 1e3) / 1e12
-        peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-        prefill_part = {"workload": pc.name, "tflops": tf, "ms": p_ms, "compress_ms": c3_ms,
-                        "algorithmic_flops": flops, "keys_per_head": keys,
-                        "roofline": {"bound": "tensor", "kernel": "prefill_pair_kernel", "achieved": tf,
-                                     "peak": peak_tf, "unit": "TFLOP/s", "frac": tf / peak_tf,
-                                     "peak_kind": pk_kind + " (bf16_tflops_sustained)",
-                                     "frac_of_burst": tf / pk["bf16_tflops"],
-                                     "traffic": traffic_for("prefill_T131072",
-                                                            ["compressed_long_context_b200/csrc/prefill.cuh",
-                                                             "compressed_long_context_b200/csrc/prefill_pair.cuh"])}}
-        # Virtual Head Attention on the prefill output (in place, bf16): one read and one write
-        # of the 8.6 GB output, HBM-bound; synthetic rank-8 factors
-        gv = torch.Generator(device=dev).manual_seed(5)
-        vu = torch.randn((pc.Hq, 8), generator=gv, device=dev) * 0.1
-        vv = torch.randn((pc.Hq, 8), generator=gv, device=dev) * 0.1
-        hca.vha(pout, vu, vv)
-        vev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(np_steps)]
-        with sampler:
-            for i in range(np_steps):
-                a, b = vev[i]
-                a.record(stream)
-                hca.vha(pout, vu, vv)
-                b.record(stream)
-            torch.cuda.synchronize()
-        hca.get_device_error()
-        v_ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in vev]), world)
-        vbytes = vha_bytes(pout.numel(), pout.element_size(), pc.Hq, vu.shape[1])
-        prefill_part["vha"] = {"ms": v_ms, "rank": 8, "algorithmic_bytes": vbytes, "bound": "hbm",
-                               "achieved_gbs": vbytes / (v_ms / 1e3) / 1e9,
-                               "frac": vbytes / (v_ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                               "peak_kind": pk_kind + " (hbm_gbs)"}
-        del pin, pkc, pvc, pout
-        torch.cuda.empty_cache()
-
+    configs = {}
+    head, configs["decode_128k"], e2e, ref_cache = bench_decode_128k(c)
     cpu_base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu_base = cpu_baseline_sample()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and ref_cache is not None:
+        cpu_base = cpu_baseline_sample(ref_cache)
+    del ref_cache
+    runners = {"tiny_prefill": bench_tiny_prefill, "prefill_128k": bench_prefill_128k,
+               "decode_1m": bench_decode_1m, "ragged_paged": bench_ragged_paged}
+    for key in CONFIG_KEYS:
+        if key in runners and key in want:
+            configs[key] = runners[key](c)
+            barrier(world)
 
-    clocks = sampler.summary()
+    clocks = c.sampler.summary()
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
-                "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        cfg = c.wl.DECODE_128K
+        line = {"metric": METRIC, "value": head["value"], "unit": "queries/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": head["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded; no dataset)",
-                "config": {"workload": cfg.name, "B": B, "L": L, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
-                           "blk": cfg.blk, "W": cfg.W, "step": "hca_compress(raw K/V) + hca_decode",
-                           "l2": "flushed (2x L2 memset) before every timed step; raw K/V 17.2 GB > L2",
+                "config": {"workload": cfg.name, "B": cfg.B, "L": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d,
+                           "blk": cfg.blk, "W": cfg.W,
+                           "step": "hca_decode of the batch (split + combine kernels), compressed cache resident",
+                           "l2": "flushed (2x L2 memset) before every timed call",
                            "parallelism": "dp%d (independent batches, no collective)" % world},
-                "roofline": roof, "decode": decode_part, "serving_step": serve_part, "prefill": prefill_part,
-                "cpu_baseline": cpu_base, "e2e": e2e,
-                "gpu_launches": 3 * args.steps, "clocks": clocks,
+                "roofline": head["roofline"], "configs": configs, "cpu_baseline": cpu_base, "e2e": e2e,
+                "gpu_launches": 2 * args.steps, "clocks": clocks,
                 "libhca": os.path.relpath(_lib.LIB_PATH, ROOT)}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -22,7 +22,8 @@ HCA_WINDOW_RING = 32
 
 # Names of every entry point declared in include/hca.h.
 EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_decode", "hca_decode_noalloc",
-           "hca_vha", "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error")
+           "hca_vha", "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error",
+           "hca_debug_set_wait_limit", "hca_debug_set_drop_slab", "hca_debug_wait_probe")
 
 _lib = None
 
@@ -64,5 +65,11 @@ def load():
     lib.hca_append_state_size.argtypes = [_i] * 4
     lib.hca_append.restype = _i
     lib.hca_append.argtypes = [_vp] * 9 + [_i] * 3 + [_vp] + [_i] * 7 + [_u, _vp]
+    lib.hca_debug_set_wait_limit.restype = _i
+    lib.hca_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong, _vp]
+    lib.hca_debug_set_drop_slab.restype = _i
+    lib.hca_debug_set_drop_slab.argtypes = [_i, _vp]
+    lib.hca_debug_wait_probe.restype = _i
+    lib.hca_debug_wait_probe.argtypes = [_vp]
     _lib = lib
     return lib

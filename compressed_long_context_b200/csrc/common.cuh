@@ -27,8 +27,19 @@ __device__ __forceinline__ void record_error(unsigned int code) {
     atomicCAS(&g_error, 0u, code);
 }
 
-// Wall-clock bound of one wait.  Legitimate waits in these kernels last microseconds.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
+// Wall-clock bound of one wait.  Legitimate waits in these kernels last microseconds.  The
+// bound lives in device memory so that a test can shorten it (hca_debug_set_wait_limit) and
+// make a wait run out in milliseconds; kernels read it only once a wait has already spun.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s, the default
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+// Debug switch set by hca_debug_set_drop_slab: when nonzero, the decode producer never
+// issues the first K slab of a launch, so the wait for it runs out (no bad address is made).
+__device__ int g_debug_drop_slab = 0;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+    return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
@@ -79,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > wait_limit_ns()) {
                 *abort = 1;
                 record_error(HCA_ERR_TIMEOUT);
                 return false;

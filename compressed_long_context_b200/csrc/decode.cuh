@@ -468,6 +468,8 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             int ks = 0, vs = 0, kdone = 0, vdone = 0, qitem = 0;
             uint32_t kring = 0, vring = 0;
             bool q_issued = false;
+            // test switch (hca_debug_set_drop_slab): the first K slab is never requested
+            bool drop = *reinterpret_cast<volatile int*>(&g_debug_drop_slab) != 0;
             uint64_t t_prog = globaltimer_ns();
             uint32_t idle = 0;
             // Page ids of the two 64-entry halves of the current compressed K (V) tile, read
@@ -522,7 +524,8 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     } else {
                         const uint32_t st = kring % kDecRingK;
                         if (mbar_test(&kempty[st], ((kring / kDecRingK) & 1) ^ 1)) {
-                            issue(ki, kpg, ks, false, sm + kSmRingK + st * kSlabBytes, &kfull[st]);
+                            if (!drop) issue(ki, kpg, ks, false, sm + kSmRingK + st * kSlabBytes, &kfull[st]);
+                            drop = false;
                             ++kring;
                             prog = true;
                             if (++ks == kDecSlabs) {
@@ -558,7 +561,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     if (*abort_flag) break;
                     const uint64_t now = globaltimer_ns();
                     if (idle == 256) t_prog = now;
-                    else if (now - t_prog > kWaitLimitNs) {
+                    else if (now - t_prog > wait_limit_ns()) {
                         *abort_flag = 1;
                         record_error(HCA_ERR_TIMEOUT);
                         break;
@@ -904,6 +907,17 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
         asm volatile("cp.async.commit_group;" ::: "memory");
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (*reinterpret_cast<volatile unsigned int*>(&g_error) == HCA_ERR_TIMEOUT) {
+        // a split CTA gave up: its records (and the unit ranges) may be stale, so the outputs are
+        // marked invalid rather than merged from whatever the workspace holds
+        for (int j = 0; j < kMergeHeads; ++j)
+            if (h0 + j < p.G) {
+                const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h0 + j) * kDecD + c;
+                *reinterpret_cast<float4*>(p.out + orow) = make_float4(NAN, NAN, NAN, NAN);
+            }
+        if (gated) asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
     const int first = __ldg(p.meta + 2 * u), last = __ldg(p.meta + 2 * u + 1);
     if (first < 0 || last < first || last >= p.nsplit) {
         if (threadIdx.x == 0 && blockIdx.y == 0) record_error(HCA_ERR_DEVICE_INPUT);

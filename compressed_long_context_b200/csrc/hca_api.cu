@@ -96,9 +96,53 @@ int num_sms() {
     return n;
 }
 
+__device__ unsigned int g_error_taken = 0;
+
+__global__ void take_error_kernel() { g_error_taken = atomicExch(&g_error, 0u); }
+
+// One CTA that waits on an mbarrier which can never complete (two arrivals expected, one
+// made), with the same bounded wait the attention kernels use: it runs out after the
+// device's wait limit, records HCA_ERR_TIMEOUT and returns.  Nothing is in flight.
+__global__ void wait_probe_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&bar, 2);
+        fence_mbar_init();
+        mbar_arrive(&bar);
+        mbar_wait(&bar, 0, &abort_flag);
+    }
+    __syncthreads();
+}
+
 }  // namespace hca
 
 extern "C" {
+
+hca_status_t hca_debug_set_wait_limit(unsigned long long limit_ns, hca_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    static const unsigned long long kDefault = hca::kWaitLimitNs;
+    const unsigned long long v = limit_ns ? limit_ns : kDefault;
+    if (cudaMemcpyToSymbolAsync(hca::g_wait_limit_ns, &v, sizeof v, 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return HCA_ERR_CUDA;
+    return HCA_OK;
+}
+
+hca_status_t hca_debug_set_drop_slab(int on, hca_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int v = on ? 1 : 0;
+    if (cudaMemcpyToSymbolAsync(hca::g_debug_drop_slab, &v, sizeof v, 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return HCA_ERR_CUDA;
+    return HCA_OK;
+}
+
+hca_status_t hca_debug_wait_probe(hca_stream_t stream) {
+    hca::wait_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    return launch_status();
+}
 
 const char* hca_status_string(hca_status_t s) {
     switch (s) {
@@ -115,10 +159,13 @@ const char* hca_status_string(hca_status_t s) {
 
 hca_status_t hca_get_device_error(hca_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    unsigned int word = 0, zero = 0;
-    if (cudaMemcpyFromSymbolAsync(&word, g_error, sizeof word, 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return HCA_ERR_CUDA;
-    if (cudaMemcpyToSymbolAsync(g_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    unsigned int word = 0;
+    // read and clear in one atomic step on the device, so that an error recorded by a kernel on
+    // another stream between a read and a separate clear cannot be lost
+    hca::take_error_kernel<<<1, 1, 0, s>>>();
+    if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
+    if (cudaMemcpyFromSymbolAsync(&word, hca::g_error_taken, sizeof word, 0, cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
         return HCA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return HCA_ERR_CUDA;
     if (word == HCA_ERR_TIMEOUT || word == HCA_ERR_DEVICE_INPUT || word == HCA_ERR_INTERNAL)

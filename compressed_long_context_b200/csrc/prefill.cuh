@@ -6,16 +6,14 @@
 // Attention").  The two segments are two runs of key tiles through the same (m, l, O)
 // state, with a per-row mask on each tile.
 //
-// Tiling.  The 128 MMA rows of a tile are (token, head) pairs of one KV group: 128 / G
-// tokens x G heads (G = Hq / Hkv), so all rows of a tile share their keys.  With d = 512
-// the fp32 accumulator of 128 rows x 512 columns would fill all of tensor memory, so a
-// CTA owns one 256-wide half of the value dimension (O: 256 TMEM columns) next to two
-// 128-column S buffers; the two halves of a row tile run on different CTAs, each
-// computing its own S.  This costs QK^T twice and is the first thing a 2-CTA variant
-// removes.
+// This single-CTA kernel serves 64-dim heads (512-dim heads run on the SM pair of
+// prefill_pair.cuh, which also takes PrefillParams and the tile helpers from here).
 //
-// Per work item (row tile, dv half), warp-specialised, persistent over a heavy-first
-// schedule:
+// Tiling.  The 128 MMA rows of a tile are (token, head) pairs of one KV group: 128 / G
+// tokens x G heads (G = Hq / Hkv), so all rows of a tile share their keys.  S (two
+// 128-column buffers), P and the 64-column O of a row tile all fit one SM's tensor memory.
+//
+// Per work item (row tile), warp-specialised, persistent over a heavy-first schedule:
 //   warp 0 (1 thread)  TMA: Q tile (d/64 slabs), then K and V tiles as 64-channel slabs
 //                      (128 keys each, 128-byte swizzle) through a ring of 16 KB slots;
 //   warp 1 (1 thread)  tcgen05.mma: S = Q K^T into TMEM (double-buffered), then
@@ -36,11 +34,11 @@ constexpr uint32_t kPfSlab = 128 * 128;
 
 template <int D>
 struct PfCfg {
+    static_assert(D == 64, "prefill_kernel serves 64-dim heads; 512-dim heads use prefill_pair_kernel");
     static constexpr int kSlabs = D / 64;                 // Q / K slabs per row
-    static constexpr int kDVC = D < 256 ? D : 256;        // value columns per CTA
-    static constexpr int kNS = D / kDVC;                  // dv halves
+    static constexpr int kDVC = D;                        // value columns
     static constexpr int kVSlabs = kDVC / 64;
-    static constexpr int kRing = D == 512 ? 6 : 8;
+    static constexpr int kRing = 8;
     static constexpr uint32_t kSmQ = 0;
     static constexpr uint32_t kSmRing = kSmQ + kSlabs * kPfSlab;
     static constexpr uint32_t kSmBar = kSmRing + kRing * kPfSlab;
@@ -50,7 +48,7 @@ struct PfCfg {
     static_assert(kSmem <= 232448, "prefill shared memory exceeds the 227 KB per-block limit");
     static_assert(kSmRing % 1024 == 0 && kSmBar % 8 == 0, "operand tiles 1024-aligned, barriers 8-aligned");
     static constexpr uint32_t kTmS = 0;       // 2 x 128 columns
-    static constexpr uint32_t kTmO = 256;     // kDVC columns
+    static constexpr uint32_t kTmO = 256;     // kDVC columns (after the two S buffers)
 };
 
 struct PrefillParams {
@@ -62,7 +60,7 @@ struct PrefillParams {
 };
 
 struct PfItem {
-    int b, g, t0, tlast, hs;
+    int b, g, t0, tlast;
     int nc_hi, ncomp, nct, wlo, nwin, nwt;
 };
 
@@ -73,10 +71,8 @@ __device__ __forceinline__ int pf_visible(int t, int W, int blk) {
 
 template <int D>
 __device__ __forceinline__ PfItem pf_item(const PrefillParams& p, long long i) {
-    using C = PfCfg<D>;
     PfItem it;
-    it.hs = (int)(i % C::kNS);
-    long long r = i / C::kNS;
+    long long r = i;
     it.g = (int)(r % p.Hkv);
     r /= p.Hkv;
     it.b = (int)(r % p.B);
@@ -175,7 +171,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                 const bool comp = j < it.nct;
                 const int row = comp ? 128 * j : it.wlo + 128 * (j - it.nct);
                 for (int s = 0; s < C::kVSlabs; ++s)
-                    if (!load_slab(comp ? &tm_vc : &tm_v, it.hs * C::kDVC + 64 * s, it.g, row, it.b)) return false;
+                    if (!load_slab(comp ? &tm_vc : &tm_v, 64 * s, it.g, row, it.b)) return false;
                 return true;
             };
             for (long long i = blockIdx.x; ok && i < p.items; i += stride, ++item_n) {
@@ -368,8 +364,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
             if (!warp_wait(o_full, item_n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const float inv = 1.f / l;
-            const size_t orow = (((size_t)it.b * p.T + tok) * p.Hq + head) * (size_t)(C::kDVC * C::kNS) +
-                                (size_t)it.hs * C::kDVC;
+            const size_t orow = (((size_t)it.b * p.T + tok) * p.Hq + head) * (size_t)C::kDVC;
 #pragma unroll 1
             for (int c = 0; c < C::kDVC; c += 16) {
                 float o[16];
@@ -393,7 +388,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
             }
-            if (row_live && p.lse && it.hs == 0)
+            if (row_live && p.lse)
                 p.lse[((size_t)it.b * p.Hq + head) * p.T + tok] = (m + log2f(l)) * 0.6931471805599453f;
             tc_fence_before();
             __syncwarp();

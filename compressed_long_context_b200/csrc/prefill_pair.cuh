@@ -11,14 +11,13 @@
 // tile need 256 more.  So the work is split by stage, not by value columns:
 //   S-CTA (cluster rank 0): Q resident in shared memory, K tiles streamed by TMA,
 //       S = Q K^T with N = 256 keys into a double-buffered S (2 x 256 TMEM columns), softmax
-//       (thread = row), and P (bf16) written to a per-pair slot in global memory (L2) in the
-//       non-swizzled K-major layout the tensor core reads (8 keys of row r at
-//       (key / 8) * 2048 + r * 16, so the 32 rows of a warp fill 512 contiguous bytes per
-//       store); the per-row rescale factors (and, after the last tile, the row sums) go
-//       straight into the O-CTA's shared memory.  P takes the L2 path because the
-//       SM-to-SM network moves only about 30 GB/s per pair, a third of what a 256-key tile
-//       needs; an O-CTA thread pulls each slot into shared memory with a bulk copy.  The
-//       hand-off granule is a P unit of 128 keys (half an S tile), four units in flight;
+//       (thread = row), and P (bf16) stored straight into a slot of the O-CTA's shared
+//       memory with st.async, in the non-swizzled K-major layout the tensor core reads (8 keys
+//       of row r at (key / 8) * 2048 + r * 16).  Every such store counts its bytes on the
+//       O-CTA's slot barrier (mbarrier::complete_tx), and each lane quarter arms that barrier
+//       with the byte total it stored, so the writers never wait for completion.  A per-unit
+//       header (each row's rescale factor, a flag per lane quarter) travels the same way.  The
+//       hand-off granule is a P unit of 128 keys (half an S tile), three slots in flight;
 //   O-CTA (cluster rank 1): V tiles streamed by TMA, O += P V with N = 256 value columns
 //       (two MMAs per 16 keys cover the 512 columns), rescale of O rows when the S-CTA moved
 //       a row's reference maximum, and the epilogue out = O / l.
@@ -27,9 +26,9 @@
 //
 // Warps (320 threads, same kernel for both ranks):
 //   S-CTA: 0 TMA (Q, K) | 1 MMA + TMEM | 2-9 softmax (two warps per TMEM lane quarter)
-//   O-CTA: 0 TMA (V)    | 1 MMA + TMEM | 2-5 rescale + epilogue | 6 P loads | 7 "P slot
-//          consumed" forwarded to the S-CTA (its own warp, so that a slot is returned the
-//          moment its PV lands, whatever the loads are waiting for) | 8, 9 idle
+//   O-CTA: 0 TMA (V)    | 1 MMA + TMEM | 2-5 rescale + epilogue | 7 "P slot consumed"
+//          forwarded to the S-CTA (its own warp, so that a slot is returned the moment its
+//          PV lands, whatever else is waiting) | 6, 8, 9 idle
 //
 // Tiles of one row tile (item): the compressed segment in tiles of 256 entries, then the
 // raw window [wlo, tlast] in tiles of 256 tokens; per-row masks [lo, hi) as in prefill.cuh.
@@ -195,7 +194,7 @@ __device__ __forceinline__ bool pp_wait_cl(uint64_t* bar, uint32_t parity, volat
         if (pp_try_wait_cl(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > wait_limit_ns()) {
                 *abort = 1;
                 record_error(HCA_ERR_TIMEOUT);
                 return false;
@@ -212,7 +211,7 @@ __device__ __forceinline__ bool pp_warp_wait_cl(uint64_t* bar, uint32_t parity, 
 __device__ __forceinline__ void pp_drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > wait_limit_ns()) {
             record_error(HCA_ERR_TIMEOUT);
             return;
         }

@@ -166,11 +166,13 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc,
  * The call allocates nothing (no cudaMalloc, no cudaFree, no allocating library routine).
  *  - Returns HCA_ERR_INVALID_ARG, before any launch, when the batch needs more scratch
  *    than the array holds, i.e. when hca_decode_workspace_size(B, Hq, Hkv, dv) exceeds
- *    HCA_DECODE_NOALLOC_MAX_BYTES (on a 148-SM B200 this allows up to about 200
+ *    HCA_DECODE_NOALLOC_MAX_BYTES (on a 148-SM B200 this allows up to 234
  *    (sequence, KV head) units).
  *  - The first call on a device looks up the array's device address on that device
  *    (once per device, with that device current); make that first call before any stream
- *    capture.
+ *    capture.  The address is cached per device ordinal for the primary context: after
+ *    cudaDeviceReset, or when calling from a context other than the device's primary one,
+ *    the cached address is no longer valid -- use hca_decode there.
  *  - Every call on a device shares the same array, and the array keeps the previous
  *    call's contents; nothing in it needs to start at zero.  Calls whose work overlaps
  *    on the GPU (for example on two streams at once) race on it: serialise them.
@@ -243,11 +245,35 @@ hca_status_t hca_append(const void* k_new, const void* v_new, const float* w_new
 const char* hca_status_string(hca_status_t status);
 
 /*
- * hca_get_device_error -- wait for `stream`, then read and clear the current device's
- * error word: HCA_OK if no kernel recorded an error since the last call,
- * HCA_ERR_TIMEOUT or HCA_ERR_DEVICE_INPUT otherwise, HCA_ERR_CUDA if the read failed.
+ * hca_get_device_error -- read and clear the current device's error word in one atomic
+ * step on `stream` (a one-thread kernel), then wait for `stream`: HCA_OK if no kernel
+ * recorded an error since the last call, HCA_ERR_TIMEOUT, HCA_ERR_DEVICE_INPUT or
+ * HCA_ERR_INTERNAL otherwise, HCA_ERR_CUDA if the read failed.  An error recorded by work on
+ * another stream is never lost: it is either returned or left for the next call.  The word
+ * is per device and the read-out slot is shared, so make one such call at a time per device.
+ * While the word holds HCA_ERR_TIMEOUT, hca_decode writes NaN to its outputs instead of
+ * merging split records that a timed-out kernel may have left incomplete.
  */
 hca_status_t hca_get_device_error(hca_stream_t stream);
+
+/*
+ * Test hooks for the bounded waits (not part of the computation; the paper has no
+ * counterpart).  Every wait inside the kernels gives up after a wall-clock limit, records
+ * HCA_ERR_TIMEOUT and lets the kernel unwind (free its tensor memory, return) instead of
+ * hanging the GPU.  These three calls let a test make that happen on purpose without any
+ * bad address, trap or endless loop.  Each synchronises `stream`.
+ *
+ * hca_debug_set_wait_limit -- set the current device's wait limit in nanoseconds
+ *   (0 restores the default of 1 s).  Affects every later launch on the device.
+ * hca_debug_set_drop_slab -- on != 0: every later hca_decode launch on the device never
+ *   requests the first key slab of each split CTA, so the wait for it runs out after the
+ *   wait limit and the whole decode reports HCA_ERR_TIMEOUT (outputs NaN); 0 turns it off.
+ * hca_debug_wait_probe -- queue one CTA that waits on a barrier that can never complete
+ *   and so records HCA_ERR_TIMEOUT after the wait limit; nothing else is in flight.
+ */
+hca_status_t hca_debug_set_wait_limit(unsigned long long limit_ns, hca_stream_t stream);
+hca_status_t hca_debug_set_drop_slab(int on, hca_stream_t stream);
+hca_status_t hca_debug_wait_probe(hca_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -85,3 +85,24 @@ def test_max_over_ranks_gloo_two_ranks():
         assert p.exitcode == 0
     res = dict(q.get(timeout=10) for _ in range(2))
     assert res == {0: 2.5, 1: 2.5}
+
+
+def test_decode_seq_bytes_gate_and_short():
+    # the gate logits add Hq * dv bf16 per query; a sequence shorter than the window has no entries
+    base = bench.decode_seq_bytes(131072, 64, 1, 512, 512, 128, 128)
+    assert bench.decode_seq_bytes(131072, 64, 1, 512, 512, 128, 128, gate=True) == base + 64 * 512 * 2
+    assert bench.decode_seq_bytes(100, 64, 1, 512, 512, 128, 128) == 64 * 1024 + 100 * 2048 + 64 * 2048 + 4
+
+
+def test_err_stats_and_within():
+    ref = np.array([[0.0, 1.0], [2.0, -1.0]])
+    got = torch.tensor([[0.0, 1.002], [2.0, -1.0]])
+    s = bench.err_stats(got, ref)
+    assert abs(s["max_abs_err"] - 0.002) < 1e-6 and s["outputs_compared"] == 4 and s["finite"]
+    assert bench.within(s)                       # max 2e-3 <= 1e-2, mean 5e-4 <= 1e-3
+    assert not bench.within(bench.err_stats(torch.tensor([[0.0, 1.02], [2.0, -1.0]]), ref))
+
+
+def test_parse_config_subset():
+    a = bench.parse(["--configs", "decode_128k,ragged_paged", "--steps", "5"])
+    assert a.steps == 5 and a.configs == "decode_128k,ragged_paged" and a.impl == "ours"

@@ -194,37 +194,30 @@ def test_decode_ragged_long_and_short(cuda_device, libhca):
     check(out, ref)
 
 
-# ------------------------------------------------------------ full-size workloads (sampled)
-
-def _oracle_decode_from_raw(k, v, w, q, L, W, blk, scale):
-    kc, vc = oracle.compress(bits(k), bits(v), w.cpu().numpy(), blk)
-    kcb, vcb = oracle.round_bf16(kc), oracle.round_bf16(vc)
-    B = k.shape[0]
-    kwin = bits(k[:, L - W:L].contiguous())
-    vwin = bits(v[:, L - W:L].contiguous())
-    return oracle.decode(bits(q), kcb, vcb, kwin, vwin, np.full((B,), L, np.int32), blk, W, scale)
-
+# ------------------------------------------------------------ full-size workloads (every output)
 
 @pytest.mark.parametrize("cfg", [wl.DECODE_128K, wl.DECODE_1M], ids=lambda c: c.name)
 def test_decode_full_size_from_raw(cuda_device, libhca, cfg):
-    """Compress + decode at full size in the benchmark's launch configuration; sampled
-    sequences checked end to end against oracle compress + oracle decode."""
+    """Compress + decode at full size in the benchmark's launch configuration; every sequence,
+    head and channel checked end to end against oracle compress + oracle decode."""
     inp = wl.decode_inputs(cfg, cuda_device)
     kc, vc = hca.compress(inp["k"], inp["v"], inp["w"], cfg.blk)
     scale = 1.0 / np.sqrt(cfg.d)
     out = hca.decode(inp["q"], kc, vc, inp["kw"], inp["vw"], inp["seqlens"], cfg.blk, cfg.W, scale)
     torch.cuda.synchronize()
     hca.get_device_error()
-    picks = [0, cfg.B - 1] + ([cfg.B // 2] if cfg.B > 2 else [])
-    for b in picks:
-        ref = _oracle_decode_from_raw(inp["k"][b:b + 1], inp["v"][b:b + 1], inp["w"][b:b + 1],
-                                      inp["q"][b:b + 1], cfg.T, cfg.W, cfg.blk, scale)
-        check(out[b:b + 1], ref)
-    del inp, kc, vc
+    rk, rv = oracle.compress(bits(inp["k"]), bits(inp["v"]), inp["w"].cpu().numpy(), cfg.blk)
+    for got, ref in ((kc, rk), (vc, rv)):
+        assert np.abs(got.float().cpu().numpy() - ref).max() <= 4e-3
+    ref = oracle.decode(bits(inp["q"]), oracle.round_bf16(rk), oracle.round_bf16(rv), bits(inp["kw"]),
+                        bits(inp["vw"]), inp["seqlens"].cpu().numpy(), cfg.blk, cfg.W, scale)
+    check(out, ref)
+    del inp, kc, vc, rk, rv
     torch.cuda.empty_cache()
 
 
 def test_decode_full_size_ragged_paged(cuda_device, libhca):
+    """The ragged paged batch with QK RMSNorm and the output gate: every output."""
     cfg = wl.RAGGED_PAGED
     inp = wl.paged_decode_inputs(cfg, cuda_device)
     scale = 1.0 / np.sqrt(cfg.d)
@@ -233,15 +226,8 @@ def test_decode_full_size_ragged_paged(cuda_device, libhca):
                      gk=inp["gk"], gate=inp["gate"])
     torch.cuda.synchronize()
     hca.get_device_error()
-    seq = inp["seqlens"].cpu()
-    order = torch.argsort(seq)
-    picks = [int(order[0]), int(order[-1]), int(order[len(order) // 2]), 0, cfg.B - 1]
-    table = inp["page_table"].cpu().numpy()
-    kc_bits, vc_bits = bits(inp["kc"]), bits(inp["vc"])
-    for b in picks:
-        ref = oracle.decode(bits(inp["q"][b:b + 1]), kc_bits, vc_bits,
-                            bits(inp["kw"][b:b + 1]), bits(inp["vw"][b:b + 1]), seq[b:b + 1].numpy(),
-                            cfg.blk, cfg.W, scale, page_table=table[b:b + 1], page_size=cfg.page_size,
-                            gq=inp["gq"].cpu().numpy(), gk=inp["gk"].cpu().numpy(), eps=1e-6,
-                            gate=bits(inp["gate"][b:b + 1]))
-        check(out[b:b + 1], ref)
+    ref = oracle.decode(bits(inp["q"]), bits(inp["kc"]), bits(inp["vc"]), bits(inp["kw"]), bits(inp["vw"]),
+                        inp["seqlens"].cpu().numpy(), cfg.blk, cfg.W, scale,
+                        page_table=inp["page_table"].cpu().numpy(), page_size=cfg.page_size,
+                        gq=inp["gq"].cpu().numpy(), gk=inp["gk"].cpu().numpy(), eps=1e-6, gate=bits(inp["gate"]))
+    check(out, ref)

@@ -3,9 +3,10 @@ decode (engine plugins that must not allocate while enqueuing, servers that forb
 allocation after warm-up, hosts that only hold pre-allocated buffers).
 
 Called through the C ABI and checked against the workspace-taking hca_decode on the same
-inputs, with the decode tolerances (max abs 1e-2, mean abs 1e-3), on two calls in a row
-(the library-owned scratch keeps the first call's contents).  This file is collected
-last on purpose.
+inputs, and against the fp64 oracle, with the decode tolerances (max abs 1e-2, mean abs
+1e-3), on two calls in a row (the library-owned scratch keeps the first call's contents).
+The device's free memory must be the same before and after the two calls: the entry point
+allocates nothing.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -14,6 +15,7 @@ import pytest
 import torch
 
 import compressed_long_context_b200 as hca
+import oracle
 from compressed_long_context_b200 import _lib
 
 pytestmark = pytest.mark.gpu
@@ -70,14 +72,28 @@ def test_decode_noalloc_matches_decode(cuda_device, libhca, kind):
                      gate=c["gate"])
     torch.cuda.synchronize()
     hca.get_device_error()
-    for _ in range(2):
-        out = torch.full_like(ref, float("nan"))
+    b = oracle.bf16_bits
+    exact = oracle.decode(b(c["q"]), b(c["kc"]), b(c["vc"]), b(c["kw"]), b(c["vw"]), c["seqlens"].cpu().numpy(),
+                          128, c["W"], scale,
+                          page_table=None if c["page_table"] is None else c["page_table"].cpu().numpy(),
+                          page_size=c["page_size"], gq=None if c["gq"] is None else c["gq"].cpu().numpy(),
+                          gk=None if c["gk"] is None else c["gk"].cpu().numpy(), eps=1e-6,
+                          gate=None if c["gate"] is None else b(c["gate"]))
+    outs = [torch.full_like(ref, float("nan")) for _ in range(2)]
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    for out in outs:
         assert _noalloc(libhca, c, out, scale) == _lib.HCA_OK
         torch.cuda.synchronize()
-        hca.get_device_error()
+    free_after = torch.cuda.mem_get_info()[0]
+    hca.get_device_error()
+    assert free_after == free_before
+    for out in outs:
         err = (out - ref).abs()
         assert torch.isfinite(out).all()
         assert err.max().item() <= MAX_TOL and err.mean().item() <= MEAN_TOL
+        e64 = np.abs(out.cpu().numpy().astype(np.float64) - exact)
+        assert e64.max() <= MAX_TOL and e64.mean() <= MEAN_TOL
 
 
 def test_decode_noalloc_rejects_batches_beyond_the_scratch(cuda_device, libhca):
