@@ -15,17 +15,25 @@
 // records of each unit with a log-sum-exp and applies the optional output gate.
 //
 // Per tile, inside a CTA (warp-specialised):
-//   warp 0 (1 thread)  TMA: K and V tiles as 16 KB slabs (128 keys x 64 channels,
-//                      128-byte swizzle) into two separate rings, polled without blocking
-//                      so the K stream never waits behind V slabs that are still waiting
-//                      for their probabilities; the query rows of each piece;
+//   warp 0 (1 thread)  TMA: K and V tiles as 16 KB slabs (128 keys x 64 channels, 128-byte
+//                      swizzle) through ONE ring of 8 slots (slot s always holds channel
+//                      slab s), in a fixed order in which K runs up to A tiles ahead of V
+//                      (A = 4 S buffers, 2 with QK normalisation): K0 .. K(A-1), V0, KA,
+//                      V1, K(A+1), ...  While the first tile's softmax runs, the next tiles'
+//                      K streams at full rate into the whole ring instead of half of it;
+//                      the query rows of each piece;
 //   warp 1 (1 thread)  tcgen05.mma  S^T[128 keys x 64 heads] = K . Q^T into TMEM (and, with
 //                      QK normalisation, diag(K K^T) for the key norms);
-//   warp 6 (1 thread)  tcgen05.mma  O^T[512 ch x 64 heads] += V^T . P^T (TMEM, 4 x 128);
-//   warps 2-5          softmax: thread = key row; per-head running max with lazy
-//                      rescaling (only when a logit exceeds the max by 2^8), P^T in bf16
-//                      to shared memory; the end-of-piece epilogue writes the record.
-// Two MMA issuers keep QK^T of the next tile from queueing behind PV of this one.
+//   warp 2 (1 thread)  tcgen05.mma  O^T[512 ch x 64 heads] += V^T . P^T (TMEM, 4 x 128);
+//   warps 3-10         softmax: thread = (key row, 32 of the 64 heads), two warps per TMEM
+//                      lane quarter; per-head running max with lazy rescaling (only when a
+//                      logit exceeds the max by 2^8), P^T in bf16 to shared memory (two
+//                      buffers); each thread keeps its rows' running sums in registers, so the
+//                      sums are reduced across threads once per piece, in the epilogue that
+//                      writes the record.
+// QK normalisation and paged caches are compile-time variants: the common path carries none of
+// their code (instruction fetch, not arithmetic, bounds the softmax of a launch's first tile).
+// Two MMA issuers keep QK^T of the next tiles from queueing behind PV of this one.
 // Every mbarrier wait is bounded (see common.cuh).
 #pragma once
 
@@ -37,27 +45,32 @@ constexpr int kDecD = 512;                 // head dim (d == dv)
 constexpr int kDecSlabs = kDecD / 64;      // 64-channel slabs per key row
 constexpr int kDecTile = 128;              // keys per tile (MMA M of S^T)
 constexpr int kDecHeads = 64;              // MMA N: query heads of one KV group (padded)
-constexpr int kDecRingK = 4;               // K slab slots
-constexpr int kDecRingV = 4;               // V slab slots (even: V^T operands are slab pairs)
-constexpr int kDecPBufs = 1;               // P^T buffers
-constexpr int kDecThreads = 224;           // 7 warps
+constexpr int kDecRing = 8;                // slab slots shared by K and V: slot s = channel slab s
+constexpr int kDecLook = 4;                // S buffers: K tiles ahead of V (2 with QK normalisation)
+constexpr int kDecLookNorm = 2;
+constexpr int kDecPBufs = 2;               // P^T buffers
+constexpr int kDecThreads = 352;           // 11 warps: TMA, QK^T MMA, PV MMA, 8 softmax
+constexpr int kDecSoftWarp0 = 3;           // first softmax warp
+constexpr int kDecSoftWarps = 8;
 constexpr uint32_t kSlabBytes = 128 * 128;                 // 128 rows x 128 B
 constexpr uint32_t kDecQBytes = kDecHeads * kDecD * 2;     // 64 KB
 constexpr uint32_t kDecPBytes = kDecTile * kDecHeads * 2;  // 16 KB
 constexpr float kRescaleThreshold = 8.0f;                  // log2 units
 
 // TMEM columns
-constexpr uint32_t kTmS = 0;      // 2 x 64  S^T buffers
+constexpr uint32_t kTmS = 0;      // S^T buffers 0, 1 (64 columns each)
 constexpr uint32_t kTmO = 128;    // 4 x 64  O^T chunks (128 channels each)
-constexpr uint32_t kTmKK = 384;   // 128     K K^T (QK normalisation only)
+constexpr uint32_t kTmS2 = 384;   // S^T buffers 2, 3 -- or, with QK normalisation,
+constexpr uint32_t kTmKK = 384;   // 128     K K^T
+
+__host__ __device__ constexpr uint32_t dec_s_col(int b) { return b < 2 ? kTmS + 64u * b : kTmS2 + 64u * (b - 2); }
 
 // shared-memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t kSmQ = 0;
 constexpr uint32_t kSmP = kSmQ + kDecQBytes;
-constexpr uint32_t kSmRingK = kSmP + kDecPBufs * kDecPBytes;
-constexpr uint32_t kSmRingV = kSmRingK + kDecRingK * kSlabBytes;
-constexpr uint32_t kSmBar = kSmRingV + kDecRingV * kSlabBytes;
-constexpr int kNumBars = 2 * kDecRingK + 2 * kDecRingV + 13;
+constexpr uint32_t kSmRing = kSmP + kDecPBufs * kDecPBytes;
+constexpr uint32_t kSmBar = kSmRing + kDecRing * kSlabBytes;
+constexpr int kNumBars = 4 * kDecRing + 2 + 2 * kDecLook + 2 * kDecPBufs + 3;
 constexpr uint32_t kSmRed = (kSmBar + kNumBars * 8 + 127) & ~127u;   // float[4][64] (read as float4)
 constexpr uint32_t kSmFin = kSmRed + 4 * 64 * 4;            // float[64] reduction result
 constexpr uint32_t kSmMax = kSmFin + 64 * 4;                // float[64] running max per head
@@ -68,9 +81,8 @@ constexpr uint32_t kDecSmemBytes = kSmMisc + 64;            // the dynamic base 
 static_assert(kDecSmemBytes <= 232448, "decode shared memory exceeds the 227 KB per-block limit");
 static_assert(kSmRed % 16 == 0 && kSmFin % 16 == 0 && kSmMax % 16 == 0 && kSmAlpha % 16 == 0 &&
               kSmSum % 16 == 0 && kSmMisc % 16 == 0, "vector-accessed shared arrays must be 16-byte aligned");
-static_assert(kSmP % 1024 == 0 && kSmRingK % 1024 == 0 && kSmRingV % 1024 == 0,
-              "swizzled operand tiles must be 1024-byte aligned");
-static_assert(kDecRingV % 2 == 0, "V^T operand pairs need an even V ring");
+static_assert(kSmP % 1024 == 0 && kSmRing % 1024 == 0, "swizzled operand tiles must be 1024-byte aligned");
+static_assert(kDecRing == kDecSlabs, "one ring slot per channel slab: a tile op fills the whole ring");
 
 struct DecodeParams {
     const __nv_bfloat16* q;      // [B, Hq, 512]
@@ -140,47 +152,46 @@ __device__ __forceinline__ int block_scan_incl(int v, int* warp_tot, int* total_
     return v + pre;
 }
 
-// Named barrier among the 128 softmax threads (warps 2-5).
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier among the 256 softmax threads.
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ bool softmax_any(bool pred) {
     uint32_t r;
     asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-                 "barrier.red.or.pred q, 2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 "barrier.red.or.pred q, 2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
                  : "=r"(r) : "r"((uint32_t)pred) : "memory");
     return r != 0;
 }
 
-// Wait by all 128 softmax threads with one verdict for the group (barrier.red.and), so
-// the four warps either all go on or all unwind -- their named barriers never strand a
+// Wait by all 256 softmax threads with one verdict for the group (barrier.red.and), so
+// the eight warps either all go on or all unwind -- their named barriers never strand a
 // warp.
 __device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
     const bool ok = mbar_wait(bar, parity, abort);
     uint32_t r;
     asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-                 "barrier.red.and.pred q, 3, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 "barrier.red.and.pred q, 3, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
                  : "=r"(r) : "r"((uint32_t)ok) : "memory");
     return r != 0;
 }
 
-// Column reduction over the 128 softmax threads of a 64-vector held by every thread:
-// warp reduce-scatter with shuffles (lane l ends with heads 2l, 2l+1), then the four
-// warps meet in shared memory.  Result (all 64 heads) left in fin[] for every thread.
+// Warp reduce-scatter of a 32-vector held by every lane: lane l ends with the reduction (max
+// or sum) of element l over the 32 lanes.  31 shuffles: at each step a lane keeps one half of
+// its remaining elements and trades the other half with its partner.
 template <bool kMax>
-__device__ __forceinline__ void colreduce64(const float (&v)[64], float* red, float* fin, int q, int lane) {
-    float t[32];
+__device__ __forceinline__ float colreduce32(const float (&v)[32], int lane) {
+    float t[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < 16; ++i) {
         const bool hi = lane & 16;
-        const float send = hi ? v[i] : v[i + 32];
-        const float keep = hi ? v[i + 32] : v[i];
+        const float send = hi ? v[i] : v[i + 16];
+        const float keep = hi ? v[i + 16] : v[i];
         const float o = __shfl_xor_sync(0xffffffffu, send, 16);
         t[i] = kMax ? fmaxf(keep, o) : keep + o;
     }
-    // 32 -> 16 -> 8 -> 4 -> 2 values per lane, exchanging with lane ^ 8, ^4, ^2, ^1
 #pragma unroll
-    for (int w = 32; w >= 4; w >>= 1) {
-        const int hf = w / 2, x = w / 4;
+    for (int w = 16; w >= 2; w >>= 1) {
+        const int hf = w / 2, x = w / 2;
         const bool hi = lane & x;
 #pragma unroll
         for (int i = 0; i < hf; ++i) {
@@ -190,15 +201,7 @@ __device__ __forceinline__ void colreduce64(const float (&v)[64], float* red, fl
             t[i] = kMax ? fmaxf(keep, o) : keep + o;
         }
     }
-    red[q * 64 + 2 * lane] = t[0];
-    red[q * 64 + 2 * lane + 1] = t[1];
-    softmax_bar();
-    const int idx = q * 32 + lane;
-    if (idx < 64) {
-        float a = red[idx], b = red[64 + idx], c = red[128 + idx], d = red[192 + idx];
-        fin[idx] = kMax ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
-    }
-    softmax_bar();
+    return t[0];
 }
 
 // Byte offset of 16-byte chunk `c` of row `r` in a 128-byte-swizzled slab.
@@ -260,6 +263,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+template <bool NORM, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -272,19 +276,21 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     }
     uint8_t* sm = dsmem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSmBar);
-    uint64_t* kfull = bars;
-    uint64_t* kempty = kfull + kDecRingK;
-    uint64_t* vfull = kempty + kDecRingK;
-    uint64_t* vempty = vfull + kDecRingV;
-    uint64_t* q_full = vempty + kDecRingV;
+    // A slot's landed / consumed barriers come in a K and a V copy: each consumer then sees only
+    // its own ops, in order, so a phase-parity wait is never two phases ahead of the barrier.
+    uint64_t* full_k = bars;                       // [kDecRing] K slab landed
+    uint64_t* full_v = full_k + kDecRing;          // [kDecRing] V slab landed
+    uint64_t* empty_k = full_v + kDecRing;         // [kDecRing] K slab consumed (QK^T issued and done)
+    uint64_t* empty_v = empty_k + kDecRing;        // [kDecRing] V slab consumed (PV issued and done)
+    uint64_t* q_full = empty_v + kDecRing;
     uint64_t* q_empty = q_full + 1;
-    uint64_t* s_full = q_full + 2;    // [2]
-    uint64_t* s_empty = q_full + 4;   // [2]
-    uint64_t* p_full = q_full + 6;    // [2]
-    uint64_t* p_empty = q_full + 8;   // [2]
-    uint64_t* o_full = q_full + 10;
-    uint64_t* o_empty = q_full + 11;
-    uint64_t* q_tma = q_full + 12;    // query slabs landed (TMA)
+    uint64_t* s_full = q_full + 2;                 // [kDecLook]
+    uint64_t* s_empty = s_full + kDecLook;         // [kDecLook]
+    uint64_t* p_full = s_empty + kDecLook;         // [kDecPBufs]
+    uint64_t* p_empty = p_full + kDecPBufs;        // [kDecPBufs]
+    uint64_t* o_full = p_empty + kDecPBufs;
+    uint64_t* o_empty = o_full + 1;
+    uint64_t* q_tma = o_full + 2;                  // query slabs landed (TMA)
     float* red = reinterpret_cast<float*>(sm + kSmRed);
     float* fin = reinterpret_cast<float*>(sm + kSmFin);
     float* m_s = reinterpret_cast<float*>(sm + kSmMax);
@@ -296,33 +302,31 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     int* sched = misc + 2;          // [0] = first unit, [2..8] scan scratch
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool norm = (p.flags & HCA_QK_NORM) != 0;
-    const bool paged = (p.flags & HCA_PAGED) != 0;
+    constexpr bool norm = NORM;
+    constexpr bool paged = PAGED;
     const int U = p.B * p.Hkv;
     const int cta = blockIdx.x;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < kDecRingK; ++i) {
-            mbar_init(&kfull[i], 1);
-            mbar_init(&kempty[i], 1);
+        for (int i = 0; i < kDecRing; ++i) {
+            mbar_init(&full_k[i], 1);
+            mbar_init(&full_v[i], 1);
+            mbar_init(&empty_k[i], 1);
+            mbar_init(&empty_v[i], 1);
         }
-        for (int i = 0; i < kDecRingV; ++i) {
-            mbar_init(&vfull[i], 1);
-            mbar_init(&vempty[i], 1);
-        }
-        mbar_init(q_full, 4);
+        mbar_init(q_full, kDecSoftWarps);
         mbar_init(q_empty, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kDecLook; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 4);
+            mbar_init(&s_empty[i], kDecSoftWarps);
         }
         for (int i = 0; i < kDecPBufs; ++i) {
-            mbar_init(&p_full[i], 4);
+            mbar_init(&p_full[i], kDecSoftWarps);
             mbar_init(&p_empty[i], 1);
         }
         mbar_init(o_full, 1);
-        mbar_init(o_empty, 4);
+        mbar_init(o_empty, kDecSoftWarps);
         mbar_init(q_tma, 1);
         fence_mbar_init();
     }
@@ -459,25 +463,23 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const uint32_t tmem = *tmem_slot;
     const bool have_work = (ts < te) && u_first >= 0;
 
+    // K tiles in flight ahead of V (the S buffers the softmax has not read yet)
+    const int look = norm ? kDecLookNorm : kDecLook;
     if (have_work && warp == 0) {
         // ===================================================== TMA producer (one thread)
         if (lane == 0) {
             TileIter ki, vi;
             ki.init(&p, u_first, p_first, ts, te);
             vi.init(&p, u_first, p_first, ts, te);
-            int ks = 0, vs = 0, kdone = 0, vdone = 0, qitem = 0;
-            uint32_t kring = 0, vring = 0;
-            bool q_issued = false;
+            int kn = 0, vn = 0, qitem = 0;
+            int last = -1;      // kind of the previous op (every op fills all slots): 0 K, 1 V
             // test switch (hca_debug_set_drop_slab): the first K slab is never requested
             bool drop = *reinterpret_cast<volatile int*>(&g_debug_drop_slab) != 0;
-            uint64_t t_prog = globaltimer_ns();
-            uint32_t idle = 0;
             // Page ids of the two 64-entry halves of the current compressed K (V) tile, read
-            // from the page table once per tile, as soon as the iterator reaches the tile
-            // (its last slab's neighbour is still in flight, so the load's latency hides
-            // behind it): each read is a dependent global load in this one thread, and one
-            // per slab costs as much as streaming the tile.  A page id outside the pool is
-            // reported and clamped into it, so every load stays inside the pool.
+            // from the page table once per tile, as soon as the iterator reaches the tile (the
+            // previous op's slabs are still in flight, so the load's latency hides behind
+            // them).  A page id outside the pool is reported and clamped into it, so every
+            // load stays inside the pool.
             int kpg[2] = {0, 0}, vpg[2] = {0, 0};
             auto pages_of = [&](const TileIter& it, int* pg) {
                 if (!paged || it.done || !it.comp()) return;
@@ -493,8 +495,10 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             };
             pages_of(ki, kpg);
             pages_of(vi, vpg);
-            // One slab of the current tile of iterator `it` (K or V) into slot `dst`.
-            auto issue = [&](const TileIter& it, const int* pg, int s, bool is_v, uint8_t* dst, uint64_t* bar) {
+            // One slab of the current tile of iterator `it` (K or V) into slot `s`.
+            auto issue = [&](const TileIter& it, const int* pg, int s, bool is_v) {
+                uint8_t* dst = sm + kSmRing + s * kSlabBytes;
+                uint64_t* bar = is_v ? &full_v[s] : &full_k[s];
                 const CUtensorMap* m = it.comp() ? (is_v ? &tm_v : &tm_k) : (is_v ? &tm_vw : &tm_kw);
                 if (it.comp() && paged) {
                     const int j0 = it.tile * kDecTile;
@@ -509,63 +513,44 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 }
             };
             while (!ki.done || !vi.done) {
-                bool prog = false;
-                if (!ki.done) {
-                    if (ks == 0 && ki.first() && !q_issued) {
-                        // the piece's 64 query rows (heads g*G ..), eight 8 KB slabs
-                        if (mbar_test(q_empty, (qitem & 1) ^ 1)) {
-                            mbar_arrive_expect_tx(q_tma, kDecQBytes);
-                            for (int s = 0; s < kDecSlabs; ++s)
-                                tma_load_4d(sm + kSmQ + s * 8192, &tm_q, q_tma, 64 * s, ki.t.g * p.G, ki.t.b, 0);
-                            q_issued = true;
-                            ++qitem;
-                            prog = true;
-                        }
-                    } else {
-                        const uint32_t st = kring % kDecRingK;
-                        if (mbar_test(&kempty[st], ((kring / kDecRingK) & 1) ^ 1)) {
-                            if (!drop) issue(ki, kpg, ks, false, sm + kSmRingK + st * kSlabBytes, &kfull[st]);
-                            drop = false;
-                            ++kring;
-                            prog = true;
-                            if (++ks == kDecSlabs) {
-                                ks = 0;
-                                ki.next();
-                                pages_of(ki, kpg);
-                                ++kdone;
-                                q_issued = false;
-                            }
-                        }
-                    }
+                // K runs up to `look` tiles ahead of V, but a piece's first K waits until every
+                // V of the previous piece is out
+                const bool do_k = !ki.done && kn < vn + look && (!ki.first() || vn == kn);
+                if (do_k && ki.first()) {
+                    // the piece's 64 query rows (heads g*G ..), eight 8 KB slabs, once the
+                    // previous piece's QK^T no longer reads them
+                    if (!mbar_wait(q_empty, (qitem & 1) ^ 1, abort_flag)) break;
+                    mbar_arrive_expect_tx(q_tma, kDecQBytes);
+                    for (int s = 0; s < kDecSlabs; ++s)
+                        tma_load_4d(sm + kSmQ + s * 8192, &tm_q, q_tma, 64 * s, ki.t.g * p.G, ki.t.b, 0);
+                    ++qitem;
                 }
-                // V of a tile only once its K has started
-                if (!vi.done && (vdone < kdone || ks > 0)) {
-                    const uint32_t st = vring % kDecRingV;
-                    if (mbar_test(&vempty[st], ((vring / kDecRingV) & 1) ^ 1)) {
-                        issue(vi, vpg, vs, true, sm + kSmRingV + st * kSlabBytes, &vfull[st]);
-                        ++vring;
-                        prog = true;
-                        if (++vs == kDecSlabs) {
-                            vs = 0;
-                            vi.next();
-                            pages_of(vi, vpg);
-                            ++vdone;
-                        }
-                    }
-                }
-                if (prog) {
-                    idle = 0;
-                } else if ((++idle & 255u) != 0) {
-                    __nanosleep(32);
-                } else {
-                    if (*abort_flag) break;
-                    const uint64_t now = globaltimer_ns();
-                    if (idle == 256) t_prog = now;
-                    else if (now - t_prog > wait_limit_ns()) {
-                        *abort_flag = 1;
-                        record_error(HCA_ERR_TIMEOUT);
+                bool ok = true;
+                for (int s = 0; s < kDecSlabs; ++s) {
+                    // the slot is free once the previous op in it (every op fills all slots) has
+                    // been consumed; all ops before that one were consumed before it was issued
+                    if (last >= 0 && !mbar_wait(last ? &empty_v[s] : &empty_k[s],
+                                                (uint32_t)((last ? vn : kn) - 1) & 1u, abort_flag)) {
+                        ok = false;
                         break;
                     }
+                    if (drop) {
+                        drop = false;
+                        continue;
+                    }
+                    if (do_k) issue(ki, kpg, s, false);
+                    else issue(vi, vpg, s, true);
+                }
+                if (!ok) break;
+                last = do_k ? 0 : 1;
+                if (do_k) {
+                    ki.next();
+                    pages_of(ki, kpg);
+                    ++kn;
+                } else {
+                    vi.next();
+                    pages_of(vi, vpg);
+                    ++vn;
                 }
             }
         }
@@ -576,33 +561,33 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         const uint32_t q_base = smem_u32(sm + kSmQ);
         TileIter it;
         it.init(&p, u_first, p_first, ts, te);
-        uint32_t kring = 0;
         int n = 0;
         while (!it.done) {
-            const int sb = n & 1;
+            const int sb = n % look;
+            const uint32_t sph = (uint32_t)(n / look) & 1u;
             if (it.first() && !warp_wait(q_full, it.item & 1, abort_flag)) break;
-            if (!warp_wait(&s_empty[sb], ((n >> 1) & 1) ^ 1, abort_flag)) break;
+            if (!warp_wait(&s_empty[sb], sph ^ 1u, abort_flag)) break;
             // the K K^T accumulator has one buffer: wait until tile n-1's softmax has read it
-            if (norm && n > 0 && !warp_wait(&s_empty[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag)) break;
+            if (norm && n > 0 &&
+                !warp_wait(&s_empty[(n - 1) % look], (uint32_t)((n - 1) / look) & 1u, abort_flag))
+                break;
             tc_fence_after();
             bool ok = true;
             for (int s = 0; s < kDecSlabs; ++s) {
-                const uint32_t st = kring % kDecRingK;
-                if (!warp_wait(&kfull[st], (kring / kDecRingK) & 1, abort_flag)) { ok = false; break; }
+                if (!warp_wait(&full_k[s], (uint32_t)n & 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t k_base = smem_u32(sm + kSmRingK + st * kSlabBytes);
+                    const uint32_t k_base = smem_u32(sm + kSmRing + s * kSlabBytes);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = smem_desc_sw128(k_base + kk * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(q_base + s * 8192 + kk * 32, 16, 1024);
-                        mma_ss(tmem + kTmS + 64 * sb, ad, bd, id_s, (s | kk) ? 1u : 0u);
+                        mma_ss(tmem + dec_s_col(sb), ad, bd, id_s, (s | kk) ? 1u : 0u);
                         if (norm) mma_ss(tmem + kTmKK, ad, ad, id_kk, (s | kk) ? 1u : 0u);
                     }
-                    mma_commit(&kempty[st]);
+                    mma_commit(&empty_k[s]);
                 }
                 __syncwarp();
-                ++kring;
             }
             if (!ok) break;
             if (lane == 0) {
@@ -613,12 +598,11 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             ++n;
             it.next();
         }
-    } else if (have_work && warp == 6) {
+    } else if (have_work && warp == 2) {
         // ===================================================== PV issuer (warp waits, lane 0 issues)
         const uint32_t id_o = idesc_bf16(128, kDecHeads, 1, 1);
         TileIter it;
         it.init(&p, u_first, p_first, ts, te);
-        uint32_t vring = 0;
         int n = 0;
         while (!it.done) {
             const int b = n % kDecPBufs;
@@ -626,24 +610,25 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             if (it.first() && !warp_wait(o_empty, (it.item & 1) ^ 1, abort_flag)) break;
             tc_fence_after();
             const int nvalid = it.nvalid();
-            const bool partial = it.comp() && nvalid < kDecTile;
+            const bool partial = nvalid < kDecTile;
             const uint32_t p_base = smem_u32(sm + kSmP + b * kDecPBytes);
             bool ok = true;
             for (int c = 0; c < 4; ++c) {
-                const uint32_t st0 = vring % kDecRingV, st1 = (vring + 1) % kDecRingV;
-                if (!warp_wait(&vfull[st0], (vring / kDecRingV) & 1, abort_flag) ||
-                    !warp_wait(&vfull[st1], ((vring + 1) / kDecRingV) & 1, abort_flag)) {
+                const int st0 = 2 * c, st1 = 2 * c + 1;
+                if (!warp_wait(&full_v[st0], (uint32_t)n & 1u, abort_flag) ||
+                    !warp_wait(&full_v[st1], (uint32_t)n & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
                 if (partial) {
                     // rows >= nvalid may hold anything (caller memory past the visible
-                    // entries): zero them so 0-probability keys contribute exactly 0
+                    // entries, or ring slots not yet written): zero them so 0-probability keys
+                    // contribute exactly 0
                     const int nz = (kDecTile - nvalid) * 8;
                     for (int i = lane; i < 2 * nz; i += 32) {
                         const int sl = i / nz, k = i - sl * nz;
                         const int r = nvalid + (k >> 3);
-                        uint8_t* slab = sm + kSmRingV + (sl ? st1 : st0) * kSlabBytes;
+                        uint8_t* slab = sm + kSmRing + (sl ? st1 : st0) * kSlabBytes;
                         *reinterpret_cast<uint4*>(slab + r * 128 + (k & 7) * 16) = make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async_smem();
@@ -651,18 +636,17 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t v_base = smem_u32(sm + kSmRingV + st0 * kSlabBytes);
+                    const uint32_t v_base = smem_u32(sm + kSmRing + st0 * kSlabBytes);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint64_t ad = smem_desc_sw128(v_base + kk * 2048, kSlabBytes, 1024);
                         const uint64_t bd = smem_desc_sw128(p_base + kk * 2048, 8192, 1024);
                         mma_ss(tmem + kTmO + 64 * c, ad, bd, id_o, (it.first() && kk == 0) ? 0u : 1u);
                     }
-                    mma_commit(&vempty[st0]);
-                    mma_commit(&vempty[st1]);
+                    mma_commit(&empty_v[st0]);
+                    mma_commit(&empty_v[st1]);
                 }
                 __syncwarp();
-                vring += 2;
             }
             if (!ok) break;
             if (lane == 0) {
@@ -673,16 +657,24 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             ++n;
             it.next();
         }
-    } else if (have_work && warp >= 2 && warp <= 5) {
-        // ===================================================== softmax / epilogue (warps 2-5)
-        const int q4 = warp & 3;                 // TMEM lane quarter
+    } else if (have_work && warp >= kDecSoftWarp0) {
+        // ===================================================== softmax / epilogue (8 warps)
+        // Two warps per TMEM lane quarter; each owns 32 of the 64 heads of the quarter's 32 key
+        // rows (a thread holds one key row's 32 logits).
+        const int q4 = warp & 3;                             // TMEM lane quarter
+        const int hh = (warp - kDecSoftWarp0) >> 2;          // head half: heads 32*hh .. 32*hh + 31
+        const int h0 = 32 * hh;
         const int r = q4 * 32 + lane;            // key row within the tile / channel within a chunk
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const int sidx = threadIdx.x - 64;       // 0..127
+        const int sidx = threadIdx.x - 32 * kDecSoftWarp0;   // 0..255
         TileIter it;
         it.init(&p, u_first, p_first, ts, te);
         int n = 0;
         bool ok = true;
+        // this thread's share of the running row sums: sum over its key rows of p, per head
+        float lsum[32];
+#pragma unroll
+        for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
         while (ok && !it.done) {
             const bool first = it.first(), last = it.last();
             if (first) {
@@ -690,11 +682,12 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 // rewritten in place as q' = q / rms(q) * g_q * g_k (bf16), since
                 // q_hat . k_hat = (q' . k) / rms(k)
                 if (!group_wait(q_tma, it.item & 1, abort_flag)) { ok = false; break; }
-                if (norm) {
-                    const int h = sidx >> 1, half = sidx & 1;
+                if (NORM) {
+                    const int h = sidx >> 2, part = sidx & 3;      // 4 threads per head, 128 channels each
                     float ss = 0.f;
-                    for (int c = 0; c < 256; c += 8) {
-                        const int cc = 256 * half + c;
+#pragma unroll 1
+                    for (int c = 0; c < 128; c += 8) {
+                        const int cc = 128 * part + c;
                         const uint4 x = *reinterpret_cast<const uint4*>(sm + kSmQ + (cc >> 6) * 8192 +
                                                                       sw128(h, (cc & 63) >> 3));
                         const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
@@ -705,9 +698,11 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                         }
                     }
                     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
                     const float inv = rsqrtf(ss * (1.f / kDecD) + p.eps);
-                    for (int c = 0; c < 256; c += 8) {
-                        const int cc = 256 * half + c;
+#pragma unroll 1
+                    for (int c = 0; c < 128; c += 8) {
+                        const int cc = 128 * part + c;
                         uint4* ptr =
                             reinterpret_cast<uint4*>(sm + kSmQ + (cc >> 6) * 8192 + sw128(h, (cc & 63) >> 3));
                         const uint4 x = *ptr;
@@ -727,15 +722,15 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 if (lane == 0) mbar_arrive(q_full);
             }
 
-            const int sb = n & 1;
+            const int sb = n % look;
             const bool valid = r < it.nvalid();
-            if (!group_wait(&s_full[sb], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!group_wait(&s_full[sb], (n / look) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            float z[64];
-#pragma unroll
-            for (int c = 0; c < 64; c += 16) tmem_ld16(tmem + lane_off + kTmS + 64 * sb + c, z + c);
+            float z[32];
+            tmem_ld16(tmem + lane_off + dec_s_col(sb) + h0, z);
+            tmem_ld16(tmem + lane_off + dec_s_col(sb) + h0 + 16, z + 16);
             float kscale = p.scale_log2;
-            if (norm) {
+            if (NORM) {
                 float d[32];
                 tmem_ld16(tmem + lane_off + kTmKK + q4 * 32, d);
                 tmem_ld16(tmem + lane_off + kTmKK + q4 * 32 + 16, d + 16);
@@ -751,7 +746,7 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[sb]);
 #pragma unroll
-            for (int h = 0; h < 64; ++h) z[h] = valid ? z[h] * kscale : -INFINITY;
+            for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * kscale : -INFINITY;
 
             // ---- running max (shared m_s[64]): full reduction on the first tile of a
             // piece; afterwards only when some logit exceeds the max by 2^threshold
@@ -761,39 +756,43 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             } else {
                 bool mine = false;
 #pragma unroll
-                for (int h = 0; h < 64; h += 4) {
-                    const float4 mm = *reinterpret_cast<const float4*>(m_s + h);
+                for (int h = 0; h < 32; h += 4) {
+                    const float4 mm = *reinterpret_cast<const float4*>(m_s + h0 + h);
                     mine |= (z[h] > mm.x + kRescaleThreshold) | (z[h + 1] > mm.y + kRescaleThreshold) |
                             (z[h + 2] > mm.z + kRescaleThreshold) | (z[h + 3] > mm.w + kRescaleThreshold);
                 }
                 need = softmax_any(mine);
             }
             if (need) {
-                colreduce64<true>(z, red, fin, q4, lane);
+                const float tmax = colreduce32<true>(z, lane);    // max of head h0 + lane over this warp's rows
+                red[q4 * 64 + h0 + lane] = tmax;
+                softmax_bar();
                 if (sidx < 64) {
                     const float mo = first ? -INFINITY : m_s[sidx];
-                    const float mn = fmaxf(mo, fin[sidx]);
-                    const float al = first ? 0.f : ex2(mo - mn);
-                    al_s[sidx] = al;
+                    const float mn = fmaxf(mo, fmaxf(fmaxf(red[sidx], red[64 + sidx]), fmaxf(red[128 + sidx], red[192 + sidx])));
+                    al_s[sidx] = first ? 0.f : ex2(mo - mn);
                     m_s[sidx] = mn;
-                    l_s[sidx] = first ? 0.f : l_s[sidx] * al;
                 }
                 softmax_bar();
                 if (!first) {
-                    // rescale O^T once the previous PV has landed
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) lsum[h] *= al_s[h0 + h];
+                    // rescale O^T (this warp's 32 head columns of each chunk) once the previous
+                    // PV has landed
                     const int pb = (n - 1) % kDecPBufs;
                     if (!group_wait(&p_empty[pb], ((n - 1) / kDecPBufs) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
+#pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                        for (int c16 = 0; c16 < 64; c16 += 16) {
+#pragma unroll 1
+                        for (int c16 = 0; c16 < 32; c16 += 16) {
                             float o[16];
-                            const uint32_t ta = tmem + lane_off + kTmO + 64 * c + c16;
+                            const uint32_t ta = tmem + lane_off + kTmO + 64 * c + h0 + c16;
                             tmem_ld16(ta, o);
                             tmem_wait_ld();
                             uint32_t w[16];
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) w[j] = __float_as_uint(o[j] * al_s[c16 + j]);
+                            for (int j = 0; j < 16; ++j) w[j] = __float_as_uint(o[j] * al_s[h0 + c16 + j]);
                             tmem_st16(ta, w);
                         }
                     }
@@ -801,15 +800,19 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     tc_fence_before();
                 }
             }
-            // ---- probabilities
-            uint32_t pk[32];
+            // ---- probabilities (and this thread's row sums)
+            uint32_t pk[16];
 #pragma unroll
-            for (int h = 0; h < 64; h += 4) {
-                const float4 mm = *reinterpret_cast<const float4*>(m_s + h);
+            for (int h = 0; h < 32; h += 4) {
+                const float4 mm = *reinterpret_cast<const float4*>(m_s + h0 + h);
                 z[h] = ex2(z[h] - mm.x);
                 z[h + 1] = ex2(z[h + 1] - mm.y);
                 z[h + 2] = ex2(z[h + 2] - mm.z);
                 z[h + 3] = ex2(z[h + 3] - mm.w);
+                lsum[h] += z[h];
+                lsum[h + 1] += z[h + 1];
+                lsum[h + 2] += z[h + 2];
+                lsum[h + 3] += z[h + 3];
                 pk[h >> 1] = pack_bf16x2(z[h], z[h + 1]);
                 pk[(h >> 1) + 1] = pack_bf16x2(z[h + 2], z[h + 3]);
             }
@@ -817,28 +820,32 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             if (!group_wait(&p_empty[pbuf], ((n / kDecPBufs) & 1) ^ 1, abort_flag)) { ok = false; break; }
             uint8_t* pt = sm + kSmP + pbuf * kDecPBytes;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(pt + sw128(r, c)) =
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4*>(pt + sw128(r, 4 * hh + c)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[pbuf]);
-            // row sums of this tile (off the MMA's critical path)
-            colreduce64<false>(z, red, fin, q4, lane);
-            if (sidx < 64) l_s[sidx] += fin[sidx];
 
             if (last) {
-                // ---- end of this CTA's piece of unit u
+                // ---- end of this CTA's piece of unit u: the row sums over all key rows, then the
+                // record (running max, sum, unnormalised O^T)
                 const int u = it.u;
                 const int rec = cta + u;
+                const float tsum = colreduce32<false>(lsum, lane);
+                red[q4 * 64 + h0 + lane] = tsum;
+                softmax_bar();
                 if (sidx == 0) {
                     if (it.tb == 0) p.meta[2 * u] = cta;
                     if (it.tend == it.ntiles) p.meta[2 * u + 1] = cta;
                 }
                 if (sidx < 64) {
                     p.rec_m[(size_t)rec * 64 + sidx] = m_s[sidx];
-                    p.rec_l[(size_t)rec * 64 + sidx] = l_s[sidx];
+                    p.rec_l[(size_t)rec * 64 + sidx] = (red[sidx] + red[64 + sidx]) + (red[128 + sidx] + red[192 + sidx]);
                 }
+                softmax_bar();     // red[] is free again before the next piece's first reduction
+#pragma unroll
+                for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
                 if (!group_wait(o_full, it.item & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 float* orec = p.rec_o + (size_t)rec * 64 * kDecD;
@@ -847,13 +854,13 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
 #pragma unroll 1
-                    for (int c16 = 0; c16 < 64; c16 += 16) {
+                    for (int c16 = 0; c16 < 32; c16 += 16) {
                         float o[16];
-                        tmem_ld16(tmem + lane_off + kTmO + 64 * c + c16, o);
+                        tmem_ld16(tmem + lane_off + kTmO + 64 * c + h0 + c16, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const int h = c16 + j;
+                            const int h = h0 + c16 + j;
                             if (h < p.G) orec[(size_t)h * kDecD + 128 * c + r] = o[j];
                         }
                     }

@@ -400,10 +400,15 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     p.scale_log2 = scale * 1.4426950408889634f;
     p.eps = eps;
 
-    if (!set_smem_attr_once(reinterpret_cast<const void*>(&decode_split_kernel), (int)kDecSmemBytes, 0))
+    // compile-time variants: QK normalisation x paged cache
+    using SplitFn = void (*)(const DecodeParams, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const CUtensorMap, const CUtensorMap);
+    const SplitFn split = norm ? (paged ? decode_split_kernel<true, true> : decode_split_kernel<true, false>)
+                               : (paged ? decode_split_kernel<false, true> : decode_split_kernel<false, false>);
+    if (!set_smem_attr_once(reinterpret_cast<const void*>(split), (int)kDecSmemBytes, 4 + 2 * norm + paged))
         return HCA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    decode_split_kernel<<<nsplit, kDecThreads, kDecSmemBytes, s>>>(p, tq, tk, tv, tkw, tvw);
+    split<<<nsplit, kDecThreads, kDecSmemBytes, s>>>(p, tq, tk, tv, tkw, tvw);
     if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
