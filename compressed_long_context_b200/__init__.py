@@ -17,7 +17,7 @@ from ._lib import (HCA_OUT_F32, HCA_OUT_GATE, HCA_PAGED, HCA_QK_NORM,  # noqa: F
                    HCA_WINDOW_RING, HCA_WRITE_LSE)
 
 __all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "append", "append_state_size",
-           "vha", "get_device_error", "status_string"]
+           "vha", "gate_logits", "get_device_error", "status_string"]
 
 
 class HCAError(RuntimeError):
@@ -127,12 +127,15 @@ def decode_workspace_size(B, Hq, Hkv, dv) -> int:
 
 
 def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size=0,
-           gq=None, gk=None, eps=1e-6, gate=None, out=None, workspace=None, window_ring=False):
+           gq=None, gk=None, eps=1e-6, gate=None, out=None, workspace=None, window_ring=False,
+           vha_u=None, vha_v=None):
     """One query per sequence at position seqlens[b]-1 over its compressed cache + raw window.
 
     q [B,Hq,d] bf16; kc/vc contiguous [B,Nmax,Hkv,d|dv] or page pools [P,page_size,Hkv,d|dv]
     with page_table [B,max_pages] int32; kw/vw [B,W,Hkv,d|dv] bf16; seqlens [B] int32;
-    gq/gk [d] fp32 for QK RMSNorm; gate [B,Hq,dv] bf16 logits.  Returns out [B,Hq,dv] fp32.
+    gq/gk [d] fp32 for QK RMSNorm; gate [B,Hq,dv] bf16 logits; vha_u/vha_v [Hq,r] fp32 Virtual
+    Head Attention factors (mixing fused into the merge, hca_decode_vha).  Returns out [B,Hq,dv]
+    fp32.
     """
     _need(q, torch.bfloat16, "q")
     dev = q.device
@@ -178,6 +181,19 @@ def decode(q, kc, vc, kw, vw, seqlens, blk, W, scale, page_table=None, page_size
     if workspace is None:
         workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=dev)
     _need(workspace, torch.uint8, "workspace", dev)
+    if vha_u is not None or vha_v is not None:
+        _need(vha_u, torch.float32, "vha_u", dev)
+        _need(vha_v, torch.float32, "vha_v", dev)
+        r = vha_u.shape[1]
+        if vha_u.shape != (Hq, r) or vha_v.shape != (Hq, r):
+            raise ValueError("vha_u and vha_v must both be [Hq, r]")
+        rc = _lib.load().hca_decode_vha(_p(q), _p(kc), _p(vc), _p(page_table), int(page_size), int(max_pages),
+                                        int(num_pages), _p(kw), _p(vw), _p(seqlens), _p(gq), _p(gk), float(eps),
+                                        _p(gate), _p(vha_u), _p(vha_v), int(r), _p(out), _p(workspace),
+                                        workspace.numel(), B, Hq, Hkv, d, dv, blk, W, Nmax, float(scale), flags,
+                                        _stream(dev))
+        _check(rc, "hca_decode_vha")
+        return out
     rc = _lib.load().hca_decode(_p(q), _p(kc), _p(vc), _p(page_table), int(page_size), int(max_pages),
                                 int(num_pages), _p(kw), _p(vw), _p(seqlens), _p(gq), _p(gk), float(eps), _p(gate), _p(out),
                                 _p(workspace), workspace.numel(), B, Hq, Hkv, d, dv, blk, W, Nmax,
@@ -260,3 +276,21 @@ def vha(out, U, V):
     _check(_lib.load().hca_vha(_p(out), _p(U), _p(V), int(n), Hq, dv, r, flags, _stream(dev)), "hca_vha")
     return out
 
+
+
+def gate_logits(cq, wg, out=None):
+    """Low-Rank Gated Attention's gate projection: gate[i, h, c] = sum_k cq[i, k] wg[k, h, c].
+    cq [n, rq] bf16 query latents, wg [rq, Hq, dv] bf16.  Returns gate logits [n, Hq, dv] bf16,
+    the ``gate`` argument of ``decode``."""
+    _need(cq, torch.bfloat16, "cq")
+    _need(wg, torch.bfloat16, "wg", cq.device)
+    n, rq = cq.shape
+    if wg.dim() != 3 or wg.shape[0] != rq:
+        raise ValueError("wg must be [rq, Hq, dv] with rq = cq.shape[1]")
+    Hq, dv = wg.shape[1], wg.shape[2]
+    if out is None:
+        out = torch.empty((n, Hq, dv), dtype=torch.bfloat16, device=cq.device)
+    _need(out, torch.bfloat16, "gate", cq.device)
+    _room(out, n * Hq * dv, "gate")
+    _check(_lib.load().hca_gate_logits(_p(cq), _p(wg), _p(out), n, rq, Hq, dv, _stream(cq.device)), "hca_gate_logits")
+    return out

@@ -21,9 +21,10 @@ HCA_OUT_F32 = 16
 HCA_WINDOW_RING = 32
 
 # Names of every entry point declared in include/hca.h.
-EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_decode", "hca_decode_noalloc",
+EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_decode", "hca_decode_vha",
+           "hca_decode_noalloc",
            "hca_vha", "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error",
-           "hca_debug_set_wait_limit", "hca_debug_set_drop_slab", "hca_debug_wait_probe")
+           "hca_debug_set_wait_limit", "hca_debug_set_drop_slab", "hca_debug_wait_probe", "hca_gate_logits")
 
 _lib = None
 
@@ -56,6 +57,9 @@ def load():
     lib.hca_decode.restype = _i
     lib.hca_decode.argtypes = ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _sz]
                                + [_i] * 8 + [_f, _u, _vp])
+    lib.hca_decode_vha.restype = _i
+    lib.hca_decode_vha.argtypes = ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _vp,
+                                    _vp, _sz] + [_i] * 8 + [_f, _u, _vp])
     lib.hca_decode_noalloc.restype = _i
     lib.hca_decode_noalloc.argtypes = ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp]
                                        + [_i] * 8 + [_f, _u, _vp])
@@ -65,6 +69,8 @@ def load():
     lib.hca_append_state_size.argtypes = [_i] * 4
     lib.hca_append.restype = _i
     lib.hca_append.argtypes = [_vp] * 9 + [_i] * 3 + [_vp] + [_i] * 7 + [_u, _vp]
+    lib.hca_gate_logits.restype = _i
+    lib.hca_gate_logits.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
     lib.hca_debug_set_wait_limit.restype = _i
     lib.hca_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong, _vp]
     lib.hca_debug_set_drop_slab.restype = _i

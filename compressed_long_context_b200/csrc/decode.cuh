@@ -97,6 +97,9 @@ struct DecodeParams {
     float* rec_m;                // [R][64]  running max (log2 units)
     float* rec_l;                // [R][64]
     float* rec_o;                // [R][64][512]
+    const float* vha_u;          // [Hq, vha_r] Virtual Head Attention factors, or null
+    const float* vha_v;
+    int vha_r;
     int B, Hq, Hkv, G, blk, W, Nmax, page_size, max_pages, num_pages, flags, nsplit;
     float scale_log2, eps;
 };
@@ -883,116 +886,142 @@ decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     }
 }
 
-// Merge the partial records of each unit (log-sum-exp), normalise, apply the gate.
-// Grid (units, heads / 4), 128 threads; a thread owns 4 heads x 4 channels.  All the
-// (m, l, O) values of a chunk of records are loaded before any is used, so a merge costs
-// about two memory round trips, and the grid fits in one wave.
-constexpr int kMergeHeads = 4;
+// Merge the partial records of each unit (log-sum-exp), normalise, apply the gate, and mix the
+// heads with Virtual Head Attention when factors are given.
+//
+// Grid (units, dv / 32), 128 threads: a CTA owns all G heads of one unit for 32 channels, so
+// the cross-head VHA mixing happens on chip.  Thread = (head h = tid / 2, 16 channels).  All
+// the (m, l, O) values of a chunk of kChunk records are loaded before any is used, so a merge
+// of up to kChunk pieces costs one memory round trip after the unit's range is known.  The
+// gate logits and the VHA factors are inputs, not products of the split kernel: they are read
+// before griddepcontrol.wait, while the split kernel still runs.  The VHA variant keeps the
+// factors, the merged outputs and V^T o in dynamic shared memory (combine_vha_smem bytes).
+constexpr int kMergeCh = 32;              // channels per combine CTA
+constexpr int kDecVhaMaxRank = 32;        // fused VHA rank limit
 
-// kMergeChunk records are loaded per round: 4 when units have many pieces (few long
-// sequences), 2 otherwise -- the smaller chunk keeps registers low enough for the whole grid
-// to fit one wave.
-template <int kMergeChunk>
+__host__ __device__ constexpr uint32_t combine_vha_smem(int r) {
+    return (uint32_t)(2 * kDecHeads * r + kDecHeads * (kMergeCh + 1) + r * (kMergeCh + 1)) * 4u;
+}
+
+template <int kChunk, bool kVha>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+    extern __shared__ float cs[];
     const int u = blockIdx.x;
-    const int h0 = blockIdx.y * kMergeHeads;
-    const int c = 4 * threadIdx.x;                // channels c .. c+3
+    const int h = threadIdx.x >> 1;
+    const int c16 = 16 * (threadIdx.x & 1);
+    const int c = blockIdx.y * kMergeCh + c16;                      // channels c .. c+15
     const int b = u / p.Hkv, g = u - (u / p.Hkv) * p.Hkv;
-    // the gate logits are an input, not a product of the split kernel: each thread copies its
-    // own into shared memory before waiting for it (cp.async: no registers held), so their
-    // DRAM latency overlaps the records' loads
-    __shared__ __align__(16) uint2 gsm[kMergeHeads][128];
+    const bool live = h < p.G;
+    const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + (live ? h : 0)) * kDecD + c;
     const bool gated = (p.flags & HCA_OUT_GATE) != 0;
-    if (gated) {
-#pragma unroll
-        for (int j = 0; j < kMergeHeads; ++j)
-            if (h0 + j < p.G) {
-                const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h0 + j) * kDecD + c;
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 8;"
-                             :: "r"(smem_u32(&gsm[j][threadIdx.x])), "l"(p.gate + orow) : "memory");
-            }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+    const int R = p.vha_r;
+    float* vs = cs;                                   // [G][R]
+    float* us = vs + kDecHeads * R;                   // [G][R]
+    float* os = us + kDecHeads * R;                   // [64][33]
+    float* ts = os + kDecHeads * (kMergeCh + 1);      // [R][33]
+    uint4 graw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    if (gated && live) {
+        graw[0] = __ldg(reinterpret_cast<const uint4*>(p.gate + orow));
+        graw[1] = __ldg(reinterpret_cast<const uint4*>(p.gate + orow) + 1);
+    }
+    if (kVha) {
+        for (int i = threadIdx.x; i < p.G * R; i += 128) {
+            vs[i] = __ldg(p.vha_v + i);
+            us[i] = __ldg(p.vha_u + i);
+        }
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (*reinterpret_cast<volatile unsigned int*>(&g_error) == HCA_ERR_TIMEOUT) {
         // a split CTA gave up: its records (and the unit ranges) may be stale, so the outputs are
         // marked invalid rather than merged from whatever the workspace holds
-        for (int j = 0; j < kMergeHeads; ++j)
-            if (h0 + j < p.G) {
-                const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h0 + j) * kDecD + c;
-                *reinterpret_cast<float4*>(p.out + orow) = make_float4(NAN, NAN, NAN, NAN);
-            }
-        if (gated) asm volatile("cp.async.wait_all;" ::: "memory");
+        if (live)
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<float4*>(p.out + orow + 4 * j) = make_float4(NAN, NAN, NAN, NAN);
         return;
     }
     const int first = __ldg(p.meta + 2 * u), last = __ldg(p.meta + 2 * u + 1);
     if (first < 0 || last < first || last >= p.nsplit) {
         if (threadIdx.x == 0 && blockIdx.y == 0) record_error(HCA_ERR_DEVICE_INPUT);
-        if (gated) asm volatile("cp.async.wait_all;" ::: "memory");
         return;
     }
-    float M[kMergeHeads], L[kMergeHeads];
-    float4 acc[kMergeHeads];
+    float M = -INFINITY, L = 0.f;
+    float acc[16];
 #pragma unroll
-    for (int j = 0; j < kMergeHeads; ++j) {
-        M[j] = -INFINITY;
-        L[j] = 0.f;
-        acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int i0 = first; i0 <= last; i0 += kMergeChunk) {
-        float m[kMergeChunk][kMergeHeads], l[kMergeChunk][kMergeHeads];
-        float4 o[kMergeChunk][kMergeHeads];
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    const int hh = live ? h : 0;
+    for (int i0 = first; i0 <= last; i0 += kChunk) {
+        float m[kChunk], l[kChunk];
+        float4 o[kChunk][4];
 #pragma unroll
-        for (int k = 0; k < kMergeChunk; ++k) {
-            const bool live = i0 + k <= last;     // ranges are contiguous: every CTA in between has a piece
+        for (int k = 0; k < kChunk; ++k) {
+            const bool ok = live && i0 + k <= last;   // ranges are contiguous: every CTA in between has a piece
             const size_t rec = (size_t)(i0 + k + u);
+            m[k] = ok ? __ldcg(p.rec_m + rec * 64 + hh) : -INFINITY;
+            l[k] = ok ? __ldcg(p.rec_l + rec * 64 + hh) : 0.f;
+            const float4* op = reinterpret_cast<const float4*>(p.rec_o + (rec * 64 + hh) * kDecD + c);
 #pragma unroll
-            for (int j = 0; j < kMergeHeads; ++j) {
-                const int h = h0 + j;
-                const bool ok = live && h < p.G;
-                m[k][j] = ok ? __ldcg(p.rec_m + rec * 64 + h) : -INFINITY;
-                l[k][j] = ok ? __ldcg(p.rec_l + rec * 64 + h) : 0.f;
-                o[k][j] = ok ? __ldcg(reinterpret_cast<const float4*>(p.rec_o + (rec * 64 + h) * kDecD + c))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < 4; ++j) o[k][j] = ok ? __ldcg(op + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float Mn = M;
+#pragma unroll
+        for (int k = 0; k < kChunk; ++k) Mn = fmaxf(Mn, m[k]);
+        if (Mn == -INFINITY) continue;
+        const float sc = M == -INFINITY ? 0.f : exp2f(M - Mn);
+        L *= sc;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] *= sc;
+#pragma unroll
+        for (int k = 0; k < kChunk; ++k) {
+            const float w = m[k] == -INFINITY ? 0.f : exp2f(m[k] - Mn);
+            L = fmaf(w, l[k], L);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc[4 * j] = fmaf(w, o[k][j].x, acc[4 * j]);
+                acc[4 * j + 1] = fmaf(w, o[k][j].y, acc[4 * j + 1]);
+                acc[4 * j + 2] = fmaf(w, o[k][j].z, acc[4 * j + 2]);
+                acc[4 * j + 3] = fmaf(w, o[k][j].w, acc[4 * j + 3]);
             }
         }
+        M = Mn;
+    }
+    const float inv = 1.f / L;
+    float r[16];
 #pragma unroll
-        for (int j = 0; j < kMergeHeads; ++j) {
-            float Mn = M[j];
+    for (int j = 0; j < 16; ++j) r[j] = acc[j] * inv;
+    if (gated) {
+        const uint32_t gw[8] = {graw[0].x, graw[0].y, graw[0].z, graw[0].w, graw[1].x, graw[1].y, graw[1].z, graw[1].w};
 #pragma unroll
-            for (int k = 0; k < kMergeChunk; ++k) Mn = fmaxf(Mn, m[k][j]);
-            if (Mn == -INFINITY) continue;
-            const float sc = M[j] == -INFINITY ? 0.f : exp2f(M[j] - Mn);
-            L[j] *= sc;
-            acc[j].x *= sc; acc[j].y *= sc; acc[j].z *= sc; acc[j].w *= sc;
-#pragma unroll
-            for (int k = 0; k < kMergeChunk; ++k) {
-                const float w = m[k][j] == -INFINITY ? 0.f : exp2f(m[k][j] - Mn);
-                L[j] = fmaf(w, l[k][j], L[j]);
-                acc[j].x = fmaf(w, o[k][j].x, acc[j].x);
-                acc[j].y = fmaf(w, o[k][j].y, acc[j].y);
-                acc[j].z = fmaf(w, o[k][j].z, acc[j].z);
-                acc[j].w = fmaf(w, o[k][j].w, acc[j].w);
-            }
-            M[j] = Mn;
+        for (int j = 0; j < 8; ++j) {
+            r[2 * j] *= 1.f / (1.f + __expf(-bf16lo(gw[j])));
+            r[2 * j + 1] *= 1.f / (1.f + __expf(-bf16hi(gw[j])));
         }
     }
-    if (gated) asm volatile("cp.async.wait_all;" ::: "memory");     // this thread's own copies
+    if (kVha) {
+        // o'[:, ch] = o[:, ch] + U (V^T o[:, ch]) over the G heads of this token
+        if (live) {
 #pragma unroll
-    for (int j = 0; j < kMergeHeads; ++j) {
-        const int h = h0 + j;
-        if (h >= p.G) continue;
-        const float inv = 1.f / L[j];
-        float4 r = make_float4(acc[j].x * inv, acc[j].y * inv, acc[j].z * inv, acc[j].w * inv);
-        const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + h) * kDecD + c;
-        if (gated) {
-            const uint2 gv = gsm[j][threadIdx.x];
-            r.x *= 1.f / (1.f + __expf(-bf16lo(gv.x)));
-            r.y *= 1.f / (1.f + __expf(-bf16hi(gv.x)));
-            r.z *= 1.f / (1.f + __expf(-bf16lo(gv.y)));
-            r.w *= 1.f / (1.f + __expf(-bf16hi(gv.y)));
+            for (int j = 0; j < 16; ++j) os[h * (kMergeCh + 1) + c16 + j] = r[j];
         }
-        *reinterpret_cast<float4*>(p.out + orow) = r;
+        __syncthreads();
+        for (int i = threadIdx.x; i < R * kMergeCh; i += 128) {
+            const int k = i / kMergeCh, ch = i - k * kMergeCh;
+            float t = 0.f;
+            for (int hd = 0; hd < p.G; ++hd) t = fmaf(vs[hd * R + k], os[hd * (kMergeCh + 1) + ch], t);
+            ts[k * (kMergeCh + 1) + ch] = t;
+        }
+        __syncthreads();
+        if (live) {
+            for (int k = 0; k < R; ++k) {
+                const float uk = us[h * R + k];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) r[j] = fmaf(uk, ts[k * (kMergeCh + 1) + c16 + j], r[j]);
+            }
+        }
+    }
+    if (live) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<float4*>(p.out + orow + 4 * j) = make_float4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
     }
 }
 

@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "decode.cuh"
+#include "gate.cuh"
 #include "prefill.cuh"
 #include "prefill_pair.cuh"
 #include "vha.cuh"
@@ -328,11 +329,18 @@ size_t hca_decode_workspace_size(int B, int Hq, int Hkv, int dv) {
     return decode_ws_layout((long long)B * Hkv, ns).bytes;
 }
 
-hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int* page_table, int page_size,
-                        int max_pages, int num_pages, const void* kw, const void* vw, const int* seqlens,
-                        const float* gq, const float* gk, float eps, const void* gate, float* out,
-                        void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int d, int dv, int blk, int W,
-                        int Nmax, float scale, unsigned flags, hca_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// hca_decode and hca_decode_vha: the split kernel, then the combine kernel (merge, gate and,
+// with factors, Virtual Head Attention).
+hca_status_t decode_impl(const void* q, const void* kc, const void* vc, const int* page_table, int page_size,
+                         int max_pages, int num_pages, const void* kw, const void* vw, const int* seqlens,
+                         const float* gq, const float* gk, float eps, const void* gate, float* out,
+                         void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int d, int dv, int blk, int W,
+                         int Nmax, float scale, unsigned flags, const float* vha_u, const float* vha_v, int vha_r,
+                         hca_stream_t stream) {
     using namespace hca;
     if (B < 0 || Hq < 1 || Hkv < 1 || blk < 1 || W < 1) return HCA_ERR_INVALID_ARG;
     if (flags & ~(unsigned)(HCA_QK_NORM | HCA_OUT_GATE | HCA_PAGED | HCA_WINDOW_RING)) return HCA_ERR_UNSUPPORTED;
@@ -356,7 +364,14 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     }
     if (norm && (!gq || !gk || (reinterpret_cast<uintptr_t>(gq) & 3) || (reinterpret_cast<uintptr_t>(gk) & 3)))
         return HCA_ERR_INVALID_ARG;
-    if (gated && (!gate || !aligned16(gate))) return HCA_ERR_INVALID_ARG;   // read 8 bytes per thread
+    if (gated && (!gate || !aligned16(gate))) return HCA_ERR_INVALID_ARG;   // read 16 bytes per thread
+    if (vha_u || vha_v) {
+        if (!vha_u || !vha_v || vha_r < 1 || (reinterpret_cast<uintptr_t>(vha_u) & 3) ||
+            (reinterpret_cast<uintptr_t>(vha_v) & 3))
+            return HCA_ERR_INVALID_ARG;
+        // the mixing spans all Hq heads of a token: one KV group must hold them all
+        if (Hkv != 1 || vha_r > kDecVhaMaxRank) return HCA_ERR_UNSUPPORTED;
+    }
     const int nsplit = num_sms();
     if (nsplit <= 0) return HCA_ERR_CUDA;
     const long long U = (long long)B * Hkv;
@@ -394,6 +409,9 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     p.rec_m = reinterpret_cast<float*>(ws + lay.m_off);
     p.rec_l = reinterpret_cast<float*>(ws + lay.l_off);
     p.rec_o = reinterpret_cast<float*>(ws + lay.o_off);
+    p.vha_u = vha_u;
+    p.vha_v = vha_v;
+    p.vha_r = vha_u ? vha_r : 0;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.blk = blk; p.W = W; p.Nmax = paged ? 0 : Nmax;
     p.page_size = paged ? page_size : 0; p.max_pages = paged ? max_pages : 0; p.num_pages = paged ? num_pages : 0;
     p.flags = (int)flags; p.nsplit = nsplit;
@@ -412,23 +430,57 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int
     if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)U, (unsigned)((p.G + kMergeHeads - 1) / kMergeHeads));
-    cfg.blockDim = dim3(kDecD / 4);
-    cfg.dynamicSmemBytes = 0;
+    cfg.gridDim = dim3((unsigned)U, (unsigned)(kDecD / kMergeCh));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = p.vha_u ? combine_vha_smem(p.vha_r) : 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // many pieces per unit (nsplit >= 3 U): load 4 records per round, else 2
-    const cudaError_t e = (long long)nsplit >= 3 * U ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<4>, p)
-                                                      : cudaLaunchKernelEx(&cfg, decode_combine_kernel<2>, p);
+    // records loaded per round, from the average number of pieces per unit (about nsplit / U)
+    const int chunk = (long long)nsplit >= 6 * U ? 8 : ((long long)nsplit >= 3 * U ? 4 : 2);
+    cudaError_t e;
+    if (p.vha_u)
+        e = chunk == 8 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<8, true>, p)
+            : chunk == 4 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<4, true>, p)
+                         : cudaLaunchKernelEx(&cfg, decode_combine_kernel<2, true>, p);
+    else
+        e = chunk == 8 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<8, false>, p)
+            : chunk == 4 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<4, false>, p)
+                         : cudaLaunchKernelEx(&cfg, decode_combine_kernel<2, false>, p);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return HCA_ERR_CUDA;
     }
     return HCA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+hca_status_t hca_decode(const void* q, const void* kc, const void* vc, const int* page_table, int page_size,
+                        int max_pages, int num_pages, const void* kw, const void* vw, const int* seqlens,
+                        const float* gq, const float* gk, float eps, const void* gate, float* out,
+                        void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int d, int dv, int blk, int W,
+                        int Nmax, float scale, unsigned flags, hca_stream_t stream) {
+    return decode_impl(q, kc, vc, page_table, page_size, max_pages, num_pages, kw, vw, seqlens, gq, gk, eps, gate,
+                       out, workspace, ws_bytes, B, Hq, Hkv, d, dv, blk, W, Nmax, scale, flags, nullptr, nullptr, 0,
+                       stream);
+}
+
+hca_status_t hca_decode_vha(const void* q, const void* kc, const void* vc, const int* page_table, int page_size,
+                            int max_pages, int num_pages, const void* kw, const void* vw, const int* seqlens,
+                            const float* gq, const float* gk, float eps, const void* gate, const float* vha_u,
+                            const float* vha_v, int vha_rank, float* out, void* workspace, size_t ws_bytes, int B,
+                            int Hq, int Hkv, int d, int dv, int blk, int W, int Nmax, float scale, unsigned flags,
+                            hca_stream_t stream) {
+    if (!vha_u || !vha_v) return HCA_ERR_INVALID_ARG;
+    return decode_impl(q, kc, vc, page_table, page_size, max_pages, num_pages, kw, vw, seqlens, gq, gk, eps, gate,
+                       out, workspace, ws_bytes, B, Hq, Hkv, d, dv, blk, W, Nmax, scale, flags, vha_u, vha_v,
+                       vha_rank, stream);
 }
 
 }  // extern "C"
@@ -615,4 +667,34 @@ extern "C" hca_status_t hca_decode_noalloc(const void* q, const void* kc, const 
     return hca_decode(q, kc, vc, page_table, page_size, max_pages, num_pages, kw, vw, seqlens, gq, gk, eps, gate,
                       out, ws, (size_t)HCA_DECODE_NOALLOC_MAX_BYTES, B, Hq, Hkv, d, dv, blk, W, Nmax, scale, flags,
                       stream);
+}
+
+// ---------------------------------------------------------------------------------------
+// hca_gate_logits: the low-rank gate projection (gate.cuh).
+extern "C" hca_status_t hca_gate_logits(const void* cq, const void* wg, void* gate, int n, int rq, int Hq, int dv,
+                                        hca_stream_t stream) {
+    if (n < 0 || rq < 1 || Hq < 1 || dv < 1) return HCA_ERR_INVALID_ARG;
+    const long long J = (long long)Hq * dv;
+    if (rq % 64 || J % hca::kGateN || J > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
+    if (n == 0) return HCA_OK;
+    if (!cq || !wg || !gate || !aligned16(cq) || !aligned16(wg) || !aligned16(gate)) return HCA_ERR_INVALID_ARG;
+    CUtensorMap ta, tb;
+    // cq [n][rq]: boxes of 64 latent values x 128 rows (rows past n read as zero)
+    if (!hca::make_tmap_4d(&ta, cq, (uint64_t)rq, (uint64_t)n, 1, 1, (uint64_t)rq, (uint64_t)rq * n, (uint64_t)rq * n,
+                           64, 128, 1, 1))
+        return HCA_ERR_CUDA;
+    // Wg [rq][J]: boxes of 64 output columns x 64 latent rows
+    if (!hca::make_tmap_4d(&tb, wg, (uint64_t)J, (uint64_t)rq, 1, 1, (uint64_t)J, (uint64_t)J * rq, (uint64_t)J * rq, 64,
+                           64, 1, 1))
+        return HCA_ERR_CUDA;
+    if (!hca::set_smem_attr_once(reinterpret_cast<const void*>(&hca::gate_logits_kernel), (int)hca::kGateSmem, 0))
+        return HCA_ERR_CUDA;
+    hca::GateParams p;
+    p.out = static_cast<__nv_bfloat16*>(gate);
+    p.n = n;
+    p.rq = rq;
+    p.J = (int)J;
+    const dim3 grid((unsigned)(J / hca::kGateN), (unsigned)((n + 127) / 128));
+    hca::gate_logits_kernel<<<grid, hca::kGateThreads, hca::kGateSmem, reinterpret_cast<cudaStream_t>(stream)>>>(p, ta, tb);
+    return launch_status();
 }

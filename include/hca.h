@@ -153,6 +153,27 @@ hca_status_t hca_decode(const void* q, const void* kc, const void* vc,
                         float scale, unsigned flags, hca_stream_t stream);
 
 /*
+ * hca_decode_vha -- hca_decode with Virtual Head Attention fused into its combine pass
+ * (official blog, section 2.1, and the Zhidx article, section "1. Latent-Gated Sparse
+ * Attention": a lightweight cross-head low-rank mixing with an identity skip, applied after the
+ * attention).  The output is that of hca_decode (with the gate, when HCA_OUT_GATE is set) mixed
+ * per sequence and channel over the Hq heads: out[b, :, c] <- (I + U V^T) out[b, :, c].
+ *   vha_u, vha_v  [Hq, vha_rank] fp32 mixing factors (4-byte aligned), 1 <= vha_rank <= 32
+ * The merge kernel already holds every head of a sequence on chip, so the mixing costs no extra
+ * pass over the output (hca_vha on an hca_decode output gives the same result).  Other
+ * arguments, layouts and errors: as hca_decode; Hkv must be 1 (one KV group holds all heads),
+ * else HCA_ERR_UNSUPPORTED.
+ */
+hca_status_t hca_decode_vha(const void* q, const void* kc, const void* vc,
+                            const int* page_table, int page_size, int max_pages, int num_pages,
+                            const void* kw, const void* vw, const int* seqlens,
+                            const float* gq, const float* gk, float eps,
+                            const void* gate, const float* vha_u, const float* vha_v, int vha_rank,
+                            float* out, void* workspace, size_t ws_bytes,
+                            int B, int Hq, int Hkv, int d, int dv, int blk, int W, int Nmax,
+                            float scale, unsigned flags, hca_stream_t stream);
+
+/*
  * hca_decode_noalloc -- hca_decode without a workspace argument.  There is no counterpart
  * in the paper: this entry point exists for callers that cannot allocate device memory
  * when they decode -- an inference-engine plugin that must not allocate inside its
@@ -240,6 +261,21 @@ hca_status_t hca_append(const void* k_new, const void* v_new, const float* w_new
                         const int* page_table, int page_size, int max_pages, int num_pages,
                         void* state, int B, int Hkv, int d, int dv, int blk, int W, int Nmax,
                         unsigned flags, hca_stream_t stream);
+
+/*
+ * hca_gate_logits -- the gate projection of Low-Rank Gated Attention (Zhidx article, section
+ * "1. Latent-Gated Sparse Attention": the output gate is computed from the attention layer's
+ * query latent, a quarter of the hidden size, so the projection has 75% fewer weights than one
+ * from the hidden state):  gate[i, h, c] = sum_k cq[i, k] * wg[k, h, c].
+ *   cq    [n, rq] bf16       query latents of n tokens (decode: one per sequence)
+ *   wg    [rq, Hq, dv] bf16  gate projection weights
+ *   gate  [n, Hq, dv] bf16   output logits (fp32 accumulation, one rounding); pass them to
+ *                            hca_decode / hca_decode_vha with HCA_OUT_GATE
+ * Supported: rq a multiple of 64, Hq * dv a multiple of 256.  Tensor-core GEMM, bound by reading
+ * wg once (64 MB at rq = 1024, Hq = 64, dv = 512).  Errors as for the other entry points.
+ */
+hca_status_t hca_gate_logits(const void* cq, const void* wg, void* gate, int n, int rq, int Hq, int dv,
+                             hca_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* hca_status_string(hca_status_t status);

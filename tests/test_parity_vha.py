@@ -138,3 +138,68 @@ def test_vha_odd_shapes(cuda_device, libhca, n, Hq, dv, r, f32):
         assert np.abs(got - ref).max() <= 1e-4
     else:
         assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
+
+
+def _decode_case(dev, seed, lengths, Hq=64, W=128, blk=128, paged_ps=0, norm=False, gate=True):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    B = len(lengths)
+    Nmax = max(1, max(oracle.visible_entries(L - 1, W, blk) for L in lengths))
+    r = lambda *s: torch.randn(s, generator=g, device=dev).to(torch.bfloat16)  # noqa: E731
+    c = dict(q=r(B, Hq, 512), kw=r(B, W, 1, 512), vw=r(B, W, 1, 512),
+             seqlens=torch.tensor(lengths, dtype=torch.int32, device=dev), gate=r(B, Hq, 512) if gate else None,
+             gq=None, gk=None, page_table=None, page_size=0, W=W, blk=blk)
+    if paged_ps:
+        npg = (Nmax + paged_ps - 1) // paged_ps
+        c["kc"], c["vc"] = r(B * npg, paged_ps, 1, 512), r(B * npg, paged_ps, 1, 512)
+        perm = torch.randperm(B * npg, generator=torch.Generator().manual_seed(seed)).to(torch.int32)
+        c["page_table"], c["page_size"] = perm.view(B, npg).to(dev), paged_ps
+    else:
+        c["kc"], c["vc"] = r(B, Nmax, 1, 512), r(B, Nmax, 1, 512)
+    if norm:
+        c["gq"] = torch.rand((512,), generator=g, device=dev) + 0.5
+        c["gk"] = torch.rand((512,), generator=g, device=dev) + 0.5
+    return c
+
+
+def _oracle_decode(c, scale):
+    n = lambda t: None if t is None else t.cpu().numpy()  # noqa: E731
+    return oracle.decode(bits(c["q"]), bits(c["kc"]), bits(c["vc"]), bits(c["kw"]), bits(c["vw"]),
+                         c["seqlens"].cpu().numpy(), c["blk"], c["W"], scale, page_table=n(c["page_table"]),
+                         page_size=c["page_size"], gq=n(c["gq"]), gk=n(c["gk"]), eps=1e-6,
+                         gate=None if c["gate"] is None else bits(c["gate"]))
+
+
+@pytest.mark.parametrize("r,lengths,gate,paged,norm", [
+    (1, [9000, 130, 20000, 700], True, 0, False),
+    (8, [131072, 5000, 1, 129, 70000], True, 0, False),
+    (32, [4096 + 17, 300, 12345], True, 64, True),
+    (5, [3000] * 40, False, 0, False),            # odd rank, no gate, many sequences (one piece each)
+    (8, [1048576], True, 0, False),               # one long sequence: many pieces merged
+])
+def test_decode_vha_fused(cuda_device, libhca, r, lengths, gate, paged, norm):
+    """Decode with the gate and Virtual Head Attention fused into the merge, against the oracle's
+    gated decode followed by the oracle's mixing; and against the unfused hca_decode + hca_vha."""
+    dev = cuda_device
+    W = 256 if paged else 128
+    c = _decode_case(dev, 120 + r + len(lengths), lengths, W=W, paged_ps=paged, norm=norm, gate=gate)
+    U, V = factors(dev, 64, r, 130 + r)
+    scale = 1.0 / np.sqrt(512)
+    kw = dict(page_table=c["page_table"], page_size=c["page_size"], gq=c["gq"], gk=c["gk"], gate=c["gate"])
+    fused = hca.decode(c["q"], c["kc"], c["vc"], c["kw"], c["vw"], c["seqlens"], c["blk"], W, scale,
+                       vha_u=U, vha_v=V, **kw)
+    plain = hca.decode(c["q"], c["kc"], c["vc"], c["kw"], c["vw"], c["seqlens"], c["blk"], W, scale, **kw)
+    hca.vha(plain, U, V)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    check(fused, oracle.vha(_oracle_decode(c, scale), U.cpu().numpy(), V.cpu().numpy()))
+    # same arithmetic up to the order of a few fp32 sums
+    assert (fused - plain).abs().max().item() <= 1e-5
+
+
+def test_decode_vha_rejects_grouped_heads(cuda_device, libhca):
+    c = _decode_case(cuda_device, 140, [3000, 700], Hq=64)
+    U, V = factors(cuda_device, 64, 4, 141)
+    kv2 = c["kc"].repeat(1, 1, 2, 1).contiguous()
+    with pytest.raises(hca.HCAError):
+        hca.decode(c["q"], kv2, kv2, c["kw"].repeat(1, 1, 2, 1).contiguous(), c["vw"].repeat(1, 1, 2, 1).contiguous(),
+                   c["seqlens"], 128, 128, 0.05, vha_u=U, vha_v=V)
