@@ -489,6 +489,42 @@ def bench_decode_128k(c):
     res["serving_step"] = serve_part
     del state, kc_s, vc_s, kw_s, vw_s
 
+    # ---- the gated layer's extras on the same batch: the low-rank gate projection (query latent
+    # 1024 -> 64 x 512 logits; 64 MB of weights read once) and the decode with the gate and
+    # Virtual Head Attention (rank 8) fused into its merge
+    gg = torch.Generator(device=c.dev).manual_seed(6)
+    cq = torch.randn((B, 1024), generator=gg, device=c.dev).to(torch.bfloat16)
+    wg = (torch.randn((1024, cfg.Hq, cfg.dv), generator=gg, device=c.dev) / 32.0).to(torch.bfloat16)
+    gate = torch.empty((B, cfg.Hq, cfg.dv), dtype=torch.bfloat16, device=c.dev)
+    vu = torch.randn((cfg.Hq, 8), generator=gg, device=c.dev) * 0.1
+    vv = torch.randn((cfg.Hq, 8), generator=gg, device=c.dev) * 0.1
+
+    def gate_proj():
+        hca.gate_logits(cq, wg, out=gate)
+
+    def dec_gated_vha():
+        hca.decode(q, kc, vc, kw, vw, seq, cfg.blk, cfg.W, scale, gate=gate, vha_u=vu, vha_v=vv, out=out,
+                   workspace=ws)
+
+    for _ in range(3):
+        gate_proj()
+        dec_gated_vha()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    g_ms = timed_calls(gate_proj, c.args.steps, c.stream, c.sampler, flush=c.flush)
+    v_ms = timed_calls(dec_gated_vha, c.args.steps, c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    t_g, t_v = c.mean_s(g_ms), c.mean_s(v_ms)
+    gbytes = (cq.numel() + wg.numel() + gate.numel()) * 2
+    vbytes = dbytes + B * cfg.Hq * cfg.dv * 2
+    res["gated_layer"] = {
+        "gate_projection": {"us": t_g * 1e6, "algorithmic_bytes": gbytes,
+                            "roofline": c.hbm_roof("gate_logits_kernel", gbytes, t_g)},
+        "decode_gate_vha_fused": {"us": t_v * 1e6, "rank": 8, "queries_per_s": B / t_v, "algorithmic_bytes": vbytes,
+                                  "roofline": c.hbm_roof("decode_split_kernel + decode_combine_kernel<.., vha>",
+                                                         vbytes, t_v)}}
+    del cq, wg, gate, vu, vv
+
     # ---- parity of the benchmarked decode (and compress) against the oracle, every output
     dec()
     torch.cuda.synchronize()
