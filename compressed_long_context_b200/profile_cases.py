@@ -4,6 +4,9 @@
     python -m compressed_long_context_b200.profile_cases decode   [--reps N]
     python -m compressed_long_context_b200.profile_cases prefill  [--reps N]
     python -m compressed_long_context_b200.profile_cases paged    [--reps N]
+    python -m compressed_long_context_b200.profile_cases vha      [--reps N]
+    python -m compressed_long_context_b200.profile_cases append   [--reps N]
+    python -m compressed_long_context_b200.profile_cases gate     [--reps N]
 
 Each case keeps its working set larger than the 126 MB L2 (so DRAM counters mean
 something) but a few GB at most, and launches the kernel `--reps` times after one
@@ -16,7 +19,8 @@ import math
 
 import torch
 
-from . import compress, decode, decode_workspace_size, get_device_error, prefill
+from . import (append, append_state_size, compress, decode, decode_workspace_size, gate_logits, get_device_error,
+               prefill, vha)
 from . import workloads as wl
 
 
@@ -81,6 +85,36 @@ def run(case: str, reps: int, B_override: int = 0, L_override: int = 0, T_overri
         keys = sum(max(0, (t - cfg.W + 1) // 128) + min(cfg.W, t + 1) for t in range(cfg.T))
         nbytes = None
         flops = 2.0 * cfg.Hq * keys * (cfg.d + cfg.dv)
+    elif case == "vha":
+        # 8192 tokens x 64 heads x 512 bf16 (512 MB, mixed in place), rank 8
+        n, Hq, d = 8192, 64, 512
+        x = torch.randn((n, Hq, d), generator=g, device=dev).to(torch.bfloat16)
+        U = torch.randn((Hq, 8), generator=g, device=dev) * 0.1
+        V = torch.randn((Hq, 8), generator=g, device=dev) * 0.1
+        fn = lambda: vha(x, U, V)  # noqa: E731
+        nbytes = 2 * x.numel() * 2
+    elif case == "append":
+        # 64 sequences of 131072 tokens appending their newest token (each completes a block)
+        B, L, d, W = 64, 131072, 512, 128
+        kn = torch.randn((B, 1, d), generator=g, device=dev).to(torch.bfloat16)
+        vn = torch.randn((B, 1, d), generator=g, device=dev).to(torch.bfloat16)
+        wn = torch.randn((B,), generator=g, device=dev)
+        seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+        kw = torch.zeros((B, W, 1, d), dtype=torch.bfloat16, device=dev)
+        vw = torch.zeros_like(kw)
+        kc = torch.zeros((B, L // 128, 1, d), dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        state = torch.zeros(append_state_size(B, 1, d, d), dtype=torch.uint8, device=dev)
+        fn = lambda: append(kn, vn, wn, seq, kw, vw, kc, vc, state, 128)  # noqa: E731
+        nbytes = B * (4 * d * 2 + 2 * (4 + 2 * d) * 4) + B * 8
+    elif case == "gate":
+        # the low-rank gate projection: 64 latents of 1024 -> 64 x 512 logits (64 MB of weights)
+        B, rq, Hq, d = 64, 1024, 64, 512
+        cq = torch.randn((B, rq), generator=g, device=dev).to(torch.bfloat16)
+        wg = (torch.randn((rq, Hq, d), generator=g, device=dev) / 32.0).to(torch.bfloat16)
+        gate = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+        fn = lambda: gate_logits(cq, wg, out=gate)  # noqa: E731
+        nbytes = (cq.numel() + wg.numel() + gate.numel()) * 2
     else:
         raise ValueError(case)
     _last_fn[0] = fn
@@ -133,7 +167,7 @@ def run_flushed(args) -> dict:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["compress", "decode", "paged", "prefill"])
+    ap.add_argument("case", choices=["compress", "decode", "paged", "prefill", "vha", "append", "gate"])
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--B", type=int, default=0, help="decode batch (default 64)")
     ap.add_argument("--L", type=int, default=0, help="decode context length (default 131072)")
