@@ -900,7 +900,7 @@ constexpr int kMergeCh = 32;              // channels per combine CTA
 constexpr int kDecVhaMaxRank = 32;        // fused VHA rank limit
 
 __host__ __device__ constexpr uint32_t combine_vha_smem(int r) {
-    return (uint32_t)(2 * kDecHeads * r + kDecHeads * (kMergeCh + 1) + r * (kMergeCh + 1)) * 4u;
+    return (uint32_t)(2 * kDecHeads * r + kDecHeads * kMergeCh + r * kMergeCh) * 4u;
 }
 
 template <int kChunk, bool kVha>
@@ -915,10 +915,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     const size_t orow = ((size_t)b * p.Hq + (size_t)g * p.G + (live ? h : 0)) * kDecD + c;
     const bool gated = (p.flags & HCA_OUT_GATE) != 0;
     const int R = p.vha_r;
-    float* vs = cs;                                   // [G][R]
+    float* os = cs;                                   // [64][32] merged, gated outputs (16-byte rows)
+    float* ts = os + kDecHeads * kMergeCh;            // [R][32]  V^T o
+    float* vs = ts + R * kMergeCh;                    // [G][R]
     float* us = vs + kDecHeads * R;                   // [G][R]
-    float* os = us + kDecHeads * R;                   // [64][33]
-    float* ts = os + kDecHeads * (kMergeCh + 1);      // [R][33]
     uint4 graw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
     if (gated && live) {
         graw[0] = __ldg(reinterpret_cast<const uint4*>(p.gate + orow));
@@ -992,29 +992,51 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
         const uint32_t gw[8] = {graw[0].x, graw[0].y, graw[0].z, graw[0].w, graw[1].x, graw[1].y, graw[1].z, graw[1].w};
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            r[2 * j] *= 1.f / (1.f + __expf(-bf16lo(gw[j])));
-            r[2 * j + 1] *= 1.f / (1.f + __expf(-bf16hi(gw[j])));
+            r[2 * j] *= __frcp_rn(1.f + __expf(-bf16lo(gw[j])));
+            r[2 * j + 1] *= __frcp_rn(1.f + __expf(-bf16hi(gw[j])));
         }
     }
     if (kVha) {
-        // o'[:, ch] = o[:, ch] + U (V^T o[:, ch]) over the G heads of this token
+        // o'[:, ch] = o[:, ch] + U (V^T o[:, ch]) over the G heads of this token.  Thread i of
+        // the V^T o step owns rank k = i / 8 and channels 4 (i % 8) .. +3: a warp reads one 128-byte
+        // row of os per head (broadcast to its four ranks) and four V values (broadcast).
         if (live) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) os[h * (kMergeCh + 1) + c16 + j] = r[j];
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<float4*>(os + h * kMergeCh + c16 + 4 * j) =
+                    make_float4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        } else if (h < kDecHeads) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<float4*>(os + h * kMergeCh + c16 + 4 * j) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         __syncthreads();
-        for (int i = threadIdx.x; i < R * kMergeCh; i += 128) {
-            const int k = i / kMergeCh, ch = i - k * kMergeCh;
-            float t = 0.f;
-            for (int hd = 0; hd < p.G; ++hd) t = fmaf(vs[hd * R + k], os[hd * (kMergeCh + 1) + ch], t);
-            ts[k * (kMergeCh + 1) + ch] = t;
+        for (int i = threadIdx.x; i < R * (kMergeCh / 4); i += 128) {
+            const int k = i >> 3, c4 = (i & 7) * 4;
+            float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int hd = 0; hd < p.G; ++hd) {
+                const float vk = vs[hd * R + k];
+                const float4 o4 = *reinterpret_cast<const float4*>(os + hd * kMergeCh + c4);
+                t.x = fmaf(vk, o4.x, t.x);
+                t.y = fmaf(vk, o4.y, t.y);
+                t.z = fmaf(vk, o4.z, t.z);
+                t.w = fmaf(vk, o4.w, t.w);
+            }
+            *reinterpret_cast<float4*>(ts + k * kMergeCh + c4) = t;
         }
         __syncthreads();
         if (live) {
             for (int k = 0; k < R; ++k) {
                 const float uk = us[h * R + k];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) r[j] = fmaf(uk, ts[k * (kMergeCh + 1) + c16 + j], r[j]);
+                for (int j = 0; j < 4; ++j) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(ts + k * kMergeCh + c16 + 4 * j);
+                    r[4 * j] = fmaf(uk, t4.x, r[4 * j]);
+                    r[4 * j + 1] = fmaf(uk, t4.y, r[4 * j + 1]);
+                    r[4 * j + 2] = fmaf(uk, t4.z, r[4 * j + 2]);
+                    r[4 * j + 3] = fmaf(uk, t4.w, r[4 * j + 3]);
+                }
             }
         }
     }
