@@ -17,7 +17,7 @@ from ._lib import (HCA_OUT_F32, HCA_OUT_GATE, HCA_PAGED, HCA_QK_NORM,  # noqa: F
                    HCA_WINDOW_RING, HCA_WRITE_LSE)
 
 __all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "append", "append_state_size",
-           "vha", "gate_logits", "get_device_error", "status_string"]
+           "vha", "gate_logits", "prefill_backward", "get_device_error", "status_string"]
 
 
 class HCAError(RuntimeError):
@@ -119,6 +119,44 @@ def prefill(q, k, v, kc, vc, blk, W, scale, out=None, want_lse=False, out_f32=Fa
                                  blk, W, float(scale), flags, _stream(q.device))
     _check(rc, "hca_prefill")
     return (out, lse) if want_lse else out
+
+
+def prefill_backward(q, k, v, w, kc, vc, out, lse, dout, blk, W, scale, want_dw=True):
+    """Gradients of sum(dout * out) for the layer (compress + prefill): dq [B,T,Hq,d],
+    dk [B,T,Hkv,d], dv [B,T,Hkv,dv] (window path plus pooling path) and dw [B,T] (None if
+    not wanted), all fp32.  ``out`` (bf16 or fp32) and ``lse`` [B,Hq,T] are the forward's
+    (prefill with want_lse=True); kc, vc the compressed cache it read."""
+    _need(q, torch.bfloat16, "q")
+    for name, t in (("k", k), ("v", v), ("kc", kc), ("vc", vc), ("dout", dout)):
+        _need(t, torch.bfloat16, name, q.device)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be bf16 or fp32")
+    _need(out, out.dtype, "out", q.device)
+    _need(lse, torch.float32, "lse", q.device)
+    if w is not None:
+        _need(w, torch.float32, "w", q.device)
+    B, T, Hq, d = q.shape
+    Hkv, dv = k.shape[2], v.shape[3]
+    Nc = T // blk if blk > 0 else 0
+    for name, t, n in (("k", k, B * T * Hkv * d), ("v", v, B * T * Hkv * dv), ("kc", kc, B * Nc * Hkv * d),
+                       ("vc", vc, B * Nc * Hkv * dv), ("out", out, B * T * Hq * dv), ("lse", lse, B * Hq * T),
+                       ("dout", dout, B * T * Hq * dv), ("w", w, B * T)):
+        _room(t, n, name)
+    dq = torch.empty((B, T, Hq, d), dtype=torch.float32, device=q.device)
+    dk = torch.empty((B, T, Hkv, d), dtype=torch.float32, device=q.device)
+    dvv = torch.empty((B, T, Hkv, dv), dtype=torch.float32, device=q.device)
+    dw = torch.empty((B, T), dtype=torch.float32, device=q.device) if want_dw else None
+    lib = _lib.load()
+    nbytes = int(lib.hca_prefill_backward_workspace_size(B, T, Hq, Hkv, dv, blk))
+    if nbytes == 0:
+        raise HCAError(_lib.HCA_ERR_UNSUPPORTED, "hca_prefill_backward_workspace_size")
+    ws = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
+    flags = HCA_OUT_F32 if out.dtype == torch.float32 else 0
+    rc = lib.hca_prefill_backward(_p(q), _p(k), _p(v), _p(w), _p(kc), _p(vc), _p(out), _p(lse), _p(dout), _p(dq),
+                                  _p(dk), _p(dvv), _p(dw), _p(ws), nbytes, B, T, Hq, Hkv, d, dv, blk, W,
+                                  float(scale), flags, _stream(q.device))
+    _check(rc, "hca_prefill_backward")
+    return dq, dk, dvv, dw
 
 
 def decode_workspace_size(B, Hq, Hkv, dv) -> int:

@@ -106,6 +106,25 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
+// Wait for a phase at exit, ignoring the abort flag: copies and MMAs already issued still
+// complete, and the CTA must not release its shared memory or tensor memory before they do.
+// Bounded by the same wall-clock limit.
+__device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > wait_limit_ns()) {
+            record_error(HCA_ERR_TIMEOUT);
+            return;
+        }
+}
+
+// Wait until the last of `issued` loads, issued round-robin into a ring of `ring` slots with
+// one full barrier each, has landed in every slot.
+__device__ __forceinline__ void mbar_drain_ring(uint64_t* full, uint32_t issued, uint32_t ring) {
+    for (uint32_t st = 0; st < ring; ++st)
+        if (issued > st) mbar_drain_wait(&full[st], ((issued - 1 - st) / ring) & 1);
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "append.cuh"
+#include "backward.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "decode.cuh"
@@ -80,9 +81,9 @@ bool make_tmap_4d_plain(CUtensorMap* m, void* base, int esize, uint64_t d0, uint
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel slot, device).
 bool set_smem_attr_once(const void* fn, int bytes, int slot) {
     static std::mutex mu;
-    static bool done[8][64] = {};
+    static bool done[16][64] = {};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 8) return false;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 16) return false;
     std::lock_guard<std::mutex> g(mu);
     if (done[slot][dev]) return true;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
@@ -696,5 +697,122 @@ extern "C" hca_status_t hca_gate_logits(const void* cq, const void* wg, void* ga
     p.J = (int)J;
     const dim3 grid((unsigned)(J / hca::kGateN), (unsigned)((n + 127) / 128));
     hca::gate_logits_kernel<<<grid, hca::kGateThreads, hca::kGateSmem, reinterpret_cast<cudaStream_t>(stream)>>>(p, ta, tb);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------------------------
+// hca_prefill_backward: the layer's gradients (backward.cuh).
+namespace {
+
+size_t bwd_align(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct BwdLayout {
+    size_t drow, dkc, dvc, total;
+};
+
+BwdLayout bwd_layout(long long B, long long T, long long Hq, long long Hkv, long long blk) {
+    BwdLayout l;
+    const long long Nc = T / blk;
+    l.drow = 0;
+    l.dkc = bwd_align((size_t)(B * T * Hq) * 4);
+    l.dvc = l.dkc + bwd_align((size_t)(B * Nc * Hkv * hca::kBwdD) * 4);
+    l.total = l.dvc + bwd_align((size_t)(B * Nc * Hkv * hca::kBwdD) * 4);
+    return l;
+}
+
+}  // namespace
+
+extern "C" size_t hca_prefill_backward_workspace_size(int B, int T, int Hq, int Hkv, int dv, int blk) {
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || dv != hca::kBwdD || blk < 1) return 0;
+    return bwd_layout(B, T, Hq, Hkv, blk).total;
+}
+
+extern "C" hca_status_t hca_prefill_backward(const void* q, const void* k, const void* v, const float* w,
+                                             const void* kc, const void* vc, const void* out, const float* lse,
+                                             const void* dout, float* dq, float* dk, float* dv, float* dw,
+                                             void* workspace, size_t workspace_bytes, int B, int T, int Hq, int Hkv,
+                                             int d, int dv_dim, int blk, int W, float scale, unsigned flags,
+                                             hca_stream_t stream) {
+    using namespace hca;
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || blk < 1 || W < 1) return HCA_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)HCA_OUT_F32) return HCA_ERR_UNSUPPORTED;
+    if (d != kBwdD || dv_dim != kBwdD || blk > 128 || Hq % Hkv) return HCA_ERR_UNSUPPORTED;
+    const int G = Hq / Hkv;
+    if (G > 128 || (G & (G - 1))) return HCA_ERR_UNSUPPORTED;
+    if (!(scale == scale)) return HCA_ERR_INVALID_ARG;
+    if ((long long)B * T == 0) return HCA_OK;
+    const int Nc = T / blk;
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace || (Nc > 0 && (!kc || !vc)))
+        return HCA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || (Nc > 0 && (!aligned16(kc) || !aligned16(vc))) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3) || (w && (reinterpret_cast<uintptr_t>(w) & 3)) ||
+        (dw && (reinterpret_cast<uintptr_t>(dw) & 3)) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return HCA_ERR_INVALID_ARG;
+    const BwdLayout lay = bwd_layout(B, T, Hq, Hkv, blk);
+    if (workspace_bytes < lay.total) return HCA_ERR_INVALID_ARG;
+    const int ns = num_sms();
+    if (ns <= 0) return HCA_ERR_CUDA;
+
+    BwdParams p;
+    char* ws = static_cast<char*>(workspace);
+    p.lse = lse;
+    p.drow = reinterpret_cast<float*>(ws + lay.drow);
+    p.out = out;
+    p.dout = static_cast<const __nv_bfloat16*>(dout);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.w = w;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dkc = reinterpret_cast<float*>(ws + lay.dkc);
+    p.dvc = reinterpret_cast<float*>(ws + lay.dvc);
+    p.dw = dw;
+    p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.tpt = 128 / G; p.blk = blk; p.W = W; p.Nc = Nc;
+    p.ntile_t = (T + p.tpt - 1) / p.tpt;
+    p.out_f32 = (flags & HCA_OUT_F32) ? 1 : 0;
+    p.dq_items = (long long)B * Hkv * p.ntile_t;
+    p.nkc = (Nc + 127) / 128;
+    p.nkw = (T + 127) / 128;
+    // query row tiles a raw key tile reaches: tokens k0 .. k0 + 127 + W - 1
+    const long long span_w = (std::min<long long>((long long)T, 128LL + W - 1) + p.tpt - 1) / p.tpt + 1;
+    const long long visits = (long long)B * Hkv * ((long long)p.nkc * p.ntile_t + (long long)p.nkw * span_w);
+    const long long chunk = std::max<long long>(1, (visits + 4LL * ns - 1) / (4LL * ns));
+    p.rt_chunk = (int)std::min<long long>(chunk, p.ntile_t);
+    p.chc = (p.ntile_t + p.rt_chunk - 1) / p.rt_chunk;
+    p.chw = (int)((span_w + p.rt_chunk - 1) / p.rt_chunk);
+    p.kv_items = (long long)B * Hkv * ((long long)p.nkc * p.chc + (long long)p.nkw * p.chw);
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    const uint64_t D = kBwdD;
+    CUtensorMap tq, tdo, tk, tv, tkc, tvc;
+    bool ok = true;
+    ok &= make_tmap_4d(&tq, q, D, Hq, T, B, D, D * Hq, D * Hq * T, 64, G, p.tpt, 1);
+    ok &= make_tmap_4d(&tdo, dout, D, Hq, T, B, D, D * Hq, D * Hq * T, 64, G, p.tpt, 1);
+    ok &= make_tmap_4d(&tk, k, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, 128, 1);
+    ok &= make_tmap_4d(&tv, v, D, Hkv, T, B, D, D * Hkv, D * Hkv * T, 64, 1, 128, 1);
+    if (Nc > 0) {
+        ok &= make_tmap_4d(&tkc, kc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, 128, 1);
+        ok &= make_tmap_4d(&tvc, vc, D, Hkv, Nc, B, D, D * Hkv, D * Hkv * Nc, 64, 1, 128, 1);
+    } else {   // never read: no entry exists when T < blk
+        tkc = tk;
+        tvc = tv;
+    }
+    if (!ok) return HCA_ERR_CUDA;
+    if (!set_smem_attr_once(reinterpret_cast<const void*>(&bwd_dq_kernel), (int)kBwdSmem, 8) ||
+        !set_smem_attr_once(reinterpret_cast<const void*>(&bwd_dkv_kernel), (int)kBwdSmem, 9))
+        return HCA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long rows = (long long)B * T * Hq;
+    const long long pre_grid = std::min<long long>((rows + 7) / 8, 8LL * ns);
+    bwd_pre_kernel<<<(unsigned)pre_grid, 256, 0, s>>>(p);
+    bwd_dq_kernel<<<(unsigned)std::min<long long>(p.dq_items, ns), kBwdThreads, kBwdSmem, s>>>(p, tq, tdo, tk, tv, tkc,
+                                                                                               tvc);
+    if (p.kv_items > 0)
+        bwd_dkv_kernel<<<(unsigned)std::min<long long>(p.kv_items, ns), kBwdThreads, kBwdSmem, s>>>(p, tq, tdo, tk, tv,
+                                                                                                    tkc, tvc);
+    if (Nc > 0) bwd_pool_kernel<<<(unsigned)((long long)B * Nc), kPoolThreads, 0, s>>>(p);
     return launch_status();
 }

@@ -110,6 +110,43 @@ hca_status_t hca_prefill(const void* q, const void* k, const void* v,
                          float scale, unsigned flags, hca_stream_t stream);
 
 /*
+ * hca_prefill_backward_workspace_size -- bytes of device workspace hca_prefill_backward
+ * needs (per-row softmax terms and the entries' gradients).  Returns 0 for invalid sizes.
+ */
+size_t hca_prefill_backward_workspace_size(int B, int T, int Hq, int Hkv, int dv, int blk);
+
+/*
+ * hca_prefill_backward -- gradients of the HCA layer for training: the gradient of
+ * sum(dout * out) with respect to q, the raw k and v (through the window and through the
+ * pooling of official blog section 2.1) and the pooling weights w.  The forward is
+ * hca_compress followed by hca_prefill; the stored bf16 cache is taken as it is (its
+ * rounding has no gradient).
+ *   q, k, v, w, kc, vc  the forward's inputs and compressed cache, as for hca_compress
+ *                       and hca_prefill (w may be NULL: mean pooling)
+ *   out  [B,T,Hq,dv]    the forward's output, bf16 or fp32 with HCA_OUT_F32
+ *   lse  [B,Hq,T] fp32  the forward's log-sum-exp (hca_prefill with HCA_WRITE_LSE)
+ *   dout [B,T,Hq,dv]    bf16 incoming gradient
+ *   dq   [B,T,Hq,d]     fp32 output
+ *   dk   [B,T,Hkv,d]    fp32 output (window path + pooling path; rows of a trailing
+ *   dv   [B,T,Hkv,dv]   fp32 output  partial block get only the window path)
+ *   dw   [B,T]          fp32 output, or NULL to skip (rows of a trailing partial block: 0)
+ *   workspace           device memory of at least hca_prefill_backward_workspace_size
+ *                       bytes, 256-byte aligned; its contents are overwritten
+ * Supported: d == dv == 512; Hq % Hkv == 0 with Hq / Hkv a power of two <= 128;
+ * 1 <= blk <= 128; W >= 1; flags 0 or HCA_OUT_F32.
+ * Arithmetic: bf16 operands on the tensor cores with fp32 accumulation; the softmax
+ * gradient dS = P * (dP - rowsum(dout * out)) is rounded once to bf16 before the dq and
+ * dk contractions, P once before the dv contraction; dk and dv are accumulated with fp32
+ * atomics, so their low bits depend on the order of the additions.
+ */
+hca_status_t hca_prefill_backward(const void* q, const void* k, const void* v, const float* w,
+                                  const void* kc, const void* vc, const void* out, const float* lse,
+                                  const void* dout, float* dq, float* dk, float* dv, float* dw,
+                                  void* workspace, size_t workspace_bytes,
+                                  int B, int T, int Hq, int Hkv, int d, int dv_dim, int blk, int W,
+                                  float scale, unsigned flags, hca_stream_t stream);
+
+/*
  * hca_decode_workspace_size -- bytes of device workspace hca_decode needs for a batch
  * of B sequences on the CURRENT device (split-KV partial results).  Returns 0 for
  * invalid sizes.

@@ -174,6 +174,37 @@ def test_vha_rejects_before_launch(libhca):
     assert libhca.hca_vha(None, None, None, 0, 64, 512, 4, 0, None) == _lib.HCA_OK          # nothing to do
 
 
+def test_prefill_backward_rejects_before_launch(libhca):
+    p = ctypes.c_void_p(256)
+    big = 1 << 30
+
+    def call(q=p, k=p, v=p, w=None, kc=p, vc=p, out=p, lse=p, dout=p, dq=p, dk=p, dv=p, dw=None, ws=p,
+             ws_bytes=big, B=1, T=256, Hq=64, Hkv=1, d=512, dvd=512, blk=128, W=128, scale=0.05, flags=0):
+        return libhca.hca_prefill_backward(q, k, v, w, kc, vc, out, lse, dout, dq, dk, dv, dw, ws, ws_bytes,
+                                           B, T, Hq, Hkv, d, dvd, blk, W, scale, flags, None)
+
+    # workspace: per-row terms plus the entries' fp32 gradients, 256-byte aligned pieces
+    assert libhca.hca_prefill_backward_workspace_size(1, 1024, 64, 1, 512, 128) == 1024 * 64 * 4 + 2 * 8 * 512 * 4
+    assert libhca.hca_prefill_backward_workspace_size(1, 1024, 64, 1, 64, 128) == 0
+    assert libhca.hca_prefill_backward_workspace_size(-1, 1024, 64, 1, 512, 128) == 0
+    # unsupported head dims, block, group size, flags
+    assert call(d=64, dvd=64) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(blk=129) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(Hq=6, Hkv=2) == _lib.HCA_ERR_UNSUPPORTED
+    assert call(flags=_lib.HCA_WRITE_LSE) == _lib.HCA_ERR_UNSUPPORTED
+    # null or misaligned pointers, bad sizes, NaN scale, a workspace too small or misaligned
+    assert call(lse=None) == _lib.HCA_ERR_INVALID_ARG
+    assert call(dout=None) == _lib.HCA_ERR_INVALID_ARG
+    assert call(dq=ctypes.c_void_p(264)) == _lib.HCA_ERR_INVALID_ARG
+    assert call(dw=ctypes.c_void_p(258)) == _lib.HCA_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(272)) == _lib.HCA_ERR_INVALID_ARG
+    assert call(ws_bytes=1024) == _lib.HCA_ERR_INVALID_ARG
+    assert call(W=0) == _lib.HCA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == _lib.HCA_ERR_INVALID_ARG
+    # nothing to do: no launch, OK
+    assert call(q=None, k=None, v=None, kc=None, vc=None, out=None, lse=None, dout=None, dq=None, dk=None,
+                dv=None, ws=None, B=0) == _lib.HCA_OK
+
 
 def test_header_compiles_as_c_and_links(tmp_path, libhca):
     """include/hca.h is a plain C header: a C99 translation unit that includes it and takes the
