@@ -23,7 +23,7 @@
 //                    added with fp32 atomics into the entries' gradients (workspace) or the raw
 //                    window keys' gradients.
 //   bwd_pool_kernel  one CTA per (sequence, block): pooling backward into dk, dv and dw.
-// Operands stream through one ring of four 32 KB slots (an A slab and a B slab of 128 rows x 64
+// Operands stream through one ring of six 32 KB slots (an A slab and a B slab of 128 rows x 64
 // channels each); the MMA issuer consumes the ops in the producer's order.  Every wait is
 // bounded (common.cuh).
 #pragma once
@@ -34,12 +34,12 @@ namespace hca {
 
 constexpr int kBwdD = 512;
 constexpr int kBwdThreads = 192;            // producer, MMA issuer, 4 softmax / epilogue warps
-constexpr int kBwdRing = 4;
+constexpr int kBwdRing = 6;
 constexpr uint32_t kBwdSlab = 16384;         // 128 rows x 64 channels bf16, 128-byte swizzle
 constexpr uint32_t kBwdSlot = 2 * kBwdSlab;  // A slab + B slab
 constexpr uint32_t kBwdSmRing = 0;
 constexpr uint32_t kBwdSmX = kBwdSmRing + kBwdRing * kBwdSlot;      // dS (or P^T / dS^T): 2 slabs
-constexpr uint32_t kBwdSmCol = kBwdSmX + 2 * kBwdSlab;              // per-column data (dkv): 4 x 128 words
+constexpr uint32_t kBwdSmCol = kBwdSmX + 2 * kBwdSlab;              // per-column data (dkv): 128 x float4
 constexpr uint32_t kBwdSmBar = kBwdSmCol + 4 * 128 * 4;
 constexpr int kBwdNumBars = 2 * kBwdRing + 8;
 constexpr uint32_t kBwdSmMisc = kBwdSmBar + kBwdNumBars * 8;
@@ -168,10 +168,20 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 
 // -------------------------------------------------------------------------------- dq
 
-// Ops of one key tile j of a dq pass: 8 x (Q slab, K slab) for S, 8 x (dO slab, V slab) for dP,
-// then the pass's four K slabs (channels 256 h ..) alone, as the N = 256 B operand of dq += dS K.
-// 20 ops: a multiple of the ring size, so the four K slabs always sit in slots 0..3.
-constexpr int kDqOps = 20;
+// Ops of one key tile of a dq pass: 8 x (Q slab, K slab) for S, 8 x (dO slab, V slab) for dP,
+// then two ops that each carry two of the pass's four K channel blocks (channels 256 h + 128 d
+// and + 64, in the slot's A and B halves): the N = 128 B operands of dq[:, 128 d ..] += dS K.
+constexpr int kDqPairs = 16;
+constexpr int kDqOps = kDqPairs + 2;
+
+// Softmax-gradient columns c0 .. c0 + 15 of row r, packed to bf16, into the K-major 128-byte-
+// swizzled operand buffer (two slabs of 64 columns).
+__device__ __forceinline__ void bwd_put16(uint8_t* xs, int r, int c0, const uint32_t* pk) {
+    uint8_t* dst = xs + (c0 >> 6) * kBwdSlab;
+    const uint32_t ch = (uint32_t)(c0 & 63) >> 3;
+    *reinterpret_cast<uint4*>(dst + bwd_sw(r, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4*>(dst + bwd_sw(r, ch + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -245,16 +255,17 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
                                 break;
                             }
                             uint8_t* base = sm + kBwdSmRing + st * kBwdSlot;
-                            if (o < 16) {
+                            mbar_arrive_expect_tx(&full[st], kBwdSlot);
+                            if (o < kDqPairs) {
                                 const int s = o & 7;
-                                mbar_arrive_expect_tx(&full[st], kBwdSlot);
                                 tma_load_4d(base, o < 8 ? &tm_q : &tm_do, &full[st], 64 * s, g * p.G, it.t0, b);
                                 tma_load_4d(base + kBwdSlab, o < 8 ? (comp ? &tm_kc : &tm_k) : (comp ? &tm_vc : &tm_v),
                                             &full[st], 64 * s, g, row, b);
                             } else {
-                                mbar_arrive_expect_tx(&full[st], kBwdSlab);
-                                tma_load_4d(base + kBwdSlab, comp ? &tm_kc : &tm_k, &full[st], 256 * h + 64 * (o - 16), g,
-                                            row, b);
+                                const int c = 256 * h + 128 * (o - kDqPairs);
+                                const CUtensorMap* km = comp ? &tm_kc : &tm_k;
+                                tma_load_4d(base, km, &full[st], c, g, row, b);
+                                tma_load_4d(base + kBwdSlab, km, &full[st], c + 64, g, row, b);
                             }
                         }
                     }
@@ -264,7 +275,7 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_q = idesc_bf16(128, 256, 0, 1);
+        const uint32_t id_q = idesc_bf16(128, 128, 0, 1);
         const uint32_t ring = smem_u32(sm + kBwdSmRing), xs = smem_u32(sm + kBwdSmX);
         uint32_t op = 0, nkt = 0, npass = 0;
         bool ok = true;
@@ -278,7 +289,7 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
                     // S and dP of the previous key tile have been read by the softmax warps
                     if (!warp_wait(sdp_empty, (nkt & 1) ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    for (int o = 0; o < 16; ++o, ++op) {
+                    for (int o = 0; o < kDqPairs; ++o, ++op) {
                         const uint32_t st = op % kBwdRing;
                         if (!warp_wait(&full[st], (op / kBwdRing) & 1, abort_flag)) { ok = false; break; }
                         tc_fence_after();
@@ -300,22 +311,30 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
                     // key tile, once the previous pass's accumulator has been read out)
                     if (j == 0 && !warp_wait(acc_empty, (npass & 1) ^ 1, abort_flag)) { ok = false; break; }
                     if (!warp_wait(ds_full, nkt & 1, abort_flag)) { ok = false; break; }
-                    for (int o = 0; o < 4; ++o)
-                        if (!warp_wait(&full[(op + o) % kBwdRing], ((op + o) / kBwdRing) & 1, abort_flag)) ok = false;
-                    if (!ok) break;
+                    if (!warp_wait(&full[op % kBwdRing], (op / kBwdRing) & 1, abort_flag) ||
+                        !warp_wait(&full[(op + 1) % kBwdRing], ((op + 1) / kBwdRing) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t kb = ring + (op % kBwdRing) * kBwdSlot + kBwdSlab;   // slot 0's B slab
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_ss(tmem + kBwdTmAcc, smem_desc_sw128(xs + (kk >> 2) * kBwdSlab + (kk & 3) * 32, 16, 1024),
-                                   smem_desc_sw128(kb + kk * 2048, kBwdSlot, 1024), id_q, (j | kk) ? 1u : 0u);
-                        for (int o = 0; o < 4; ++o) mma_commit(&empty[(op + o) % kBwdRing]);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t ad = smem_desc_sw128(xs + (kk >> 2) * kBwdSlab + (kk & 3) * 32, 16, 1024);
+#pragma unroll
+                            for (int d = 0; d < 2; ++d)
+                                mma_ss(tmem + kBwdTmAcc + 128 * d, ad,
+                                       smem_desc_sw128(ring + ((op + d) % kBwdRing) * kBwdSlot + kk * 2048, kBwdSlab,
+                                                       1024),
+                                       id_q, (j | kk) ? 1u : 0u);
+                        }
+                        mma_commit(&empty[op % kBwdRing]);
+                        mma_commit(&empty[(op + 1) % kBwdRing]);
                         mma_commit(ds_empty);
                         if (j == nt - 1) mma_commit(acc_full);
                     }
                     __syncwarp();
-                    op += 4;
+                    op += 2;
                 }
             }
         }
@@ -330,6 +349,7 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        uint8_t* xsp = sm + kBwdSmX;
         uint32_t nkt = 0, npass = 0;
         bool ok = true;
         for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride) {
@@ -347,6 +367,8 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
             for (int h = 0; ok && h < 2; ++h, ++npass) {
                 for (int j = 0; ok && j < nt; ++j, ++nkt) {
                     if (!bwd_group_wait(sdp_full, nkt & 1, abort_flag)) { ok = false; break; }
+                    // the previous key tile's dS has been consumed
+                    if (!bwd_group_wait(ds_empty, (nkt & 1) ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     int lo, hi;   // valid columns of this row in the tile
                     if (j < it.nct) {
@@ -358,33 +380,29 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
                         hi = min(128, t - u0 + 1);
                     }
                     if (!live) hi = lo;
-                    uint32_t pk[64];
-#pragma unroll
+#pragma unroll 1
                     for (int c0 = 0; c0 < 128; c0 += 16) {
                         float sv[16], dpv[16];
                         tmem_ld16(tmem + lane_off + kBwdTmS + c0, sv);
                         tmem_ld16(tmem + lane_off + kBwdTmP + c0, dpv);
                         tmem_wait_ld();
+                        uint32_t pk[8];
 #pragma unroll
                         for (int e = 0; e < 16; e += 2) {
                             const int c = c0 + e;
                             const float p0 = (c >= lo && c < hi) ? ex2(fmaf(sv[e], p.scale_log2, -lse2)) : 0.f;
                             const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2(fmaf(sv[e + 1], p.scale_log2, -lse2)) : 0.f;
-                            pk[(c0 + e) >> 1] = pack_bf16x2(p0 * (dpv[e] - Dr), p1 * (dpv[e + 1] - Dr));
+                            pk[e >> 1] = pack_bf16x2(p0 * (dpv[e] - Dr), p1 * (dpv[e + 1] - Dr));
                         }
+                        bwd_put16(xsp, r, c0, pk);
                     }
                     tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(sdp_empty);
-                    // dS (bf16, K-major: keys along the row) into the operand buffer
-                    if (!bwd_group_wait(ds_empty, (nkt & 1) ^ 1, abort_flag)) { ok = false; break; }
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        *reinterpret_cast<uint4*>(sm + kBwdSmX + (c >> 3) * kBwdSlab + bwd_sw(r, c & 7)) =
-                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(ds_full);
+                    if (lane == 0) {
+                        mbar_arrive(sdp_empty);
+                        mbar_arrive(ds_full);
+                    }
                 }
                 if (!ok) break;
                 // ---- the pass's dq half: scale * accumulator -> dq[b, t, head, 256 h ..]
@@ -465,10 +483,29 @@ __device__ __forceinline__ bool bwd_keys(const BwdParams& p, long long i, BwdKey
     return kk.rt_lo < kk.rt_hi && kk.nk > 0;
 }
 
+// Per query row (column of S^T) of row tile rt: its log2-domain LSE, D, and the key rows of the
+// tile it sees, [rlo, rhi) relative to k0 (empty for rows past the sequence end).
+__device__ __forceinline__ float4 bwd_col(const BwdParams& p, const BwdKeys& kk, int rt, int c) {
+    const int tok = rt * p.tpt + c / p.G;
+    if (tok >= p.T) return make_float4(0.f, 0.f, __int_as_float(0), __int_as_float(0));
+    const int head = kk.g * p.G + c % p.G;
+    const float l2 = __ldg(p.lse + ((size_t)kk.b * p.Hq + head) * p.T + tok) * 1.4426950408889634f;
+    const float D = __ldg(p.drow + ((size_t)kk.b * p.T + tok) * p.Hq + head);
+    int rlo, rhi;
+    if (kk.comp) {
+        rlo = 0;
+        rhi = bwd_visible(tok, p.W, p.blk) - kk.k0;
+    } else {
+        rlo = tok - p.W + 1 - kk.k0;
+        rhi = tok - kk.k0 + 1;
+    }
+    return make_float4(l2, D, __int_as_float(rlo), __int_as_float(rhi));
+}
+
 // Ops of one query row tile in pass ps (0, 1: dV halves; 2, 3: dK halves): 8 x (K slab, Q slab)
-// for S^T; for dK, 8 x (V slab, dO slab) for dP^T; then the half's four dO (dV) or Q (dK) slabs
-// alone as the N = 256 B operand.  12 or 20 ops: multiples of the ring size.
-__device__ __forceinline__ int bwd_kv_ops(int ps) { return ps < 2 ? 12 : 20; }
+// for S^T; for dK, 8 x (V slab, dO slab) for dP^T; then two ops carrying the half's four dO (dV)
+// or Q (dK) channel blocks, two per op, as the N = 128 B operands of the accumulation.
+__device__ __forceinline__ int bwd_kv_pairs(int ps) { return ps < 2 ? 8 : 16; }
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -489,9 +526,7 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
     uint64_t* acc_full = sdp_full + 4;
     uint64_t* acc_empty = sdp_full + 5;
     uint64_t* drain = sdp_full + 6;
-    float* col_lse = reinterpret_cast<float*>(sm + kBwdSmCol);     // [128] per query row (column)
-    float* col_d = col_lse + 128;                                    // [128]
-    int* col_t = reinterpret_cast<int*>(col_d + 128);                // [128] token (-1: no row)
+    float4* colv = reinterpret_cast<float4*>(sm + kBwdSmCol);      // [128] per query row (column)
     int* misc = reinterpret_cast<int*>(sm + kBwdSmMisc);
     volatile int* abort_flag = misc;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
@@ -528,27 +563,26 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
                 for (int ps = 0; ok && ps < 4; ++ps)
                     for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt) {
                         const int t0 = rt * p.tpt;
-                        const int nops = bwd_kv_ops(ps);
-                        for (int o = 0; o < nops; ++o, ++op) {
+                        const int pairs = bwd_kv_pairs(ps);
+                        for (int o = 0; o < pairs + 2; ++o, ++op) {
                             const uint32_t st = op % kBwdRing;
                             if (!mbar_wait(&empty[st], ((op / kBwdRing) & 1) ^ 1, abort_flag)) {
                                 ok = false;
                                 break;
                             }
                             uint8_t* base = sm + kBwdSmRing + st * kBwdSlot;
-                            const int pair_ops = nops - 4;
-                            if (o < pair_ops) {
+                            mbar_arrive_expect_tx(&full[st], kBwdSlot);
+                            if (o < pairs) {
                                 const int s = o & 7;
                                 const bool sk = o < 8;        // S^T: (K, Q); dP^T: (V, dO)
-                                mbar_arrive_expect_tx(&full[st], kBwdSlot);
                                 tma_load_4d(base, sk ? (kk.comp ? &tm_kc : &tm_k) : (kk.comp ? &tm_vc : &tm_v), &full[st],
                                             64 * s, kk.g, kk.k0, kk.b);
                                 tma_load_4d(base + kBwdSlab, sk ? &tm_q : &tm_do, &full[st], 64 * s, kk.g * p.G, t0, kk.b);
                             } else {
-                                const int half = ps & 1;
-                                mbar_arrive_expect_tx(&full[st], kBwdSlab);
-                                tma_load_4d(base + kBwdSlab, ps < 2 ? &tm_do : &tm_q, &full[st],
-                                            256 * half + 64 * (o - pair_ops), kk.g * p.G, t0, kk.b);
+                                const int c = 256 * (ps & 1) + 128 * (o - pairs);
+                                const CUtensorMap* m = ps < 2 ? &tm_do : &tm_q;
+                                tma_load_4d(base, m, &full[st], c, kk.g * p.G, t0, kk.b);
+                                tma_load_4d(base + kBwdSlab, m, &full[st], c + 64, kk.g * p.G, t0, kk.b);
                             }
                         }
                     }
@@ -557,7 +591,7 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
         }
     } else if (warp == 1) {
         const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_a = idesc_bf16(128, 256, 0, 1);
+        const uint32_t id_a = idesc_bf16(128, 128, 0, 1);
         const uint32_t ring = smem_u32(sm + kBwdSmRing), xs = smem_u32(sm + kBwdSmX);
         uint32_t op = 0, nrt = 0, npass = 0;
         bool ok = true;
@@ -565,11 +599,11 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
             BwdKeys kk;
             if (!bwd_keys(p, i, kk)) continue;
             for (int ps = 0; ok && ps < 4; ++ps, ++npass) {
-                const int nops = bwd_kv_ops(ps), pair_ops = nops - 4;
+                const int pairs = bwd_kv_pairs(ps);
                 for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt, ++nrt) {
                     if (!warp_wait(sdp_empty, (nrt & 1) ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    for (int o = 0; o < pair_ops; ++o, ++op) {
+                    for (int o = 0; o < pairs; ++o, ++op) {
                         const uint32_t st = op % kBwdRing;
                         if (!warp_wait(&full[st], (op / kBwdRing) & 1, abort_flag)) { ok = false; break; }
                         tc_fence_after();
@@ -590,22 +624,29 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
                     const bool first_rt = rt == kk.rt_lo;
                     if (first_rt && !warp_wait(acc_empty, (npass & 1) ^ 1, abort_flag)) { ok = false; break; }
                     if (!warp_wait(x_full, nrt & 1, abort_flag)) { ok = false; break; }
-                    for (int o = 0; o < 4; ++o)
-                        if (!warp_wait(&full[(op + o) % kBwdRing], ((op + o) / kBwdRing) & 1, abort_flag)) ok = false;
-                    if (!ok) break;
+                    if (!warp_wait(&full[op % kBwdRing], (op / kBwdRing) & 1, abort_flag) ||
+                        !warp_wait(&full[(op + 1) % kBwdRing], ((op + 1) / kBwdRing) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t xb = ring + (op % kBwdRing) * kBwdSlot + kBwdSlab;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            mma_ss(tmem + kBwdTmAcc, smem_desc_sw128(xs + (q >> 2) * kBwdSlab + (q & 3) * 32, 16, 1024),
-                                   smem_desc_sw128(xb + q * 2048, kBwdSlot, 1024), id_a, (!first_rt || q) ? 1u : 0u);
-                        for (int o = 0; o < 4; ++o) mma_commit(&empty[(op + o) % kBwdRing]);
+                        for (int q = 0; q < 8; ++q) {
+                            const uint64_t ad = smem_desc_sw128(xs + (q >> 2) * kBwdSlab + (q & 3) * 32, 16, 1024);
+#pragma unroll
+                            for (int d = 0; d < 2; ++d)
+                                mma_ss(tmem + kBwdTmAcc + 128 * d, ad,
+                                       smem_desc_sw128(ring + ((op + d) % kBwdRing) * kBwdSlot + q * 2048, kBwdSlab, 1024),
+                                       id_a, (!first_rt || q) ? 1u : 0u);
+                        }
+                        mma_commit(&empty[op % kBwdRing]);
+                        mma_commit(&empty[(op + 1) % kBwdRing]);
                         mma_commit(x_empty);
                         if (rt == kk.rt_hi - 1) mma_commit(acc_full);
                     }
                     __syncwarp();
-                    op += 4;
+                    op += 2;
                 }
             }
         }
@@ -618,8 +659,9 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
     } else {
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;              // key row of the tile
-        const int sidx = threadIdx.x - 64;         // 0..127: column (query row) for the staging
+        const int sidx = threadIdx.x - 64;         // 0..127: column (query row) this thread stages
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        uint8_t* xsp = sm + kBwdSmX;
         uint32_t nrt = 0, npass = 0;
         bool ok = true;
         for (long long i = blockIdx.x; ok && i < p.kv_items; i += stride) {
@@ -627,61 +669,46 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
             if (!bwd_keys(p, i, kk)) continue;
             const int key = kk.k0 + r;
             const bool key_live = r < kk.nk;
+            float4 nx = bwd_col(p, kk, kk.rt_lo, sidx);
             for (int ps = 0; ok && ps < 4; ++ps, ++npass) {
                 const bool dkpass = ps >= 2;
                 for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt, ++nrt) {
-                    // the row tile's per-column data: token, LSE (log2 units), D
-                    {
-                        const int c = sidx;
-                        const int tok = rt * p.tpt + c / p.G;
-                        const int head = kk.g * p.G + c % p.G;
-                        bwd_bar();    // the previous row tile's columns have been used
-                        if (tok < p.T) {
-                            col_t[c] = tok;
-                            col_lse[c] = __ldg(p.lse + ((size_t)kk.b * p.Hq + head) * p.T + tok) * 1.4426950408889634f;
-                            col_d[c] = __ldg(p.drow + ((size_t)kk.b * p.T + tok) * p.Hq + head);
-                        } else {
-                            col_t[c] = -1;
-                            col_lse[c] = 0.f;
-                            col_d[c] = 0.f;
-                        }
-                        bwd_bar();
-                    }
+                    bwd_bar();    // every thread is done with the previous row tile's columns
+                    colv[sidx] = nx;
+                    bwd_bar();
+                    // the next row tile's columns load while this one is computed
+                    nx = bwd_col(p, kk, rt + 1 < kk.rt_hi ? rt + 1 : kk.rt_lo, sidx);
                     if (!bwd_group_wait(sdp_full, nrt & 1, abort_flag)) { ok = false; break; }
+                    if (!bwd_group_wait(x_empty, (nrt & 1) ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    uint32_t pk[64];
-#pragma unroll
+#pragma unroll 1
                     for (int c0 = 0; c0 < 128; c0 += 16) {
                         float sv[16], dpv[16];
                         tmem_ld16(tmem + lane_off + kBwdTmS + c0, sv);
                         if (dkpass) tmem_ld16(tmem + lane_off + kBwdTmP + c0, dpv);
                         tmem_wait_ld();
+                        uint32_t pk[8];
 #pragma unroll
                         for (int e = 0; e < 16; e += 2) {
                             float x[2];
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
-                                const int c = c0 + e + u;
-                                const int t = col_t[c];
-                                bool vis = key_live && t >= 0;
-                                if (vis) vis = kk.comp ? key < bwd_visible(t, p.W, p.blk) : (key <= t && key >= t - p.W + 1);
-                                const float pr = vis ? ex2(fmaf(sv[e + u], p.scale_log2, -col_lse[c])) : 0.f;
-                                x[u] = dkpass ? pr * (dpv[e + u] - col_d[c]) : pr;
+                                const float4 cd = colv[c0 + e + u];
+                                const bool vis = r >= __float_as_int(cd.z) && r < __float_as_int(cd.w);
+                                const float pr = vis ? ex2(fmaf(sv[e + u], p.scale_log2, -cd.x)) : 0.f;
+                                x[u] = dkpass ? pr * (dpv[e + u] - cd.y) : pr;
                             }
-                            pk[(c0 + e) >> 1] = pack_bf16x2(x[0], x[1]);
+                            pk[e >> 1] = pack_bf16x2(x[0], x[1]);
                         }
+                        bwd_put16(xsp, r, c0, pk);
                     }
                     tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(sdp_empty);
-                    if (!bwd_group_wait(x_empty, (nrt & 1) ^ 1, abort_flag)) { ok = false; break; }
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        *reinterpret_cast<uint4*>(sm + kBwdSmX + (c >> 3) * kBwdSlab + bwd_sw(r, c & 7)) =
-                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(x_full);
+                    if (lane == 0) {
+                        mbar_arrive(sdp_empty);
+                        mbar_arrive(x_full);
+                    }
                 }
                 if (!ok) break;
                 // ---- the pass's half of dV (ps 0, 1) or dK (ps 2, 3), added to the key's gradient
