@@ -147,7 +147,7 @@ def prefill_backward(q, k, v, w, kc, vc, out, lse, dout, blk, W, scale, want_dw=
     dvv = torch.empty((B, T, Hkv, dv), dtype=torch.float32, device=q.device)
     dw = torch.empty((B, T), dtype=torch.float32, device=q.device) if want_dw else None
     lib = _lib.load()
-    nbytes = int(lib.hca_prefill_backward_workspace_size(B, T, Hq, Hkv, dv, blk))
+    nbytes = int(lib.hca_prefill_backward_workspace_size(B, T, Hq, Hkv, dv, blk, W))
     if nbytes == 0:
         raise HCAError(_lib.HCA_ERR_UNSUPPORTED, "hca_prefill_backward_workspace_size")
     ws = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)

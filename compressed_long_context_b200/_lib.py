@@ -25,7 +25,7 @@ EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_deco
            "hca_decode_noalloc",
            "hca_vha", "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error",
            "hca_debug_set_wait_limit", "hca_debug_set_drop_slab", "hca_debug_wait_probe", "hca_gate_logits",
-           "hca_prefill_backward_workspace_size", "hca_prefill_backward")
+           "hca_prefill_backward_workspace_size", "hca_prefill_backward", "hca_debug_set_backward_segment")
 
 _lib = None
 
@@ -73,9 +73,11 @@ def load():
     lib.hca_gate_logits.restype = _i
     lib.hca_gate_logits.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
     lib.hca_prefill_backward_workspace_size.restype = _sz
-    lib.hca_prefill_backward_workspace_size.argtypes = [_i] * 6
+    lib.hca_prefill_backward_workspace_size.argtypes = [_i] * 7
     lib.hca_prefill_backward.restype = _i
     lib.hca_prefill_backward.argtypes = [_vp] * 13 + [_vp, _sz] + [_i] * 8 + [_f, _u, _vp]
+    lib.hca_debug_set_backward_segment.restype = _i
+    lib.hca_debug_set_backward_segment.argtypes = [_i]
     lib.hca_debug_set_wait_limit.restype = _i
     lib.hca_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong, _vp]
     lib.hca_debug_set_drop_slab.restype = _i

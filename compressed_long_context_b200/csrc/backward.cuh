@@ -12,19 +12,26 @@
 // dw_i = alpha_i (dalpha_i - sum_i' alpha_i' dalpha_i'), dalpha_i = K_i . dKc + V_i . dVc.
 // The stored cache is bf16; its rounding has no gradient (the entries are taken as stored).
 //
-// Kernels (every contraction on tcgen05, 512-dim heads):
-//   bwd_pre_kernel   D for every (token, head) row (one warp per row).
-//   bwd_dq_kernel    one CTA per row tile of 128 (token, head) rows: for every key tile it
-//                    recomputes S = Q K^T and dP = dO V^T (TMEM, 128 columns each), the
-//                    softmax warps form dS (bf16, shared memory), and dq += dS K accumulates in
-//                    TMEM -- 256 columns, so the 512 channels take two passes.
-//   bwd_dkv_kernel   one CTA per (key tile, range of query row tiles): S^T = K Q^T and, for dK,
-//                    dP^T = V dO^T; dV += P^T dO and dK += dS^T Q in channel halves (four passes),
-//                    added with fp32 atomics into the entries' gradients (workspace) or the raw
-//                    window keys' gradients.
-//   bwd_pool_kernel  one CTA per (sequence, block): pooling backward into dk, dv and dw.
-// Operands stream through one ring of six 32 KB slots (an A slab and a B slab of 128 rows x 64
-// channels each); the MMA issuer consumes the ops in the producer's order.  Every wait is
+// Work unit: a row tile of 128 (token, head) rows -- tpt = 128 / G tokens times the G query heads
+// of one KV head -- against a key tile of 128 keys: entries 128 j .. of the cache, or raw tokens
+// 128 kt .. (tiles aligned to multiples of 128, so that both kernels below name the same tiles).
+// A 512-dim head makes one key tile's dK and dV accumulators (2 x 128 x 512 fp32) twice the
+// tensor memory of an SM, so P and dS are formed once and kept in global memory instead of being
+// recomputed per accumulator:
+//   bwd_pre_kernel  D for every (token, head) row (one warp per row); clears the accumulators.
+//   bwd_dq_kernel   one CTA per row tile.  Phase S: per key tile, S = Q K^T and dP = dO V^T into
+//                   one of two tensor-memory buffers (the MMAs of the next tile overlap the
+//                   softmax of this one); eight softmax warps form P and dS in bf16 and write the
+//                   pair to the tile's record (64 KB, the operand layout of the tensor cores).
+//                   Phase A: dq = scale sum_j dS_j K_j, all 512 channels in tensor memory, dS
+//                   read back from the records just written (L2).
+//   bwd_dkv_kernel  one CTA per (key tile, dV or dK, range of row tiles): dV = sum P^T dO or
+//                   dK = scale sum dS^T Q from the records, 512 channels in tensor memory, added
+//                   with fp32 atomics into the entries' gradients (workspace) or the raw keys'.
+//   bwd_pool_kernel one CTA per (sequence, block): pooling backward into dk, dv and dw.
+// The records of a segment of row tiles are written by one dq launch and read by the dk/dv launch
+// that follows, which bounds the workspace; the host walks the segments.  Operands stream through
+// a ring of six 32 KB slots; the MMA issuer consumes ops in the producer's order.  Every wait is
 // bounded (common.cuh).
 #pragma once
 
@@ -33,24 +40,19 @@
 namespace hca {
 
 constexpr int kBwdD = 512;
-constexpr int kBwdThreads = 192;            // producer, MMA issuer, 4 softmax / epilogue warps
+constexpr int kDqThreads = 320;             // producer, MMA issuer, 8 softmax / epilogue warps
+constexpr int kKvThreads = 192;             // producer, MMA issuer, 4 epilogue warps
 constexpr int kBwdRing = 6;
-constexpr uint32_t kBwdSlab = 16384;         // 128 rows x 64 channels bf16, 128-byte swizzle
-constexpr uint32_t kBwdSlot = 2 * kBwdSlab;  // A slab + B slab
+constexpr uint32_t kBwdSlab = 16384;         // 128 rows x 64 columns bf16, 128-byte swizzle
+constexpr uint32_t kBwdSlot = 2 * kBwdSlab;  // two slabs
+constexpr uint32_t kBwdRec = 2 * kBwdSlot;   // one (row tile, key tile) record: P, then dS
 constexpr uint32_t kBwdSmRing = 0;
-constexpr uint32_t kBwdSmX = kBwdSmRing + kBwdRing * kBwdSlot;      // dS (or P^T / dS^T): 2 slabs
-constexpr uint32_t kBwdSmCol = kBwdSmX + 2 * kBwdSlab;              // per-column data (dkv): 128 x float4
-constexpr uint32_t kBwdSmBar = kBwdSmCol + 4 * 128 * 4;
-constexpr int kBwdNumBars = 2 * kBwdRing + 8;
+constexpr uint32_t kBwdSmBar = kBwdSmRing + kBwdRing * kBwdSlot;
+constexpr int kBwdNumBars = 2 * kBwdRing + 12;
 constexpr uint32_t kBwdSmMisc = kBwdSmBar + kBwdNumBars * 8;
 constexpr uint32_t kBwdSmem = kBwdSmMisc + 16;
 static_assert(kBwdSmem <= 232448, "backward shared memory exceeds the per-block limit");
-static_assert(kBwdSmX % 1024 == 0 && kBwdSlot % 1024 == 0, "swizzled operands 1024-aligned");
-
-// TMEM columns
-constexpr uint32_t kBwdTmS = 0;      // S (or S^T): 128 columns
-constexpr uint32_t kBwdTmP = 128;    // dP (or dP^T): 128 columns
-constexpr uint32_t kBwdTmAcc = 256;  // dq / dk / dv half: 256 columns
+static_assert(kBwdSlot % 1024 == 0, "swizzled operands 1024-aligned");
 
 struct BwdParams {
     const float* lse;             // [B, Hq, T] natural log
@@ -66,11 +68,13 @@ struct BwdParams {
     float* dkc;                   // [B, Nc, Hkv, 512] (workspace)
     float* dvc;
     float* dw;                    // [B, T]
+    uint8_t* rec;                 // [B, Hkv, seg, nt_max] records of kBwdRec bytes (workspace)
     int B, T, Hq, Hkv, G, tpt, blk, W, Nc, ntile_t, out_f32;
-    long long dq_items;           // B * Hkv * ntile_t
-    int nkc, nkw;                 // compressed / raw key tiles per (b, g)
-    int chc, chw;                 // row-tile chunks per compressed / raw key tile
-    int rt_chunk;                 // row tiles per chunk
+    int nkc, nkw, nt_max, seg;    // compressed / raw key tiles; record slots per row tile; segment
+    int s0, s1;                   // this launch's segment of row tiles
+    long long dq_items;           // B * Hkv * (s1 - s0)
+    int ch_rows, nch;             // dk/dv: row tiles per chunk of a compressed key tile, chunks
+    int kta, nraw;                // dk/dv: first raw key tile touching the segment, their count
     long long kv_items;
     float scale, scale_log2;
 };
@@ -80,34 +84,38 @@ __device__ __forceinline__ int bwd_visible(int t, int W, int blk) {
     return a > 0 ? a / blk : 0;
 }
 
-// Row tile of a dq item: rows (token t0 + r / G, head g * G + r % G).
+// Row tile rt of (b, g): rows (token t0 + r / G, head g G + r % G); its key tiles j < nct are the
+// entry tiles, then raw tiles kw0, kw0 + 1, .. (128-aligned) covering the window of every token.
 struct BwdRows {
-    int b, g, t0, tlast, ncomp, nct, wlo, nwin, nwt;
+    int t0, tlast, nct, wlo, kw0, nt;
 };
 
-__device__ __forceinline__ BwdRows bwd_rows(const BwdParams& p, int b, int g, int rt) {
+__device__ __forceinline__ BwdRows bwd_rows(const BwdParams& p, int rt) {
     BwdRows it;
-    it.b = b;
-    it.g = g;
     it.t0 = rt * p.tpt;
     it.tlast = min(it.t0 + p.tpt, p.T) - 1;
-    it.ncomp = bwd_visible(it.tlast, p.W, p.blk);
-    it.nct = (it.ncomp + 127) / 128;
+    it.nct = (bwd_visible(it.tlast, p.W, p.blk) + 127) / 128;
     it.wlo = max(0, it.t0 - p.W + 1);
-    it.nwin = it.tlast - it.wlo + 1;
-    it.nwt = (it.nwin + 127) / 128;
+    it.kw0 = it.wlo / 128;
+    it.nt = it.nct + it.tlast / 128 - it.kw0 + 1;
     return it;
 }
 
-// Named barrier among the four softmax / epilogue warps.
-__device__ __forceinline__ void bwd_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ uint8_t* bwd_record(const BwdParams& p, int b, int g, int rt, int j) {
+    return p.rec + ((((size_t)b * p.Hkv + g) * p.seg + (rt - p.s0)) * p.nt_max + j) * (size_t)kBwdRec;
+}
 
+// Named barrier among the softmax / epilogue warps (n threads).
+template <int n>
+__device__ __forceinline__ void bwd_bar() { asm volatile("bar.sync 1, %0;" :: "n"(n) : "memory"); }
+
+template <int n>
 __device__ __forceinline__ bool bwd_group_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
     const bool ok = mbar_wait(bar, parity, abort);
     uint32_t r;
     asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-                 "barrier.red.and.pred q, 2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r) : "r"((uint32_t)ok) : "memory");
+                 "barrier.red.and.pred q, 2, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)ok), "n"(n) : "memory");
     return r != 0;
 }
 
@@ -168,22 +176,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 
 // -------------------------------------------------------------------------------- dq
 
-// Ops of one key tile of a dq pass: 8 x (Q slab, K slab) for S, 8 x (dO slab, V slab) for dP,
-// then two ops that each carry two of the pass's four K channel blocks (channels 256 h + 128 d
-// and + 64, in the slot's A and B halves): the N = 128 B operands of dq[:, 128 d ..] += dS K.
+// Phase S ops of a key tile: 8 x (Q slab, K slab) for S, then 8 x (dO slab, V slab) for dP.
+// Phase A ops of a key tile: its dS (32 KB from the record), then the key tile's 512 channels as
+// four ops of two 64-channel blocks, the N = 128 B operands of dq[:, 128 d ..] += dS K.
 constexpr int kDqPairs = 16;
-constexpr int kDqOps = kDqPairs + 2;
 
-// Softmax-gradient columns c0 .. c0 + 15 of row r, packed to bf16, into the K-major 128-byte-
-// swizzled operand buffer (two slabs of 64 columns).
-__device__ __forceinline__ void bwd_put16(uint8_t* xs, int r, int c0, const uint32_t* pk) {
-    uint8_t* dst = xs + (c0 >> 6) * kBwdSlab;
-    const uint32_t ch = (uint32_t)(c0 & 63) >> 3;
-    *reinterpret_cast<uint4*>(dst + bwd_sw(r, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    *reinterpret_cast<uint4*>(dst + bwd_sw(r, ch + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-}
-
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
 bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc) {
@@ -195,13 +193,12 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
     uint8_t* sm = dsmem;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBwdSmBar);
     uint64_t* empty = full + kBwdRing;
-    uint64_t* sdp_full = empty + kBwdRing;
-    uint64_t* sdp_empty = sdp_full + 1;
-    uint64_t* ds_full = sdp_full + 2;
-    uint64_t* ds_empty = sdp_full + 3;
-    uint64_t* acc_full = sdp_full + 4;
-    uint64_t* acc_empty = sdp_full + 5;
-    uint64_t* drain = sdp_full + 6;
+    uint64_t* sdp_full = empty + kBwdRing;      // [2]
+    uint64_t* sdp_empty = sdp_full + 2;         // [2]
+    uint64_t* rec_ready = sdp_full + 4;
+    uint64_t* acc_full = sdp_full + 5;
+    uint64_t* acc_empty = sdp_full + 6;
+    uint64_t* drain = sdp_full + 7;
     int* misc = reinterpret_cast<int*>(sm + kBwdSmMisc);
     volatile int* abort_flag = misc;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
@@ -212,12 +209,13 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        mbar_init(sdp_full, 1);
-        mbar_init(sdp_empty, 4);
-        mbar_init(ds_full, 4);
-        mbar_init(ds_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sdp_full[i], 1);
+            mbar_init(&sdp_empty[i], 8);
+        }
+        mbar_init(rec_ready, 1);
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
+        mbar_init(acc_empty, 8);
         mbar_init(drain, 1);
         fence_mbar_init();
     }
@@ -229,113 +227,127 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
     const long long stride = gridDim.x;
     auto decode_item = [&](long long i, int& b, int& g, int& rt) {
         g = (int)(i % p.Hkv);
-        long long r = i / p.Hkv;
+        const long long r = i / p.Hkv;
         b = (int)(r % p.B);
-        rt = p.ntile_t - 1 - (int)(r / p.B);        // heavy (late) row tiles first
+        rt = p.s1 - 1 - (int)(r / p.B);        // heavy (late) row tiles first
     };
 
     if (warp == 0) {
         // ================================================================ TMA producer
         if (lane == 0) {
-            uint32_t op = 0;
+            uint32_t op = 0, nitem = 0;
             bool ok = true;
-            for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride) {
+            auto slot = [&](uint32_t& st) -> uint8_t* {
+                st = op % kBwdRing;
+                if (!mbar_wait(&empty[st], ((op / kBwdRing) & 1) ^ 1, abort_flag)) return nullptr;
+                return sm + kBwdSmRing + st * kBwdSlot;
+            };
+            for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride, ++nitem) {
                 int b, g, rt;
                 decode_item(i, b, g, rt);
-                const BwdRows it = bwd_rows(p, b, g, rt);
-                const int nt = it.nct + it.nwt;
-                for (int h = 0; ok && h < 2; ++h)
-                    for (int j = 0; ok && j < nt; ++j) {
-                        const bool comp = j < it.nct;
-                        const int row = comp ? 128 * j : it.wlo + 128 * (j - it.nct);
-                        for (int o = 0; o < kDqOps; ++o, ++op) {
-                            const uint32_t st = op % kBwdRing;
-                            if (!mbar_wait(&empty[st], ((op / kBwdRing) & 1) ^ 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            uint8_t* base = sm + kBwdSmRing + st * kBwdSlot;
-                            mbar_arrive_expect_tx(&full[st], kBwdSlot);
-                            if (o < kDqPairs) {
-                                const int s = o & 7;
-                                tma_load_4d(base, o < 8 ? &tm_q : &tm_do, &full[st], 64 * s, g * p.G, it.t0, b);
-                                tma_load_4d(base + kBwdSlab, o < 8 ? (comp ? &tm_kc : &tm_k) : (comp ? &tm_vc : &tm_v),
-                                            &full[st], 64 * s, g, row, b);
-                            } else {
-                                const int c = 256 * h + 128 * (o - kDqPairs);
-                                const CUtensorMap* km = comp ? &tm_kc : &tm_k;
-                                tma_load_4d(base, km, &full[st], c, g, row, b);
-                                tma_load_4d(base + kBwdSlab, km, &full[st], c + 64, g, row, b);
-                            }
+                const BwdRows it = bwd_rows(p, rt);
+                for (int j = 0; ok && j < it.nt; ++j) {
+                    const bool comp = j < it.nct;
+                    const int row = 128 * (comp ? j : it.kw0 + j - it.nct);
+                    for (int o = 0; o < kDqPairs; ++o, ++op) {
+                        uint32_t st;
+                        uint8_t* base = slot(st);
+                        if (!base) { ok = false; break; }
+                        const int s = o & 7;
+                        mbar_arrive_expect_tx(&full[st], kBwdSlot);
+                        tma_load_4d(base, o < 8 ? &tm_q : &tm_do, &full[st], 64 * s, g * p.G, it.t0, b);
+                        tma_load_4d(base + kBwdSlab, o < 8 ? (comp ? &tm_kc : &tm_k) : (comp ? &tm_vc : &tm_v),
+                                    &full[st], 64 * s, g, row, b);
+                    }
+                }
+                // phase A reads the dS the softmax warps have written for this item
+                if (ok && !mbar_wait(rec_ready, nitem & 1, abort_flag)) ok = false;
+                for (int j = 0; ok && j < it.nt; ++j) {
+                    const bool comp = j < it.nct;
+                    const int row = 128 * (comp ? j : it.kw0 + j - it.nct);
+                    const CUtensorMap* km = comp ? &tm_kc : &tm_k;
+                    for (int o = 0; o < 5; ++o, ++op) {
+                        uint32_t st;
+                        uint8_t* base = slot(st);
+                        if (!base) { ok = false; break; }
+                        mbar_arrive_expect_tx(&full[st], kBwdSlot);
+                        if (o == 0) {
+                            bulk_load(base, bwd_record(p, b, g, rt, j) + kBwdSlot, kBwdSlot, &full[st]);
+                        } else {
+                            const int c = 128 * (o - 1);
+                            tma_load_4d(base, km, &full[st], c, g, row, b);
+                            tma_load_4d(base + kBwdSlab, km, &full[st], c + 64, g, row, b);
                         }
                     }
+                }
             }
             mbar_drain_ring(full, op, kBwdRing);
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_q = idesc_bf16(128, 128, 0, 1);
-        const uint32_t ring = smem_u32(sm + kBwdSmRing), xs = smem_u32(sm + kBwdSmX);
-        uint32_t op = 0, nkt = 0, npass = 0;
+        const uint32_t id_a = idesc_bf16(128, 128, 0, 1);
+        const uint32_t ring = smem_u32(sm + kBwdSmRing);
+        uint32_t op = 0, ns = 0, nitem = 0;
         bool ok = true;
-        for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride) {
+        for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride, ++nitem) {
             int b, g, rt;
             decode_item(i, b, g, rt);
-            const BwdRows it = bwd_rows(p, b, g, rt);
-            const int nt = it.nct + it.nwt;
-            for (int h = 0; ok && h < 2; ++h, ++npass) {
-                for (int j = 0; ok && j < nt; ++j, ++nkt) {
-                    // S and dP of the previous key tile have been read by the softmax warps
-                    if (!warp_wait(sdp_empty, (nkt & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int o = 0; o < kDqPairs; ++o, ++op) {
-                        const uint32_t st = op % kBwdRing;
-                        if (!warp_wait(&full[st], (op / kBwdRing) & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        if (lane == 0) {
-                            const uint32_t a = ring + st * kBwdSlot, bb = a + kBwdSlab;
-                            const uint32_t d = tmem + (o < 8 ? kBwdTmS : kBwdTmP);
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_ss(d, smem_desc_sw128(a + kk * 32, 16, 1024), smem_desc_sw128(bb + kk * 32, 16, 1024),
-                                       id_s, ((o & 7) | kk) ? 1u : 0u);
-                            mma_commit(&empty[st]);
-                        }
-                        __syncwarp();
-                    }
-                    if (!ok) break;
-                    if (lane == 0) mma_commit(sdp_full);
-                    __syncwarp();
-                    // dq half += dS K_half, once dS is in shared memory (and, on the pass's first
-                    // key tile, once the previous pass's accumulator has been read out)
-                    if (j == 0 && !warp_wait(acc_empty, (npass & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    if (!warp_wait(ds_full, nkt & 1, abort_flag)) { ok = false; break; }
-                    if (!warp_wait(&full[op % kBwdRing], (op / kBwdRing) & 1, abort_flag) ||
-                        !warp_wait(&full[(op + 1) % kBwdRing], ((op + 1) / kBwdRing) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+            const BwdRows it = bwd_rows(p, rt);
+            // tensor memory is free once the previous item's dq has been read out
+            if (!warp_wait(acc_empty, (nitem & 1) ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            for (int j = 0; ok && j < it.nt; ++j, ++ns) {
+                const uint32_t buf = ns & 1;
+                // the softmax warps have read this buffer's previous tile
+                if (!warp_wait(&sdp_empty[buf], ((ns >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int o = 0; o < kDqPairs; ++o, ++op) {
+                    const uint32_t st = op % kBwdRing;
+                    if (!warp_wait(&full[st], (op / kBwdRing) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     if (lane == 0) {
+                        const uint32_t a = ring + st * kBwdSlot, bb = a + kBwdSlab;
+                        const uint32_t d = tmem + 256 * buf + (o < 8 ? 0 : 128);
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t ad = smem_desc_sw128(xs + (kk >> 2) * kBwdSlab + (kk & 3) * 32, 16, 1024);
-#pragma unroll
-                            for (int d = 0; d < 2; ++d)
-                                mma_ss(tmem + kBwdTmAcc + 128 * d, ad,
-                                       smem_desc_sw128(ring + ((op + d) % kBwdRing) * kBwdSlot + kk * 2048, kBwdSlab,
-                                                       1024),
-                                       id_q, (j | kk) ? 1u : 0u);
-                        }
-                        mma_commit(&empty[op % kBwdRing]);
-                        mma_commit(&empty[(op + 1) % kBwdRing]);
-                        mma_commit(ds_empty);
-                        if (j == nt - 1) mma_commit(acc_full);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(d, smem_desc_sw128(a + kk * 32, 16, 1024), smem_desc_sw128(bb + kk * 32, 16, 1024),
+                                   id_s, ((o & 7) | kk) ? 1u : 0u);
+                        mma_commit(&empty[st]);
                     }
                     __syncwarp();
-                    op += 2;
                 }
+                if (!ok) break;
+                if (lane == 0) mma_commit(&sdp_full[buf]);
+                __syncwarp();
+            }
+            if (!ok) break;
+            // phase A overwrites both buffers: the softmax warps have read the last two tiles
+            for (int m = (int)ns - 1; ok && m >= 0 && m >= (int)ns - 2; --m)
+                if (!warp_wait(&sdp_empty[m & 1], (m >> 1) & 1, abort_flag)) ok = false;
+            if (!ok) break;
+            tc_fence_after();
+            for (int j = 0; ok && j < it.nt; ++j) {
+                for (int o = 0; o < 5; ++o)
+                    if (!warp_wait(&full[(op + o) % kBwdRing], ((op + o) / kBwdRing) & 1, abort_flag)) ok = false;
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t ds = ring + (op % kBwdRing) * kBwdSlot;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(ds + (kk >> 2) * kBwdSlab + (kk & 3) * 32, 16, 1024);
+#pragma unroll
+                        for (int d = 0; d < 4; ++d)
+                            mma_ss(tmem + 128 * d, ad,
+                                   smem_desc_sw128(ring + ((op + 1 + d) % kBwdRing) * kBwdSlot + kk * 2048, kBwdSlab, 1024),
+                                   id_a, (j | kk) ? 1u : 0u);
+                    }
+                    for (int o = 0; o < 5; ++o) mma_commit(&empty[(op + o) % kBwdRing]);
+                    if (j == it.nt - 1) mma_commit(acc_full);
+                }
+                __syncwarp();
+                op += 5;
             }
         }
         // every MMA has completed before the CTA releases its shared and tensor memory
@@ -345,18 +357,17 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
         }
         __syncwarp();
     } else {
-        // ================================================================ dS and the epilogue
-        const int q4 = warp & 3;
+        // ================================================================ P, dS and the epilogue
+        const int q4 = warp & 3;                  // tensor-memory lane quarter
+        const int hc = (warp - 2) >> 2;           // column half
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        uint8_t* xsp = sm + kBwdSmX;
-        uint32_t nkt = 0, npass = 0;
+        uint32_t ns = 0, nitem = 0;
         bool ok = true;
-        for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride) {
+        for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride, ++nitem) {
             int b, g, rt;
             decode_item(i, b, g, rt);
-            const BwdRows it = bwd_rows(p, b, g, rt);
-            const int nt = it.nct + it.nwt;
+            const BwdRows it = bwd_rows(p, rt);
             const int tok = it.t0 + r / p.G;
             const bool live = tok < p.T;
             const int t = live ? tok : p.T - 1;
@@ -364,66 +375,75 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
             const float lse2 = live ? __ldg(p.lse + ((size_t)b * p.Hq + head) * p.T + t) * 1.4426950408889634f : 0.f;
             const float Dr = live ? __ldg(p.drow + ((size_t)b * p.T + t) * p.Hq + head) : 0.f;
             const int nc_t = bwd_visible(t, p.W, p.blk);
-            for (int h = 0; ok && h < 2; ++h, ++npass) {
-                for (int j = 0; ok && j < nt; ++j, ++nkt) {
-                    if (!bwd_group_wait(sdp_full, nkt & 1, abort_flag)) { ok = false; break; }
-                    // the previous key tile's dS has been consumed
-                    if (!bwd_group_wait(ds_empty, (nkt & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    int lo, hi;   // valid columns of this row in the tile
-                    if (j < it.nct) {
-                        lo = 0;
-                        hi = min(128, nc_t - 128 * j);
-                    } else {
-                        const int u0 = it.wlo + 128 * (j - it.nct);
-                        lo = max(0, t - p.W + 1 - u0);
-                        hi = min(128, t - u0 + 1);
-                    }
-                    if (!live) hi = lo;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < 128; c0 += 16) {
-                        float sv[16], dpv[16];
-                        tmem_ld16(tmem + lane_off + kBwdTmS + c0, sv);
-                        tmem_ld16(tmem + lane_off + kBwdTmP + c0, dpv);
-                        tmem_wait_ld();
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int e = 0; e < 16; e += 2) {
-                            const int c = c0 + e;
-                            const float p0 = (c >= lo && c < hi) ? ex2(fmaf(sv[e], p.scale_log2, -lse2)) : 0.f;
-                            const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2(fmaf(sv[e + 1], p.scale_log2, -lse2)) : 0.f;
-                            pk[e >> 1] = pack_bf16x2(p0 * (dpv[e] - Dr), p1 * (dpv[e + 1] - Dr));
-                        }
-                        bwd_put16(xsp, r, c0, pk);
-                    }
-                    tc_fence_before();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(sdp_empty);
-                        mbar_arrive(ds_full);
-                    }
-                }
-                if (!ok) break;
-                // ---- the pass's dq half: scale * accumulator -> dq[b, t, head, 256 h ..]
-                if (!bwd_group_wait(acc_full, npass & 1, abort_flag)) { ok = false; break; }
+            for (int j = 0; ok && j < it.nt; ++j, ++ns) {
+                const uint32_t buf = ns & 1;
+                if (!bwd_group_wait<256>(&sdp_full[buf], (ns >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                float* dst = p.dq + (((size_t)b * p.T + t) * p.Hq + head) * kBwdD + 256 * h;
+                int lo, hi;   // valid key columns of this row in the tile
+                if (j < it.nct) {
+                    lo = 0;
+                    hi = min(128, nc_t - 128 * j);
+                } else {
+                    const int u0 = 128 * (it.kw0 + j - it.nct);
+                    lo = max(0, t - p.W + 1 - u0);
+                    hi = min(128, t - u0 + 1);
+                }
+                if (!live) hi = lo;
+                uint8_t* rp = bwd_record(p, b, g, rt, j) + hc * kBwdSlab;
 #pragma unroll 1
-                for (int c0 = 0; c0 < 256; c0 += 16) {
-                    float a[16];
-                    tmem_ld16(tmem + lane_off + kBwdTmAcc + c0, a);
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int c0 = 64 * hc + 32 * h2;
+                    float sv[32], dpv[32];
+                    const uint32_t tb = tmem + lane_off + 256 * buf + c0;
+                    tmem_ld16(tb, sv);
+                    tmem_ld16(tb + 16, sv + 16);
+                    tmem_ld16(tb + 128, dpv);
+                    tmem_ld16(tb + 144, dpv + 16);
                     tmem_wait_ld();
-                    if (live)
+                    uint32_t pp[16], pd[16];
 #pragma unroll
-                        for (int e = 0; e < 16; e += 4)
-                            *reinterpret_cast<float4*>(dst + c0 + e) =
-                                make_float4(p.scale * a[e], p.scale * a[e + 1], p.scale * a[e + 2], p.scale * a[e + 3]);
+                    for (int e = 0; e < 32; e += 2) {
+                        const int c = c0 + e;
+                        const float p0 = (c >= lo && c < hi) ? ex2(fmaf(sv[e], p.scale_log2, -lse2)) : 0.f;
+                        const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2(fmaf(sv[e + 1], p.scale_log2, -lse2)) : 0.f;
+                        pp[e >> 1] = pack_bf16x2(p0, p1);
+                        pd[e >> 1] = pack_bf16x2(p0 * (dpv[e] - Dr), p1 * (dpv[e + 1] - Dr));
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t off = bwd_sw(r, 4 * h2 + q);
+                        *reinterpret_cast<uint4*>(rp + off) = make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
+                        *reinterpret_cast<uint4*>(rp + kBwdSlot + off) =
+                            make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                if (lane == 0) mbar_arrive(&sdp_empty[buf]);
             }
+            if (!ok) break;
+            // the records are complete: hand them to the async proxy (the producer's bulk loads)
+            fence_proxy_async_global();
+            bwd_bar<256>();
+            if (threadIdx.x == 64) mbar_arrive(rec_ready);
+            // ---- dq = scale * accumulator, channels 256 hc ..
+            if (!bwd_group_wait<256>(acc_full, nitem & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            float* dst = p.dq + (((size_t)b * p.T + t) * p.Hq + head) * kBwdD + 256 * hc;
+#pragma unroll 1
+            for (int c0 = 0; c0 < 256; c0 += 16) {
+                float a[16];
+                tmem_ld16(tmem + lane_off + 256 * hc + c0, a);
+                tmem_wait_ld();
+                if (live)
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4*>(dst + c0 + e) =
+                            make_float4(p.scale * a[e], p.scale * a[e + 1], p.scale * a[e + 2], p.scale * a[e + 3]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
         }
     }
     __syncwarp();
@@ -437,80 +457,59 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
 
 // -------------------------------------------------------------------------------- dk, dv
 
-// Key tile kt of (b, g): kt < nkc are entries 128 kt .., else raw tokens 128 (kt - nkc) ..; its
-// query row tiles [lo, hi), cut into chunks of rt_chunk.
+// Item of a dk/dv launch: key tile kt (entries 128 kt .. when comp, else raw tokens 128 kt ..),
+// which = 0 for dV (from P and dO) or 1 for dK (from dS and Q), over row tiles [rt_lo, rt_hi).
+// Per (b, g): the entry tiles' items first, ordered (chunk of ch_rows row tiles, kt, which) so
+// that the CTAs running at once share those rows of Q and dO in L2; then the raw tiles' (kt, which).
 struct BwdKeys {
-    int b, g, kt, comp, k0, nk, rt_lo, rt_hi;
+    int b, g, kt, comp, which, k0, nk, rt_lo, rt_hi;
 };
 
 __device__ __forceinline__ bool bwd_keys(const BwdParams& p, long long i, BwdKeys& kk) {
-    const long long ncomp_items = (long long)p.B * p.Hkv * p.nkc * p.chc;
-    int chunk;
-    long long r;
-    if (i < ncomp_items) {
-        kk.comp = 1;
-        chunk = (int)(i % p.chc);
-        r = i / p.chc;
-        kk.kt = (int)(r % p.nkc);
-        r /= p.nkc;
-    } else {
-        i -= ncomp_items;
-        kk.comp = 0;
-        chunk = (int)(i % p.chw);
-        r = i / p.chw;
-        kk.kt = (int)(r % p.nkw);
-        r /= p.nkw;
-    }
-    kk.g = (int)(r % p.Hkv);
-    kk.b = (int)(r / p.Hkv);
+    const long long per_c = 2LL * p.nkc * p.nch, per_bg = per_c + 2LL * p.nraw;
+    const long long bg = i / per_bg;
+    long long rem = i - bg * per_bg;
+    kk.b = (int)(bg / p.Hkv);
+    kk.g = (int)(bg % p.Hkv);
+    kk.which = (int)(rem & 1);
     int lo, hi;
-    if (kk.comp) {
+    if (rem < per_c) {
+        kk.comp = 1;
+        rem >>= 1;
+        kk.kt = (int)(rem % p.nkc);
+        const int c = (int)(rem / p.nkc);
         kk.k0 = 128 * kk.kt;
         kk.nk = min(128, p.Nc - kk.k0);
         // the first token that sees entry k0: n_c(t) > k0  <=>  t >= blk (k0 + 1) + W - 1
         const long long tmin = (long long)p.blk * (kk.k0 + 1) + p.W - 1;
         lo = tmin >= p.T ? p.ntile_t : (int)(tmin / p.tpt);
         hi = p.ntile_t;
+        lo = max(lo, p.s0 + c * p.ch_rows);
+        hi = min(hi, min(p.s1, p.s0 + (c + 1) * p.ch_rows));
     } else {
+        kk.comp = 0;
+        kk.kt = p.kta + (int)((rem - per_c) >> 1);
+        if (kk.kt >= p.nkw) return false;
         kk.k0 = 128 * kk.kt;
         kk.nk = min(128, p.T - kk.k0);
         const int tmax = min(p.T - 1, kk.k0 + kk.nk - 1 + p.W - 1);
-        lo = kk.k0 / p.tpt;
-        hi = tmax / p.tpt + 1;
+        lo = max(kk.k0 / p.tpt, p.s0);
+        hi = min(tmax / p.tpt + 1, p.s1);
     }
-    kk.rt_lo = lo + chunk * p.rt_chunk;
-    kk.rt_hi = min(hi, kk.rt_lo + p.rt_chunk);
-    return kk.rt_lo < kk.rt_hi && kk.nk > 0;
+    kk.rt_lo = lo;
+    kk.rt_hi = hi;
+    return lo < hi && kk.nk > 0;
 }
 
-// Per query row (column of S^T) of row tile rt: its log2-domain LSE, D, and the key rows of the
-// tile it sees, [rlo, rhi) relative to k0 (empty for rows past the sequence end).
-__device__ __forceinline__ float4 bwd_col(const BwdParams& p, const BwdKeys& kk, int rt, int c) {
-    const int tok = rt * p.tpt + c / p.G;
-    if (tok >= p.T) return make_float4(0.f, 0.f, __int_as_float(0), __int_as_float(0));
-    const int head = kk.g * p.G + c % p.G;
-    const float l2 = __ldg(p.lse + ((size_t)kk.b * p.Hq + head) * p.T + tok) * 1.4426950408889634f;
-    const float D = __ldg(p.drow + ((size_t)kk.b * p.T + tok) * p.Hq + head);
-    int rlo, rhi;
-    if (kk.comp) {
-        rlo = 0;
-        rhi = bwd_visible(tok, p.W, p.blk) - kk.k0;
-    } else {
-        rlo = tok - p.W + 1 - kk.k0;
-        rhi = tok - kk.k0 + 1;
-    }
-    return make_float4(l2, D, __int_as_float(rlo), __int_as_float(rhi));
+// Record slot of key tile kt in row tile rt (the dq kernel's order).
+__device__ __forceinline__ int bwd_slot(const BwdParams& p, const BwdKeys& kk, int rt) {
+    if (kk.comp) return kk.kt;
+    const BwdRows it = bwd_rows(p, rt);
+    return it.nct + kk.kt - it.kw0;
 }
 
-// Ops of one query row tile in pass ps (0, 1: dV halves; 2, 3: dK halves): 8 x (K slab, Q slab)
-// for S^T; for dK, 8 x (V slab, dO slab) for dP^T; then two ops carrying the half's four dO (dV)
-// or Q (dK) channel blocks, two per op, as the N = 128 B operands of the accumulation.
-__device__ __forceinline__ int bwd_kv_pairs(int ps) { return ps < 2 ? 8 : 16; }
-
-__global__ void __launch_bounds__(kBwdThreads, 1)
-bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc) {
+__global__ void __launch_bounds__(kKvThreads, 1)
+bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do) {
     extern __shared__ __align__(1024) uint8_t dsmem[];
     if (smem_u32(dsmem) & 1023u) {
         if (threadIdx.x == 0) record_error(HCA_ERR_INTERNAL);
@@ -519,14 +518,9 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
     uint8_t* sm = dsmem;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBwdSmBar);
     uint64_t* empty = full + kBwdRing;
-    uint64_t* sdp_full = empty + kBwdRing;
-    uint64_t* sdp_empty = sdp_full + 1;
-    uint64_t* x_full = sdp_full + 2;
-    uint64_t* x_empty = sdp_full + 3;
-    uint64_t* acc_full = sdp_full + 4;
-    uint64_t* acc_empty = sdp_full + 5;
-    uint64_t* drain = sdp_full + 6;
-    float4* colv = reinterpret_cast<float4*>(sm + kBwdSmCol);      // [128] per query row (column)
+    uint64_t* acc_full = empty + kBwdRing;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* drain = acc_full + 2;
     int* misc = reinterpret_cast<int*>(sm + kBwdSmMisc);
     volatile int* abort_flag = misc;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
@@ -537,10 +531,6 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        mbar_init(sdp_full, 1);
-        mbar_init(sdp_empty, 4);
-        mbar_init(x_full, 4);
-        mbar_init(x_empty, 1);
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 4);
         mbar_init(drain, 1);
@@ -554,185 +544,110 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
     const long long stride = gridDim.x;
 
     if (warp == 0) {
+        // ops of one row tile: the record's P (dV) or dS (dK), then dO (dV) or Q (dK) rows as four
+        // ops of two 64-channel blocks
         if (lane == 0) {
             uint32_t op = 0;
             bool ok = true;
             for (long long i = blockIdx.x; ok && i < p.kv_items; i += stride) {
                 BwdKeys kk;
                 if (!bwd_keys(p, i, kk)) continue;
-                for (int ps = 0; ok && ps < 4; ++ps)
-                    for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt) {
-                        const int t0 = rt * p.tpt;
-                        const int pairs = bwd_kv_pairs(ps);
-                        for (int o = 0; o < pairs + 2; ++o, ++op) {
-                            const uint32_t st = op % kBwdRing;
-                            if (!mbar_wait(&empty[st], ((op / kBwdRing) & 1) ^ 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            uint8_t* base = sm + kBwdSmRing + st * kBwdSlot;
-                            mbar_arrive_expect_tx(&full[st], kBwdSlot);
-                            if (o < pairs) {
-                                const int s = o & 7;
-                                const bool sk = o < 8;        // S^T: (K, Q); dP^T: (V, dO)
-                                tma_load_4d(base, sk ? (kk.comp ? &tm_kc : &tm_k) : (kk.comp ? &tm_vc : &tm_v), &full[st],
-                                            64 * s, kk.g, kk.k0, kk.b);
-                                tma_load_4d(base + kBwdSlab, sk ? &tm_q : &tm_do, &full[st], 64 * s, kk.g * p.G, t0, kk.b);
-                            } else {
-                                const int c = 256 * (ps & 1) + 128 * (o - pairs);
-                                const CUtensorMap* m = ps < 2 ? &tm_do : &tm_q;
-                                tma_load_4d(base, m, &full[st], c, kk.g * p.G, t0, kk.b);
-                                tma_load_4d(base + kBwdSlab, m, &full[st], c + 64, kk.g * p.G, t0, kk.b);
-                            }
+                const CUtensorMap* m = kk.which ? &tm_q : &tm_do;
+                for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt) {
+                    const uint8_t* rec = bwd_record(p, kk.b, kk.g, rt, bwd_slot(p, kk, rt)) + kk.which * kBwdSlot;
+                    for (int o = 0; o < 5; ++o, ++op) {
+                        const uint32_t st = op % kBwdRing;
+                        if (!mbar_wait(&empty[st], ((op / kBwdRing) & 1) ^ 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t* base = sm + kBwdSmRing + st * kBwdSlot;
+                        mbar_arrive_expect_tx(&full[st], kBwdSlot);
+                        if (o == 0) {
+                            bulk_load(base, rec, kBwdSlot, &full[st]);
+                        } else {
+                            const int c = 128 * (o - 1);
+                            tma_load_4d(base, m, &full[st], c, kk.g * p.G, rt * p.tpt, kk.b);
+                            tma_load_4d(base + kBwdSlab, m, &full[st], c + 64, kk.g * p.G, rt * p.tpt, kk.b);
                         }
                     }
+                }
             }
             mbar_drain_ring(full, op, kBwdRing);
         }
     } else if (warp == 1) {
-        const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_a = idesc_bf16(128, 128, 0, 1);
-        const uint32_t ring = smem_u32(sm + kBwdSmRing), xs = smem_u32(sm + kBwdSmX);
-        uint32_t op = 0, nrt = 0, npass = 0;
+        // D[key, channel] += sum over the tile's 128 query rows of X[row, key] Y[row, channel]:
+        // A = the record's tile read MN-major (keys contiguous), B = dO / Q MN-major
+        const uint32_t id_a = idesc_bf16(128, 128, 1, 1);
+        const uint32_t ring = smem_u32(sm + kBwdSmRing);
+        uint32_t op = 0, nitem = 0;
         bool ok = true;
         for (long long i = blockIdx.x; ok && i < p.kv_items; i += stride) {
             BwdKeys kk;
             if (!bwd_keys(p, i, kk)) continue;
-            for (int ps = 0; ok && ps < 4; ++ps, ++npass) {
-                const int pairs = bwd_kv_pairs(ps);
-                for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt, ++nrt) {
-                    if (!warp_wait(sdp_empty, (nrt & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int o = 0; o < pairs; ++o, ++op) {
-                        const uint32_t st = op % kBwdRing;
-                        if (!warp_wait(&full[st], (op / kBwdRing) & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        if (lane == 0) {
-                            const uint32_t a = ring + st * kBwdSlot, bb = a + kBwdSlab;
-                            const uint32_t d = tmem + (o < 8 ? kBwdTmS : kBwdTmP);
+            if (!warp_wait(acc_empty, (nitem & 1) ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt) {
+                for (int o = 0; o < 5; ++o)
+                    if (!warp_wait(&full[(op + o) % kBwdRing], ((op + o) / kBwdRing) & 1, abort_flag)) ok = false;
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t x = ring + (op % kBwdRing) * kBwdSlot;
+                    const bool first = rt == kk.rt_lo;
 #pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                mma_ss(d, smem_desc_sw128(a + q * 32, 16, 1024), smem_desc_sw128(bb + q * 32, 16, 1024),
-                                       id_s, ((o & 7) | q) ? 1u : 0u);
-                            mma_commit(&empty[st]);
-                        }
-                        __syncwarp();
-                    }
-                    if (!ok) break;
-                    if (lane == 0) mma_commit(sdp_full);
-                    __syncwarp();
-                    const bool first_rt = rt == kk.rt_lo;
-                    if (first_rt && !warp_wait(acc_empty, (npass & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    if (!warp_wait(x_full, nrt & 1, abort_flag)) { ok = false; break; }
-                    if (!warp_wait(&full[op % kBwdRing], (op / kBwdRing) & 1, abort_flag) ||
-                        !warp_wait(&full[(op + 1) % kBwdRing], ((op + 1) / kBwdRing) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (lane == 0) {
+                    for (int q = 0; q < 8; ++q) {
+                        const uint64_t ad = smem_desc_sw128(x + q * 2048, kBwdSlab, 1024);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const uint64_t ad = smem_desc_sw128(xs + (q >> 2) * kBwdSlab + (q & 3) * 32, 16, 1024);
-#pragma unroll
-                            for (int d = 0; d < 2; ++d)
-                                mma_ss(tmem + kBwdTmAcc + 128 * d, ad,
-                                       smem_desc_sw128(ring + ((op + d) % kBwdRing) * kBwdSlot + q * 2048, kBwdSlab, 1024),
-                                       id_a, (!first_rt || q) ? 1u : 0u);
-                        }
-                        mma_commit(&empty[op % kBwdRing]);
-                        mma_commit(&empty[(op + 1) % kBwdRing]);
-                        mma_commit(x_empty);
-                        if (rt == kk.rt_hi - 1) mma_commit(acc_full);
+                        for (int d = 0; d < 4; ++d)
+                            mma_ss(tmem + 128 * d, ad,
+                                   smem_desc_sw128(ring + ((op + 1 + d) % kBwdRing) * kBwdSlot + q * 2048, kBwdSlab, 1024),
+                                   id_a, (first && q == 0) ? 0u : 1u);
                     }
-                    __syncwarp();
-                    op += 2;
+                    for (int o = 0; o < 5; ++o) mma_commit(&empty[(op + o) % kBwdRing]);
+                    if (rt == kk.rt_hi - 1) mma_commit(acc_full);
                 }
+                __syncwarp();
+                op += 5;
             }
+            ++nitem;
         }
-        // every MMA has completed before the CTA releases its shared and tensor memory
         if (lane == 0) {
             mma_commit(drain);
             mbar_drain_wait(drain, 0);
         }
         __syncwarp();
     } else {
+        // ================================================================ epilogue: one key row per thread
         const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;              // key row of the tile
-        const int sidx = threadIdx.x - 64;         // 0..127: column (query row) this thread stages
+        const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        uint8_t* xsp = sm + kBwdSmX;
-        uint32_t nrt = 0, npass = 0;
-        bool ok = true;
-        for (long long i = blockIdx.x; ok && i < p.kv_items; i += stride) {
+        uint32_t nitem = 0;
+        for (long long i = blockIdx.x; i < p.kv_items; i += stride) {
             BwdKeys kk;
             if (!bwd_keys(p, i, kk)) continue;
-            const int key = kk.k0 + r;
+            if (!bwd_group_wait<128>(acc_full, nitem & 1, abort_flag)) break;
+            tc_fence_after();
             const bool key_live = r < kk.nk;
-            float4 nx = bwd_col(p, kk, kk.rt_lo, sidx);
-            for (int ps = 0; ok && ps < 4; ++ps, ++npass) {
-                const bool dkpass = ps >= 2;
-                for (int rt = kk.rt_lo; ok && rt < kk.rt_hi; ++rt, ++nrt) {
-                    bwd_bar();    // every thread is done with the previous row tile's columns
-                    colv[sidx] = nx;
-                    bwd_bar();
-                    // the next row tile's columns load while this one is computed
-                    nx = bwd_col(p, kk, rt + 1 < kk.rt_hi ? rt + 1 : kk.rt_lo, sidx);
-                    if (!bwd_group_wait(sdp_full, nrt & 1, abort_flag)) { ok = false; break; }
-                    if (!bwd_group_wait(x_empty, (nrt & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
+            const float mul = kk.which ? p.scale : 1.f;
+            float* base = kk.comp ? (kk.which ? p.dkc : p.dvc) : (kk.which ? p.dk : p.dv);
+            const size_t rows = kk.comp ? (size_t)p.Nc : (size_t)p.T;
+            float* dst = base + (((size_t)kk.b * rows + (key_live ? kk.k0 + r : 0)) * p.Hkv + kk.g) * kBwdD;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < 128; c0 += 16) {
-                        float sv[16], dpv[16];
-                        tmem_ld16(tmem + lane_off + kBwdTmS + c0, sv);
-                        if (dkpass) tmem_ld16(tmem + lane_off + kBwdTmP + c0, dpv);
-                        tmem_wait_ld();
-                        uint32_t pk[8];
+            for (int c0 = 0; c0 < kBwdD; c0 += 16) {
+                float a[16];
+                tmem_ld16(tmem + lane_off + c0, a);
+                tmem_wait_ld();
+                if (key_live)
 #pragma unroll
-                        for (int e = 0; e < 16; e += 2) {
-                            float x[2];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const float4 cd = colv[c0 + e + u];
-                                const bool vis = r >= __float_as_int(cd.z) && r < __float_as_int(cd.w);
-                                const float pr = vis ? ex2(fmaf(sv[e + u], p.scale_log2, -cd.x)) : 0.f;
-                                x[u] = dkpass ? pr * (dpv[e + u] - cd.y) : pr;
-                            }
-                            pk[e >> 1] = pack_bf16x2(x[0], x[1]);
-                        }
-                        bwd_put16(xsp, r, c0, pk);
-                    }
-                    tc_fence_before();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(sdp_empty);
-                        mbar_arrive(x_full);
-                    }
-                }
-                if (!ok) break;
-                // ---- the pass's half of dV (ps 0, 1) or dK (ps 2, 3), added to the key's gradient
-                if (!bwd_group_wait(acc_full, npass & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const float mul = dkpass ? p.scale : 1.f;
-                float* base = kk.comp ? (dkpass ? p.dkc : p.dvc) : (dkpass ? p.dk : p.dv);
-                const size_t rows = kk.comp ? (size_t)p.Nc : (size_t)p.T;
-                float* dst = base + (((size_t)kk.b * rows + (key_live ? key : 0)) * p.Hkv + kk.g) * kBwdD + 256 * (ps & 1);
-#pragma unroll 1
-                for (int c0 = 0; c0 < 256; c0 += 16) {
-                    float a[16];
-                    tmem_ld16(tmem + lane_off + kBwdTmAcc + c0, a);
-                    tmem_wait_ld();
-                    if (key_live)
-#pragma unroll
-                        for (int e = 0; e < 16; e += 4)
-                            atomicAdd(reinterpret_cast<float4*>(dst + c0 + e),
-                                      make_float4(mul * a[e], mul * a[e + 1], mul * a[e + 2], mul * a[e + 3]));
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                    for (int e = 0; e < 16; e += 4)
+                        atomicAdd(reinterpret_cast<float4*>(dst + c0 + e),
+                                  make_float4(mul * a[e], mul * a[e + 1], mul * a[e + 2], mul * a[e + 3]));
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            ++nitem;
         }
     }
     __syncwarp();

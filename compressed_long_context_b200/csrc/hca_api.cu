@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "append.cuh"
@@ -706,25 +707,54 @@ namespace {
 
 size_t bwd_align(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Bytes of P / dS records one segment may hold: the records of a segment are written by its dq
+// launch and read by its dk/dv launch, so this bounds the workspace whatever the length.
+constexpr size_t kBwdRecordCap = (size_t)2 << 30;
+
+// Row tiles per segment forced by hca_debug_set_backward_segment (0: from the cap).
+std::atomic<int> g_bwd_seg_rows{0};
+
 struct BwdLayout {
-    size_t drow, dkc, dvc, total;
+    int tpt, ntile, nkc, nkw, nt_max, seg;
+    size_t drow, dkc, dvc, rec, total;
 };
 
-BwdLayout bwd_layout(long long B, long long T, long long Hq, long long Hkv, long long blk) {
+BwdLayout bwd_layout(long long B, long long T, long long Hq, long long Hkv, long long blk, long long W) {
     BwdLayout l;
     const long long Nc = T / blk;
+    l.tpt = (int)(128 / (Hq / Hkv));
+    l.ntile = (int)((T + l.tpt - 1) / l.tpt);
+    l.nkc = (int)((Nc + 127) / 128);
+    l.nkw = (int)((T + 127) / 128);
+    // key tiles of one row tile: the entry tiles, then the 128-aligned raw tiles that hold the
+    // windows of its tpt tokens
+    const long long nwt = std::min<long long>((l.tpt + W - 2) / 128 + 2, l.nkw);
+    l.nt_max = (int)(l.nkc + nwt);
+    const long long per_row_tile = B * Hkv * (long long)l.nt_max * hca::kBwdRec;
+    l.seg = (int)std::max<long long>(1, std::min<long long>(l.ntile, (long long)(kBwdRecordCap / per_row_tile)));
+    const int forced = g_bwd_seg_rows.load();
+    if (forced > 0) l.seg = std::min(l.seg, forced);
     l.drow = 0;
     l.dkc = bwd_align((size_t)(B * T * Hq) * 4);
     l.dvc = l.dkc + bwd_align((size_t)(B * Nc * Hkv * hca::kBwdD) * 4);
-    l.total = l.dvc + bwd_align((size_t)(B * Nc * Hkv * hca::kBwdD) * 4);
+    l.rec = l.dvc + bwd_align((size_t)(B * Nc * Hkv * hca::kBwdD) * 4);
+    l.total = l.rec + (size_t)per_row_tile * l.seg;
     return l;
 }
 
 }  // namespace
 
-extern "C" size_t hca_prefill_backward_workspace_size(int B, int T, int Hq, int Hkv, int dv, int blk) {
-    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || dv != hca::kBwdD || blk < 1) return 0;
-    return bwd_layout(B, T, Hq, Hkv, blk).total;
+extern "C" hca_status_t hca_debug_set_backward_segment(int rows) {
+    if (rows < 0) return HCA_ERR_INVALID_ARG;
+    g_bwd_seg_rows.store(rows);
+    return HCA_OK;
+}
+
+extern "C" size_t hca_prefill_backward_workspace_size(int B, int T, int Hq, int Hkv, int dv, int blk, int W) {
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || dv != hca::kBwdD || blk < 1 || W < 1 || Hq % Hkv) return 0;
+    const int G = Hq / Hkv;
+    if (G > 128 || (G & (G - 1))) return 0;
+    return bwd_layout(B, T, Hq, Hkv, blk, W).total;
 }
 
 extern "C" hca_status_t hca_prefill_backward(const void* q, const void* k, const void* v, const float* w,
@@ -749,7 +779,7 @@ extern "C" hca_status_t hca_prefill_backward(const void* q, const void* k, const
         (reinterpret_cast<uintptr_t>(lse) & 3) || (w && (reinterpret_cast<uintptr_t>(w) & 3)) ||
         (dw && (reinterpret_cast<uintptr_t>(dw) & 3)) || (reinterpret_cast<uintptr_t>(workspace) & 255))
         return HCA_ERR_INVALID_ARG;
-    const BwdLayout lay = bwd_layout(B, T, Hq, Hkv, blk);
+    const BwdLayout lay = bwd_layout(B, T, Hq, Hkv, blk, W);
     if (workspace_bytes < lay.total) return HCA_ERR_INVALID_ARG;
     const int ns = num_sms();
     if (ns <= 0) return HCA_ERR_CUDA;
@@ -769,20 +799,18 @@ extern "C" hca_status_t hca_prefill_backward(const void* q, const void* k, const
     p.dkc = reinterpret_cast<float*>(ws + lay.dkc);
     p.dvc = reinterpret_cast<float*>(ws + lay.dvc);
     p.dw = dw;
-    p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.tpt = 128 / G; p.blk = blk; p.W = W; p.Nc = Nc;
-    p.ntile_t = (T + p.tpt - 1) / p.tpt;
+    p.rec = reinterpret_cast<uint8_t*>(ws + lay.rec);
+    p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.tpt = lay.tpt; p.blk = blk; p.W = W; p.Nc = Nc;
+    p.ntile_t = lay.ntile;
     p.out_f32 = (flags & HCA_OUT_F32) ? 1 : 0;
-    p.dq_items = (long long)B * Hkv * p.ntile_t;
-    p.nkc = (Nc + 127) / 128;
-    p.nkw = (T + 127) / 128;
-    // query row tiles a raw key tile reaches: tokens k0 .. k0 + 127 + W - 1
-    const long long span_w = (std::min<long long>((long long)T, 128LL + W - 1) + p.tpt - 1) / p.tpt + 1;
-    const long long visits = (long long)B * Hkv * ((long long)p.nkc * p.ntile_t + (long long)p.nkw * span_w);
-    const long long chunk = std::max<long long>(1, (visits + 4LL * ns - 1) / (4LL * ns));
-    p.rt_chunk = (int)std::min<long long>(chunk, p.ntile_t);
-    p.chc = (p.ntile_t + p.rt_chunk - 1) / p.rt_chunk;
-    p.chw = (int)((span_w + p.rt_chunk - 1) / p.rt_chunk);
-    p.kv_items = (long long)B * Hkv * ((long long)p.nkc * p.chc + (long long)p.nkw * p.chw);
+    p.nkc = lay.nkc;
+    p.nkw = lay.nkw;
+    p.nt_max = lay.nt_max;
+    p.seg = lay.seg;
+    // row tiles per item of an entry tile: about the rows a raw key tile reaches, so that items
+    // are of similar length
+    const int raw_span = (127 + W - 1) / p.tpt + 2;
+    p.ch_rows = std::max(16, std::min(128, raw_span));
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
 
@@ -808,11 +836,21 @@ extern "C" hca_status_t hca_prefill_backward(const void* q, const void* k, const
     const long long rows = (long long)B * T * Hq;
     const long long pre_grid = std::min<long long>((rows + 7) / 8, 8LL * ns);
     bwd_pre_kernel<<<(unsigned)pre_grid, 256, 0, s>>>(p);
-    bwd_dq_kernel<<<(unsigned)std::min<long long>(p.dq_items, ns), kBwdThreads, kBwdSmem, s>>>(p, tq, tdo, tk, tv, tkc,
-                                                                                               tvc);
-    if (p.kv_items > 0)
-        bwd_dkv_kernel<<<(unsigned)std::min<long long>(p.kv_items, ns), kBwdThreads, kBwdSmem, s>>>(p, tq, tdo, tk, tv,
-                                                                                                    tkc, tvc);
+    for (int s0 = 0; s0 < p.ntile_t; s0 += p.seg) {
+        p.s0 = s0;
+        p.s1 = std::min(p.ntile_t, s0 + p.seg);
+        p.dq_items = (long long)B * Hkv * (p.s1 - s0);
+        p.nch = (p.s1 - s0 + p.ch_rows - 1) / p.ch_rows;
+        const long long num = (long long)s0 * p.tpt - 126 - W;
+        p.kta = num > 0 ? (int)(num / 128) : 0;
+        const int ktb = std::min(p.nkw - 1, (int)(((long long)p.s1 * p.tpt - 1) / 128));
+        p.nraw = std::max(0, ktb - p.kta + 1);
+        p.kv_items = (long long)B * Hkv * (2LL * p.nkc * p.nch + 2LL * p.nraw);
+        bwd_dq_kernel<<<(unsigned)std::min<long long>(p.dq_items, ns), kDqThreads, kBwdSmem, s>>>(p, tq, tdo, tk, tv,
+                                                                                                  tkc, tvc);
+        if (p.kv_items > 0)
+            bwd_dkv_kernel<<<(unsigned)std::min<long long>(p.kv_items, ns), kKvThreads, kBwdSmem, s>>>(p, tq, tdo);
+    }
     if (Nc > 0) bwd_pool_kernel<<<(unsigned)((long long)B * Nc), kPoolThreads, 0, s>>>(p);
     return launch_status();
 }

@@ -111,9 +111,11 @@ hca_status_t hca_prefill(const void* q, const void* k, const void* v,
 
 /*
  * hca_prefill_backward_workspace_size -- bytes of device workspace hca_prefill_backward
- * needs (per-row softmax terms and the entries' gradients).  Returns 0 for invalid sizes.
+ * needs: per-row softmax terms, the entries' gradients, and the bf16 P / dS tiles of one
+ * segment of row tiles (at most about 2 GiB; the call walks the sequence segment by
+ * segment).  Returns 0 for invalid or unsupported sizes.
  */
-size_t hca_prefill_backward_workspace_size(int B, int T, int Hq, int Hkv, int dv, int blk);
+size_t hca_prefill_backward_workspace_size(int B, int T, int Hq, int Hkv, int dv, int blk, int W);
 
 /*
  * hca_prefill_backward -- gradients of the HCA layer for training: the gradient of
@@ -328,6 +330,15 @@ const char* hca_status_string(hca_status_t status);
  * merging split records that a timed-out kernel may have left incomplete.
  */
 hca_status_t hca_get_device_error(hca_stream_t stream);
+
+/*
+ * hca_debug_set_backward_segment -- test hook: hca_prefill_backward (and its workspace size)
+ * processes at most `rows` row tiles per segment, so that short sequences exercise the
+ * segment walk that long ones take; 0 restores the default (segments sized by a 2 GiB bound
+ * on the P / dS records).  Process-wide; call it only while no backward is being enqueued.
+ * HCA_ERR_INVALID_ARG for rows < 0.
+ */
+hca_status_t hca_debug_set_backward_segment(int rows);
 
 /*
  * Test hooks for the bounded waits (not part of the computation; the paper has no

@@ -183,10 +183,22 @@ def test_prefill_backward_rejects_before_launch(libhca):
         return libhca.hca_prefill_backward(q, k, v, w, kc, vc, out, lse, dout, dq, dk, dv, dw, ws, ws_bytes,
                                            B, T, Hq, Hkv, d, dvd, blk, W, scale, flags, None)
 
-    # workspace: per-row terms plus the entries' fp32 gradients, 256-byte aligned pieces
-    assert libhca.hca_prefill_backward_workspace_size(1, 1024, 64, 1, 512, 128) == 1024 * 64 * 4 + 2 * 8 * 512 * 4
-    assert libhca.hca_prefill_backward_workspace_size(1, 1024, 64, 1, 64, 128) == 0
-    assert libhca.hca_prefill_backward_workspace_size(-1, 1024, 64, 1, 512, 128) == 0
+    # workspace: per-row terms, the entries' fp32 gradients, then 64 KB P / dS records for
+    # every (row tile, key tile slot) of a segment: 512 row tiles of 2 tokens, one entry tile and
+    # up to three 128-aligned raw tiles each
+    assert libhca.hca_prefill_backward_workspace_size(1, 1024, 64, 1, 512, 128, 128) == (
+        1024 * 64 * 4 + 2 * 8 * 512 * 4 + 512 * 4 * 65536)
+    assert libhca.hca_prefill_backward_workspace_size(1, 1024, 64, 1, 64, 128, 128) == 0
+    assert libhca.hca_prefill_backward_workspace_size(-1, 1024, 64, 1, 512, 128, 128) == 0
+    assert libhca.hca_prefill_backward_workspace_size(1, 1024, 48, 1, 512, 128, 128) == 0
+    # a forced segment of 7 row tiles bounds the records to 7 row tiles
+    assert libhca.hca_debug_set_backward_segment(7) == _lib.HCA_OK
+    try:
+        assert libhca.hca_prefill_backward_workspace_size(1, 1024, 64, 1, 512, 128, 128) == (
+            1024 * 64 * 4 + 2 * 8 * 512 * 4 + 7 * 4 * 65536)
+    finally:
+        assert libhca.hca_debug_set_backward_segment(0) == _lib.HCA_OK
+    assert libhca.hca_debug_set_backward_segment(-1) == _lib.HCA_ERR_INVALID_ARG
     # unsupported head dims, block, group size, flags
     assert call(d=64, dvd=64) == _lib.HCA_ERR_UNSUPPORTED
     assert call(blk=129) == _lib.HCA_ERR_UNSUPPORTED

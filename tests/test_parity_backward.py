@@ -138,3 +138,17 @@ def test_backward_rejects_unsupported(cuda_device, libhca):
     out, lse = hca.prefill(q, k, v, kc, vc, 128, 128, 0.05, want_lse=True)
     with pytest.raises(hca.HCAError):
         hca.prefill_backward(q, k, v, w, kc, vc, out, lse, dout, 256, 128, 0.05)   # blk > 128
+
+
+@pytest.mark.parametrize("seg,B,T,Hq,Hkv,blk,W", [
+    (5, 1, 640, 64, 1, 128, 128),
+    (3, 2, 1000, 16, 2, 32, 200),
+])
+def test_backward_segments(cuda_device, libhca, seg, B, T, Hq, Hkv, blk, W):
+    """Long sequences are processed in segments of row tiles (the P / dS records of one segment
+    at a time); forcing a few row tiles per segment walks the same path on a short sequence."""
+    assert libhca.hca_debug_set_backward_segment(seg) == 0
+    try:
+        run_case(cuda_device, B, T, Hq, Hkv, blk, W, seed=7 * T + seg)
+    finally:
+        assert libhca.hca_debug_set_backward_segment(0) == 0
