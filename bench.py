@@ -636,6 +636,7 @@ def bench_prefill_128k(c):
     res["vha"] = {"ms": tv * 1e3, "rank": 8, "algorithmic_bytes": vbytes,
                   "roofline": c.hbm_roof("vha_kernel<false,8>", vbytes, tv)}
     del vout
+    res["backward"] = bench_backward_128k(c, pc, pin, pkc, pvc, scale, flops, keys, n)
     if c.oracle_on:
         import oracle
         T = pc.T
@@ -670,6 +671,109 @@ def bench_prefill_128k(c):
         res["parity"] = dict(e, cache_max_abs_err=ek["max_abs_err"], bf16_within_bar_plus_half_ulp=ok_bf16,
                              within_tolerance=ok_bf16 and e["mean_abs_err"] <= 1e-3 and ek["max_abs_err"] <= 4e-3)
     del pin, pkc, pvc, pout
+    torch.cuda.empty_cache()
+    return res
+
+
+class RowsF64:
+    """Read-only fp64 view of a bf16 device tensor, converted on indexing, so that the oracle's
+    row-by-row reads of a 128K-token input need no host copy of the whole tensor."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, idx):
+        import oracle
+        return oracle.bits_to_f64(oracle.bf16_bits(self.t[idx]))
+
+
+def backward_segments(B, T, Hq, Hkv, blk, W, cap=2 << 30):
+    """Segments of row tiles hca_prefill_backward walks (each one dq and one dk/dv launch)."""
+    tpt = 128 // (Hq // Hkv)
+    ntile = (T + tpt - 1) // tpt
+    nkc, nkw = (T // blk + 127) // 128, (T + 127) // 128
+    nt_max = nkc + min((tpt + W - 2) // 128 + 2, nkw)
+    seg = max(1, min(ntile, cap // (B * Hkv * nt_max * 65536)))
+    return (ntile + seg - 1) // seg
+
+
+def bench_backward_128k(c, pc, pin, pkc, pvc, scale, fwd_flops, keys, n):
+    """Training step of the prefill workload: hca_prefill with the log-sum-exp, then
+    hca_prefill_backward (dq, dk, dv, dw) for a synthetic dout."""
+    hca = c.hca
+    g = torch.Generator(device=c.dev).manual_seed(9)
+    dout = torch.empty_like(pin["q"])
+    flat = dout.view(-1)
+    for i in range(0, flat.numel(), 1 << 28):
+        m = min(1 << 28, flat.numel() - i)
+        flat[i:i + m] = torch.randn(m, generator=g, device=c.dev).to(torch.bfloat16)
+    # the forward output in fp32: D = rowsum(dout * out) then carries no bf16 rounding of out, which
+    # rows dominated by one key (the boosted ones) would turn into a large relative error of dS
+    out, lse = hca.prefill(pin["q"], pin["k"], pin["v"], pkc, pvc, pc.blk, pc.W, scale, want_lse=True,
+                           out_f32=True)
+    grads = {}
+
+    def bwd():
+        grads["g"] = hca.prefill_backward(pin["q"], pin["k"], pin["v"], pin["w"], pkc, pvc, out, lse, dout,
+                                          pc.blk, pc.W, scale)
+
+    for _ in range(2):
+        bwd()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    b_ms = timed_calls(bwd, n, c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    tb = c.median_s(b_ms)
+    # five contractions of the forward's size: S, dP, dq, dk, dv (2.5x the forward's flops)
+    flops = 2.5 * fwd_flops
+    tf = flops / tb / 1e12
+    burst = c.pk["bf16_tflops"]
+    res = {"what": "hca_prefill_backward: dq, dk, dv, dw of the prefill workload (forward output fp32, "
+                   "its LSE, synthetic bf16 dout)",
+           "ms": tb * 1e3, "tflops": tf, "algorithmic_flops": flops,
+           "flops_per_row_key": 5 * 2 * pc.Hq * pc.d,
+           "roofline": {"bound": "tensor", "kernel": "bwd_dq_kernel + bwd_dkv_kernel", "achieved": tf,
+                        "peak": burst, "unit": "TFLOP/s", "frac": tf / burst,
+                        "peak_kind": c.pk_kind + " (bf16_tflops, burst)", "traffic": None}}
+    from compressed_long_context_b200 import _lib
+    res["workspace_bytes"] = int(_lib.load().hca_prefill_backward_workspace_size(1, pc.T, pc.Hq, pc.Hkv, pc.dv,
+                                                                                  pc.blk, pc.W))
+    res["launches_per_call"] = 2 + 2 * backward_segments(1, pc.T, pc.Hq, pc.Hkv, pc.blk, pc.W)
+    if c.oracle_on:
+        from oracle import backward as ob
+        import oracle
+        T, blk, W = pc.T, pc.blk, pc.W
+        Nc = T // blk
+        rows = [0, 127, 128, 255, 16511, 16512, 65537, T - 2, T - 1]
+        raw = [blk * (Nc - 3), blk * (Nc - 3) + 77, T - 128, T - 1]
+        tm = OracleTimer()
+        f64 = lambda t: oracle.bits_to_f64(oracle.bf16_bits(t))  # noqa: E731
+        # q and dout are widened row by row on access (the oracle reads one (t, h) row at a time)
+        qn, don = RowsF64(pin["q"]), RowsF64(dout)
+        kn, vn = f64(pin["k"]), f64(pin["v"])
+        ref = tm(ob.backward_sampled, qn, kn, vn, pin["w"].cpu().numpy(), blk, W, scale, don, 0, rows=rows, raw=raw)
+        dq, dk, dv, dw = grads["g"]
+
+        def rel(got, r):
+            g64 = got.double().cpu().numpy()
+            return float(np.sqrt(((g64 - r) ** 2).sum() / max((r ** 2).sum(), 1e-300))), \
+                float(np.abs(g64 - r).max() / max(np.abs(r).max(), 1e-300))
+
+        out_rel = {}
+        for name, got, r in (("dq", dq[0, rows], np.stack([ref["dq"][t] for t in rows])),
+                             ("dk", dk[0, raw], np.stack([ref["dk"][u] for u in raw])),
+                             ("dv", dv[0, raw], np.stack([ref["dv"][u] for u in raw]))):
+            nr, mr = rel(got, r)
+            out_rel[name] = {"normwise_rel_err": nr, "max_err_over_max_ref": mr}
+        ok = all(v["normwise_rel_err"] <= 2 ** -7 and v["max_err_over_max_ref"] <= 2 ** -5 for v in out_rel.values())
+        res["oracle"] = {"seconds": tm.s, "rows": len(rows), "raw_positions": len(raw), "cores": oracle.num_threads(),
+                         "scope": "oracle.backward.backward_sampled: dq of %d query positions, dk/dv of %d raw "
+                                  "positions (window path, and the pooling path of a late block)" % (len(rows), len(raw))}
+        res["parity"] = dict(out_rel, within_tolerance=ok,
+                             bar="normwise <= 2^-7 and max <= 2^-5 of the largest reference value")
+        del qn, kn, vn, don
+    del dout, out, lse, grads
     torch.cuda.empty_cache()
     return res
 

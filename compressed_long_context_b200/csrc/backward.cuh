@@ -174,6 +174,24 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     }
 }
 
+// One K-step (16 rows of the contraction, step kk) of D[:, 0:512] += A B, B being 512 channels held
+// as four ops of two 64-channel blocks in ring slots op0 .. op0 + 3: a pair of ops in adjacent
+// slots is one N = 256 operand (blocks 16 KB apart), otherwise two N = 128 operands.
+__device__ __forceinline__ void bwd_mma_blocks(uint32_t tmem, uint64_t ad, uint32_t ring, uint32_t op0, int kk,
+                                               uint32_t id_n128, uint32_t id_n256, uint32_t acc) {
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+        const uint32_t sa = (op0 + 2 * pr) % kBwdRing, sb = (op0 + 2 * pr + 1) % kBwdRing;
+        const uint32_t ba = ring + sa * kBwdSlot + kk * 2048, bb = ring + sb * kBwdSlot + kk * 2048;
+        if (sb == sa + 1) {
+            mma_ss(tmem + 256 * pr, ad, smem_desc_sw128(ba, kBwdSlab, 1024), id_n256, acc);
+        } else {
+            mma_ss(tmem + 256 * pr, ad, smem_desc_sw128(ba, kBwdSlab, 1024), id_n128, acc);
+            mma_ss(tmem + 256 * pr + 128, ad, smem_desc_sw128(bb, kBwdSlab, 1024), id_n128, acc);
+        }
+    }
+}
+
 // -------------------------------------------------------------------------------- dq
 
 // Phase S ops of a key tile: 8 x (Q slab, K slab) for S, then 8 x (dO slab, V slab) for dP.
@@ -286,7 +304,7 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_a = idesc_bf16(128, 128, 0, 1);
+        const uint32_t id_a = idesc_bf16(128, 128, 0, 1), id_a2 = idesc_bf16(128, 256, 0, 1);
         const uint32_t ring = smem_u32(sm + kBwdSmRing);
         uint32_t op = 0, ns = 0, nitem = 0;
         bool ok = true;
@@ -334,14 +352,10 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t ds = ring + (op % kBwdRing) * kBwdSlot;
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint64_t ad = smem_desc_sw128(ds + (kk >> 2) * kBwdSlab + (kk & 3) * 32, 16, 1024);
-#pragma unroll
-                        for (int d = 0; d < 4; ++d)
-                            mma_ss(tmem + 128 * d, ad,
-                                   smem_desc_sw128(ring + ((op + 1 + d) % kBwdRing) * kBwdSlot + kk * 2048, kBwdSlab, 1024),
-                                   id_a, (j | kk) ? 1u : 0u);
+                        bwd_mma_blocks(tmem, ad, ring, op + 1, kk, id_a, id_a2, (j | kk) ? 1u : 0u);
                     }
                     for (int o = 0; o < 5; ++o) mma_commit(&empty[(op + o) % kBwdRing]);
                     if (j == it.nt - 1) mma_commit(acc_full);
@@ -578,7 +592,7 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
     } else if (warp == 1) {
         // D[key, channel] += sum over the tile's 128 query rows of X[row, key] Y[row, channel]:
         // A = the record's tile read MN-major (keys contiguous), B = dO / Q MN-major
-        const uint32_t id_a = idesc_bf16(128, 128, 1, 1);
+        const uint32_t id_a = idesc_bf16(128, 128, 1, 1), id_a2 = idesc_bf16(128, 256, 1, 1);
         const uint32_t ring = smem_u32(sm + kBwdSmRing);
         uint32_t op = 0, nitem = 0;
         bool ok = true;
@@ -595,15 +609,10 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
                 if (lane == 0) {
                     const uint32_t x = ring + (op % kBwdRing) * kBwdSlot;
                     const bool first = rt == kk.rt_lo;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint64_t ad = smem_desc_sw128(x + q * 2048, kBwdSlab, 1024);
-#pragma unroll
-                        for (int d = 0; d < 4; ++d)
-                            mma_ss(tmem + 128 * d, ad,
-                                   smem_desc_sw128(ring + ((op + 1 + d) % kBwdRing) * kBwdSlot + q * 2048, kBwdSlab, 1024),
-                                   id_a, (first && q == 0) ? 0u : 1u);
-                    }
+#pragma unroll 1
+                    for (int q = 0; q < 8; ++q)
+                        bwd_mma_blocks(tmem, smem_desc_sw128(x + q * 2048, kBwdSlab, 1024), ring, op + 1, q, id_a, id_a2,
+                                       (first && q == 0) ? 0u : 1u);
                     for (int o = 0; o < 5; ++o) mma_commit(&empty[(op + o) % kBwdRing]);
                     if (rt == kk.rt_hi - 1) mma_commit(acc_full);
                 }

@@ -7,6 +7,7 @@
     python -m compressed_long_context_b200.profile_cases vha      [--reps N]
     python -m compressed_long_context_b200.profile_cases append   [--reps N]
     python -m compressed_long_context_b200.profile_cases gate     [--reps N]
+    python -m compressed_long_context_b200.profile_cases backward [--reps N] [--T tokens]
 
 Each case keeps its working set larger than the 126 MB L2 (so DRAM counters mean
 something) but a few GB at most, and launches the kernel `--reps` times after one
@@ -20,7 +21,7 @@ import math
 import torch
 
 from . import (append, append_state_size, compress, decode, decode_workspace_size, gate_logits, get_device_error,
-               prefill, vha)
+               prefill, prefill_backward, vha)
 from . import workloads as wl
 
 
@@ -115,6 +116,19 @@ def run(case: str, reps: int, B_override: int = 0, L_override: int = 0, T_overri
         gate = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
         fn = lambda: gate_logits(cq, wg, out=gate)  # noqa: E731
         nbytes = (cq.numel() + wg.numel() + gate.numel()) * 2
+    elif case == "backward":
+        # default T = 8192 tokens, 64 heads of 512: 512 MB each of Q, dO and the bf16 output
+        cfg = wl.PREFILL_128K.scaled(T=T_override or 8192)
+        inp = wl.prefill_inputs(cfg, dev)
+        kc, vc = compress(inp["k"], inp["v"], inp["w"], 128)
+        sc = 1 / math.sqrt(cfg.d)
+        out, lse = prefill(inp["q"], inp["k"], inp["v"], kc, vc, 128, cfg.W, sc, want_lse=True)
+        dout = torch.randn(inp["q"].shape, generator=g, device=dev).to(torch.bfloat16)
+        fn = lambda: prefill_backward(inp["q"], inp["k"], inp["v"], inp["w"], kc, vc, out, lse,  # noqa: E731
+                                      dout, 128, cfg.W, sc)
+        keys = sum(max(0, (t - cfg.W + 1) // 128) + min(cfg.W, t + 1) for t in range(cfg.T))
+        nbytes = None
+        flops = 5 * 2.0 * cfg.Hq * keys * cfg.d
     else:
         raise ValueError(case)
     _last_fn[0] = fn
@@ -135,7 +149,7 @@ def run(case: str, reps: int, B_override: int = 0, L_override: int = 0, T_overri
     if nbytes:
         res["bytes"] = nbytes
         res["GB_per_s"] = nbytes / (ms / 1e3) / 1e9
-    if case == "prefill":
+    if case in ("prefill", "backward"):
         res["T"] = cfg.T
         res["TFLOP_per_s"] = flops / (ms / 1e3) / 1e12
     return res
@@ -167,11 +181,11 @@ def run_flushed(args) -> dict:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["compress", "decode", "paged", "prefill", "vha", "append", "gate"])
+    ap.add_argument("case", choices=["compress", "decode", "paged", "prefill", "vha", "append", "gate", "backward"])
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--B", type=int, default=0, help="decode batch (default 64)")
     ap.add_argument("--L", type=int, default=0, help="decode context length (default 131072)")
-    ap.add_argument("--T", type=int, default=0, help="prefill tokens (default 16384)")
+    ap.add_argument("--T", type=int, default=0, help="prefill tokens (default 16384; backward 8192)")
     ap.add_argument("--flush", action="store_true", help="flush L2 before every launch (events per launch)")
     args = ap.parse_args()
     print(json.dumps(run(args.case, args.reps, args.B, args.L, args.T) if not args.flush else run_flushed(args)))

@@ -51,11 +51,14 @@ def check(got, ref, what):
     assert err.max() <= MAX_TOL * scale, (what, "max", err.max(), scale)
 
 
-def inputs(dev, B, T, Hq, Hkv, seed, wstd=0.5, zero_w=False):
+def inputs(dev, B, T, Hq, Hkv, seed, wstd=0.5, zero_w=False, boost=0):
     g = torch.Generator(device=dev).manual_seed(seed)
     d = 512
     q = torch.randn((B, T, Hq, d), generator=g, device=dev).to(torch.bfloat16)
     k = torch.randn((B, T, Hkv, d), generator=g, device=dev).to(torch.bfloat16)
+    if boost:
+        # every boost-th raw key row times 8 (exact in bf16): softmax rows dominated by one key
+        k[:, ::boost] = (k[:, ::boost].float() * 8).to(torch.bfloat16)
     v = torch.randn((B, T, Hkv, d), generator=g, device=dev).to(torch.bfloat16)
     w = None if zero_w else torch.randn((B, T), generator=g, device=dev) * wstd
     dout = torch.randn((B, T, Hq, d), generator=g, device=dev).to(torch.bfloat16)
@@ -81,8 +84,8 @@ def oracle_grads(q, k, v, w, dout, blk, W, scale):
     return dq, dk_w + dk_p, dv_w + dv_p, dw
 
 
-def run_case(dev, B, T, Hq, Hkv, blk, W, seed, out_f32=True, wstd=0.5, zero_w=False):
-    q, k, v, w, dout = inputs(dev, B, T, Hq, Hkv, seed, wstd, zero_w)
+def run_case(dev, B, T, Hq, Hkv, blk, W, seed, out_f32=True, wstd=0.5, zero_w=False, boost=0):
+    q, k, v, w, dout = inputs(dev, B, T, Hq, Hkv, seed, wstd, zero_w, boost)
     scale = 1.0 / np.sqrt(512)
     got = gpu_grads(q, k, v, w, dout, blk, W, scale, out_f32)
     ref = oracle_grads(q, k, v, w, dout, blk, W, scale)
@@ -99,6 +102,12 @@ def run_case(dev, B, T, Hq, Hkv, blk, W, seed, out_f32=True, wstd=0.5, zero_w=Fa
 ])
 def test_backward_d512(cuda_device, libhca, B, T, Hq, Hkv, blk, W):
     run_case(cuda_device, B, T, Hq, Hkv, blk, W, seed=3 * T + Hq, out_f32=(T % 2 == 0))
+
+
+def test_backward_boosted_keys(cuda_device, libhca):
+    """One raw key in 97 scaled by 8 (the prefill workload's boosted keys): rows whose softmax
+    one key dominates, where dS = P (dP - D) cancels; fp32 forward output."""
+    run_case(cuda_device, 1, 1000, 64, 1, 128, 128, seed=41, out_f32=True, boost=97)
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,blk,W,zero_w", [
