@@ -47,7 +47,9 @@ constexpr uint32_t kBwdSlab = 16384;         // 128 rows x 64 columns bf16, 128-
 constexpr uint32_t kBwdSlot = 2 * kBwdSlab;  // two slabs
 constexpr uint32_t kBwdRec = 2 * kBwdSlot;   // one (row tile, key tile) record: P, then dS
 constexpr uint32_t kBwdSmRing = 0;
-constexpr uint32_t kBwdSmBar = kBwdSmRing + kBwdRing * kBwdSlot;
+constexpr uint32_t kBwdSmStage = kBwdSmRing + kBwdRing * kBwdSlot;   // 4 KB per softmax / epilogue warp
+constexpr uint32_t kBwdStageBytes = 4096;
+constexpr uint32_t kBwdSmBar = kBwdSmStage + 8 * kBwdStageBytes;
 constexpr int kBwdNumBars = 2 * kBwdRing + 12;
 constexpr uint32_t kBwdSmMisc = kBwdSmBar + kBwdNumBars * 8;
 constexpr uint32_t kBwdSmem = kBwdSmMisc + 16;
@@ -121,6 +123,45 @@ __device__ __forceinline__ bool bwd_group_wait(uint64_t* bar, uint32_t parity, v
 
 // Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled slab.
 __device__ __forceinline__ uint32_t bwd_sw(uint32_t r, uint32_t c) { return r * 128u + (((c ^ r) & 7u) << 4); }
+
+// A warp's 32 rows x 128 bytes of a record (rows 32 q .. 32 q + 31 of a slab: 4 KB, contiguous in
+// the record), lane = row: written through the warp's staging buffer so that every global store
+// instruction covers four whole 128-byte lines (a store per lane and row would touch 32 lines).
+// v holds the row's eight 16-byte chunks in column order; the record keeps the slab's swizzle.
+__device__ __forceinline__ void bwd_warp_rows_out(uint8_t* stg, uint8_t* dst, const uint32_t* v, int lane) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(stg + bwd_sw(lane, c)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<uint4*>(dst + i * 512 + lane * 16) = *reinterpret_cast<const uint4*>(stg + i * 512 + lane * 16);
+    __syncwarp();
+}
+
+// 32 consecutive fp32 channels of each of a warp's 32 rows (lane = row, v = its 32 values) to
+// row-major global rows, through the staging buffer: lane l then writes 16 bytes of row
+// 4 i + l / 8, so each instruction covers four whole 128-byte lines.  row_ptr(i) gives the
+// destination of the warp's row i (null: skip the row); kAtomic adds with fp32 vector atomics.
+template <bool kAtomic, class RowPtr>
+__device__ __forceinline__ void bwd_warp_f32_out(uint8_t* stg, const float* v, int lane, RowPtr row_ptr) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(stg + bwd_sw(lane, c)) = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    __syncwarp();
+    const int k = lane & 7;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int row = 4 * i + (lane >> 3);
+        float* d = row_ptr(row);
+        const float4 x = *reinterpret_cast<const float4*>(stg + bwd_sw(row, k));
+        if (d) {
+            if (kAtomic) atomicAdd(reinterpret_cast<float4*>(d + 4 * k), x);
+            else *reinterpret_cast<float4*>(d + 4 * k) = x;
+        }
+    }
+    __syncwarp();
+}
 
 // -------------------------------------------------------------------------------- D = rowsum(dO O)
 
@@ -376,6 +417,7 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
         const int hc = (warp - 2) >> 2;           // column half
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        uint8_t* stg = sm + kBwdSmStage + (warp - 2) * kBwdStageBytes;
         uint32_t ns = 0, nitem = 0;
         bool ok = true;
         for (long long i = blockIdx.x; ok && i < p.dq_items; i += stride, ++nitem) {
@@ -403,8 +445,12 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
                     hi = min(128, t - u0 + 1);
                 }
                 if (!live) hi = lo;
-                uint8_t* rp = bwd_record(p, b, g, rt, j) + hc * kBwdSlab;
-#pragma unroll 1
+                // this warp's 32 rows of slab hc: 4 KB, contiguous in the record
+                uint8_t* rp = bwd_record(p, b, g, rt, j) + hc * kBwdSlab + q4 * 32 * 128;
+                // P goes straight into the staging buffer (the row's chunks at their swizzled
+                // places), dS stays in registers until P is out
+                uint32_t pd[32];
+#pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     const int c0 = 64 * hc + 32 * h2;
                     float sv[32], dpv[32];
@@ -414,26 +460,29 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
                     tmem_ld16(tb + 128, dpv);
                     tmem_ld16(tb + 144, dpv + 16);
                     tmem_wait_ld();
-                    uint32_t pp[16], pd[16];
+                    uint32_t pp[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int c = c0 + e;
                         const float p0 = (c >= lo && c < hi) ? ex2(fmaf(sv[e], p.scale_log2, -lse2)) : 0.f;
                         const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2(fmaf(sv[e + 1], p.scale_log2, -lse2)) : 0.f;
                         pp[e >> 1] = pack_bf16x2(p0, p1);
-                        pd[e >> 1] = pack_bf16x2(p0 * (dpv[e] - Dr), p1 * (dpv[e + 1] - Dr));
+                        pd[16 * h2 + (e >> 1)] = pack_bf16x2(p0 * (dpv[e] - Dr), p1 * (dpv[e + 1] - Dr));
                     }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t off = bwd_sw(r, 4 * h2 + q);
-                        *reinterpret_cast<uint4*>(rp + off) = make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
-                        *reinterpret_cast<uint4*>(rp + kBwdSlot + off) =
-                            make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
-                    }
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4*>(stg + bwd_sw(lane, 4 * h2 + q)) =
+                            make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
                 }
+                // S and dP are read: the MMAs of the tile after next may use the buffer
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sdp_empty[buf]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<uint4*>(rp + i * 512 + lane * 16) = *reinterpret_cast<const uint4*>(stg + i * 512 + lane * 16);
+                __syncwarp();
+                bwd_warp_rows_out(stg, rp + kBwdSlot, pd, lane);
             }
             if (!ok) break;
             // the records are complete: hand them to the async proxy (the producer's bulk loads)
@@ -443,17 +492,21 @@ bwd_dq_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, const
             // ---- dq = scale * accumulator, channels 256 hc ..
             if (!bwd_group_wait<256>(acc_full, nitem & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            float* dst = p.dq + (((size_t)b * p.T + t) * p.Hq + head) * kBwdD + 256 * hc;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 16) {
-                float a[16];
+            for (int c0 = 0; c0 < 256; c0 += 32) {
+                float a[32];
                 tmem_ld16(tmem + lane_off + 256 * hc + c0, a);
+                tmem_ld16(tmem + lane_off + 256 * hc + c0 + 16, a + 16);
                 tmem_wait_ld();
-                if (live)
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *reinterpret_cast<float4*>(dst + c0 + e) =
-                            make_float4(p.scale * a[e], p.scale * a[e + 1], p.scale * a[e + 2], p.scale * a[e + 3]);
+                for (int e = 0; e < 32; ++e) a[e] *= p.scale;
+                const int ch = 256 * hc + c0;
+                bwd_warp_f32_out<false>(stg, a, lane, [&](int row) -> float* {
+                    const int rr = q4 * 32 + row;
+                    const int tk = it.t0 + rr / p.G;
+                    if (tk >= p.T) return nullptr;
+                    return p.dq + (((size_t)b * p.T + tk) * p.Hq + g * p.G + rr % p.G) * kBwdD + ch;
+                });
             }
             tc_fence_before();
             __syncwarp();
@@ -629,29 +682,30 @@ bwd_dkv_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tm_q, cons
     } else {
         // ================================================================ epilogue: one key row per thread
         const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        uint8_t* stg = sm + kBwdSmStage + (warp - 2) * kBwdStageBytes;
         uint32_t nitem = 0;
         for (long long i = blockIdx.x; i < p.kv_items; i += stride) {
             BwdKeys kk;
             if (!bwd_keys(p, i, kk)) continue;
             if (!bwd_group_wait<128>(acc_full, nitem & 1, abort_flag)) break;
             tc_fence_after();
-            const bool key_live = r < kk.nk;
             const float mul = kk.which ? p.scale : 1.f;
             float* base = kk.comp ? (kk.which ? p.dkc : p.dvc) : (kk.which ? p.dk : p.dv);
             const size_t rows = kk.comp ? (size_t)p.Nc : (size_t)p.T;
-            float* dst = base + (((size_t)kk.b * rows + (key_live ? kk.k0 + r : 0)) * p.Hkv + kk.g) * kBwdD;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kBwdD; c0 += 16) {
-                float a[16];
+            for (int c0 = 0; c0 < kBwdD; c0 += 32) {
+                float a[32];
                 tmem_ld16(tmem + lane_off + c0, a);
+                tmem_ld16(tmem + lane_off + c0 + 16, a + 16);
                 tmem_wait_ld();
-                if (key_live)
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        atomicAdd(reinterpret_cast<float4*>(dst + c0 + e),
-                                  make_float4(mul * a[e], mul * a[e + 1], mul * a[e + 2], mul * a[e + 3]));
+                for (int e = 0; e < 32; ++e) a[e] *= mul;
+                bwd_warp_f32_out<true>(stg, a, lane, [&](int row) -> float* {
+                    const int key = q4 * 32 + row;
+                    if (key >= kk.nk) return nullptr;
+                    return base + (((size_t)kk.b * rows + kk.k0 + key) * p.Hkv + kk.g) * kBwdD + c0;
+                });
             }
             tc_fence_before();
             __syncwarp();
