@@ -11,7 +11,8 @@
 
 Each case keeps its working set larger than the 126 MB L2 (so DRAM counters mean
 something) but a few GB at most, and launches the kernel `--reps` times after one
-warm-up launch.  Prints the per-launch time from CUDA events (not meaningful under a
+warm-up launch.  The size options (--B, --L, --T) are for timing and for one-pass launch
+lists; multi-metric captures use the default sizes and scale.  Prints the per-launch time from CUDA events (not meaningful under a
 profiler).
 """
 import argparse
