@@ -17,7 +17,8 @@ from ._lib import (HCA_OUT_F32, HCA_OUT_GATE, HCA_PAGED, HCA_QK_NORM,  # noqa: F
                    HCA_WINDOW_RING, HCA_WRITE_LSE)
 
 __all__ = ["HCAError", "compress", "prefill", "decode", "decode_workspace_size", "append", "append_state_size",
-           "vha", "gate_logits", "prefill_backward", "get_device_error", "status_string"]
+           "vha", "gate_logits", "prefill_backward", "dsa_index", "dsa_topk", "dsa_attend", "dsa_decode",
+           "get_device_error", "status_string"]
 
 
 class HCAError(RuntimeError):
@@ -157,6 +158,72 @@ def prefill_backward(q, k, v, w, kc, vc, out, lse, dout, blk, W, scale, want_dw=
                                   float(scale), flags, _stream(q.device))
     _check(rc, "hca_prefill_backward")
     return dq, dk, dvv, dw
+
+
+def dsa_index(q_idx, w_idx, k_idx, seqlens, scores=None):
+    """Indexer scores of the sparse-attention decode step: q_idx [B,H_I,64] bf16, w_idx [B,H_I]
+    fp32, k_idx [B,Lmax,64] bf16, seqlens [B] int32.  Returns scores [B,Lmax] fp32."""
+    _need(q_idx, torch.bfloat16, "q_idx")
+    dev = q_idx.device
+    _need(w_idx, torch.float32, "w_idx", dev)
+    _need(k_idx, torch.bfloat16, "k_idx", dev)
+    _need(seqlens, torch.int32, "seqlens", dev)
+    B, HI, dI = q_idx.shape
+    Lmax = k_idx.shape[1]
+    if scores is None:
+        scores = torch.empty((B, Lmax), dtype=torch.float32, device=dev)
+    _need(scores, torch.float32, "scores", dev)
+    for name, t, n in (("w_idx", w_idx, B * HI), ("k_idx", k_idx, B * Lmax * dI), ("seqlens", seqlens, B),
+                       ("scores", scores, B * Lmax)):
+        _room(t, n, name)
+    _check(_lib.load().hca_dsa_index(_p(q_idx), _p(w_idx), _p(k_idx), _p(seqlens), _p(scores), B, HI, dI, Lmax,
+                                     _stream(dev)), "hca_dsa_index")
+    return scores
+
+
+def dsa_topk(scores, seqlens, k, idx=None):
+    """Positions of the k largest scores per sequence (ascending, -1 padded): [B,k] int32."""
+    _need(scores, torch.float32, "scores")
+    dev = scores.device
+    _need(seqlens, torch.int32, "seqlens", dev)
+    B, Lmax = scores.shape
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+    _need(idx, torch.int32, "idx", dev)
+    _room(idx, B * k, "idx")
+    _room(seqlens, B, "seqlens")
+    _check(_lib.load().hca_dsa_topk(_p(scores), _p(seqlens), _p(idx), B, Lmax, int(k), _stream(dev)), "hca_dsa_topk")
+    return idx
+
+
+def dsa_attend(q, k, v, idx, seqlens, scale, out=None):
+    """Core attention over the kept positions: q [B,Hq,256], k / v [B,Lmax,256] bf16,
+    idx [B,kmax] int32.  Returns out [B,Hq,256] fp32."""
+    _need(q, torch.bfloat16, "q")
+    dev = q.device
+    for name, t in (("k", k), ("v", v)):
+        _need(t, torch.bfloat16, name, dev)
+    _need(idx, torch.int32, "idx", dev)
+    _need(seqlens, torch.int32, "seqlens", dev)
+    B, Hq, d = q.shape
+    Lmax, kmax = k.shape[1], idx.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    _need(out, torch.float32, "out", dev)
+    for name, t, n in (("k", k, B * Lmax * d), ("v", v, B * Lmax * d), ("seqlens", seqlens, B),
+                       ("out", out, B * Hq * d)):
+        _room(t, n, name)
+    _check(_lib.load().hca_dsa_attend(_p(q), _p(k), _p(v), _p(idx), _p(seqlens), _p(out), B, Hq, d, Lmax, kmax,
+                                      float(scale), _stream(dev)), "hca_dsa_attend")
+    return out
+
+
+def dsa_decode(q_idx, w_idx, k_idx, q, k, v, seqlens, topk, scale):
+    """The whole sparse-attention decode step: scores, selection, attention.  Returns
+    (out, idx, scores)."""
+    scores = dsa_index(q_idx, w_idx, k_idx, seqlens)
+    idx = dsa_topk(scores, seqlens, topk)
+    return dsa_attend(q, k, v, idx, seqlens, scale), idx, scores
 
 
 def decode_workspace_size(B, Hq, Hkv, dv) -> int:

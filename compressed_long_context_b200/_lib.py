@@ -25,7 +25,8 @@ EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_deco
            "hca_decode_noalloc",
            "hca_vha", "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error",
            "hca_debug_set_wait_limit", "hca_debug_set_drop_slab", "hca_debug_wait_probe", "hca_gate_logits",
-           "hca_prefill_backward_workspace_size", "hca_prefill_backward", "hca_debug_set_backward_segment")
+           "hca_prefill_backward_workspace_size", "hca_prefill_backward", "hca_debug_set_backward_segment",
+           "hca_dsa_index", "hca_dsa_topk", "hca_dsa_attend")
 
 _lib = None
 
@@ -76,6 +77,12 @@ def load():
     lib.hca_prefill_backward_workspace_size.argtypes = [_i] * 7
     lib.hca_prefill_backward.restype = _i
     lib.hca_prefill_backward.argtypes = [_vp] * 13 + [_vp, _sz] + [_i] * 8 + [_f, _u, _vp]
+    lib.hca_dsa_index.restype = _i
+    lib.hca_dsa_index.argtypes = [_vp] * 5 + [_i] * 4 + [_vp]
+    lib.hca_dsa_topk.restype = _i
+    lib.hca_dsa_topk.argtypes = [_vp] * 3 + [_i] * 3 + [_vp]
+    lib.hca_dsa_attend.restype = _i
+    lib.hca_dsa_attend.argtypes = [_vp] * 6 + [_i] * 5 + [_f, _vp]
     lib.hca_debug_set_backward_segment.restype = _i
     lib.hca_debug_set_backward_segment.argtypes = [_i]
     lib.hca_debug_set_wait_limit.restype = _i

@@ -1,0 +1,701 @@
+// dsa.cuh -- the sparse-attention layers' decode step (sm_100a): a lightweight indexer scores every
+// past position, the top-k positions are kept, and the core attention of the query's heads runs
+// over those positions only (Zhidx article "280B Total Parameters, 14B Activated ...", section
+// "1. Latent-Gated Sparse Attention", DSA paragraph; wiki summary "Key claims": DeepSeek-style
+// DSA in the full-context MLA layers, whose query, key and value are 256-dim).
+//
+// Forms (the pages leave them open; the oracle takes the same readings):
+//   I(s) = sum_j w_j * max(0, q_I[j] . k_I[s])   (H_I indexer heads, one d_I = 64 key per position)
+//   keep the k positions of largest I, equal scores in increasing position order
+//   out[h] = softmax_s(scale * q[h] . k[s]) v[s] over the kept s, one key / value row per position
+//
+// Kernels:
+//   dsa_index_kernel   one persistent CTA per SM over all (sequence, 128-position tile) pairs:
+//                      a tile's indexer keys (128 x 64 bf16, 16 KB) arrive by TMA into an 8-slot
+//                      ring, one tcgen05 MMA chain gives the 128 x H_I dot products in tensor
+//                      memory (two buffers), four epilogue warps apply ReLU and the head weights
+//                      and write the scores (fp32).  HBM-bound on the keys.
+//   dsa_topk_kernel    one CTA per sequence: radix select of the k-th largest score (three
+//                      digit passes of 11 / 11 / 10 bits over order-preserving integer keys,
+//                      warp-aggregated shared-memory histograms), then one ordered pass that keeps
+//                      every larger score and the first equal ones, positions ascending.
+//   dsa_attend_kernel  one CTA per sequence: the query heads (64 x 256 bf16) stay in shared
+//                      memory; per tile of 128 kept positions, the key rows and then the value
+//                      rows are gathered with 16-byte asynchronous copies into 128-byte-swizzled
+//                      slabs (a warp copies one 512-byte row per instruction), S^T = K Q^T and
+//                      O^T += V^T P^T run on tcgen05 (as in the HCA decode), and four warps run an
+//                      online softmax with a lazily moved reference maximum.
+// Every wait is bounded (common.cuh).
+#pragma once
+
+#include "common.cuh"
+
+namespace hca {
+
+constexpr int kDsaDI = 64;                 // indexer key / query dimension (one 128-byte row)
+constexpr int kDsaD = 256;                 // core attention head dimension
+constexpr int kDsaHeads = 64;              // query heads of a sequence (MMA N, padded)
+constexpr int kDsaMaxHI = 64;              // indexer heads (MMA N, multiple of 16)
+
+// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled slab (the TMA / tcgen05 layout).
+__device__ __forceinline__ uint32_t dsa_sw(uint32_t r, uint32_t c) { return r * 128u + (((c ^ r) & 7u) << 4); }
+
+// Bounded wait by a group of 128 threads (named barrier 2) with one verdict for the group, so
+// that the group either goes on together or unwinds together.
+__device__ __forceinline__ bool dsa_group_wait128(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    const bool ok = mbar_wait(bar, parity, abort);
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "barrier.red.and.pred q, 2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)ok) : "memory");
+    return r != 0;
+}
+
+// ------------------------------------------------------------------------------------- indexer
+
+constexpr int kIdxThreads = 192;           // producer, MMA issuer, 4 epilogue warps
+constexpr int kIdxRing = 8;
+constexpr uint32_t kIdxSlab = 128 * 128;   // 128 positions x 64 dims bf16
+constexpr uint32_t kIdxQBytes = kDsaMaxHI * 128;
+constexpr uint32_t kIdxSmRing = 0;
+constexpr uint32_t kIdxSmQ = kIdxSmRing + kIdxRing * kIdxSlab;          // two query buffers
+constexpr uint32_t kIdxSmBar = kIdxSmQ + 2 * kIdxQBytes;
+constexpr uint32_t kIdxSmW = kIdxSmBar + 256;                           // two weight buffers [64]
+constexpr uint32_t kIdxSmem = kIdxSmW + 2 * kDsaMaxHI * 4 + 16;
+static_assert(kIdxSmQ % 1024 == 0 && kIdxSlab % 1024 == 0, "swizzled operands 1024-aligned");
+
+struct DsaIndexParams {
+    const float* w;          // [B, HI]
+    const int* seqlens;      // [B]
+    float* scores;           // [B, Lmax]
+    int B, HI, Lmax, ntile;  // ntile = ceil(Lmax / 128)
+    long long total;         // B * ntile
+};
+
+__device__ __forceinline__ int dsa_len(const DsaIndexParams& p, int b) {
+    const int L = __ldg(p.seqlens + b);
+    return L < 0 ? 0 : (L > p.Lmax ? p.Lmax : L);
+}
+
+__global__ void __launch_bounds__(kIdxThreads, 1)
+dsa_index_kernel(const DsaIndexParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k) {
+    extern __shared__ __align__(1024) uint8_t dsmem[];
+    if (smem_u32(dsmem) & 1023u) {
+        if (threadIdx.x == 0) record_error(HCA_ERR_INTERNAL);
+        return;
+    }
+    uint8_t* sm = dsmem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kIdxSmBar);
+    uint64_t* empty = full + kIdxRing;
+    uint64_t* q_full = empty + kIdxRing;       // [2]
+    uint64_t* q_empty = q_full + 2;            // [2]
+    uint64_t* acc_full = q_full + 4;           // [2]
+    uint64_t* acc_empty = q_full + 6;          // [2]
+    uint64_t* drain = q_full + 8;
+    int* misc = reinterpret_cast<int*>(sm + kIdxSmW + 2 * kDsaMaxHI * 4);
+    volatile int* abort_flag = misc;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
+    float* wsm = reinterpret_cast<float*>(sm + kIdxSmW);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int i = 0; i < kIdxRing; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // this CTA's contiguous range of (sequence, tile) pairs
+    const long long per = (p.total + gridDim.x - 1) / gridDim.x;
+    const long long t_begin = per * blockIdx.x;
+    const long long t_end = min(p.total, t_begin + per);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t op = 0, nq = 0;
+            int cur_b = -1;
+            bool ok = true;
+            for (long long i = t_begin; ok && i < t_end; ++i) {
+                const int b = (int)(i / p.ntile), t = (int)(i - (long long)b * p.ntile);
+                if (128 * t >= dsa_len(p, b)) continue;           // past the sequence: no keys to read
+                if (b != cur_b) {
+                    const uint32_t qb = nq & 1;
+                    if (!mbar_wait(&q_empty[qb], ((nq >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&q_full[qb], (uint32_t)p.HI * 128);
+                    tma_load_4d(sm + kIdxSmQ + qb * kIdxQBytes, &tm_q, &q_full[qb], 0, 0, b, 0);
+                    ++nq;
+                    cur_b = b;
+                }
+                const uint32_t st = op % kIdxRing;
+                if (!mbar_wait(&empty[st], ((op / kIdxRing) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                mbar_arrive_expect_tx(&full[st], kIdxSlab);
+                tma_load_4d(sm + kIdxSmRing + st * kIdxSlab, &tm_k, &full[st], 0, 128 * t, b, 0);
+                ++op;
+            }
+            mbar_drain_ring(full, op, kIdxRing);
+            // the last query load has landed too (it was consumed unless a wait gave up)
+            if (nq) mbar_drain_wait(&q_full[(nq - 1) & 1], ((nq - 1) >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        const uint32_t id = idesc_bf16(128, p.HI, 0, 0);
+        uint32_t op = 0, nq = 0, na = 0;
+        int cur_b = -1;
+        bool ok = true;
+        for (long long i = t_begin; ok && i < t_end; ++i) {
+            const int b = (int)(i / p.ntile), t = (int)(i - (long long)b * p.ntile);
+            if (128 * t >= dsa_len(p, b)) continue;
+            if (b != cur_b) {
+                if (cur_b >= 0 && lane == 0) mma_commit(&q_empty[(nq - 1) & 1]);   // previous query buffer free
+                if (!warp_wait(&q_full[nq & 1], (nq >> 1) & 1, abort_flag)) { ok = false; break; }
+                ++nq;
+                cur_b = b;
+            }
+            const uint32_t st = op % kIdxRing, ab = na & 1;
+            if (!warp_wait(&acc_empty[ab], ((na >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!warp_wait(&full[st], (op / kIdxRing) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t a = smem_u32(sm + kIdxSmRing + st * kIdxSlab);
+                const uint32_t q = smem_u32(sm + kIdxSmQ + ((nq - 1) & 1) * kIdxQBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem + 64 * ab, smem_desc_sw128(a + kk * 32, 16, 1024), smem_desc_sw128(q + kk * 32, 16, 1024), id,
+                           kk ? 1u : 0u);
+                mma_commit(&empty[st]);
+                mma_commit(&acc_full[ab]);
+            }
+            __syncwarp();
+            ++op;
+            ++na;
+        }
+        if (lane == 0) {
+            mma_commit(drain);
+            mbar_drain_wait(drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ================================================================ epilogue: thread = position
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int et = threadIdx.x - 64;          // 0..127
+        uint32_t na = 0, nb = 0;
+        int cur_b = -1;
+        for (long long i = t_begin; i < t_end; ++i) {
+            const int b = (int)(i / p.ntile), t = (int)(i - (long long)b * p.ntile);
+            const int L = dsa_len(p, b);
+            const int pos = 128 * t + r;
+            if (128 * t >= L) {
+                if (pos < p.Lmax) p.scores[(size_t)b * p.Lmax + pos] = -INFINITY;
+                continue;
+            }
+            if (b != cur_b) {
+                // the sequence's head weights, in the other of two buffers
+                float* wb = wsm + (nb & 1) * kDsaMaxHI;
+                if (et < p.HI) wb[et] = __ldg(p.w + (size_t)b * p.HI + et);
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                ++nb;
+                cur_b = b;
+            }
+            const float* wb = wsm + ((nb - 1) & 1) * kDsaMaxHI;
+            const uint32_t ab = na & 1;
+            if (!dsa_group_wait128(&acc_full[ab], (na >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            float s = 0.f;
+            for (int c0 = 0; c0 < p.HI; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem + lane_off + 64 * ab + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) s = fmaf(wb[c0 + j], fmaxf(v[j], 0.f), s);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            ++na;
+            if (pos < p.Lmax) p.scores[(size_t)b * p.Lmax + pos] = pos < L ? s : -INFINITY;
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+// ------------------------------------------------------------------------------------- top-k
+
+constexpr int kTopkThreads = 1024;
+
+struct DsaTopkParams {
+    const float* scores;     // [B, Lmax]
+    const int* seqlens;
+    int* idx;                // [B, k]
+    int B, Lmax, k;
+};
+
+// Order-preserving integer image of an fp32 score: larger scores give larger keys.
+__device__ __forceinline__ uint32_t dsa_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive scan of one int per thread (1024 threads); returns the exclusive prefix
+// and the block total through *total.
+__device__ __forceinline__ int dsa_block_scan(int v, int* wsum, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += n;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = wsum[lane];
+        int y = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, y, off);
+            if (lane >= off) y += n;
+        }
+        wsum[lane] = y - w;                 // exclusive prefix of the warp totals
+        if (lane == 31) wsum[32] = y;
+    }
+    __syncthreads();
+    const int r = wsum[warp] + x - v;
+    *total = wsum[32];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopkParams p) {
+    __shared__ int hist[2048];
+    __shared__ int wsum[33];
+    __shared__ uint32_t sel[2];             // [0] digit chosen, [1] remaining after the pass
+    const int b = blockIdx.x;
+    int L = __ldg(p.seqlens + b);
+    L = L < 0 ? 0 : (L > p.Lmax ? p.Lmax : L);
+    const float* sc = p.scores + (size_t)b * p.Lmax;
+    int* out = p.idx + (size_t)b * p.k;
+    const int kk = min(p.k, L);
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = kk;                     // how many of the largest keys still to place
+    if (kk < L) {
+        // three digit passes, most significant first: 11, 11 and 10 bits
+        for (int pass = 0; pass < 3; ++pass) {
+            const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+            const int nbins = pass == 2 ? 1024 : 2048;
+            for (int i = tid; i < 2048; i += kTopkThreads) hist[i] = 0;
+            __syncthreads();
+            for (int base = 0; base < L; base += kTopkThreads) {
+                const int s = base + tid;
+                bool in = false;
+                uint32_t bin = 0;
+                if (s < L) {
+                    const uint32_t key = dsa_key(__ldg(sc + s));
+                    in = (key & pmask) == prefix;
+                    bin = (key >> shift) & (uint32_t)(nbins - 1);
+                }
+                // warp-aggregated increments: lanes with the same bin add once
+                const uint32_t act = __ballot_sync(0xffffffffu, in);
+                if (in) {
+                    const uint32_t peers = __match_any_sync(act, bin);
+                    if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
+                }
+            }
+            __syncthreads();
+            // the digit holding the remaining-th largest key: suffix sums over bins, high to low
+            // (thread i takes bins 2i and 2i + 1, counted from the top)
+            const int hi_bin = nbins - 1 - 2 * tid;
+            const int c0 = (2 * tid < nbins) ? hist[hi_bin] : 0;
+            const int c1 = (2 * tid + 1 < nbins) ? hist[hi_bin - 1] : 0;
+            int tot;
+            const int before = dsa_block_scan(c0 + c1, wsum, &tot);     // keys in higher bins
+            if (2 * tid < nbins) {
+                if (before < remaining && before + c0 >= remaining) {
+                    sel[0] = (uint32_t)hi_bin;
+                    sel[1] = (uint32_t)(remaining - before);
+                } else if (2 * tid + 1 < nbins && before + c0 < remaining && before + c0 + c1 >= remaining) {
+                    sel[0] = (uint32_t)(hi_bin - 1);
+                    sel[1] = (uint32_t)(remaining - before - c0);
+                }
+            }
+            __syncthreads();
+            prefix |= sel[0] << shift;
+            pmask |= (uint32_t)(nbins - 1) << shift;
+            remaining = (int)sel[1];
+            __syncthreads();
+        }
+    }
+    // keep every key above the threshold key `prefix` and the first `remaining` keys equal to
+    // it, in position order (each thread takes a contiguous chunk of positions).  With all
+    // positions kept, prefix = 0 and remaining = 0: every finite score's key is above 0.
+    const int chunk = (L + kTopkThreads - 1) / kTopkThreads;
+    const int s0 = min(L, tid * chunk), s1 = min(L, s0 + chunk);
+    int n_gt = 0, n_eq = 0;
+    for (int s = s0; s < s1; ++s) {
+        const uint32_t key = dsa_key(__ldg(sc + s));
+        n_gt += key > prefix;
+        n_eq += key == prefix;
+    }
+    int tot;
+    const int eq_before = dsa_block_scan(n_eq, wsum, &tot);
+    const int keep_eq = max(0, min(n_eq, remaining - eq_before));
+    int o = dsa_block_scan(n_gt + keep_eq, wsum, &tot);
+    int eq_rank = eq_before;
+    for (int s = s0; s < s1; ++s) {
+        const uint32_t key = dsa_key(__ldg(sc + s));
+        if (key > prefix) {
+            out[o++] = s;
+        } else if (key == prefix) {
+            if (eq_rank < remaining) out[o++] = s;
+            ++eq_rank;
+        }
+    }
+    for (int i = kk + tid; i < p.k; i += kTopkThreads) out[i] = -1;
+}
+
+// ------------------------------------------------------------------------------------- attention
+
+constexpr int kAttThreads = 160;           // MMA issuer, 4 gather / softmax warps
+constexpr uint32_t kAttSlab = 128 * 128;   // 128 rows x 64 channels bf16
+constexpr uint32_t kAttQSlab = 64 * 128;   // 64 heads x 64 channels
+constexpr uint32_t kAttSmQ = 0;                                  // 4 x 8 KB
+constexpr uint32_t kAttSmK = kAttSmQ + 4 * kAttQSlab;            // 4 x 16 KB
+constexpr uint32_t kAttSmV = kAttSmK + 4 * kAttSlab;             // 4 x 16 KB
+constexpr uint32_t kAttSmP = kAttSmV + 4 * kAttSlab;             // 128 keys x 64 heads bf16
+constexpr uint32_t kAttSmRed = kAttSmP + kAttSlab;               // float [4][64]
+constexpr uint32_t kAttSmM = kAttSmRed + 4 * 64 * 4;             // float [64] reference max
+constexpr uint32_t kAttSmA = kAttSmM + 64 * 4;                   // float [64] rescale factors
+constexpr uint32_t kAttSmBar = kAttSmA + 64 * 4;
+constexpr uint32_t kAttSmem = kAttSmBar + 16 * 8 + 32;
+static_assert(kAttSmem <= 232448, "attention shared memory exceeds the per-block limit");
+constexpr float kAttRescale = 8.0f;        // move the reference max only when exceeded by 2^8
+
+struct DsaAttendParams {
+    const __nv_bfloat16* k;  // [B, Lmax, 256]
+    const __nv_bfloat16* v;
+    const int* idx;          // [B, kmax] ascending, -1 padding
+    const int* seqlens;
+    float* out;              // [B, Hq, 256]
+    int B, Hq, Lmax, kmax;
+    float scale_log2;
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int n>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(n) : "memory"); }
+
+// Column reduction of 32 values per lane across a warp: returns, in lane c, the max (or sum)
+// over the 32 lanes of column c (a butterfly that halves the columns kept at each step).
+template <bool kMax>
+__device__ __forceinline__ float dsa_colred32(float* t, int lane) {
+#pragma unroll
+    for (int x = 16; x >= 1; x >>= 1) {
+        const bool hi = (lane & x) != 0;
+#pragma unroll
+        for (int i = 0; i < x; ++i) {
+            const float send = hi ? t[i] : t[i + x];
+            const float keep = hi ? t[i + x] : t[i];
+            const float o = __shfl_xor_sync(0xffffffffu, send, x);
+            t[i] = kMax ? fmaxf(keep, o) : keep + o;
+        }
+    }
+    return t[0];
+}
+
+// Rows 32 w .. 32 w + 31 of a 128-row tile of gathered 512-byte rows (positions idx[row], -1 or
+// past `count`: zeros) into four 128-byte-swizzled slabs of 64 channels; lane l copies 16 bytes
+// of channel chunk l of a row, so one instruction moves one whole row.
+__device__ __forceinline__ void dsa_gather_rows(uint8_t* dst, const __nv_bfloat16* src_b, const int* idx_t, int nvalid,
+                                                int Lmax, int w, int lane) {
+    const int slab = lane >> 3, c = lane & 7;
+#pragma unroll 4
+    for (int i = 0; i < 32; ++i) {
+        const int row = 32 * w + i;
+        uint8_t* d = dst + slab * kAttSlab + dsa_sw(row, c);
+        int pos = row < nvalid ? __ldg(idx_t + row) : -1;
+        if (pos >= Lmax) {                      // a position past the buffer: reported, not read
+            if (lane == 0) record_error(HCA_ERR_DEVICE_INPUT);
+            pos = -1;
+        }
+        if (pos >= 0) cp_async16(d, src_b + (size_t)pos * kDsaD + 8 * lane);
+        else *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
+    }
+}
+
+__global__ void __launch_bounds__(kAttThreads, 1)
+dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap tm_q) {
+    extern __shared__ __align__(1024) uint8_t dsmem[];
+    if (smem_u32(dsmem) & 1023u) {
+        if (threadIdx.x == 0) record_error(HCA_ERR_INTERNAL);
+        return;
+    }
+    uint8_t* sm = dsmem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kAttSmBar);
+    uint64_t* q_full = bars + 0;
+    uint64_t* k_full = bars + 1;        // 4 worker warps: the tile's key rows are in place
+    uint64_t* s_full = bars + 2;        // S^T of the tile is in tensor memory (commit)
+    uint64_t* s_read = bars + 3;        // 4 worker warps: S^T read
+    uint64_t* p_full = bars + 4;        // 4 worker warps: P^T and the value rows are in place
+    uint64_t* pv_done = bars + 5;       // O^T += V^T P^T done (commit)
+    uint64_t* drain = bars + 6;
+    int* misc = reinterpret_cast<int*>(sm + kAttSmBar + 16 * 8);
+    volatile int* abort_flag = misc;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
+    float* red = reinterpret_cast<float*>(sm + kAttSmRed);
+    float* mref = reinterpret_cast<float*>(sm + kAttSmM);
+    float* alpha = reinterpret_cast<float*>(sm + kAttSmA);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x;
+    int L = __ldg(p.seqlens + b);
+    L = L < 0 ? 0 : (L > p.Lmax ? p.Lmax : L);
+    const int count = min(p.kmax, L);
+    const int nt = (count + 127) / 128;
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(q_full, 1);
+        mbar_init(k_full, 4);
+        mbar_init(s_full, 1);
+        mbar_init(s_read, 4);
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = 0, tO = 64;     // S^T: 64 columns; O^T: two chunks of 128 channels x 64 heads
+    const int* idx_b = p.idx + (size_t)b * p.kmax;
+
+    if (warp == 0) {
+        // ================================================================ MMA issuer (+ query load)
+        if (lane == 0 && nt > 0) {
+            mbar_arrive_expect_tx(q_full, 4 * kAttQSlab);
+            for (int s = 0; s < 4; ++s) tma_load_4d(sm + kAttSmQ + s * kAttQSlab, &tm_q, q_full, 64 * s, 0, b, 0);
+        }
+        const uint32_t id_s = idesc_bf16(128, kDsaHeads, 0, 0);
+        const uint32_t id_o = idesc_bf16(128, kDsaHeads, 1, 1);
+        bool ok = nt == 0 || warp_wait(q_full, 0, abort_flag);
+        for (int j = 0; ok && j < nt; ++j) {
+            if (!warp_wait(k_full, j & 1, abort_flag)) { ok = false; break; }
+            if (j > 0 && !warp_wait(s_read, (j - 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t kb = smem_u32(sm + kAttSmK), qb = smem_u32(sm + kAttSmQ);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + tS, smem_desc_sw128(kb + s * kAttSlab + kk * 32, 16, 1024),
+                               smem_desc_sw128(qb + s * kAttQSlab + kk * 32, 16, 1024), id_s, (s | kk) ? 1u : 0u);
+                mma_commit(s_full);
+            }
+            __syncwarp();
+            if (!warp_wait(p_full, j & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t vb = smem_u32(sm + kAttSmV), pb = smem_u32(sm + kAttSmP);
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tmem + tO + 64 * c, smem_desc_sw128(vb + 2 * c * kAttSlab + kk * 2048, kAttSlab, 1024),
+                               smem_desc_sw128(pb + kk * 2048, 8192, 1024), id_o, (j | kk) ? 1u : 0u);
+                mma_commit(pv_done);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            mma_commit(drain);
+            mbar_drain_wait(drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ================================================================ gathers, softmax, epilogue
+        // a warp reaches only the TMEM lane quarter (warp id mod 4): rows / lanes 32 w .. 32 w + 31
+        const int w = warp & 3;
+        const int r = 32 * w + lane;
+        const uint32_t lane_off = (uint32_t)(32 * w) << 16;
+        const __nv_bfloat16* kb = p.k + (size_t)b * p.Lmax * kDsaD;
+        const __nv_bfloat16* vb = p.v + (size_t)b * p.Lmax * kDsaD;
+        float lsum[64];
+#pragma unroll
+        for (int h = 0; h < 64; ++h) lsum[h] = 0.f;
+        bool ok = true;
+        if (nt > 0) {
+            dsa_gather_rows(sm + kAttSmK, kb, idx_b, count, p.Lmax, w, lane);
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(k_full);
+        }
+        for (int j = 0; ok && j < nt; ++j) {
+            const int* idx_t = idx_b + 128 * j;
+            const int nvalid = count - 128 * j;
+            // the value rows of this tile (the previous PV is done: waited at the end of the last tile)
+            dsa_gather_rows(sm + kAttSmV, vb, idx_t, nvalid, p.Lmax, w, lane);
+            cp_async_commit();
+            if (!dsa_group_wait128(s_full, j & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            // S^T is in tensor memory, so the key buffer is free: the next tile's keys start now
+            if (j + 1 < nt) {
+                dsa_gather_rows(sm + kAttSmK, kb, idx_t + 128, nvalid - 128, p.Lmax, w, lane);
+                cp_async_commit();
+            }
+            float z[64];
+#pragma unroll
+            for (int c = 0; c < 64; c += 16) tmem_ld16(tmem + lane_off + tS + c, z + c);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_read);
+            const bool valid = r < nvalid;
+#pragma unroll
+            for (int h = 0; h < 64; ++h) z[h] = valid ? z[h] * p.scale_log2 : -INFINITY;
+            // tile max per head over the 128 rows, then the reference max (moved lazily)
+            {
+                float t[32];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) t[i] = z[32 * half + i];
+                    red[w * 64 + 32 * half + lane] = dsa_colred32<true>(t, lane);
+                }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (threadIdx.x >= 32 && threadIdx.x < 96) {
+                const int h = threadIdx.x - 32;
+                const float tm = fmaxf(fmaxf(red[h], red[64 + h]), fmaxf(red[128 + h], red[192 + h]));
+                const float mo = j == 0 ? -INFINITY : mref[h];
+                if (j == 0 || tm > mo + kAttRescale) {
+                    alpha[h] = j == 0 ? 1.f : ex2(mo - tm);
+                    mref[h] = tm;
+                } else {
+                    alpha[h] = 1.f;
+                }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            bool any = false;
+            if (j > 0)
+#pragma unroll
+                for (int h = 0; h < 64; ++h) any |= alpha[h] != 1.f;
+            if (any) {
+                // O^T rows (channels 128 c + r) times alpha per head column; PV of the last tile is done
+#pragma unroll
+                for (int h = 0; h < 64; ++h) lsum[h] *= alpha[h];
+#pragma unroll 1
+                for (int c = 0; c < 2; ++c)
+#pragma unroll 1
+                    for (int c16 = 0; c16 < 64; c16 += 16) {
+                        float o[16];
+                        uint32_t wv[16];
+                        const uint32_t ta = tmem + lane_off + tO + 64 * c + c16;
+                        tmem_ld16(ta, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) wv[i] = __float_as_uint(o[i] * alpha[c16 + i]);
+                        tmem_st16(ta, wv);
+                    }
+                tmem_wait_st();
+                tc_fence_before();
+            }
+            // probabilities: P^T row r (64 heads) in bf16, and this thread's share of the sums of
+            // the same rounded values (numerator and normaliser use identical weights)
+            uint32_t pk[32];
+#pragma unroll
+            for (int h = 0; h < 64; h += 2) {
+                const uint32_t u = pack_bf16x2(ex2(z[h] - mref[h]), ex2(z[h + 1] - mref[h + 1]));
+                lsum[h] += bf16lo(u);
+                lsum[h + 1] += bf16hi(u);
+                pk[h >> 1] = u;
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(sm + kAttSmP + dsa_sw(r, c)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            // this tile's value rows have landed (the next tile's keys may still be in flight)
+            if (j + 1 < nt) cp_async_wait<1>();
+            else cp_async_wait<0>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+            if (j + 1 < nt) {
+                cp_async_wait<0>();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(k_full);
+            }
+            // PV of this tile done: the value and P buffers are free and O^T is stable
+            if (!dsa_group_wait128(pv_done, j & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+        }
+        cp_async_wait<0>();
+        // ---- out[h][ch] = O^T[ch][h] / l[h]; l from every row's share (column sums, then 4 warps)
+        {
+            float t[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) t[i] = lsum[32 * half + i];
+                red[w * 64 + 32 * half + lane] = dsa_colred32<false>(t, lane);
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x >= 32 && threadIdx.x < 96) {
+            const int h = threadIdx.x - 32;
+            alpha[h] = (ok && nt > 0) ? 1.f / ((red[h] + red[64 + h]) + (red[128 + h] + red[192 + h])) : NAN;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (nt > 0) {
+            float* ob = p.out + (size_t)b * p.Hq * kDsaD;
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c)
+#pragma unroll 1
+                for (int c16 = 0; c16 < 64; c16 += 16) {
+                    float o[16];
+                    tmem_ld16(tmem + lane_off + tO + 64 * c + c16, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int h = c16 + i;
+                        if (h < p.Hq) ob[(size_t)h * kDsaD + 128 * c + r] = o[i] * alpha[h];
+                    }
+                }
+        }
+        tc_fence_before();
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace hca

@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "decode.cuh"
+#include "dsa.cuh"
 #include "gate.cuh"
 #include "prefill.cuh"
 #include "prefill_pair.cuh"
@@ -852,5 +853,81 @@ extern "C" hca_status_t hca_prefill_backward(const void* q, const void* k, const
             bwd_dkv_kernel<<<(unsigned)std::min<long long>(p.kv_items, ns), kKvThreads, kBwdSmem, s>>>(p, tq, tdo);
     }
     if (Nc > 0) bwd_pool_kernel<<<(unsigned)((long long)B * Nc), kPoolThreads, 0, s>>>(p);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------------------------
+// The sparse-attention decode step (dsa.cuh): indexer scores, top-k selection, core attention.
+extern "C" hca_status_t hca_dsa_index(const void* q_idx, const float* w_idx, const void* k_idx, const int* seqlens,
+                                      float* scores, int B, int HI, int dI, int Lmax, hca_stream_t stream) {
+    using namespace hca;
+    if (B < 0 || Lmax < 1 || HI < 1) return HCA_ERR_INVALID_ARG;
+    if (dI != kDsaDI || HI % 16 || HI > kDsaMaxHI) return HCA_ERR_UNSUPPORTED;
+    if (B == 0) return HCA_OK;
+    if (!q_idx || !w_idx || !k_idx || !seqlens || !scores || !aligned16(q_idx) || !aligned16(k_idx) ||
+        (reinterpret_cast<uintptr_t>(w_idx) & 3) || (reinterpret_cast<uintptr_t>(seqlens) & 3) ||
+        (reinterpret_cast<uintptr_t>(scores) & 3))
+        return HCA_ERR_INVALID_ARG;
+    const int ns = num_sms();
+    if (ns <= 0) return HCA_ERR_CUDA;
+    CUtensorMap tq, tk;
+    bool ok = make_tmap_4d(&tq, q_idx, kDsaDI, HI, B, 1, kDsaDI, (uint64_t)kDsaDI * HI, (uint64_t)kDsaDI * HI * B, 64, HI, 1, 1);
+    ok &= make_tmap_4d(&tk, k_idx, kDsaDI, Lmax, B, 1, kDsaDI, (uint64_t)kDsaDI * Lmax, (uint64_t)kDsaDI * Lmax * B, 64, 128,
+                       1, 1);
+    if (!ok) return HCA_ERR_CUDA;
+    if (!set_smem_attr_once(reinterpret_cast<const void*>(&dsa_index_kernel), (int)kIdxSmem, 10)) return HCA_ERR_CUDA;
+    DsaIndexParams p;
+    p.w = w_idx;
+    p.seqlens = seqlens;
+    p.scores = scores;
+    p.B = B; p.HI = HI; p.Lmax = Lmax; p.ntile = (Lmax + 127) / 128;
+    p.total = (long long)B * p.ntile;
+    const long long grid = std::min<long long>(p.total, ns);
+    dsa_index_kernel<<<(unsigned)grid, kIdxThreads, kIdxSmem, reinterpret_cast<cudaStream_t>(stream)>>>(p, tq, tk);
+    return launch_status();
+}
+
+extern "C" hca_status_t hca_dsa_topk(const float* scores, const int* seqlens, int* idx, int B, int Lmax, int k,
+                                     hca_stream_t stream) {
+    using namespace hca;
+    if (B < 0 || Lmax < 1 || k < 1) return HCA_ERR_INVALID_ARG;
+    if (B == 0) return HCA_OK;
+    if (!scores || !seqlens || !idx || (reinterpret_cast<uintptr_t>(scores) & 3) ||
+        (reinterpret_cast<uintptr_t>(seqlens) & 3) || (reinterpret_cast<uintptr_t>(idx) & 3))
+        return HCA_ERR_INVALID_ARG;
+    DsaTopkParams p;
+    p.scores = scores;
+    p.seqlens = seqlens;
+    p.idx = idx;
+    p.B = B; p.Lmax = Lmax; p.k = k;
+    dsa_topk_kernel<<<(unsigned)B, kTopkThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    return launch_status();
+}
+
+extern "C" hca_status_t hca_dsa_attend(const void* q, const void* k, const void* v, const int* idx, const int* seqlens,
+                                       float* out, int B, int Hq, int d, int Lmax, int kmax, float scale,
+                                       hca_stream_t stream) {
+    using namespace hca;
+    if (B < 0 || Hq < 1 || Lmax < 1 || kmax < 1) return HCA_ERR_INVALID_ARG;
+    if (d != kDsaD || Hq > kDsaHeads) return HCA_ERR_UNSUPPORTED;
+    if (!(scale == scale)) return HCA_ERR_INVALID_ARG;
+    if (B == 0) return HCA_OK;
+    if (!q || !k || !v || !idx || !seqlens || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        (reinterpret_cast<uintptr_t>(idx) & 3) || (reinterpret_cast<uintptr_t>(seqlens) & 3) ||
+        (reinterpret_cast<uintptr_t>(out) & 3))
+        return HCA_ERR_INVALID_ARG;
+    CUtensorMap tq;
+    if (!make_tmap_4d(&tq, q, kDsaD, Hq, B, 1, kDsaD, (uint64_t)kDsaD * Hq, (uint64_t)kDsaD * Hq * B, 64, 64, 1, 1))
+        return HCA_ERR_CUDA;
+    if (!set_smem_attr_once(reinterpret_cast<const void*>(&dsa_attend_kernel), (int)kAttSmem, 11)) return HCA_ERR_CUDA;
+    DsaAttendParams p;
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.idx = idx;
+    p.seqlens = seqlens;
+    p.out = out;
+    p.B = B; p.Hq = Hq; p.Lmax = Lmax; p.kmax = kmax;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    dsa_attend_kernel<<<(unsigned)B, kAttThreads, kAttSmem, reinterpret_cast<cudaStream_t>(stream)>>>(p, tq);
     return launch_status();
 }

@@ -149,6 +149,47 @@ hca_status_t hca_prefill_backward(const void* q, const void* k, const void* v, c
                                   float scale, unsigned flags, hca_stream_t stream);
 
 /*
+ * The sparse-attention layers' decode step, in three calls (Zhidx article, section
+ * "1. Latent-Gated Sparse Attention", DSA paragraph: a lightweight indexer scores the past
+ * positions of each query and core attention runs over the highest-scoring Top-K only; the
+ * model card: those layers use 256-dim query, key and value).  Readings where the pages are
+ * silent: H_I indexer heads of d_I dims and one d_I-dim indexer key per position, the score
+ * I(s) = sum_j w_j * max(0, q_I[j] . k_I[s]); the k largest scores kept, equal scores in
+ * increasing position order; core attention of Hq heads over one key and one value row per
+ * kept position, shared by the heads.  One decode query per sequence, at position L_b - 1,
+ * sees positions 0 .. L_b - 1.
+ *
+ * hca_dsa_index -- indexer scores.
+ *   q_idx  [B,H_I,d_I] bf16, w_idx [B,H_I] fp32, k_idx [B,Lmax,d_I] bf16
+ *   seqlens [B] int32 (device; clamped into [0, Lmax])
+ *   scores [B,Lmax] fp32 output, -inf at positions >= L_b
+ * Supported: d_I == 64, H_I a multiple of 16 up to 64.  bf16 products, fp32 sums.
+ */
+hca_status_t hca_dsa_index(const void* q_idx, const float* w_idx, const void* k_idx, const int* seqlens,
+                           float* scores, int B, int HI, int dI, int Lmax, hca_stream_t stream);
+
+/*
+ * hca_dsa_topk -- the k positions of largest score of each sequence among 0 .. L_b - 1.
+ *   scores [B,Lmax] fp32 (as hca_dsa_index writes them), seqlens [B] int32
+ *   idx    [B,k] int32 output: kept positions in increasing order, then -1 where L_b < k
+ * Equal scores are taken in increasing position order, so the result is unique.
+ */
+hca_status_t hca_dsa_topk(const float* scores, const int* seqlens, int* idx, int B, int Lmax, int k,
+                          hca_stream_t stream);
+
+/*
+ * hca_dsa_attend -- core attention of each sequence's Hq query heads over its kept positions.
+ *   q    [B,Hq,d] bf16;  k, v [B,Lmax,d] bf16 (one row per position, shared by the heads)
+ *   idx  [B,kmax] int32 from hca_dsa_topk (-1 entries and entries past min(kmax, L_b) unused;
+ *        an entry >= Lmax is reported as HCA_ERR_DEVICE_INPUT and not read)
+ *   seqlens [B] int32;  out [B,Hq,d] fp32;  scale: logit scale (typically 1/sqrt(d))
+ * Supported: d == 256, Hq <= 64.  bf16 operands, fp32 accumulation, P rounded to bf16.
+ */
+hca_status_t hca_dsa_attend(const void* q, const void* k, const void* v, const int* idx, const int* seqlens,
+                            float* out, int B, int Hq, int d, int Lmax, int kmax, float scale,
+                            hca_stream_t stream);
+
+/*
  * hca_decode_workspace_size -- bytes of device workspace hca_decode needs for a batch
  * of B sequences on the CURRENT device (split-KV partial results).  Returns 0 for
  * invalid sizes.
