@@ -38,7 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "HCA decode queries/s, prefill TFLOP/s, % of HBM/TC roofline (1 B200)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-CONFIG_KEYS = ("tiny_prefill", "decode_128k", "prefill_128k", "decode_1m", "ragged_paged")
+CONFIG_KEYS = ("tiny_prefill", "decode_128k", "prefill_128k", "decode_1m", "ragged_paged", "dsa_decode_128k")
 
 
 def parse(argv=None):
@@ -882,6 +882,94 @@ def bench_ragged_paged(c):
     return res
 
 
+def bench_dsa_decode_128k(c):
+    """The sparse-attention decode step: indexer scores, top-k selection, core attention."""
+    hca, wl = c.hca, c.wl
+    cfg = wl.DSA_DECODE_128K
+    inp = wl.dsa_inputs(cfg, c.dev)
+    B, L = cfg.B, cfg.L
+    scale = 1.0 / np.sqrt(cfg.d)
+    scores = torch.empty((B, L), dtype=torch.float32, device=c.dev)
+    idx = torch.empty((B, cfg.topk), dtype=torch.int32, device=c.dev)
+    out = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.float32, device=c.dev)
+
+    def index():
+        hca.dsa_index(inp["q_idx"], inp["w_idx"], inp["k_idx"], inp["seqlens"], scores=scores)
+
+    def topk():
+        hca.dsa_topk(scores, inp["seqlens"], cfg.topk, idx=idx)
+
+    def attend():
+        hca.dsa_attend(inp["q"], inp["k"], inp["v"], idx, inp["seqlens"], scale, out=out)
+
+    def step():
+        index()
+        topk()
+        attend()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    n = max(5, min(c.args.steps, 20))
+    s_ms = timed_calls(step, n, c.stream, c.sampler, flush=c.flush)
+    i_ms = timed_calls(index, n, c.stream, c.sampler, flush=c.flush)
+    k_ms = timed_calls(topk, n, c.stream, c.sampler, flush=c.flush)
+    a_ms = timed_calls(attend, n, c.stream, c.sampler, flush=c.flush)
+    hca.get_device_error()
+    ts, ti, tk, ta = (c.median_s(x) for x in (s_ms, i_ms, k_ms, a_ms))
+    # algorithmic bytes: the indexer reads every indexer key once and writes the scores; the
+    # selection reads the scores; the attention reads the kept key and value rows, q, writes out
+    i_bytes = B * L * cfg.dI * 2 + B * cfg.HI * (cfg.dI * 2 + 4) + B * L * 4
+    k_bytes = B * L * 4 + B * cfg.topk * 4
+    a_bytes = B * cfg.topk * (2 * cfg.d * 2 + 4) + B * cfg.Hq * cfg.d * (2 + 4)
+    res = {"workload": cfg.name, "what": "hca_dsa_index + hca_dsa_topk + hca_dsa_attend, inputs resident",
+           "B": B, "L": L, "HI": cfg.HI, "dI": cfg.dI, "topk": cfg.topk, "Hq": cfg.Hq, "d": cfg.d,
+           "us": ts * 1e6, "queries_per_s": B / ts,
+           "algorithmic_bytes": i_bytes + k_bytes + a_bytes,
+           "index": {"us": ti * 1e6, "algorithmic_bytes": i_bytes, "roofline": c.hbm_roof("dsa_index_kernel", i_bytes, ti)},
+           "topk": {"us": tk * 1e6, "algorithmic_bytes": k_bytes, "roofline": c.hbm_roof("dsa_topk_kernel", k_bytes, tk)},
+           "attend": {"us": ta * 1e6, "algorithmic_bytes": a_bytes, "roofline": c.hbm_roof("dsa_attend_kernel", a_bytes, ta)},
+           "roofline": c.hbm_roof("dsa_index_kernel + dsa_topk_kernel + dsa_attend_kernel",
+                                  i_bytes + k_bytes + a_bytes, ts)}
+    if c.oracle_on:
+        import oracle
+        from oracle import dsa as od
+        f64 = lambda t: oracle.bits_to_f64(oracle.bf16_bits(t))  # noqa: E731
+        tm = OracleTimer()
+        sel_b = [0, 31, 63]
+        worst = {"scores_rel": 0.0, "out_max_abs": 0.0, "out_mean_abs": 0.0, "kept_outside_bound": 0}
+        for b in sel_b:
+            qi, ki, wi = f64(inp["q_idx"][b:b + 1]), f64(inp["k_idx"][b:b + 1]), inp["w_idx"][b:b + 1].cpu().numpy()
+            lens = np.array([L])
+            ref_s = tm(od.index_scores, qi, wi, ki, lens)[0]
+            got_s = scores[b].double().cpu().numpy()
+            bound = 2.0 ** -20 * (np.abs(ki[0] @ qi[0].T) @ np.abs(wi[0].astype(np.float64))) + 1e-6
+            worst["scores_rel"] = max(worst["scores_rel"], float(np.max(np.abs(got_s - ref_s) / bound)))
+            ridx = tm(od.select_topk, ref_s[None], lens, cfg.topk)[0]
+            kept = idx[b].cpu().numpy()
+            kth = np.sort(ref_s)[::-1][cfg.topk - 1]
+            worst["kept_outside_bound"] += int(np.sum(ref_s[kept] < kth - 2 * bound.max()))
+            # the attention over the GPU's kept positions (its selection is checked just above)
+            ro = tm(od.sparse_attend, f64(inp["q"][b:b + 1]), f64(inp["k"][b:b + 1]), f64(inp["v"][b:b + 1]),
+                    kept[None], scale)[0]
+            e = np.abs(out[b].double().cpu().numpy() - ro)
+            worst["out_max_abs"] = max(worst["out_max_abs"], float(e.max()))
+            worst["out_mean_abs"] = max(worst["out_mean_abs"], float(e.mean()))
+            worst["same_selection_as_oracle"] = worst.get("same_selection_as_oracle", True) and bool(np.array_equal(kept, ridx))
+        res["oracle"] = {"seconds": tm.s, "sequences": len(sel_b), "cores": oracle.num_threads(),
+                         "seconds_full_extrapolated": tm.s * B / len(sel_b),
+                         "scope": "oracle.dsa on 3 of the 64 sequences (scores, selection, attention)"}
+        res["parity"] = dict(worst, within_tolerance=bool(worst["scores_rel"] <= 1.0 and worst["kept_outside_bound"] == 0
+                                                          and worst["out_max_abs"] <= 1e-2
+                                                          and worst["out_mean_abs"] <= 1e-3),
+                             bar="scores within 2^-20 sum|w||q.k|; kept positions a top-k within that bound; "
+                                 "attention max abs 1e-2, mean abs 1e-3")
+    del inp, scores, idx, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline_sample(ref_cache, target_s=10.0):
     """The oracle as it stands, on this host, for a bounded sample of the headline workload: the
     oracle's decode of the whole 64-query batch over its own compressed cache, repeated for about
@@ -922,7 +1010,8 @@ def main(argv=None):
         cpu_base = cpu_baseline_sample(ref_cache)
     del ref_cache
     runners = {"tiny_prefill": bench_tiny_prefill, "prefill_128k": bench_prefill_128k,
-               "decode_1m": bench_decode_1m, "ragged_paged": bench_ragged_paged}
+               "decode_1m": bench_decode_1m, "ragged_paged": bench_ragged_paged,
+               "dsa_decode_128k": bench_dsa_decode_128k}
     for key in CONFIG_KEYS:
         if key in runners and key in want:
             configs[key] = runners[key](c)

@@ -297,6 +297,17 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
     const int tid = threadIdx.x, lane = tid & 31;
     uint32_t prefix = 0, pmask = 0;
     int remaining = kk;                     // how many of the largest keys still to place
+    // 4 consecutive positions per thread and round: 16-byte loads when the row is 16-byte aligned
+    const bool vec = ((reinterpret_cast<uintptr_t>(sc) & 15u) == 0);
+    auto load4 = [&](int s, float* f) {
+        if (vec && s + 3 < L) {
+            const float4 x = __ldg(reinterpret_cast<const float4*>(sc + s));
+            f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) f[e] = s + e < L ? __ldg(sc + s + e) : -INFINITY;
+        }
+    };
     if (kk < L) {
         // three digit passes, most significant first: 11, 11 and 10 bits
         for (int pass = 0; pass < 3; ++pass) {
@@ -304,20 +315,21 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
             const int nbins = pass == 2 ? 1024 : 2048;
             for (int i = tid; i < 2048; i += kTopkThreads) hist[i] = 0;
             __syncthreads();
-            for (int base = 0; base < L; base += kTopkThreads) {
-                const int s = base + tid;
-                bool in = false;
-                uint32_t bin = 0;
-                if (s < L) {
-                    const uint32_t key = dsa_key(__ldg(sc + s));
-                    in = (key & pmask) == prefix;
-                    bin = (key >> shift) & (uint32_t)(nbins - 1);
-                }
-                // warp-aggregated increments: lanes with the same bin add once
-                const uint32_t act = __ballot_sync(0xffffffffu, in);
-                if (in) {
-                    const uint32_t peers = __match_any_sync(act, bin);
-                    if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
+            for (int base = 0; base < L; base += 4 * kTopkThreads) {
+                const int s = base + 4 * tid;
+                float f[4];
+                load4(s, f);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t key = dsa_key(f[e]);
+                    const bool in = s + e < L && (key & pmask) == prefix;
+                    const uint32_t bin = (key >> shift) & (uint32_t)(nbins - 1);
+                    // warp-aggregated increments: lanes with the same bin add once
+                    const uint32_t act = __ballot_sync(0xffffffffu, in);
+                    if (in) {
+                        const uint32_t peers = __match_any_sync(act, bin);
+                        if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
+                    }
                 }
             }
             __syncthreads();
@@ -344,30 +356,41 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
             __syncthreads();
         }
     }
-    // keep every key above the threshold key `prefix` and the first `remaining` keys equal to
-    // it, in position order (each thread takes a contiguous chunk of positions).  With all
-    // positions kept, prefix = 0 and remaining = 0: every finite score's key is above 0.
-    const int chunk = (L + kTopkThreads - 1) / kTopkThreads;
-    const int s0 = min(L, tid * chunk), s1 = min(L, s0 + chunk);
-    int n_gt = 0, n_eq = 0;
-    for (int s = s0; s < s1; ++s) {
-        const uint32_t key = dsa_key(__ldg(sc + s));
-        n_gt += key > prefix;
-        n_eq += key == prefix;
-    }
-    int tot;
-    const int eq_before = dsa_block_scan(n_eq, wsum, &tot);
-    const int keep_eq = max(0, min(n_eq, remaining - eq_before));
-    int o = dsa_block_scan(n_gt + keep_eq, wsum, &tot);
-    int eq_rank = eq_before;
-    for (int s = s0; s < s1; ++s) {
-        const uint32_t key = dsa_key(__ldg(sc + s));
-        if (key > prefix) {
-            out[o++] = s;
-        } else if (key == prefix) {
-            if (eq_rank < remaining) out[o++] = s;
-            ++eq_rank;
+    // keep every key above the threshold key `prefix` and the first `remaining` keys equal to it,
+    // in position order, rounds of 4096 positions: one block scan per round gives each thread the
+    // larger and equal keys before its four.  With all positions kept, prefix = 0 and remaining =
+    // 0: every finite score's key is above 0.
+    int o_base = 0, eq_seen = 0;
+    for (int base = 0; base < L; base += 4 * kTopkThreads) {
+        const int s = base + 4 * tid;
+        float f[4];
+        load4(s, f);
+        uint32_t key[4];
+        int n_gt = 0, n_eq = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            key[e] = dsa_key(f[e]);
+            const bool live = s + e < L;
+            n_gt += live && key[e] > prefix;
+            n_eq += live && key[e] == prefix;
         }
+        int tot;
+        const int pre = dsa_block_scan(n_gt + (n_eq << 16), wsum, &tot);
+        int gt_before = pre & 0xffff, eq_before = eq_seen + (pre >> 16);
+        int o = o_base + gt_before + max(0, min(eq_before - eq_seen, remaining - eq_seen));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (s + e >= L) break;
+            if (key[e] > prefix) {
+                out[o++] = s + e;
+            } else if (key[e] == prefix) {
+                if (eq_before < remaining) out[o++] = s + e;
+                ++eq_before;
+            }
+        }
+        const int tot_gt = tot & 0xffff, tot_eq = tot >> 16;
+        o_base += tot_gt + max(0, min(tot_eq, remaining - eq_seen));
+        eq_seen += tot_eq;
     }
     for (int i = kk + tid; i < p.k; i += kTopkThreads) out[i] = -1;
 }
@@ -430,11 +453,13 @@ __device__ __forceinline__ float dsa_colred32(float* t, int lane) {
 __device__ __forceinline__ void dsa_gather_rows(uint8_t* dst, const __nv_bfloat16* src_b, const int* idx_t, int nvalid,
                                                 int Lmax, int w, int lane) {
     const int slab = lane >> 3, c = lane & 7;
-#pragma unroll 4
+    // the warp's 32 positions in one coalesced load, handed to the whole warp row by row
+    const int mine = 32 * w + lane < nvalid ? __ldg(idx_t + 32 * w + lane) : -1;
+#pragma unroll 8
     for (int i = 0; i < 32; ++i) {
         const int row = 32 * w + i;
         uint8_t* d = dst + slab * kAttSlab + dsa_sw(row, c);
-        int pos = row < nvalid ? __ldg(idx_t + row) : -1;
+        int pos = __shfl_sync(0xffffffffu, mine, i);
         if (pos >= Lmax) {                      // a position past the buffer: reported, not read
             if (lane == 0) record_error(HCA_ERR_DEVICE_INPUT);
             pos = -1;

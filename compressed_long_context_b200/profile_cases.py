@@ -8,6 +8,7 @@
     python -m compressed_long_context_b200.profile_cases append   [--reps N]
     python -m compressed_long_context_b200.profile_cases gate     [--reps N]
     python -m compressed_long_context_b200.profile_cases backward [--reps N] [--T tokens]
+    python -m compressed_long_context_b200.profile_cases dsa      [--reps N]   (index + topk + attend)
 
 Each case keeps its working set larger than the 126 MB L2 (so DRAM counters mean
 something) but a few GB at most, and launches the kernel `--reps` times after one
@@ -21,8 +22,8 @@ import math
 
 import torch
 
-from . import (append, append_state_size, compress, decode, decode_workspace_size, gate_logits, get_device_error,
-               prefill, prefill_backward, vha)
+from . import (append, append_state_size, compress, decode, decode_workspace_size, dsa_attend, dsa_index, dsa_topk,
+               gate_logits, get_device_error, prefill, prefill_backward, vha)
 from . import workloads as wl
 
 
@@ -130,6 +131,22 @@ def run(case: str, reps: int, B_override: int = 0, L_override: int = 0, T_overri
         keys = sum(max(0, (t - cfg.W + 1) // 128) + min(cfg.W, t + 1) for t in range(cfg.T))
         nbytes = None
         flops = 5 * 2.0 * cfg.Hq * keys * cfg.d
+    elif case == "dsa":
+        # the sparse-attention decode step at 16 sequences of 32768 positions (64 MB of indexer
+        # keys, 512 MB of key / value rows)
+        cfg = wl.DSA_DECODE_128K
+        cfg = wl.DsaWorkload(cfg.name, B=B_override or 16, L=L_override or 32768, HI=cfg.HI, dI=cfg.dI, topk=cfg.topk,
+                             Hq=cfg.Hq, d=cfg.d, seed=cfg.seed)
+        inp = wl.dsa_inputs(cfg, dev)
+        scores = torch.empty((cfg.B, cfg.L), dtype=torch.float32, device=dev)
+        idx = torch.empty((cfg.B, cfg.topk), dtype=torch.int32, device=dev)
+        out = torch.empty((cfg.B, cfg.Hq, cfg.d), dtype=torch.float32, device=dev)
+
+        def fn():
+            dsa_index(inp["q_idx"], inp["w_idx"], inp["k_idx"], inp["seqlens"], scores=scores)
+            dsa_topk(scores, inp["seqlens"], cfg.topk, idx=idx)
+            dsa_attend(inp["q"], inp["k"], inp["v"], idx, inp["seqlens"], 1 / math.sqrt(cfg.d), out=out)
+        nbytes = cfg.B * cfg.L * (cfg.dI * 2 + 8) + cfg.B * cfg.topk * (4 * cfg.d + 8)
     else:
         raise ValueError(case)
     _last_fn[0] = fn
@@ -182,7 +199,7 @@ def run_flushed(args) -> dict:
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["compress", "decode", "paged", "prefill", "vha", "append", "gate", "backward"])
+    ap.add_argument("case", choices=["compress", "decode", "paged", "prefill", "vha", "append", "gate", "backward", "dsa"])
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--B", type=int, default=0, help="decode batch (default 64)")
     ap.add_argument("--L", type=int, default=0, help="decode context length (default 131072)")

@@ -179,3 +179,41 @@ def paged_decode_inputs(wl: Workload, device="cpu", seqlens=None):
     return {"q": q, "kc": kc, "vc": vc, "page_table": table.to(device), "kw": kw, "vw": vw,
             "seqlens": seqlens.to(device), "gq": gq, "gk": gk, "gate": gate,
             "page_size": ps, "max_pages": maxp}
+
+
+@dataclass(frozen=True)
+class DsaWorkload:
+    """The sparse-attention layers' decode step: B sequences of context L, an indexer of H_I
+    heads of d_I dims, the top-k positions kept, Hq query heads of d dims over one key and one
+    value row per position (the pages' MLA layers use 256-dim heads)."""
+    name: str
+    B: int
+    L: int
+    HI: int
+    dI: int
+    topk: int
+    Hq: int
+    d: int
+    seed: int
+
+
+DSA_DECODE_128K = DsaWorkload("dsa_decode_B64_L131072_topk2048_d256", B=64, L=131072, HI=16, dI=64, topk=2048,
+                              Hq=64, d=256, seed=6)
+
+
+def dsa_inputs(wl: DsaWorkload, device="cpu"):
+    """Draw order: indexer queries, indexer weights, indexer keys, queries, keys, values.
+
+    q_idx [B,H_I,d_I] ~ N(0,1) bf16, w_idx [B,H_I] ~ U(0.5,1.5) fp32, k_idx [B,L,d_I] ~ N(0,1)
+    bf16, q [B,Hq,d], k, v [B,L,d] ~ N(0,1) bf16, seqlens [B] int32 (= L).
+    """
+    g = _gen(device, wl.seed)
+    B, L = wl.B, wl.L
+    q_idx = _normal_bf16((B, wl.HI, wl.dI), g, device)
+    w_idx = torch.rand((B, wl.HI), generator=g, device=device, dtype=torch.float32) + 0.5
+    k_idx = _normal_bf16_chunked((B, L, wl.dI), g, device)
+    q = _normal_bf16((B, wl.Hq, wl.d), g, device)
+    k = _normal_bf16_chunked((B, L, wl.d), g, device)
+    v = _normal_bf16_chunked((B, L, wl.d), g, device)
+    seqlens = torch.full((B,), L, dtype=torch.int32, device=device)
+    return {"q_idx": q_idx, "w_idx": w_idx, "k_idx": k_idx, "q": q, "k": k, "v": v, "seqlens": seqlens}
