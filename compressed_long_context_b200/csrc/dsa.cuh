@@ -11,7 +11,7 @@
 //
 // Kernels:
 //   dsa_index_kernel   one persistent CTA per SM over all (sequence, 128-position tile) pairs:
-//                      a tile's indexer keys (128 x 64 bf16, 16 KB) arrive by TMA into an 8-slot
+//                      a tile's indexer keys (128 x 64 bf16, 16 KB) arrive by TMA into a 12-slot
 //                      ring, one tcgen05 MMA chain gives the 128 x H_I dot products in tensor
 //                      memory (two buffers), four epilogue warps apply ReLU and the head weights
 //                      and write the scores (fp32).  HBM-bound on the keys.
@@ -54,15 +54,17 @@ __device__ __forceinline__ bool dsa_group_wait128(uint64_t* bar, uint32_t parity
 // ------------------------------------------------------------------------------------- indexer
 
 constexpr int kIdxThreads = 192;           // producer, MMA issuer, 4 epilogue warps
-constexpr int kIdxRing = 8;
+constexpr int kIdxRing = 12;
 constexpr uint32_t kIdxSlab = 128 * 128;   // 128 positions x 64 dims bf16
 constexpr uint32_t kIdxQBytes = kDsaMaxHI * 128;
 constexpr uint32_t kIdxSmRing = 0;
 constexpr uint32_t kIdxSmQ = kIdxSmRing + kIdxRing * kIdxSlab;          // two query buffers
 constexpr uint32_t kIdxSmBar = kIdxSmQ + 2 * kIdxQBytes;
-constexpr uint32_t kIdxSmW = kIdxSmBar + 256;                           // two weight buffers [64]
+constexpr int kIdxNumBars = 2 * kIdxRing + 9;                           // ring full / empty, q, acc, drain
+constexpr uint32_t kIdxSmW = kIdxSmBar + ((kIdxNumBars * 8 + 15) & ~15);  // two weight buffers [64]
 constexpr uint32_t kIdxSmem = kIdxSmW + 2 * kDsaMaxHI * 4 + 16;
 static_assert(kIdxSmQ % 1024 == 0 && kIdxSlab % 1024 == 0, "swizzled operands 1024-aligned");
+static_assert(kIdxSmem <= 232448, "indexer shared memory exceeds the per-block limit");
 
 struct DsaIndexParams {
     const float* w;          // [B, HI]
@@ -492,11 +494,18 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
     float* mref = reinterpret_cast<float*>(sm + kAttSmM);
     float* alpha = reinterpret_cast<float*>(sm + kAttSmA);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.x;
+    // a cluster of two CTAs per sequence: rank 0 takes the first half of the kept tiles, rank 1
+    // the rest; rank 1 hands its partial (max, sum, O^T) to rank 0, which merges and writes out
+    const int b = blockIdx.x >> 1;
+    uint32_t rank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
     int L = __ldg(p.seqlens + b);
     L = L < 0 ? 0 : (L > p.Lmax ? p.Lmax : L);
     const int count = min(p.kmax, L);
-    const int nt = (count + 127) / 128;
+    const int nt_all = (count + 127) / 128;
+    const int nt_first = (nt_all + 1) / 2;
+    const int jt0 = rank ? nt_first : 0;                  // this CTA's first tile of the sequence
+    const int nt = rank ? nt_all - nt_first : nt_first;   // and its number of tiles
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         mbar_init(q_full, 1);
@@ -572,7 +581,7 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
         for (int h = 0; h < 64; ++h) lsum[h] = 0.f;
         bool ok = true;
         if (nt > 0) {
-            dsa_gather_rows(sm + kAttSmK, kb, idx_b, count, p.Lmax, w, lane);
+            dsa_gather_rows(sm + kAttSmK, kb, idx_b + 128 * jt0, count - 128 * jt0, p.Lmax, w, lane);
             cp_async_commit();
             cp_async_wait<0>();
             fence_proxy_async_smem();
@@ -580,8 +589,8 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             if (lane == 0) mbar_arrive(k_full);
         }
         for (int j = 0; ok && j < nt; ++j) {
-            const int* idx_t = idx_b + 128 * j;
-            const int nvalid = count - 128 * j;
+            const int* idx_t = idx_b + 128 * (jt0 + j);
+            const int nvalid = count - 128 * (jt0 + j);
             // the value rows of this tile (the previous PV is done: waited at the end of the last tile)
             dsa_gather_rows(sm + kAttSmV, vb, idx_t, nvalid, p.Lmax, w, lane);
             cp_async_commit();
@@ -680,7 +689,7 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             tc_fence_after();
         }
         cp_async_wait<0>();
-        // ---- out[h][ch] = O^T[ch][h] / l[h]; l from every row's share (column sums, then 4 warps)
+        // ---- this CTA's softmax sums per head (column sums, then the 4 warps) and its max
         {
             float t[32];
 #pragma unroll
@@ -693,25 +702,87 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x >= 32 && threadIdx.x < 96) {
             const int h = threadIdx.x - 32;
-            alpha[h] = (ok && nt > 0) ? 1.f / ((red[h] + red[64 + h]) + (red[128 + h] + red[192 + h])) : NAN;
+            alpha[h] = nt > 0 ? (red[h] + red[64 + h]) + (red[128 + h] + red[192 + h]) : 0.f;   // l
+            if (nt == 0) mref[h] = -INFINITY;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (nt > 0) {
-            float* ob = p.out + (size_t)b * p.Hq * kDsaD;
+        if (threadIdx.x == 32) misc[2] = ok ? 1 : 0;
+        tc_fence_before();
+    }
+    // ---- merge the two halves in rank 0: out = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M))
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // rank 0 no longer reads its key / value buffers (its MMAs are drained): rank 1 may write there
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    float* o1 = reinterpret_cast<float*>(sm + kAttSmK);              // rank 1's O^T [256 ch][64 heads]
+    float* ml1 = reinterpret_cast<float*>(sm + kAttSmV);             // rank 1's max [64], sum [64], ok
+    if (rank == 1 && warp >= 1) {
+        const int w = warp & 3;
+        const int r = 32 * w + lane;
+        const uint32_t lane_off = (uint32_t)(32 * w) << 16;
+        uint32_t ro, rml;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(ro) : "r"(smem_u32(o1)));
+        asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(rml) : "r"(smem_u32(ml1)));
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll 1
-                for (int c16 = 0; c16 < 64; c16 += 16) {
-                    float o[16];
+            for (int c16 = 0; c16 < 64; c16 += 16) {
+                float o[16];
+                if (nt > 0) {
                     tmem_ld16(tmem + lane_off + tO + 64 * c + c16, o);
                     tmem_wait_ld();
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int h = c16 + i;
-                        if (h < p.Hq) ob[(size_t)h * kDsaD + 128 * c + r] = o[i] * alpha[h];
-                    }
+                    for (int i = 0; i < 16; ++i) o[i] = 0.f;
                 }
+                const uint32_t dst = ro + (uint32_t)(((128 * c + r) * 64 + c16) * 4);
+#pragma unroll
+                for (int i = 0; i < 16; i += 4)
+                    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                                 :: "r"(dst + 4 * i), "f"(o[i]), "f"(o[i + 1]), "f"(o[i + 2]), "f"(o[i + 3]) : "memory");
+            }
+        if (threadIdx.x >= 32 && threadIdx.x < 96) {
+            const int h = threadIdx.x - 32;
+            asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(rml + 4 * h), "f"(mref[h]) : "memory");
+            asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(rml + 256 + 4 * h), "f"(alpha[h]) : "memory");
         }
+        if (threadIdx.x == 32)
+            asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(rml + 512), "f"(misc[2] ? 1.f : 0.f) : "memory");
+        tc_fence_before();
+    }
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (rank == 0 && warp >= 1) {
+        const int w = warp & 3;
+        const int r = 32 * w + lane;
+        const uint32_t lane_off = (uint32_t)(32 * w) << 16;
+        tc_fence_after();
+        if (threadIdx.x >= 32 && threadIdx.x < 96) {
+            const int h = threadIdx.x - 32;
+            const float m0 = mref[h], m1 = ml1[h];
+            const float M = fmaxf(m0, m1);
+            const float e0 = ex2(m0 - M), e1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+            const float inv = 1.f / (alpha[h] * e0 + ml1[64 + h] * e1);
+            const bool good = misc[2] && ml1[128] != 0.f;
+            red[h] = good ? e0 * inv : NAN;          // weight of this CTA's O^T
+            red[64 + h] = good ? e1 * inv : NAN;     // weight of rank 1's
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        float* ob = p.out + (size_t)b * p.Hq * kDsaD;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c)
+#pragma unroll 1
+            for (int c16 = 0; c16 < 64; c16 += 16) {
+                float o[16];
+                tmem_ld16(tmem + lane_off + tO + 64 * c + c16, o);
+                tmem_wait_ld();
+                const float* x1 = o1 + (128 * c + r) * 64 + c16;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int h = c16 + i;
+                    if (h < p.Hq) ob[(size_t)h * kDsaD + 128 * c + r] = fmaf(o[i], red[h], x1[i] * red[64 + h]);
+                }
+            }
         tc_fence_before();
     }
     __syncwarp();

@@ -910,6 +910,7 @@ extern "C" hca_status_t hca_dsa_attend(const void* q, const void* k, const void*
     using namespace hca;
     if (B < 0 || Hq < 1 || Lmax < 1 || kmax < 1) return HCA_ERR_INVALID_ARG;
     if (d != kDsaD || Hq > kDsaHeads) return HCA_ERR_UNSUPPORTED;
+    if (B > (1 << 30)) return HCA_ERR_INVALID_ARG;
     if (!(scale == scale)) return HCA_ERR_INVALID_ARG;
     if (B == 0) return HCA_OK;
     if (!q || !k || !v || !idx || !seqlens || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
@@ -928,6 +929,22 @@ extern "C" hca_status_t hca_dsa_attend(const void* q, const void* k, const void*
     p.out = out;
     p.B = B; p.Hq = Hq; p.Lmax = Lmax; p.kmax = kmax;
     p.scale_log2 = scale * 1.4426950408889634f;
-    dsa_attend_kernel<<<(unsigned)B, kAttThreads, kAttSmem, reinterpret_cast<cudaStream_t>(stream)>>>(p, tq);
-    return launch_status();
+    // a cluster of two CTAs per sequence (each takes half of the kept positions)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * B), 1, 1);
+    cfg.blockDim = dim3(kAttThreads, 1, 1);
+    cfg.dynamicSmemBytes = kAttSmem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, dsa_attend_kernel, p, tq) != cudaSuccess) {
+        cudaGetLastError();
+        return HCA_ERR_CUDA;
+    }
+    return HCA_OK;
 }
