@@ -171,3 +171,32 @@ def test_dsa_rejects_unsupported(cuda_device, libhca):
     q, w, k = int_inputs(cuda_device, 1, 24, 100, seed=1)     # 24 indexer heads: not a multiple of 16
     with pytest.raises(hca.HCAError):
         hca.dsa_index(q, w, k, torch.tensor([100], dtype=torch.int32, device=cuda_device))
+
+
+def test_dsa_128k_sequences_sampled(cuda_device, libhca):
+    """Four sequences of the bench's 128K sparse-attention workload shape (H_I = 16, d_I = 64,
+    top-2048, 64 heads of 256), two of them checked in full against the oracle: scores within
+    the rounding bound, the kept positions a top-k of the oracle's scores within it, and the
+    attention over the kept positions within the attention bar."""
+    from compressed_long_context_b200 import workloads as wl
+    cfg = wl.DsaWorkload("dsa_test", B=4, L=131072, HI=16, dI=64, topk=2048, Hq=64, d=256, seed=12)
+    inp = wl.dsa_inputs(cfg, cuda_device)
+    scale = 1.0 / np.sqrt(cfg.d)
+    out, idx, sc = hca.dsa_decode(inp["q_idx"], inp["w_idx"], inp["k_idx"], inp["q"], inp["k"], inp["v"],
+                                  inp["seqlens"], cfg.topk, scale)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    for b in (0, 3):
+        qi, ki = f64(inp["q_idx"][b:b + 1]), f64(inp["k_idx"][b:b + 1])
+        wi = inp["w_idx"][b:b + 1].cpu().numpy().astype(np.float64)
+        ref = od.index_scores(qi, wi, ki, np.array([cfg.L]))[0]
+        got = sc[b].double().cpu().numpy()
+        bound = 2.0 ** -20 * (np.abs(ki[0] @ qi[0].T) @ np.abs(wi[0])) + 1e-6
+        assert np.all(np.abs(got - ref) <= bound)
+        kept = idx[b].cpu().numpy()
+        kth = np.sort(ref)[::-1][cfg.topk - 1]
+        assert np.all(kept >= 0) and np.all(np.diff(kept) > 0)
+        assert np.all(ref[kept] >= kth - 2 * bound.max())
+        ro = od.sparse_attend(f64(inp["q"][b:b + 1]), f64(inp["k"][b:b + 1]), f64(inp["v"][b:b + 1]), kept[None], scale)[0]
+        err = np.abs(out[b].double().cpu().numpy() - ro)
+        assert err.max() <= MAX_TOL and err.mean() <= MEAN_TOL
