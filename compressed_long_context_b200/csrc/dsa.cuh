@@ -10,8 +10,8 @@
 //   out[h] = softmax_s(scale * q[h] . k[s]) v[s] over the kept s, one key / value row per position
 //
 // Kernels:
-//   dsa_index_kernel   one persistent CTA per SM over all (sequence, 128-position tile) pairs:
-//                      a tile's indexer keys (128 x 64 bf16, 16 KB) arrive by TMA into a 12-slot
+//   dsa_index_kernel   two persistent CTAs per SM over all (sequence, 128-position tile) pairs:
+//                      a tile's indexer keys (128 x 64 bf16, 16 KB) arrive by TMA into a 6-slot
 //                      ring, one tcgen05 MMA chain gives the 128 x H_I dot products in tensor
 //                      memory (two buffers), four epilogue warps apply ReLU and the head weights
 //                      and write the scores (fp32).  HBM-bound on the keys.
@@ -54,7 +54,7 @@ __device__ __forceinline__ bool dsa_group_wait128(uint64_t* bar, uint32_t parity
 // ------------------------------------------------------------------------------------- indexer
 
 constexpr int kIdxThreads = 192;           // producer, MMA issuer, 4 epilogue warps
-constexpr int kIdxRing = 12;
+constexpr int kIdxRing = 6;                // two CTAs per SM: 12 slots per SM
 constexpr uint32_t kIdxSlab = 128 * 128;   // 128 positions x 64 dims bf16
 constexpr uint32_t kIdxQBytes = kDsaMaxHI * 128;
 constexpr uint32_t kIdxSmRing = 0;
@@ -79,7 +79,24 @@ __device__ __forceinline__ int dsa_len(const DsaIndexParams& p, int b) {
     return L < 0 ? 0 : (L > p.Lmax ? p.Lmax : L);
 }
 
-__global__ void __launch_bounds__(kIdxThreads, 1)
+// Walks (sequence, tile) pairs in order from a flat index, with the sequence's length cached.
+struct DsaTileWalk {
+    int b, t, L;
+    __device__ DsaTileWalk(const DsaIndexParams& p, long long i) {
+        b = (int)(i / p.ntile);
+        t = (int)(i - (long long)b * p.ntile);
+        L = b < p.B ? dsa_len(p, b) : 0;
+    }
+    __device__ void next(const DsaIndexParams& p) {
+        if (++t == p.ntile) {
+            t = 0;
+            ++b;
+            L = b < p.B ? dsa_len(p, b) : 0;
+        }
+    }
+};
+
+__global__ void __launch_bounds__(kIdxThreads, 2)
 dsa_index_kernel(const DsaIndexParams p, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k) {
     extern __shared__ __align__(1024) uint8_t dsmem[];
     if (smem_u32(dsmem) & 1023u) {
@@ -129,9 +146,10 @@ dsa_index_kernel(const DsaIndexParams p, const __grid_constant__ CUtensorMap tm_
             uint32_t op = 0, nq = 0;
             int cur_b = -1;
             bool ok = true;
-            for (long long i = t_begin; ok && i < t_end; ++i) {
-                const int b = (int)(i / p.ntile), t = (int)(i - (long long)b * p.ntile);
-                if (128 * t >= dsa_len(p, b)) continue;           // past the sequence: no keys to read
+            DsaTileWalk wk(p, t_begin);
+            for (long long i = t_begin; ok && i < t_end; ++i, wk.next(p)) {
+                const int b = wk.b, t = wk.t;
+                if (128 * t >= wk.L) continue;                    // past the sequence: no keys to read
                 if (b != cur_b) {
                     const uint32_t qb = nq & 1;
                     if (!mbar_wait(&q_empty[qb], ((nq >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -155,9 +173,10 @@ dsa_index_kernel(const DsaIndexParams p, const __grid_constant__ CUtensorMap tm_
         uint32_t op = 0, nq = 0, na = 0;
         int cur_b = -1;
         bool ok = true;
-        for (long long i = t_begin; ok && i < t_end; ++i) {
-            const int b = (int)(i / p.ntile), t = (int)(i - (long long)b * p.ntile);
-            if (128 * t >= dsa_len(p, b)) continue;
+        DsaTileWalk wk(p, t_begin);
+        for (long long i = t_begin; ok && i < t_end; ++i, wk.next(p)) {
+            const int b = wk.b, t = wk.t;
+            if (128 * t >= wk.L) continue;
             if (b != cur_b) {
                 if (cur_b >= 0 && lane == 0) mma_commit(&q_empty[(nq - 1) & 1]);   // previous query buffer free
                 if (!warp_wait(&q_full[nq & 1], (nq >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -195,9 +214,10 @@ dsa_index_kernel(const DsaIndexParams p, const __grid_constant__ CUtensorMap tm_
         const int et = threadIdx.x - 64;          // 0..127
         uint32_t na = 0, nb = 0;
         int cur_b = -1;
-        for (long long i = t_begin; i < t_end; ++i) {
-            const int b = (int)(i / p.ntile), t = (int)(i - (long long)b * p.ntile);
-            const int L = dsa_len(p, b);
+        DsaTileWalk wk(p, t_begin);
+        for (long long i = t_begin; i < t_end; ++i, wk.next(p)) {
+            const int b = wk.b, t = wk.t;
+            const int L = wk.L;
             const int pos = 128 * t + r;
             if (128 * t >= L) {
                 if (pos < p.Lmax) p.scores[(size_t)b * p.Lmax + pos] = -INFINITY;
@@ -286,28 +306,56 @@ __device__ __forceinline__ int dsa_block_scan(int v, int* wsum, int* total) {
     return r;
 }
 
+constexpr int kTopkCluster = 4;            // CTAs per sequence, each over a quarter of the positions
+
+__device__ __forceinline__ void dsa_cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t dsa_mapa(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ int dsa_ld_cluster(uint32_t a) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void dsa_st_cluster(uint32_t a, int v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" :: "r"(a), "r"(v) : "memory");
+}
+
+// A cluster of kTopkCluster CTAs per sequence: each builds the digit histograms of its quarter of
+// the positions, rank 0 adds the four through distributed shared memory and picks the digit, and
+// in the last pass each CTA writes the kept positions of its quarter after those of the ranks
+// before it.
 __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopkParams p) {
     __shared__ int hist[2048];
     __shared__ int wsum[33];
-    __shared__ uint32_t sel[2];             // [0] digit chosen, [1] remaining after the pass
-    const int b = blockIdx.x;
+    __shared__ int sel[2];                  // [0] digit chosen, [1] remaining after the pass
+    __shared__ int counts[2 * kTopkCluster];   // rank 0: each rank's larger / equal key counts
+    uint32_t rank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    const int b = blockIdx.x / kTopkCluster;
     int L = __ldg(p.seqlens + b);
     L = L < 0 ? 0 : (L > p.Lmax ? p.Lmax : L);
     const float* sc = p.scores + (size_t)b * p.Lmax;
     int* out = p.idx + (size_t)b * p.k;
     const int kk = min(p.k, L);
     const int tid = threadIdx.x, lane = tid & 31;
+    // this CTA's quarter of the positions (a multiple of 4 long, for 16-byte loads)
+    const int qsize = (((L + kTopkCluster - 1) / kTopkCluster) + 3) & ~3;
+    const int q0 = min(L, (int)rank * qsize), q1 = min(L, q0 + qsize);
     uint32_t prefix = 0, pmask = 0;
     int remaining = kk;                     // how many of the largest keys still to place
-    // 4 consecutive positions per thread and round: 16-byte loads when the row is 16-byte aligned
     const bool vec = ((reinterpret_cast<uintptr_t>(sc) & 15u) == 0);
     auto load4 = [&](int s, float* f) {
-        if (vec && s + 3 < L) {
+        if (vec && s + 3 < q1) {
             const float4 x = __ldg(reinterpret_cast<const float4*>(sc + s));
             f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
         } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) f[e] = s + e < L ? __ldg(sc + s + e) : -INFINITY;
+            for (int e = 0; e < 4; ++e) f[e] = s + e < q1 ? __ldg(sc + s + e) : -INFINITY;
         }
     };
     if (kk < L) {
@@ -317,14 +365,14 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
             const int nbins = pass == 2 ? 1024 : 2048;
             for (int i = tid; i < 2048; i += kTopkThreads) hist[i] = 0;
             __syncthreads();
-            for (int base = 0; base < L; base += 4 * kTopkThreads) {
+            for (int base = q0; base < q1; base += 4 * kTopkThreads) {
                 const int s = base + 4 * tid;
                 float f[4];
                 load4(s, f);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const uint32_t key = dsa_key(f[e]);
-                    const bool in = s + e < L && (key & pmask) == prefix;
+                    const bool in = s + e < q1 && (key & pmask) == prefix;
                     const uint32_t bin = (key >> shift) & (uint32_t)(nbins - 1);
                     // warp-aggregated increments: lanes with the same bin add once
                     const uint32_t act = __ballot_sync(0xffffffffu, in);
@@ -334,55 +382,90 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
                     }
                 }
             }
-            __syncthreads();
-            // the digit holding the remaining-th largest key: suffix sums over bins, high to low
-            // (thread i takes bins 2i and 2i + 1, counted from the top)
-            const int hi_bin = nbins - 1 - 2 * tid;
-            const int c0 = (2 * tid < nbins) ? hist[hi_bin] : 0;
-            const int c1 = (2 * tid + 1 < nbins) ? hist[hi_bin - 1] : 0;
-            int tot;
-            const int before = dsa_block_scan(c0 + c1, wsum, &tot);     // keys in higher bins
-            if (2 * tid < nbins) {
-                if (before < remaining && before + c0 >= remaining) {
-                    sel[0] = (uint32_t)hi_bin;
-                    sel[1] = (uint32_t)(remaining - before);
-                } else if (2 * tid + 1 < nbins && before + c0 < remaining && before + c0 + c1 >= remaining) {
-                    sel[0] = (uint32_t)(hi_bin - 1);
-                    sel[1] = (uint32_t)(remaining - before - c0);
+            dsa_cluster_sync();             // every quarter's histogram is complete
+            if (rank == 0) {
+                // the digit holding the remaining-th largest key: suffix sums over the bins of the
+                // four histograms, high to low (thread i takes bins 2i and 2i + 1 from the top)
+                const int hi_bin = nbins - 1 - 2 * tid;
+                int c0 = 0, c1 = 0;
+                for (int r = 0; r < kTopkCluster; ++r) {
+                    if (2 * tid < nbins) c0 += dsa_ld_cluster(dsa_mapa(&hist[hi_bin], r));
+                    if (2 * tid + 1 < nbins) c1 += dsa_ld_cluster(dsa_mapa(&hist[hi_bin - 1], r));
                 }
+                int tot;
+                const int before = dsa_block_scan(c0 + c1, wsum, &tot);     // keys in higher bins
+                int dig = -1, rem = 0;
+                if (2 * tid < nbins) {
+                    if (before < remaining && before + c0 >= remaining) {
+                        dig = hi_bin;
+                        rem = remaining - before;
+                    } else if (2 * tid + 1 < nbins && before + c0 < remaining && before + c0 + c1 >= remaining) {
+                        dig = hi_bin - 1;
+                        rem = remaining - before - c0;
+                    }
+                }
+                if (dig >= 0)
+                    for (int r = 0; r < kTopkCluster; ++r) {
+                        dsa_st_cluster(dsa_mapa(&sel[0], r), dig);
+                        dsa_st_cluster(dsa_mapa(&sel[1], r), rem);
+                    }
             }
-            __syncthreads();
-            prefix |= sel[0] << shift;
+            dsa_cluster_sync();             // the digit is known everywhere; rank 0 is done reading
+            prefix |= (uint32_t)sel[0] << shift;
             pmask |= (uint32_t)(nbins - 1) << shift;
-            remaining = (int)sel[1];
-            __syncthreads();
+            remaining = sel[1];
         }
     }
     // keep every key above the threshold key `prefix` and the first `remaining` keys equal to it,
-    // in position order, rounds of 4096 positions: one block scan per round gives each thread the
-    // larger and equal keys before its four.  With all positions kept, prefix = 0 and remaining =
-    // 0: every finite score's key is above 0.
-    int o_base = 0, eq_seen = 0;
-    for (int base = 0; base < L; base += 4 * kTopkThreads) {
+    // in position order.  With all positions kept the passes are skipped (prefix = 0, remaining =
+    // kk = L): every key is at least 0, so every position is kept.  First the ranks' counts, to
+    // place each quarter after the previous ones.
+    int n_gt = 0, n_eq = 0;
+    for (int base = q0; base < q1; base += 4 * kTopkThreads) {
+        const int s = base + 4 * tid;
+        float f[4];
+        load4(s, f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t key = dsa_key(f[e]);
+            n_gt += s + e < q1 && key > prefix;
+            n_eq += s + e < q1 && key == prefix;
+        }
+    }
+    int tot, tot_eq_q;
+    dsa_block_scan(n_gt, wsum, &tot);       // the quarter's counts: two scans, as a quarter may
+    dsa_block_scan(n_eq, wsum, &tot_eq_q);  // hold 2^16 positions or more
+    if (tid == 0) {
+        dsa_st_cluster(dsa_mapa(&counts[2 * rank], 0), tot);
+        dsa_st_cluster(dsa_mapa(&counts[2 * rank + 1], 0), tot_eq_q);
+    }
+    dsa_cluster_sync();
+    int gt_pre = 0, eq_pre = 0;
+    for (uint32_t r = 0; r < rank; ++r) {
+        gt_pre += dsa_ld_cluster(dsa_mapa(&counts[2 * r], 0));
+        eq_pre += dsa_ld_cluster(dsa_mapa(&counts[2 * r + 1], 0));
+    }
+    int o_base = gt_pre + max(0, min(eq_pre, remaining)), eq_seen = eq_pre;
+    for (int base = q0; base < q1; base += 4 * kTopkThreads) {
         const int s = base + 4 * tid;
         float f[4];
         load4(s, f);
         uint32_t key[4];
-        int n_gt = 0, n_eq = 0;
+        int ng = 0, ne = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             key[e] = dsa_key(f[e]);
-            const bool live = s + e < L;
-            n_gt += live && key[e] > prefix;
-            n_eq += live && key[e] == prefix;
+            const bool live = s + e < q1;
+            ng += live && key[e] > prefix;
+            ne += live && key[e] == prefix;
         }
-        int tot;
-        const int pre = dsa_block_scan(n_gt + (n_eq << 16), wsum, &tot);
-        int gt_before = pre & 0xffff, eq_before = eq_seen + (pre >> 16);
+        const int pre = dsa_block_scan(ng + (ne << 16), wsum, &tot);
+        const int gt_before = pre & 0xffff;
+        int eq_before = eq_seen + (pre >> 16);
         int o = o_base + gt_before + max(0, min(eq_before - eq_seen, remaining - eq_seen));
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            if (s + e >= L) break;
+            if (s + e >= q1) break;
             if (key[e] > prefix) {
                 out[o++] = s + e;
             } else if (key[e] == prefix) {
@@ -394,7 +477,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
         o_base += tot_gt + max(0, min(tot_eq, remaining - eq_seen));
         eq_seen += tot_eq;
     }
-    for (int i = kk + tid; i < p.k; i += kTopkThreads) out[i] = -1;
+    if (rank == 0)
+        for (int i = kk + tid; i < p.k; i += kTopkThreads) out[i] = -1;
+    dsa_cluster_sync();                     // rank 0's counts stay readable until every rank is done
 }
 
 // ------------------------------------------------------------------------------------- attention

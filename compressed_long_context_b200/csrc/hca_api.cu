@@ -882,7 +882,7 @@ extern "C" hca_status_t hca_dsa_index(const void* q_idx, const float* w_idx, con
     p.scores = scores;
     p.B = B; p.HI = HI; p.Lmax = Lmax; p.ntile = (Lmax + 127) / 128;
     p.total = (long long)B * p.ntile;
-    const long long grid = std::min<long long>(p.total, ns);
+    const long long grid = std::min<long long>(p.total, 2LL * ns);   // two CTAs per SM
     dsa_index_kernel<<<(unsigned)grid, kIdxThreads, kIdxSmem, reinterpret_cast<cudaStream_t>(stream)>>>(p, tq, tk);
     return launch_status();
 }
@@ -890,7 +890,7 @@ extern "C" hca_status_t hca_dsa_index(const void* q_idx, const float* w_idx, con
 extern "C" hca_status_t hca_dsa_topk(const float* scores, const int* seqlens, int* idx, int B, int Lmax, int k,
                                      hca_stream_t stream) {
     using namespace hca;
-    if (B < 0 || Lmax < 1 || k < 1) return HCA_ERR_INVALID_ARG;
+    if (B < 0 || Lmax < 1 || k < 1 || B > (1 << 28)) return HCA_ERR_INVALID_ARG;
     if (B == 0) return HCA_OK;
     if (!scores || !seqlens || !idx || (reinterpret_cast<uintptr_t>(scores) & 3) ||
         (reinterpret_cast<uintptr_t>(seqlens) & 3) || (reinterpret_cast<uintptr_t>(idx) & 3))
@@ -900,8 +900,24 @@ extern "C" hca_status_t hca_dsa_topk(const float* scores, const int* seqlens, in
     p.seqlens = seqlens;
     p.idx = idx;
     p.B = B; p.Lmax = Lmax; p.k = k;
-    dsa_topk_kernel<<<(unsigned)B, kTopkThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
-    return launch_status();
+    // a cluster of kTopkCluster CTAs per sequence
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kTopkCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)((long long)kTopkCluster * B), 1, 1);
+    cfg.blockDim = dim3(kTopkThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, dsa_topk_kernel, p) != cudaSuccess) {
+        cudaGetLastError();
+        return HCA_ERR_CUDA;
+    }
+    return HCA_OK;
 }
 
 extern "C" hca_status_t hca_dsa_attend(const void* q, const void* k, const void* v, const int* idx, const int* seqlens,
