@@ -19,10 +19,10 @@
 //                      digit passes of 11 / 11 / 10 bits over order-preserving integer keys,
 //                      warp-aggregated shared-memory histograms), then one ordered pass that keeps
 //                      every larger score and the first equal ones, positions ascending.
-//   dsa_attend_kernel  one CTA per sequence: the query heads (64 x 256 bf16) stay in shared
+//   dsa_attend_kernel  two CTAs per sequence: the query heads (64 x 256 bf16) stay in shared
 //                      memory; per tile of 128 kept positions, the key rows and then the value
-//                      rows are gathered with 16-byte asynchronous copies into 128-byte-swizzled
-//                      slabs (a warp copies one 512-byte row per instruction), S^T = K Q^T and
+//                      rows are gathered by TMA (tile::gather4: four 128-byte row segments per
+//                      copy) into 128-byte-swizzled slabs, S^T = K Q^T and
 //                      O^T += V^T P^T run on tcgen05 (as in the HCA decode), and four warps run an
 //                      online softmax with a lazily moved reference maximum.
 // Every wait is bounded (common.cuh).
@@ -506,15 +506,22 @@ struct DsaAttendParams {
     const int* seqlens;
     float* out;              // [B, Hq, 256]
     int B, Hq, Lmax, kmax;
+    int rows;                // rows of the key / value maps (B * Lmax): a row index past every row
     float scale_log2;
 };
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
+// Four rows of a 2-D map (one row high box of 64 bf16 channels, 128-byte swizzle) gathered into
+// four consecutive 128-byte rows of a swizzled slab; completion counted in bytes on `bar`.  A row
+// index past the map's rows reads zeros.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int r0, int r1,
+                                            int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)),
+           "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int n>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(n) : "memory"); }
 
 // Column reduction of 32 values per lane across a warp: returns, in lane c, the max (or sum)
 // over the 32 lanes of column c (a butterfly that halves the columns kept at each step).
@@ -534,30 +541,27 @@ __device__ __forceinline__ float dsa_colred32(float* t, int lane) {
     return t[0];
 }
 
-// Rows 32 w .. 32 w + 31 of a 128-row tile of gathered 512-byte rows (positions idx[row], -1 or
-// past `count`: zeros) into four 128-byte-swizzled slabs of 64 channels; lane l copies 16 bytes
-// of channel chunk l of a row, so one instruction moves one whole row.
-__device__ __forceinline__ void dsa_gather_rows(uint8_t* dst, const __nv_bfloat16* src_b, const int* idx_t, int nvalid,
-                                                int Lmax, int w, int lane) {
-    const int slab = lane >> 3, c = lane & 7;
-    // the warp's 32 positions in one coalesced load, handed to the whole warp row by row
+// Rows 32 w .. 32 w + 31 of a 128-row tile of gathered 512-byte rows (positions idx[row] of the
+// sequence whose first map row is row0) into four 128-byte-swizzled slabs of 64 channels: lane l
+// issues one gather4 of rows 32 w + 4 (l >> 2) .. + 3 for slab l & 3.  Positions -1, rows past
+// `nvalid` and positions past Lmax (reported) read zeros (row index `oob`, past the map).  The
+// warp's 16 KB are announced on `bar` before any copy is issued.
+__device__ __forceinline__ void dsa_gather_tile(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int row0,
+                                                const int* idx_t, int nvalid, int Lmax, int oob, int w, int lane) {
     const int mine = 32 * w + lane < nvalid ? __ldg(idx_t + 32 * w + lane) : -1;
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) {
-        const int row = 32 * w + i;
-        uint8_t* d = dst + slab * kAttSlab + dsa_sw(row, c);
-        int pos = __shfl_sync(0xffffffffu, mine, i);
-        if (pos >= Lmax) {                      // a position past the buffer: reported, not read
-            if (lane == 0) record_error(HCA_ERR_DEVICE_INPUT);
-            pos = -1;
-        }
-        if (pos >= 0) cp_async16(d, src_b + (size_t)pos * kDsaD + 8 * lane);
-        else *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
-    }
+    if (__any_sync(0xffffffffu, mine >= Lmax) && lane == 0) record_error(HCA_ERR_DEVICE_INPUT);
+    const int row = (mine >= 0 && mine < Lmax) ? row0 + mine : oob;
+    if (lane == 0) mbar_arrive_expect_tx(bar, 32 * 4 * 128);
+    __syncwarp();
+    const int g = lane >> 2, slab = lane & 3;
+    const int r0 = __shfl_sync(0xffffffffu, row, 4 * g), r1 = __shfl_sync(0xffffffffu, row, 4 * g + 1);
+    const int r2 = __shfl_sync(0xffffffffu, row, 4 * g + 2), r3 = __shfl_sync(0xffffffffu, row, 4 * g + 3);
+    tma_gather4(dst + slab * kAttSlab + (32 * w + 4 * g) * 128, m, bar, 64 * slab, r0, r1, r2, r3);
 }
 
 __global__ void __launch_bounds__(kAttThreads, 1)
-dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap tm_q) {
+dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     extern __shared__ __align__(1024) uint8_t dsmem[];
     if (smem_u32(dsmem) & 1023u) {
         if (threadIdx.x == 0) record_error(HCA_ERR_INTERNAL);
@@ -566,12 +570,13 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
     uint8_t* sm = dsmem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kAttSmBar);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;        // 4 worker warps: the tile's key rows are in place
+    uint64_t* k_full = bars + 1;        // 4 worker warps' gathers: the tile's key rows are in place
     uint64_t* s_full = bars + 2;        // S^T of the tile is in tensor memory (commit)
     uint64_t* s_read = bars + 3;        // 4 worker warps: S^T read
     uint64_t* p_full = bars + 4;        // 4 worker warps: P^T and the value rows are in place
     uint64_t* pv_done = bars + 5;       // O^T += V^T P^T done (commit)
     uint64_t* drain = bars + 6;
+    uint64_t* v_full = bars + 7;        // 4 worker warps' gathers: the tile's value rows are in place
     int* misc = reinterpret_cast<int*>(sm + kAttSmBar + 16 * 8);
     volatile int* abort_flag = misc;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 1);
@@ -600,6 +605,7 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
         mbar_init(p_full, 4);
         mbar_init(pv_done, 1);
         mbar_init(drain, 1);
+        mbar_init(v_full, 4);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, 256);
@@ -613,6 +619,8 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
     if (warp == 0) {
         // ================================================================ MMA issuer (+ query load)
         if (lane == 0 && nt > 0) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(q_full, 4 * kAttQSlab);
             for (int s = 0; s < 4; ++s) tma_load_4d(sm + kAttSmQ + s * kAttQSlab, &tm_q, q_full, 64 * s, 0, b, 0);
         }
@@ -635,6 +643,7 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             }
             __syncwarp();
             if (!warp_wait(p_full, j & 1, abort_flag)) { ok = false; break; }
+            if (!warp_wait(v_full, j & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t vb = smem_u32(sm + kAttSmV), pb = smem_u32(sm + kAttSmP);
@@ -659,32 +668,30 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
         const int w = warp & 3;
         const int r = 32 * w + lane;
         const uint32_t lane_off = (uint32_t)(32 * w) << 16;
-        const __nv_bfloat16* kb = p.k + (size_t)b * p.Lmax * kDsaD;
-        const __nv_bfloat16* vb = p.v + (size_t)b * p.Lmax * kDsaD;
+        const int row0 = b * p.Lmax;    // the sequence's first row in the key / value maps
+        int n_issued = 0;               // tiles whose key gathers were issued (value: one fewer or equal)
+        int v_issued = 0;
         float lsum[64];
 #pragma unroll
         for (int h = 0; h < 64; ++h) lsum[h] = 0.f;
         bool ok = true;
         if (nt > 0) {
-            dsa_gather_rows(sm + kAttSmK, kb, idx_b + 128 * jt0, count - 128 * jt0, p.Lmax, w, lane);
-            cp_async_commit();
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(k_full);
+            dsa_gather_tile(sm + kAttSmK, &tm_k, k_full, row0, idx_b + 128 * jt0, count - 128 * jt0, p.Lmax, p.rows, w,
+                            lane);
+            n_issued = 1;
         }
         for (int j = 0; ok && j < nt; ++j) {
             const int* idx_t = idx_b + 128 * (jt0 + j);
             const int nvalid = count - 128 * (jt0 + j);
             // the value rows of this tile (the previous PV is done: waited at the end of the last tile)
-            dsa_gather_rows(sm + kAttSmV, vb, idx_t, nvalid, p.Lmax, w, lane);
-            cp_async_commit();
+            dsa_gather_tile(sm + kAttSmV, &tm_v, v_full, row0, idx_t, nvalid, p.Lmax, p.rows, w, lane);
+            ++v_issued;
             if (!dsa_group_wait128(s_full, j & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             // S^T is in tensor memory, so the key buffer is free: the next tile's keys start now
             if (j + 1 < nt) {
-                dsa_gather_rows(sm + kAttSmK, kb, idx_t + 128, nvalid - 128, p.Lmax, w, lane);
-                cp_async_commit();
+                dsa_gather_tile(sm + kAttSmK, &tm_k, k_full, row0, idx_t + 128, nvalid - 128, p.Lmax, p.rows, w, lane);
+                ++n_issued;
             }
             float z[64];
 #pragma unroll
@@ -757,23 +764,19 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<uint4*>(sm + kAttSmP + dsa_sw(r, c)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            // this tile's value rows have landed (the next tile's keys may still be in flight)
-            if (j + 1 < nt) cp_async_wait<1>();
-            else cp_async_wait<0>();
+            // P^T is written (the MMA issuer also waits for the value rows)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
-            if (j + 1 < nt) {
-                cp_async_wait<0>();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(k_full);
-            }
             // PV of this tile done: the value and P buffers are free and O^T is stable
             if (!dsa_group_wait128(pv_done, j & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
         }
-        cp_async_wait<0>();
+        // gathers still in flight after an abort land before the buffers are reused or released
+        if (threadIdx.x == 32) {
+            if (n_issued) mbar_drain_wait(k_full, (n_issued - 1) & 1);
+            if (v_issued) mbar_drain_wait(v_full, (v_issued - 1) & 1);
+        }
         // ---- this CTA's softmax sums per head (column sums, then the 4 warps) and its max
         {
             float t[32];

@@ -80,6 +80,21 @@ bool make_tmap_4d_plain(CUtensorMap* m, void* base, int esize, uint64_t d0, uint
     return r == CUDA_SUCCESS;
 }
 
+// 2-D bf16 tensor map over `rows` rows of d0 contiguous elements, box {b0, 1} (one row high, as
+// tile::gather4 copies need), 128-byte swizzle (b0 * 2 bytes must be 128).
+bool make_tmap_rows(CUtensorMap* m, const void* base, uint64_t d0, uint64_t rows, uint32_t b0) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {d0, rows};
+    cuuint64_t strides[1] = {d0 * 2};
+    cuuint32_t box[2] = {b0, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel slot, device).
 bool set_smem_attr_once(const void* fn, int bytes, int slot) {
     static std::mutex mu;
@@ -933,34 +948,47 @@ extern "C" hca_status_t hca_dsa_attend(const void* q, const void* k, const void*
         (reinterpret_cast<uintptr_t>(idx) & 3) || (reinterpret_cast<uintptr_t>(seqlens) & 3) ||
         (reinterpret_cast<uintptr_t>(out) & 3))
         return HCA_ERR_INVALID_ARG;
-    CUtensorMap tq;
-    if (!make_tmap_4d(&tq, q, kDsaD, Hq, B, 1, kDsaD, (uint64_t)kDsaD * Hq, (uint64_t)kDsaD * Hq * B, 64, 64, 1, 1))
-        return HCA_ERR_CUDA;
     if (!set_smem_attr_once(reinterpret_cast<const void*>(&dsa_attend_kernel), (int)kAttSmem, 11)) return HCA_ERR_CUDA;
-    DsaAttendParams p;
-    p.k = static_cast<const __nv_bfloat16*>(k);
-    p.v = static_cast<const __nv_bfloat16*>(v);
-    p.idx = idx;
-    p.seqlens = seqlens;
-    p.out = out;
-    p.B = B; p.Hq = Hq; p.Lmax = Lmax; p.kmax = kmax;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    // a cluster of two CTAs per sequence (each takes half of the kept positions)
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(2 * B), 1, 1);
-    cfg.blockDim = dim3(kAttThreads, 1, 1);
-    cfg.dynamicSmemBytes = kAttSmem;
-    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, dsa_attend_kernel, p, tq) != cudaSuccess) {
-        cudaGetLastError();
-        return HCA_ERR_CUDA;
+    // the key / value maps index rows with 32-bit coordinates, one past the last row meaning
+    // "zeros": launch over groups of sequences whose rows stay below 2^31
+    const long long per = std::max<long long>(1, std::min<long long>(B, (long long)INT32_MAX / Lmax - 1));
+    for (long long b0 = 0; b0 < B; b0 += per) {
+        const int nb = (int)std::min<long long>(per, B - b0);
+        const size_t row_off = (size_t)b0 * Lmax * kDsaD;
+        const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k) + row_off;
+        const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v) + row_off;
+        const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q) + (size_t)b0 * Hq * kDsaD;
+        CUtensorMap tq, tk, tv;
+        if (!make_tmap_4d(&tq, qb, kDsaD, Hq, nb, 1, kDsaD, (uint64_t)kDsaD * Hq, (uint64_t)kDsaD * Hq * nb, 64, 64, 1, 1) ||
+            !make_tmap_rows(&tk, kb, kDsaD, (uint64_t)nb * Lmax, 64) ||
+            !make_tmap_rows(&tv, vb, kDsaD, (uint64_t)nb * Lmax, 64))
+            return HCA_ERR_CUDA;
+        DsaAttendParams p;
+        p.k = kb;
+        p.v = vb;
+        p.idx = idx + (size_t)b0 * kmax;
+        p.seqlens = seqlens + b0;
+        p.out = out + (size_t)b0 * Hq * kDsaD;
+        p.B = nb; p.Hq = Hq; p.Lmax = Lmax; p.kmax = kmax;
+        p.rows = (int)((long long)nb * Lmax);
+        p.scale_log2 = scale * 1.4426950408889634f;
+        // a cluster of two CTAs per sequence (each takes half of the kept positions)
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(2 * nb), 1, 1);
+        cfg.blockDim = dim3(kAttThreads, 1, 1);
+        cfg.dynamicSmemBytes = kAttSmem;
+        cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, dsa_attend_kernel, p, tq, tk, tv) != cudaSuccess) {
+            cudaGetLastError();
+            return HCA_ERR_CUDA;
+        }
     }
     return HCA_OK;
 }

@@ -184,6 +184,9 @@ hca_status_t hca_dsa_topk(const float* scores, const int* seqlens, int* idx, int
  *        an entry >= Lmax is reported as HCA_ERR_DEVICE_INPUT and not read)
  *   seqlens [B] int32;  out [B,Hq,d] fp32;  scale: logit scale (typically 1/sqrt(d))
  * Supported: d == 256, Hq <= 64.  bf16 operands, fp32 accumulation, P rounded to bf16.
+ * A sequence with L_b = 0 keeps no position: its output is NaN (a softmax over nothing).
+ * Sequences are launched in groups whose B_group * Lmax stays below 2^31 (one launch at the
+ * usual sizes).
  */
 hca_status_t hca_dsa_attend(const void* q, const void* k, const void* v, const int* idx, const int* seqlens,
                             float* out, int B, int Hq, int d, int Lmax, int kmax, float scale,
