@@ -23,8 +23,9 @@
 //                      memory; per tile of 128 kept positions, the key rows and then the value
 //                      rows are gathered by TMA (tile::gather4: four 128-byte row segments per
 //                      copy) into 128-byte-swizzled slabs, S^T = K Q^T and
-//                      O^T += V^T P^T run on tcgen05 (as in the HCA decode), and four warps run an
-//                      online softmax with a lazily moved reference maximum.
+//                      O^T += V^T P^T run on tcgen05 (as in the HCA decode), four warps run an
+//                      online softmax with a lazily moved reference maximum, and four more issue
+//                      the gathers as soon as a buffer is free.
 // Every wait is bounded (common.cuh).
 #pragma once
 
@@ -484,7 +485,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
 
 // ------------------------------------------------------------------------------------- attention
 
-constexpr int kAttThreads = 160;           // MMA issuer, 4 gather / softmax warps
+constexpr int kAttThreads = 288;           // MMA issuer, 4 softmax warps, 4 gather warps
 constexpr uint32_t kAttSlab = 128 * 128;   // 128 rows x 64 channels bf16
 constexpr uint32_t kAttQSlab = 64 * 128;   // 64 heads x 64 channels
 constexpr uint32_t kAttSmQ = 0;                                  // 4 x 8 KB
@@ -494,7 +495,8 @@ constexpr uint32_t kAttSmP = kAttSmV + 4 * kAttSlab;             // 128 keys x 6
 constexpr uint32_t kAttSmRed = kAttSmP + kAttSlab;               // float [4][64]
 constexpr uint32_t kAttSmM = kAttSmRed + 4 * 64 * 4;             // float [64] reference max
 constexpr uint32_t kAttSmA = kAttSmM + 64 * 4;                   // float [64] rescale factors
-constexpr uint32_t kAttSmBar = kAttSmA + 64 * 4;
+constexpr uint32_t kAttSmL = kAttSmA + 64 * 4;                   // float4 [16][128] running sums
+constexpr uint32_t kAttSmBar = kAttSmL + 16 * 128 * 16;
 constexpr uint32_t kAttSmem = kAttSmBar + 16 * 8 + 32;
 static_assert(kAttSmem <= 232448, "attention shared memory exceeds the per-block limit");
 constexpr float kAttRescale = 8.0f;        // move the reference max only when exceeded by 2^8
@@ -541,14 +543,19 @@ __device__ __forceinline__ float dsa_colred32(float* t, int lane) {
     return t[0];
 }
 
-// Rows 32 w .. 32 w + 31 of a 128-row tile of gathered 512-byte rows (positions idx[row] of the
-// sequence whose first map row is row0) into four 128-byte-swizzled slabs of 64 channels: lane l
-// issues one gather4 of rows 32 w + 4 (l >> 2) .. + 3 for slab l & 3.  Positions -1, rows past
-// `nvalid` and positions past Lmax (reported) read zeros (row index `oob`, past the map).  The
-// warp's 16 KB are announced on `bar` before any copy is issued.
+// The position of row 32 w + lane of kept-position tile jj (-1 past the tile count or the kept count).
+__device__ __forceinline__ int dsa_tile_pos(const int* idx_b, int jj, int count, int w, int lane) {
+    const int row = 128 * jj + 32 * w + lane;
+    return row < count ? __ldg(idx_b + row) : -1;
+}
+
+// Rows 32 w .. 32 w + 31 of a 128-row tile of gathered 512-byte rows (lane l holds the position
+// `mine` of row 32 w + l, in the sequence whose first map row is row0) into four 128-byte-swizzled
+// slabs of 64 channels: lane l issues one gather4 of rows 32 w + 4 (l >> 2) .. + 3 for slab l & 3.
+// Positions -1 and positions past Lmax (reported) read zeros (row index `oob`, past the map).
+// The warp's 16 KB are announced on `bar` before any copy is issued.
 __device__ __forceinline__ void dsa_gather_tile(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int row0,
-                                                const int* idx_t, int nvalid, int Lmax, int oob, int w, int lane) {
-    const int mine = 32 * w + lane < nvalid ? __ldg(idx_t + 32 * w + lane) : -1;
+                                                int mine, int Lmax, int oob, int w, int lane) {
     if (__any_sync(0xffffffffu, mine >= Lmax) && lane == 0) record_error(HCA_ERR_DEVICE_INPUT);
     const int row = (mine >= 0 && mine < Lmax) ? row0 + mine : oob;
     if (lane == 0) mbar_arrive_expect_tx(bar, 32 * 4 * 128);
@@ -662,37 +669,54 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             mbar_drain_wait(drain, 0);
         }
         __syncwarp();
+    } else if (warp >= 5) {
+        // ================================================================ gathers
+        // warp 5 + w fetches rows 32 w .. 32 w + 31 of every tile: the keys of tile j + 1 as soon
+        // as S^T of tile j is in tensor memory, the values of tile j once PV of tile j - 1 is done
+        const int w = warp - 5;
+        const int row0 = b * p.Lmax;    // the sequence's first row in the key / value maps
+        int k_issued = 0, v_issued = 0;
+        // each tile's positions are loaded one tile ahead of their key gather (the value gather
+        // of the same tile reuses them)
+        int cur = nt > 0 ? dsa_tile_pos(idx_b, jt0, count, w, lane) : -1;
+        if (nt > 0) {
+            dsa_gather_tile(sm + kAttSmK, &tm_k, k_full, row0, cur, p.Lmax, p.rows, w, lane);
+            k_issued = 1;
+        }
+        for (int j = 0; j < nt; ++j) {
+            const int nxt = j + 1 < nt ? dsa_tile_pos(idx_b, jt0 + j + 1, count, w, lane) : -1;
+            if (j > 0 && !warp_wait(pv_done, (j - 1) & 1, abort_flag)) break;
+            dsa_gather_tile(sm + kAttSmV, &tm_v, v_full, row0, cur, p.Lmax, p.rows, w, lane);
+            ++v_issued;
+            if (j + 1 < nt) {
+                if (!warp_wait(s_full, j & 1, abort_flag)) break;
+                dsa_gather_tile(sm + kAttSmK, &tm_k, k_full, row0, nxt, p.Lmax, p.rows, w, lane);
+                ++k_issued;
+            }
+            cur = nxt;
+        }
+        // gathers still in flight (after an abort) land before the buffers are reused or released
+        if (lane == 0) {
+            if (k_issued) mbar_drain_wait(k_full, (k_issued - 1) & 1);
+            if (v_issued) mbar_drain_wait(v_full, (v_issued - 1) & 1);
+        }
+        __syncwarp();
     } else {
-        // ================================================================ gathers, softmax, epilogue
+        // ================================================================ softmax, epilogue
         // a warp reaches only the TMEM lane quarter (warp id mod 4): rows / lanes 32 w .. 32 w + 31
         const int w = warp & 3;
         const int r = 32 * w + lane;
         const uint32_t lane_off = (uint32_t)(32 * w) << 16;
-        const int row0 = b * p.Lmax;    // the sequence's first row in the key / value maps
-        int n_issued = 0;               // tiles whose key gathers were issued (value: one fewer or equal)
-        int v_issued = 0;
-        float lsum[64];
+        // this thread's running softmax sums of heads 4 i .. 4 i + 3 at lsum[128 i + r] (shared
+        // memory, consecutive threads on consecutive 16-byte words)
+        float4* lsum = reinterpret_cast<float4*>(sm + kAttSmL);
 #pragma unroll
-        for (int h = 0; h < 64; ++h) lsum[h] = 0.f;
+        for (int i = 0; i < 16; ++i) lsum[128 * i + r] = make_float4(0.f, 0.f, 0.f, 0.f);
         bool ok = true;
-        if (nt > 0) {
-            dsa_gather_tile(sm + kAttSmK, &tm_k, k_full, row0, idx_b + 128 * jt0, count - 128 * jt0, p.Lmax, p.rows, w,
-                            lane);
-            n_issued = 1;
-        }
         for (int j = 0; ok && j < nt; ++j) {
-            const int* idx_t = idx_b + 128 * (jt0 + j);
             const int nvalid = count - 128 * (jt0 + j);
-            // the value rows of this tile (the previous PV is done: waited at the end of the last tile)
-            dsa_gather_tile(sm + kAttSmV, &tm_v, v_full, row0, idx_t, nvalid, p.Lmax, p.rows, w, lane);
-            ++v_issued;
             if (!dsa_group_wait128(s_full, j & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            // S^T is in tensor memory, so the key buffer is free: the next tile's keys start now
-            if (j + 1 < nt) {
-                dsa_gather_tile(sm + kAttSmK, &tm_k, k_full, row0, idx_t + 128, nvalid - 128, p.Lmax, p.rows, w, lane);
-                ++n_issued;
-            }
             float z[64];
 #pragma unroll
             for (int c = 0; c < 64; c += 16) tmem_ld16(tmem + lane_off + tS + c, z + c);
@@ -726,6 +750,9 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
                 }
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
+            // PV of the previous tile done: O^T is stable and the P buffer free
+            if (j > 0 && !dsa_group_wait128(pv_done, (j - 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
             bool any = false;
             if (j > 0)
 #pragma unroll
@@ -733,7 +760,11 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             if (any) {
                 // O^T rows (channels 128 c + r) times alpha per head column; PV of the last tile is done
 #pragma unroll
-                for (int h = 0; h < 64; ++h) lsum[h] *= alpha[h];
+                for (int i = 0; i < 16; ++i) {
+                    float4 l = lsum[128 * i + r];
+                    l.x *= alpha[4 * i]; l.y *= alpha[4 * i + 1]; l.z *= alpha[4 * i + 2]; l.w *= alpha[4 * i + 3];
+                    lsum[128 * i + r] = l;
+                }
 #pragma unroll 1
                 for (int c = 0; c < 2; ++c)
 #pragma unroll 1
@@ -754,11 +785,14 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             // the same rounded values (numerator and normaliser use identical weights)
             uint32_t pk[32];
 #pragma unroll
-            for (int h = 0; h < 64; h += 2) {
-                const uint32_t u = pack_bf16x2(ex2(z[h] - mref[h]), ex2(z[h + 1] - mref[h + 1]));
-                lsum[h] += bf16lo(u);
-                lsum[h + 1] += bf16hi(u);
-                pk[h >> 1] = u;
+            for (int h = 0; h < 64; h += 2)
+                pk[h >> 1] = pack_bf16x2(ex2(z[h] - mref[h]), ex2(z[h + 1] - mref[h + 1]));
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float4 l = lsum[128 * i + r];
+                l.x += bf16lo(pk[2 * i]); l.y += bf16hi(pk[2 * i]);
+                l.z += bf16lo(pk[2 * i + 1]); l.w += bf16hi(pk[2 * i + 1]);
+                lsum[128 * i + r] = l;
             }
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -768,22 +802,20 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
-            // PV of this tile done: the value and P buffers are free and O^T is stable
-            if (!dsa_group_wait128(pv_done, j & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
         }
-        // gathers still in flight after an abort land before the buffers are reused or released
-        if (threadIdx.x == 32) {
-            if (n_issued) mbar_drain_wait(k_full, (n_issued - 1) & 1);
-            if (v_issued) mbar_drain_wait(v_full, (v_issued - 1) & 1);
-        }
+        // the last PV is done before O^T is read
+        if (ok && nt > 0 && !dsa_group_wait128(pv_done, (nt - 1) & 1, abort_flag)) ok = false;
+        tc_fence_after();
         // ---- this CTA's softmax sums per head (column sums, then the 4 warps) and its max
         {
             float t[32];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) t[i] = lsum[32 * half + i];
+                for (int i = 0; i < 8; ++i) {
+                    const float4 l = lsum[128 * (8 * half + i) + r];
+                    t[4 * i] = l.x; t[4 * i + 1] = l.y; t[4 * i + 2] = l.z; t[4 * i + 3] = l.w;
+                }
                 red[w * 64 + 32 * half + lane] = dsa_colred32<false>(t, lane);
             }
         }
@@ -803,9 +835,11 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
     tc_fence_after();
     // rank 0 no longer reads its key / value buffers (its MMAs are drained): rank 1 may write there
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    float* o1 = reinterpret_cast<float*>(sm + kAttSmK);              // rank 1's O^T [256 ch][64 heads]
+    // rank 1's O^T [256 ch][64 heads], each 256-byte channel row's 16-byte chunks XOR-swizzled by
+    // the row's low four bits, so that 32 threads on 32 consecutive rows touch all banks
+    float* o1 = reinterpret_cast<float*>(sm + kAttSmK);
     float* ml1 = reinterpret_cast<float*>(sm + kAttSmV);             // rank 1's max [64], sum [64], ok
-    if (rank == 1 && warp >= 1) {
+    if (rank == 1 && warp >= 1 && warp <= 4) {
         const int w = warp & 3;
         const int r = 32 * w + lane;
         const uint32_t lane_off = (uint32_t)(32 * w) << 16;
@@ -824,11 +858,13 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
 #pragma unroll
                     for (int i = 0; i < 16; ++i) o[i] = 0.f;
                 }
-                const uint32_t dst = ro + (uint32_t)(((128 * c + r) * 64 + c16) * 4);
+                const int row = 128 * c + r;
+                const uint32_t dst = ro + (uint32_t)(row * 256);
 #pragma unroll
                 for (int i = 0; i < 16; i += 4)
                     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
-                                 :: "r"(dst + 4 * i), "f"(o[i]), "f"(o[i + 1]), "f"(o[i + 2]), "f"(o[i + 3]) : "memory");
+                                 :: "r"(dst + 16 * (((c16 + i) >> 2) ^ (row & 15))), "f"(o[i]), "f"(o[i + 1]),
+                                    "f"(o[i + 2]), "f"(o[i + 3]) : "memory");
             }
         if (threadIdx.x >= 32 && threadIdx.x < 96) {
             const int h = threadIdx.x - 32;
@@ -840,7 +876,7 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
         tc_fence_before();
     }
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (rank == 0 && warp >= 1) {
+    if (rank == 0 && warp >= 1 && warp <= 4) {
         const int w = warp & 3;
         const int r = 32 * w + lane;
         const uint32_t lane_off = (uint32_t)(32 * w) << 16;
@@ -864,11 +900,17 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
                 float o[16];
                 tmem_ld16(tmem + lane_off + tO + 64 * c + c16, o);
                 tmem_wait_ld();
-                const float* x1 = o1 + (128 * c + r) * 64 + c16;
+                const int row = 128 * c + r;
+                float x1[16];
+#pragma unroll
+                for (int i = 0; i < 16; i += 4) {
+                    const float4 t = *reinterpret_cast<const float4*>(o1 + row * 64 + 4 * (((c16 + i) >> 2) ^ (row & 15)));
+                    x1[i] = t.x; x1[i + 1] = t.y; x1[i + 2] = t.z; x1[i + 3] = t.w;
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int h = c16 + i;
-                    if (h < p.Hq) ob[(size_t)h * kDsaD + 128 * c + r] = fmaf(o[i], red[h], x1[i] * red[64 + h]);
+                    if (h < p.Hq) ob[(size_t)h * kDsaD + row] = fmaf(o[i], red[h], x1[i] * red[64 + h]);
                 }
             }
         tc_fence_before();
