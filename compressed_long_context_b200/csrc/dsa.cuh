@@ -326,11 +326,12 @@ __device__ __forceinline__ void dsa_st_cluster(uint32_t a, int v) {
     asm volatile("st.shared::cluster.s32 [%0], %1;" :: "r"(a), "r"(v) : "memory");
 }
 
-// A cluster of kTopkCluster CTAs per sequence: each builds the digit histograms of its quarter of
-// the positions, rank 0 adds the four through distributed shared memory and picks the digit, and
-// in the last pass each CTA writes the kept positions of its quarter after those of the ranks
-// before it.
-__global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopkParams p) {
+// A cluster of kTopkCluster CTAs per sequence (two CTAs per SM, so that 64 sequences run in one
+// wave): each builds the digit histograms of its quarter of the positions, rank 0 adds the four
+// through distributed shared memory and picks the digit, each CTA counts its keys above the
+// digit from its own histogram, and in the last pass each CTA writes the kept positions of its
+// quarter after those of the ranks before it.
+__global__ void __launch_bounds__(kTopkThreads, 2) dsa_topk_kernel(const DsaTopkParams p) {
     __shared__ int hist[2048];
     __shared__ int wsum[33];
     __shared__ int sel[2];                  // [0] digit chosen, [1] remaining after the pass
@@ -349,6 +350,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
     const int q0 = min(L, (int)rank * qsize), q1 = min(L, q0 + qsize);
     uint32_t prefix = 0, pmask = 0;
     int remaining = kk;                     // how many of the largest keys still to place
+    int n_gt_q = 0, n_eq_q = 0;             // this quarter's keys above / equal to the threshold
     const bool vec = ((reinterpret_cast<uintptr_t>(sc) & 15u) == 0);
     auto load4 = [&](int s, float* f) {
         if (vec && s + 3 < q1) {
@@ -415,27 +417,25 @@ __global__ void __launch_bounds__(kTopkThreads, 1) dsa_topk_kernel(const DsaTopk
             prefix |= (uint32_t)sel[0] << shift;
             pmask |= (uint32_t)(nbins - 1) << shift;
             remaining = sel[1];
+            // this quarter's keys in bins above the chosen digit are all kept: their count, from its
+            // own histogram (the scan's barriers end the reads before the next pass clears it)
+            {
+                int c = 0;
+                for (int bin = sel[0] + 1 + tid; bin < nbins; bin += kTopkThreads) c += hist[bin];
+                if (pass == 2) n_eq_q = hist[sel[0]];
+                int t;
+                dsa_block_scan(c, wsum, &t);
+                n_gt_q += t;
+            }
         }
     }
     // keep every key above the threshold key `prefix` and the first `remaining` keys equal to it,
     // in position order.  With all positions kept the passes are skipped (prefix = 0, remaining =
-    // kk = L): every key is at least 0, so every position is kept.  First the ranks' counts, to
-    // place each quarter after the previous ones.
-    int n_gt = 0, n_eq = 0;
-    for (int base = q0; base < q1; base += 4 * kTopkThreads) {
-        const int s = base + 4 * tid;
-        float f[4];
-        load4(s, f);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const uint32_t key = dsa_key(f[e]);
-            n_gt += s + e < q1 && key > prefix;
-            n_eq += s + e < q1 && key == prefix;
-        }
-    }
-    int tot, tot_eq_q;
-    dsa_block_scan(n_gt, wsum, &tot);       // the quarter's counts: two scans, as a quarter may
-    dsa_block_scan(n_eq, wsum, &tot_eq_q);  // hold 2^16 positions or more
+    // kk = L): every key is at least 0, so every position is kept.  Each quarter's output starts
+    // after the kept positions of the quarters before it, from the ranks' counts.
+    // with every position kept (no passes), all count as above the threshold
+    int tot = kk < L ? n_gt_q : q1 - q0;
+    const int tot_eq_q = kk < L ? n_eq_q : 0;
     if (tid == 0) {
         dsa_st_cluster(dsa_mapa(&counts[2 * rank], 0), tot);
         dsa_st_cluster(dsa_mapa(&counts[2 * rank + 1], 0), tot_eq_q);
