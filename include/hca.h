@@ -28,9 +28,10 @@
  * Conventions for every entry point:
  *  - all tensor pointers are DEVICE pointers owned by the caller, dense row-major in the
  *    stated layout, 16-byte aligned; bf16 means IEEE bfloat16 bit patterns;
- *  - the library allocates no device memory and copies nothing between host and device
- *    (hca_get_device_error excepted); work is queued on `stream` and the call returns
- *    without waiting for it;
+ *  - no call allocates device memory and none copies between host and device
+ *    (hca_get_device_error excepted); the library's image holds one fixed 48 MiB device
+ *    array per GPU, the scratch of hca_decode_noalloc; work is queued on `stream` and the
+ *    call returns without waiting for it;
  *  - a call returns HCA_OK once the work is queued; HCA_ERR_INVALID_ARG for a NULL
  *    pointer, a misaligned pointer or a size out of range; HCA_ERR_UNSUPPORTED for a
  *    shape outside the supported set (nothing is launched in either case);
