@@ -26,6 +26,7 @@ EXPORTS = ("hca_compress", "hca_prefill", "hca_decode_workspace_size", "hca_deco
            "hca_vha", "hca_append_state_size", "hca_append", "hca_status_string", "hca_get_device_error",
            "hca_debug_set_wait_limit", "hca_debug_set_drop_slab", "hca_debug_wait_probe", "hca_gate_logits",
            "hca_prefill_backward_workspace_size", "hca_prefill_backward", "hca_debug_set_backward_segment",
+           "hca_debug_set_dsa_rows_limit",
            "hca_dsa_index", "hca_dsa_topk", "hca_dsa_attend")
 
 _lib = None
@@ -85,6 +86,8 @@ def load():
     lib.hca_dsa_attend.argtypes = [_vp] * 6 + [_i] * 5 + [_f, _vp]
     lib.hca_debug_set_backward_segment.restype = _i
     lib.hca_debug_set_backward_segment.argtypes = [_i]
+    lib.hca_debug_set_dsa_rows_limit.restype = _i
+    lib.hca_debug_set_dsa_rows_limit.argtypes = [ctypes.c_longlong]
     lib.hca_debug_set_wait_limit.restype = _i
     lib.hca_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong, _vp]
     lib.hca_debug_set_drop_slab.restype = _i

@@ -760,6 +760,18 @@ BwdLayout bwd_layout(long long B, long long T, long long Hq, long long Hkv, long
 
 }  // namespace
 
+namespace {
+// Row bound of one attention launch's key / value maps forced by hca_debug_set_dsa_rows_limit
+// (0: 2^31 - 1, the 32-bit coordinate range).
+std::atomic<long long> g_dsa_rows_limit{0};
+}  // namespace
+
+extern "C" hca_status_t hca_debug_set_dsa_rows_limit(long long rows) {
+    if (rows < 0) return HCA_ERR_INVALID_ARG;
+    g_dsa_rows_limit.store(rows);
+    return HCA_OK;
+}
+
 extern "C" hca_status_t hca_debug_set_backward_segment(int rows) {
     if (rows < 0) return HCA_ERR_INVALID_ARG;
     g_bwd_seg_rows.store(rows);
@@ -951,7 +963,9 @@ extern "C" hca_status_t hca_dsa_attend(const void* q, const void* k, const void*
     if (!set_smem_attr_once(reinterpret_cast<const void*>(&dsa_attend_kernel), (int)kAttSmem, 11)) return HCA_ERR_CUDA;
     // the key / value maps index rows with 32-bit coordinates, one past the last row meaning
     // "zeros": launch over groups of sequences whose rows stay below 2^31
-    const long long per = std::max<long long>(1, std::min<long long>(B, (long long)INT32_MAX / Lmax - 1));
+    const long long forced = g_dsa_rows_limit.load();
+    const long long limit = forced > 0 ? std::min<long long>(forced, INT32_MAX) : (long long)INT32_MAX;
+    const long long per = std::max<long long>(1, std::min<long long>(B, limit / Lmax - 1));
     for (long long b0 = 0; b0 < B; b0 += per) {
         const int nb = (int)std::min<long long>(per, B - b0);
         const size_t row_off = (size_t)b0 * Lmax * kDsaD;

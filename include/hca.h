@@ -386,6 +386,15 @@ hca_status_t hca_get_device_error(hca_stream_t stream);
 hca_status_t hca_debug_set_backward_segment(int rows);
 
 /*
+ * hca_debug_set_dsa_rows_limit -- test hook: hca_dsa_attend launches over groups of
+ * sequences whose B_group * Lmax stays below `rows` instead of below 2^31, so that small
+ * batches exercise the grouped launches that very large ones take; 0 restores the default.
+ * Process-wide; call it only while no attention call is being enqueued.
+ * HCA_ERR_INVALID_ARG for rows < 0.
+ */
+hca_status_t hca_debug_set_dsa_rows_limit(long long rows);
+
+/*
  * Test hooks for the bounded waits (not part of the computation; the paper has no
  * counterpart).  Every wait inside the kernels gives up after a wall-clock limit, records
  * HCA_ERR_TIMEOUT and lets the kernel unwind (free its tensor memory, return) instead of

@@ -199,6 +199,9 @@ def test_prefill_backward_rejects_before_launch(libhca):
     finally:
         assert libhca.hca_debug_set_backward_segment(0) == _lib.HCA_OK
     assert libhca.hca_debug_set_backward_segment(-1) == _lib.HCA_ERR_INVALID_ARG
+    assert libhca.hca_debug_set_dsa_rows_limit(1 << 20) == _lib.HCA_OK
+    assert libhca.hca_debug_set_dsa_rows_limit(0) == _lib.HCA_OK
+    assert libhca.hca_debug_set_dsa_rows_limit(-1) == _lib.HCA_ERR_INVALID_ARG
     # unsupported head dims, block, group size, flags
     assert call(d=64, dvd=64) == _lib.HCA_ERR_UNSUPPORTED
     assert call(blk=129) == _lib.HCA_ERR_UNSUPPORTED

@@ -138,6 +138,28 @@ def test_attend_matches_oracle(cuda_device, libhca, Hq, lengths, kmax, boost):
     assert err.max() <= MAX_TOL and err.mean() <= MEAN_TOL, (err.max(), err.mean())
 
 
+def test_attend_grouped_launches_match_one_launch(cuda_device, libhca):
+    """Sequences launched in groups (forced small row bound on the key / value maps): the
+    output equals the single launch's bit for bit, and the oracle's within the bar."""
+    lengths = [3000, 700, 2049, 1, 2500, 130, 3000]
+    B, Lmax, kmax = len(lengths), max(lengths), 1024
+    q, k, v, idx = attend_case(cuda_device, B, 64, Lmax, lengths, kmax, seed=41)
+    seq = torch.tensor(lengths, dtype=torch.int32, device=cuda_device)
+    idx_t = torch.tensor(idx, device=cuda_device)
+    one = hca.dsa_attend(q, k, v, idx_t, seq, 0.0625)
+    assert libhca.hca_debug_set_dsa_rows_limit(3 * Lmax) == 0      # two sequences per launch
+    try:
+        grouped = hca.dsa_attend(q, k, v, idx_t, seq, 0.0625)
+        torch.cuda.synchronize()
+    finally:
+        assert libhca.hca_debug_set_dsa_rows_limit(0) == 0
+    hca.get_device_error()
+    assert torch.equal(one, grouped)
+    ref = od.sparse_attend(f64(q), f64(k), f64(v), idx, 0.0625)
+    err = np.abs(grouped.cpu().numpy().astype(np.float64) - ref)
+    assert err.max() <= MAX_TOL and err.mean() <= MEAN_TOL, (err.max(), err.mean())
+
+
 def test_whole_step_matches_oracle(cuda_device, libhca):
     """Indexer inputs exact (small integers), attention inputs normal: the selection is
     bit-exact and the output within the attention bar."""
