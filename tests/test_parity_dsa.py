@@ -59,7 +59,10 @@ def test_index_and_topk_exact(cuda_device, libhca, HI, lengths, topk):
     assert np.array_equal(idx.cpu().numpy(), ridx)                    # bit-exact, ties included
 
 
-@pytest.mark.parametrize("topk,lengths", [(100, [5000, 3000, 7]), (1000, [5000, 1001, 999]), (4096, [3000, 5000])])
+@pytest.mark.parametrize("topk,lengths", [
+    (100, [5000, 3000, 7]), (1000, [5000, 1001, 999]), (4096, [3000, 5000]),
+    (70000, [300001, 150000, 70001, 69999]),    # quarters of 75K positions, k far above 2^16
+])
 def test_topk_exact_on_given_scores(cuda_device, libhca, topk, lengths):
     """Scores drawn by the test (coarse values: many ties, some -inf), the same array for both."""
     rs = np.random.RandomState(topk)
@@ -73,6 +76,19 @@ def test_topk_exact_on_given_scores(cuda_device, libhca, topk, lengths):
     hca.get_device_error()
     ref = od.select_topk(s.astype(np.float64), seq, topk)
     assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_all_equal_scores(cuda_device, libhca):
+    """Every score equal (one digit in every pass): the first k positions are kept, and with
+    more than 2^16 equal keys in a quarter the counts still place each quarter's output."""
+    lengths = np.array([280000, 5, 4097], dtype=np.int32)
+    s = torch.full((3, 280000), 0.75, device=cuda_device)
+    idx = hca.dsa_topk(s, torch.tensor(lengths, device=cuda_device), 100000)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    ref = od.select_topk(s.cpu().numpy().astype(np.float64), lengths, 100000)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+    assert np.array_equal(ref[0], np.arange(100000))
 
 
 def test_index_rounding_bound(cuda_device, libhca):
