@@ -271,9 +271,11 @@ struct DsaTopkParams {
     int B, Lmax, k;
 };
 
-// Order-preserving integer image of an fp32 score: larger scores give larger keys.
+// Order-preserving integer image of an fp32 score: larger scores give larger keys, equal
+// scores equal keys (-0 is taken as +0, as the two compare equal).
 __device__ __forceinline__ uint32_t dsa_key(float f) {
-    const uint32_t u = __float_as_uint(f);
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

@@ -173,7 +173,8 @@ hca_status_t hca_dsa_index(const void* q_idx, const float* w_idx, const void* k_
  * hca_dsa_topk -- the k positions of largest score of each sequence among 0 .. L_b - 1.
  *   scores [B,Lmax] fp32 (as hca_dsa_index writes them), seqlens [B] int32
  *   idx    [B,k] int32 output: kept positions in increasing order, then -1 where L_b < k
- * Equal scores are taken in increasing position order, so the result is unique.
+ * Equal scores are taken in increasing position order, so the result is unique (-0.0 and
+ * +0.0 are equal scores; scores must not be NaN).
  */
 hca_status_t hca_dsa_topk(const float* scores, const int* seqlens, int* idx, int B, int Lmax, int k,
                           hca_stream_t stream);

@@ -91,6 +91,20 @@ def test_topk_all_equal_scores(cuda_device, libhca):
     assert np.array_equal(ref[0], np.arange(100000))
 
 
+def test_topk_signed_zeros_are_equal(cuda_device, libhca):
+    """-0.0 and +0.0 are the same score: with the threshold at zero, the zeros are kept in
+    position order whatever their sign."""
+    rs = np.random.RandomState(5)
+    s = np.where(rs.rand(2, 20000) < 0.5, np.float32(0.0), np.float32(-0.0)).astype(np.float32)
+    s[:, ::7] = 1.0
+    lengths = np.array([20000, 9999], dtype=np.int32)
+    idx = hca.dsa_topk(torch.tensor(s, device=cuda_device), torch.tensor(lengths, device=cuda_device), 5000)
+    torch.cuda.synchronize()
+    hca.get_device_error()
+    ref = od.select_topk(s.astype(np.float64), lengths, 5000)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
 def test_index_rounding_bound(cuda_device, libhca):
     B, HI, Lmax = 2, 16, 3000
     g = torch.Generator(device=cuda_device).manual_seed(5)
