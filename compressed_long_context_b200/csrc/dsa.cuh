@@ -15,10 +15,12 @@
 //                      ring, one tcgen05 MMA chain gives the 128 x H_I dot products in tensor
 //                      memory (two buffers), four epilogue warps apply ReLU and the head weights
 //                      and write the scores (fp32).  HBM-bound on the keys.
-//   dsa_topk_kernel    one CTA per sequence: radix select of the k-th largest score (three
-//                      digit passes of 11 / 11 / 10 bits over order-preserving integer keys,
-//                      warp-aggregated shared-memory histograms), then one ordered pass that keeps
-//                      every larger score and the first equal ones, positions ascending.
+//   dsa_topk_kernel    a cluster of four CTAs per sequence, each over a quarter of the
+//                      positions: radix select of the k-th largest score (three digit passes of
+//                      11 / 11 / 10 bits over order-preserving integer keys, warp-aggregated
+//                      shared-memory histograms summed by rank 0 through distributed shared
+//                      memory), then one ordered pass that keeps every larger score and the
+//                      first equal ones, positions ascending.
 //   dsa_attend_kernel  two CTAs per sequence: the query heads (64 x 256 bf16) stay in shared
 //                      memory; per tile of 128 kept positions, the key rows and then the value
 //                      rows are gathered by TMA (tile::gather4: four 128-byte row segments per

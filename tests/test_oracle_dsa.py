@@ -107,6 +107,15 @@ def test_topk_bruteforce_small():
             assert list(got[got >= 0]) == ref
 
 
+def test_topk_signed_zeros_tie():
+    """-0.0 and +0.0 compare equal, so they are one score and tie by position."""
+    s = np.array([[-0.0, 0.0, -0.0, 1.0, 0.0, -0.0]])
+    got = dsa.select_topk(s, np.array([6]), 3)[0]
+    assert list(got) == [0, 1, 3]
+    ref = sorted(sorted(range(6), key=lambda i: (-s[0, i], i))[:3])     # brute force
+    assert list(got) == ref
+
+
 def _sdpa(q, kk, vv, sel, scale):
     """torch SDPA (float64) of one sequence over the positions in sel (a boolean mask)."""
     Hq = q.shape[0]
