@@ -596,7 +596,7 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
     float* alpha = reinterpret_cast<float*>(sm + kAttSmA);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // a cluster of two CTAs per sequence: rank 0 takes the first half of the kept tiles, rank 1
-    // the rest; rank 1 hands its partial (max, sum, O^T) to rank 0, which merges and writes out
+    // the rest; at the end they exchange partials and each merges and writes half the channels
     const int b = blockIdx.x >> 1;
     uint32_t rank;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
@@ -832,44 +832,46 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
         if (threadIdx.x == 32) misc[2] = ok ? 1 : 0;
         tc_fence_before();
     }
-    // ---- merge the two halves in rank 0: out = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M))
+    // ---- merge the two halves: out = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M)).
+    // Rank r writes the output channels 128 r .. 128 r + 127: each rank sends the other its
+    // (max, sum, ok) and its O^T rows of the other's channel half, then both merge the same way.
     __syncwarp();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // rank 0 no longer reads its key / value buffers (its MMAs are drained): rank 1 may write there
+    // neither rank reads its key / value buffers any more (its MMAs are drained): the peer may
+    // write there
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    // rank 1's O^T [256 ch][64 heads], each 256-byte channel row's 16-byte chunks XOR-swizzled by
-    // the row's low four bits, so that 32 threads on 32 consecutive rows touch all banks
-    float* o1 = reinterpret_cast<float*>(sm + kAttSmK);
-    float* ml1 = reinterpret_cast<float*>(sm + kAttSmV);             // rank 1's max [64], sum [64], ok
-    if (rank == 1 && warp >= 1 && warp <= 4) {
+    // the peer's O^T rows of this rank's channel half [128 ch][64 heads], each 256-byte row's
+    // 16-byte chunks XOR-swizzled by the row's low four bits, so that 32 threads on 32
+    // consecutive rows touch all banks; the peer's max [64], sum [64] and ok flag
+    float* ox = reinterpret_cast<float*>(sm + kAttSmK);
+    float* mlx = reinterpret_cast<float*>(sm + kAttSmV);
+    if (warp >= 1 && warp <= 4) {
         const int w = warp & 3;
         const int r = 32 * w + lane;
         const uint32_t lane_off = (uint32_t)(32 * w) << 16;
+        const uint32_t peer = rank ^ 1u;
         uint32_t ro, rml;
-        asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(ro) : "r"(smem_u32(o1)));
-        asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(rml) : "r"(smem_u32(ml1)));
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ro) : "r"(smem_u32(ox)), "r"(peer));
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rml) : "r"(smem_u32(mlx)), "r"(peer));
+        const uint32_t dst = ro + (uint32_t)(r * 256);
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c)
-#pragma unroll 1
-            for (int c16 = 0; c16 < 64; c16 += 16) {
-                float o[16];
-                if (nt > 0) {
-                    tmem_ld16(tmem + lane_off + tO + 64 * c + c16, o);
-                    tmem_wait_ld();
-                } else {
+        for (int c16 = 0; c16 < 64; c16 += 16) {
+            float o[16];
+            if (nt > 0) {
+                tmem_ld16(tmem + lane_off + tO + 64 * peer + c16, o);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] = 0.f;
-                }
-                const int row = 128 * c + r;
-                const uint32_t dst = ro + (uint32_t)(row * 256);
-#pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
-                                 :: "r"(dst + 16 * (((c16 + i) >> 2) ^ (row & 15))), "f"(o[i]), "f"(o[i + 1]),
-                                    "f"(o[i + 2]), "f"(o[i + 3]) : "memory");
+                for (int i = 0; i < 16; ++i) o[i] = 0.f;
             }
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                             :: "r"(dst + 16 * (((c16 + i) >> 2) ^ (r & 15))), "f"(o[i]), "f"(o[i + 1]),
+                                "f"(o[i + 2]), "f"(o[i + 3]) : "memory");
+        }
         if (threadIdx.x >= 32 && threadIdx.x < 96) {
             const int h = threadIdx.x - 32;
             asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(rml + 4 * h), "f"(mref[h]) : "memory");
@@ -880,43 +882,48 @@ dsa_attend_kernel(const DsaAttendParams p, const __grid_constant__ CUtensorMap t
         tc_fence_before();
     }
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (rank == 0 && warp >= 1 && warp <= 4) {
+    if (warp >= 1 && warp <= 4) {
         const int w = warp & 3;
         const int r = 32 * w + lane;
         const uint32_t lane_off = (uint32_t)(32 * w) << 16;
         tc_fence_after();
         if (threadIdx.x >= 32 && threadIdx.x < 96) {
             const int h = threadIdx.x - 32;
-            const float m0 = mref[h], m1 = ml1[h];
+            // rank 0's and rank 1's (max, sum), whichever this rank is
+            const float m0 = rank ? mlx[h] : mref[h], l0 = rank ? mlx[64 + h] : alpha[h];
+            const float m1 = rank ? mref[h] : mlx[h], l1 = rank ? alpha[h] : mlx[64 + h];
             const float M = fmaxf(m0, m1);
             const float e0 = ex2(m0 - M), e1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
-            const float inv = 1.f / (alpha[h] * e0 + ml1[64 + h] * e1);
-            const bool good = misc[2] && ml1[128] != 0.f;
-            red[h] = good ? e0 * inv : NAN;          // weight of this CTA's O^T
+            const float inv = 1.f / (l0 * e0 + l1 * e1);
+            const bool good = misc[2] && mlx[128] != 0.f;
+            red[h] = good ? e0 * inv : NAN;          // weight of rank 0's O^T
             red[64 + h] = good ? e1 * inv : NAN;     // weight of rank 1's
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        float* ob = p.out + (size_t)b * p.Hq * kDsaD;
+        float* ob = p.out + (size_t)b * p.Hq * kDsaD + 128 * rank + r;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c)
-#pragma unroll 1
-            for (int c16 = 0; c16 < 64; c16 += 16) {
-                float o[16];
-                tmem_ld16(tmem + lane_off + tO + 64 * c + c16, o);
+        for (int c16 = 0; c16 < 64; c16 += 16) {
+            float o[16];
+            if (nt > 0) {
+                tmem_ld16(tmem + lane_off + tO + 64 * rank + c16, o);
                 tmem_wait_ld();
-                const int row = 128 * c + r;
-                float x1[16];
+            } else {
 #pragma unroll
-                for (int i = 0; i < 16; i += 4) {
-                    const float4 t = *reinterpret_cast<const float4*>(o1 + row * 64 + 4 * (((c16 + i) >> 2) ^ (row & 15)));
-                    x1[i] = t.x; x1[i + 1] = t.y; x1[i + 2] = t.z; x1[i + 3] = t.w;
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int h = c16 + i;
-                    if (h < p.Hq) ob[(size_t)h * kDsaD + row] = fmaf(o[i], red[h], x1[i] * red[64 + h]);
-                }
+                for (int i = 0; i < 16; ++i) o[i] = 0.f;
             }
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                const float4 t = *reinterpret_cast<const float4*>(ox + r * 64 + 4 * (((c16 + i) >> 2) ^ (r & 15)));
+                x[i] = t.x; x[i + 1] = t.y; x[i + 2] = t.z; x[i + 3] = t.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int h = c16 + i;
+                const float o0 = rank ? x[i] : o[i], o1 = rank ? o[i] : x[i];
+                if (h < p.Hq) ob[(size_t)h * kDsaD] = fmaf(o0, red[h], o1 * red[64 + h]);
+            }
+        }
         tc_fence_before();
     }
     __syncwarp();
